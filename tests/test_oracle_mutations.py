@@ -1,0 +1,53 @@
+"""Each plausible mistake planted in a temporary copy of the oracle must make
+at least one oracle pin fail.  Runs the pin suite on the mutated copy in a
+subprocess; CPU only."""
+
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "verification row scored": (
+        "rows = list(range(1, Qn)) if Qn > 1 else [0]", "rows = list(range(0, Qn))"),
+    "kmin term dropped": (
+        "np.maximum(qs[:, None, :] * lo[None], qs[:, None, :] * hi[None])", "qs[:, None, :] * hi[None]"),
+    "ties to the higher index": (
+        "key=lambda n: (-float(s[n]), n)", "key=lambda n: (-float(s[n]), -n)"),
+    "most recently used evicted": (
+        "stale.sort(key=lambda slot: (int(lu[b, h, slot]), int(st[b, h, slot])))",
+        "stale.sort(key=lambda slot: (-int(lu[b, h, slot]), int(st[b, h, slot])))"),
+    "stale slots before free ones": ("victims = free + stale", "victims = stale + free"),
+    "lowest-ranked misses fetched": (
+        "fetch = missing[:min(C, len(missing))]",
+        "fetch = missing[-min(C, len(missing)):] if missing and C else []"),
+    "masked tokens summarised": ("valid = min(P, ctx - n * P)\n            tokens", "valid = P\n            tokens"),
+    "hits not stamped": ("lu[b, h, resident[blk]] = step", "pass"),
+    "softmax scale dropped": ("logits = scale * (qh @ kt.T)  ", "logits = (qh @ kt.T)  "),
+    "output rows transposed": (
+        "reshape(Qn, G, D)\n            lse[b, :, h * G:(h + 1) * G] = (m + np.log(l)).reshape(Qn, G)\n"
+        "    return o, lse\n\n\ndef dense_attention",
+        "reshape(G, Qn, D).transpose(1, 0, 2)\n"
+        "            lse[b, :, h * G:(h + 1) * G] = (m + np.log(l)).reshape(Qn, G)\n"
+        "    return o, lse\n\n\ndef dense_attention"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTATIONS[name]
+    for sub in ("oracle", "tests", "lookahead_sparse_kv_b200"):
+        shutil.copytree(os.path.join(ROOT, sub), tmp_path / sub,
+                        ignore=shutil.ignore_patterns("*.so", "__pycache__", "_build"))
+    src_path = tmp_path / "oracle" / "oasis_oracle.py"
+    src = src_path.read_text()
+    assert src.count(old) == 1, f"mutation anchor not found once: {name}"
+    src_path.write_text(src.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        str(tmp_path / "tests" / "test_oracle.py")],
+                       cwd=tmp_path, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"no pin failed for planted mistake: {name}\n{r.stdout[-2000:]}"
