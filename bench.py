@@ -1,0 +1,608 @@
+"""Benchmark of the lookahead sparse-KV decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workload: Llama-3.1-8B-shaped attention layers at 32K context (batch 16,
+32 query / 8 KV heads, head dim 128, 2,048 blocks of 16 tokens per KV head,
+budget 2,048 tokens = 128 blocks, 1 verification + 4 draft queries, fetch cap
+16 blocks per head per step, AR(1)-drifting queries), synthetic bf16 data,
+stacked --layers deep (default 8, each layer with its own 2 GiB host KV) so
+that a layer's host-to-HBM transfer overlaps the other layers' work as in
+the OasisKV pipeline (Figure 8).  One step = one decode step through every
+layer: per layer, sparse attention over the resident pool, lookahead scores,
+top-K selection, the capped fetch plan and the gather of the missing blocks
+from pinned host memory.  Metric: layer-steps/s = layers x steps / time
+(whole job; weak scaling - every rank runs its own batch, no collective on
+the data path).
+
+Prints one JSON line (rank 0).  With --impl reference the CPU oracle runs the
+same configuration on the host cores (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import lookahead_sparse_kv_b200 as lsk                                    # noqa: E402
+from lookahead_sparse_kv_b200 import workloads as W                        # noqa: E402
+from lookahead_sparse_kv_b200.pipeline import DecodePipeline, LayerState  # noqa: E402
+
+WORKLOAD = "llama8b_32k"
+QUERY_RING = 256
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic_llama8b_32k.json")
+KERNELS = ("sparse_attn", "score_select", "plan_fetch", "prefetch")
+
+
+# ------------------------------------------------------------------ setup
+def ring_index(t: int, n: int) -> int:
+    """Index into a ring of n pre-generated query steps walked back and forth,
+    so consecutive steps stay consecutive points of the AR(1) path."""
+    if n <= 1:
+        return 0
+    p = t % (2 * n - 2)
+    return p if p < n else 2 * n - 2 - p
+
+
+def build_workload_state(w, steps: int, device="cuda", n_queries: int | None = None, layers: int = 1):
+    """Pinned host KV, per-layer device state, pipeline and resident queries
+    for `layers` layers of workload `w` (layer l draws its own KV and queries)."""
+    d = lsk.dims_for(w)
+    states, qrings, hosts = [], [], []
+    nq = n_queries if n_queries is not None else min(QUERY_RING, max(steps, 1))
+    for l in range(layers):
+        host = torch.empty((w.batch, w.n_kv_heads, w.max_blocks, 2, w.block_tokens, w.head_dim),
+                           dtype=torch.bfloat16, pin_memory=True)
+        W.make_host_kv(w, layer=l, device=device, out=host)
+        torch.cuda.synchronize()
+        states.append(LayerState(d, host, device))
+        qs = W.QueryStream(w, l, device)
+        qrings.append([qs.next() for _ in range(max(nq, 1))])
+        hosts.append(host)
+    pipe = DecodePipeline(d, states, W.initial_ctx_len(w, device), 1.0 / math.sqrt(w.head_dim), device)
+    pipe.build_summaries()
+    torch.cuda.synchronize()
+    return {"dims": d, "layers": states, "layer": states[0], "pipe": pipe, "qrings": qrings,
+            "queries": qrings[0], "host": hosts[0]}
+
+
+class KernelTimer:
+    """CUDA events around each library call, on the stream it runs on."""
+
+    def __init__(self, n):
+        self.ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(n)] for k in KERNELS}
+        self.i = {k: 0 for k in KERNELS}
+        self.on = False
+
+    def begin(self, name, stream):
+        if self.on and self.i[name] < len(self.ev[name]):
+            self.ev[name][self.i[name]][0].record(stream)
+
+    def end(self, name, stream):
+        if self.on and self.i[name] < len(self.ev[name]):
+            self.ev[name][self.i[name]][1].record(stream)
+            self.i[name] += 1
+
+    def mean_ms(self, name):
+        n = self.i[name]
+        if n == 0:
+            return None
+        return sum(a.elapsed_time(b) for a, b in self.ev[name][:n]) / n
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.lines = index, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# -------------------------------------------------------------- measures
+def measure_h2d_peak(device) -> dict:
+    """Best of a 1 GiB pinned cudaMemcpyAsync and the zero-copy gather kernel
+    over 16K distinct 8 KiB blocks (128 MiB)."""
+    n = 1 << 30
+    src = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    src.fill_(1)
+    dst = torch.empty(n, dtype=torch.uint8, device=device)
+    best_copy = 0.0
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        b.synchronize()
+        best_copy = max(best_copy, n / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del dst
+    # zero-copy: 128 units x 128 blocks, every entry valid
+    d = lsk.make_dims(batch=16, n_q_heads=8, n_kv_heads=8, max_blocks=128, budget_blocks=128,
+                      n_queries=1, fetch_cap=128)
+    host = src[: 16 * 8 * 128 * 8192].view(torch.bfloat16).view(16, 8, 128, 2, 16, 128)
+    pool = torch.empty((16, 8, 128, 2, 16, 128), dtype=torch.bfloat16, device=device)
+    ids = torch.arange(128, dtype=torch.int32, device=device).repeat(16, 8, 1).contiguous()
+    nf = torch.full((16, 8), 128, dtype=torch.int32, device=device)
+    best_zc = 0.0
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        lsk.prefetch(d, host, ids, ids, nf, pool)
+        b.record()
+        b.synchronize()
+        best_zc = max(best_zc, pool.numel() * 2 / (a.elapsed_time(b) * 1e-3) / 1e9)
+    return {"memcpy_gbs": best_copy, "zero_copy_gbs": best_zc, "peak_gbs": max(best_copy, best_zc)}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lookahead_sparse_kv_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    try:
+        with open(TRAFFIC_PATH) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    return t.get("kernels", {}) if t.get("source_hash") == kernel_source_hash() else {}
+
+
+# ------------------------------------------------------------------- run
+def isolated_kernel_ms(st, reps: int = 20) -> dict:
+    """Each library call of one layer-step timed alone on one stream (no
+    concurrent kernels), for per-kernel rooflines."""
+    pipe, L, d = st["pipe"], st["layers"][0], st["dims"]
+    q = st["qrings"][0][0]
+    s = torch.cuda.current_stream()
+    ctx = pipe.ctx_len
+    st_c, lu_c = L.slot_table.clone(), L.last_used.clone()
+    calls = {
+        "sparse_attn": lambda: lsk.sparse_attn(d, q, L.pool, L.slot_table, ctx, pipe.scale, L.out, L.lse, pipe.ws,
+                                               stream=s),
+        # the gather of the last plan of the timed run (re-copies the same blocks)
+        "prefetch": lambda: lsk.prefetch(d, L.host_kv, L.fetch_slot, L.fetch_block, L.n_fetch, L.pool, stream=s),
+        "score_select": lambda: lsk.score_select(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, pipe.ws, stream=s),
+        "select_only": lambda: lsk.select_topk(d, pipe.ws.view(torch.float32), ctx, L.sel, L.sel_score, stream=s),
+        "plan_fetch": lambda: lsk.plan_fetch(d, L.sel, st_c, lu_c, 10 ** 6, L.fetch_slot, L.fetch_block,
+                                             L.n_fetch, stream=s),
+    }
+    fetched = int(L.n_fetch.sum().item())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=q.device)
+    out = {}
+    torch.cuda.synchronize()
+    for name, fn in calls.items():
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()                                  # evict L2 between launches
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            fn()
+            b.record(s)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        out[name] = tot / reps
+    out["_prefetch_blocks"] = fetched
+    return out
+
+
+def run_gpu(args, rank, world, device):
+    w = W.WORKLOADS[WORKLOAD]
+    if rank:
+        w = w.with_(seed=w.seed + 1000 * rank)
+    st = build_workload_state(w, args.warmup + args.steps, device, n_queries=args.query_ring,
+                              layers=args.layers)
+    d, layers, pipe, qrings = st["dims"], st["layers"], st["pipe"], st["qrings"]
+    nl, nq = len(layers), len(qrings[0])
+    timer = KernelTimer(args.steps * nl)
+    pipe.timer = timer
+    main = pipe.main
+    fetch_hist = torch.zeros((args.steps, nl, w.batch, w.n_kv_heads), dtype=torch.int32, device=device)
+
+    def qs_at(t):
+        i = ring_index(t, nq)
+        return [r[i] for r in qrings]
+
+    pipe.prime(qs_at(0))
+    t = 1
+    for _ in range(args.warmup):
+        pipe.step(t, qs_at(t))
+        t += 1
+    pipe.wait_all()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    timer.on = True
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev0.record(main)
+        for i in range(args.steps):
+            pipe.step(t, qs_at(t))
+            for l, L in enumerate(layers):
+                fetch_hist[i, l].copy_(L.n_fetch, non_blocking=True)
+            t += 1
+        pipe.wait_all()
+        ev1.record(main)
+        torch.cuda.synchronize()
+    timer.on = False
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        torch.distributed.barrier()
+        m = torch.tensor([ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(m, op=torch.distributed.ReduceOp.MAX)
+        ms = float(m.item())
+
+    # reuse of the selected set between consecutive steps (untimed)
+    reuse = []
+    prev = [L.sel.clone() for L in layers]
+    for _ in range(16):
+        pipe.step(t, qs_at(t))
+        t += 1
+        pipe.wait_all()
+        for l, L in enumerate(layers):
+            cur = L.sel.clone()
+            same = (cur.unsqueeze(-1) == prev[l].unsqueeze(-2)) & (cur.unsqueeze(-1) >= 0)
+            reuse.append(same.any(-1).sum().item() / max(1, (cur >= 0).sum().item()))
+            prev[l] = cur
+    torch.cuda.synchronize()
+
+    # end-to-end through the API: every step copies its queries in from pinned
+    # host memory and reads every layer's outputs back, synchronised
+    e2e_steps = min(args.steps, 200)
+    hq = [[q.cpu().pin_memory() for q in r[: min(nq, 32)]] for r in qrings]
+    qdev = [torch.empty_like(r[0]) for r in qrings]
+    hout = [torch.empty(L.out.shape, dtype=L.out.dtype, pin_memory=True) for L in layers]
+    hlse = [torch.empty(L.lse.shape, dtype=L.lse.dtype, pin_memory=True) for L in layers]
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for i in range(e2e_steps):
+        j = ring_index(i, len(hq[0]))
+        for l in range(nl):
+            qdev[l].copy_(hq[l][j], non_blocking=True)
+        pipe.step(t, qdev)
+        t += 1
+        for l, L in enumerate(layers):
+            hout[l].copy_(L.out, non_blocking=True)
+            hlse[l].copy_(L.lse, non_blocking=True)
+        main.synchronize()
+    pipe.wait_all()
+    e1.record(main)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        m = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(m, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(m.item())
+
+    iso = isolated_kernel_ms(st)
+    h2d = measure_h2d_peak(device) if rank == 0 else None
+    err = lsk.read_device_error(clear=True)
+    return {"w": w, "d": d, "ms": ms, "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
+            "e2e_ms": e2e_ms, "e2e_steps": e2e_steps, "h2d": h2d, "clocks": clk.summary(), "dev_err": err,
+            "layer": layers[0], "layers": layers, "queries": qrings[0], "iso": iso}
+
+
+def algorithmic_bytes(w, fetched_blocks_per_layer_step):
+    """Bytes each kernel must move per launch (the whole batch, one layer)."""
+    units = w.batch * w.n_kv_heads
+    nv = math.ceil(w.context / w.block_tokens)
+    q_bytes = w.batch * w.n_queries * w.n_q_heads * w.head_dim * 2
+    out_bytes = w.batch * w.n_queries * w.n_q_heads * (w.head_dim + 1) * 4
+    block = w.block_bytes
+    return {
+        # resident KV (every slot is occupied after warm-up) + queries + outputs
+        "sparse_attn": units * w.budget_blocks * block + q_bytes + out_bytes,
+        # min/max summaries of every valid block + draft queries + scores written and read + selection
+        "score_select": units * nv * 2 * w.head_dim * 2 + q_bytes + 2 * units * nv * 4 + units * w.budget_blocks * 8,
+        "select_only": units * nv * 4 + units * w.budget_blocks * 8,
+        # slot table + last-used read and written, selection read, fetch lists written
+        "plan_fetch": units * w.budget_blocks * 4 * 5 + units * w.fetch_cap * 8 + units * 4,
+        # fetched blocks: read over PCIe and written to HBM (counted once, as H2D bytes)
+        "prefetch": fetched_blocks_per_layer_step * block,
+    }
+
+
+def emit_gpu(args, res, world):
+    w, timer = res["w"], res["timer"]
+    nl = len(res["layers"])
+    peaks, peak_src = load_peaks()
+    layer_steps = args.steps * nl
+    fetched = res["fetch_hist"].sum().item() / layer_steps            # blocks per layer-step (this rank)
+    ab = algorithmic_bytes(w, fetched)
+    h2d_peak = res["h2d"]["peak_gbs"] if res["h2d"] else None
+    traffic = load_traffic()
+
+    def roof(k, ms):
+        gbs = ab[k] / (ms * 1e-3) / 1e9
+        if k == "prefetch":
+            bound, peak, src = "h2d", h2d_peak, "measured in this run (best of 1 GiB pinned memcpy, zero-copy gather)"
+        else:
+            bound, peak, src = "hbm", peaks["hbm_gbs"], f"{peak_src} hbm_gbs (MEASURED_PEAKS)"
+        return {"ms": ms, "bytes": ab[k], "achieved_gbs": gbs, "bound": bound, "peak_gbs": peak,
+                "frac": (gbs / peak) if peak else None, "peak_source": src, "traffic": traffic.get(k)}
+
+    kernels = {k: roof(k, timer.mean_ms(k)) for k in KERNELS if timer.mean_ms(k) is not None}
+    iso = dict(res["iso"])
+    iso_blocks = iso.pop("_prefetch_blocks")
+    isolated = {k: roof(k, v) for k, v in iso.items()}
+    isolated["prefetch"]["bytes"] = iso_blocks * w.block_bytes
+    isolated["prefetch"]["achieved_gbs"] = iso_blocks * w.block_bytes / (iso["prefetch"] * 1e-3) / 1e9
+    if h2d_peak:
+        isolated["prefetch"]["frac"] = isolated["prefetch"]["achieved_gbs"] / h2d_peak
+    dominant = max(kernels, key=lambda k: kernels[k]["ms"])
+    kd = kernels[dominant]
+    value = world * layer_steps / (res["ms"] * 1e-3)
+    e2e_value = world * res["e2e_steps"] * nl / (res["e2e_ms"] * 1e-3)
+    q_bytes = w.batch * w.n_queries * w.n_q_heads * w.head_dim * 2
+    L = res["layer"]
+    line = {
+        "metric": "sparse decode layer-steps/s (score+select+plan+prefetch+attn)",
+        "value": value,
+        "unit": "layer-steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": res["ms"] / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded bf16 KV ~N(0,1) with 4 outlier channels x8, AR(1)-drifting queries)",
+        "config": {"workload": f"{WORKLOAD}: {nl} Llama-3.1-8B-shaped attention layers at 32K context, "
+                               f"pipelined across layers",
+                   "batch": w.batch, "seq_len": w.context, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim, "block_tokens": w.block_tokens, "budget_blocks": w.budget_blocks,
+                   "queries": w.n_queries, "fetch_cap": w.fetch_cap, "layers": nl,
+                   "parallelism": f"dp{world} (independent replicas)",
+                   "l2": "inputs larger than L2: per layer-step 128 MiB summaries + 128 MiB pool read"},
+        "roofline": {"kernel": dominant, "bound": kd["bound"], "achieved": kd["achieved_gbs"],
+                     "peak": kd["peak_gbs"], "unit": "GB/s", "frac": kd["frac"], "traffic": kd["traffic"],
+                     "peak_source": kd["peak_source"]},
+        "kernels": kernels,
+        "kernels_isolated": isolated,
+        "tokens_per_s": value / nl * w.batch,
+        "fetched_blocks_per_layer_step": fetched,
+        "h2d_gbs_avg": ab["prefetch"] * layer_steps / (res["ms"] * 1e-3) / 1e9,
+        "reuse": sum(res["reuse"]) / len(res["reuse"]),
+        "h2d_peak": res["h2d"],
+        "e2e": {"value": e2e_value, "unit": "layer-steps/s",
+                "h2d_bytes_per_step": nl * (q_bytes + int(ab["prefetch"])),
+                "d2h_bytes_per_step": nl * (L.out.numel() * 4 + L.lse.numel() * 4),
+                "note": "per step: every layer's queries copied in from pinned host memory and its outputs read "
+                        "back, then synchronised; h2d bytes include the zero-copy gather of fetched blocks"},
+        "gpu_launches": 5 * layer_steps,
+        "clocks": res["clocks"],
+        "device_error_word": res["dev_err"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, res)
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------- oracle
+class OracleUnit:
+    """The CPU oracle driving one (sequence, KV head) unit through decode
+    layer-steps: attention over its pool, scores, top-K, plan, gather."""
+
+    def __init__(self, w, host_bits):
+        import numpy as np
+
+        import oracle as O
+        self.O, self.np, self.w = O, np, w
+        self.host_bits = host_bits                          # uint16 [1, 1, N, 2, P, D]
+        kv = O.bf16_bits_to_f64(host_bits)
+        self.keys, self.vals = kv[:, :, :, 0], kv[:, :, :, 1]
+        self.ctx = np.array([w.context], dtype=np.int64)
+        self.kmin, self.kmax = O.block_summaries(self.keys, self.ctx)   # admission, not timed
+        K, P, D = w.budget_blocks, w.block_tokens, w.head_dim
+        self.st = np.full((1, 1, K), -1, np.int32)
+        self.lu = np.full((1, 1, K), -1, np.int32)
+        self.pool_k = np.zeros((1, 1, K, P, D))
+        self.pool_v = np.zeros((1, 1, K, P, D))
+        self.scale = 1.0 / math.sqrt(D)
+
+    def step(self, q, t, attend=True):
+        O, w = self.O, self.w
+        if attend:
+            O.sparse_attention(q, self.pool_k, self.pool_v, self.st, self.ctx, self.scale)
+        sc = O.lookahead_scores(q, self.kmin, self.kmax, self.ctx, w.block_tokens)
+        sel, _ = O.select_topk(sc, self.ctx, w.budget_blocks, w.block_tokens)
+        plan = O.plan_fetch(sel, self.st, self.lu, t, w.fetch_cap)
+        self.pool_k = O.prefetch(self.keys, self.pool_k, plan["fetch_slot"], plan["fetch_block"], plan["n_fetch"])
+        self.pool_v = O.prefetch(self.vals, self.pool_v, plan["fetch_slot"], plan["fetch_block"], plan["n_fetch"])
+        self.st, self.lu = plan["slot_table"], plan["last_used"]
+
+
+def time_oracle(w, unit_bits, unit_queries, fill_steps, timed_steps):
+    """Seconds per decode layer-step per unit, BLAS limited to one thread.
+    unit_bits: list of host-KV bit arrays of single units; unit_queries:
+    list (per unit) of per-step float64 queries [1, Qn, G, D]."""
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=1)
+    except ImportError:                       # pragma: no cover
+        lim = None
+    times = []
+    try:
+        for bits, qs in zip(unit_bits, unit_queries):
+            u = OracleUnit(w, bits)
+            u.step(qs[0], 0, attend=False)                  # priming
+            for i in range(1, fill_steps + 1):
+                u.step(qs[i % len(qs)], i)
+            for i in range(fill_steps + 1, fill_steps + 1 + timed_steps):
+                t0 = time.perf_counter()
+                u.step(qs[i % len(qs)], i)
+                times.append(time.perf_counter() - t0)
+    finally:
+        if lim is not None:
+            lim.__exit__(None, None, None)
+    return sum(times) / len(times), len(times)
+
+
+def cpu_baseline(w, res, n_units=6, fill_steps=8, timed_steps=24):
+    """The oracle, as it stands, on this host's cores, on a sample of the
+    benchmarked workload: a few (sequence, KV head) units of the same KV and
+    queries, layer-steps/s scaled to the whole batch."""
+    import numpy as np
+
+    import oracle as O
+    L = res["layer"]
+    G = w.group
+    rng = np.random.default_rng(0)
+    units = [(int(rng.integers(w.batch)), int(rng.integers(w.n_kv_heads))) for _ in range(n_units)]
+    qs_all = [O.bf16_bits_to_f64(W.bf16_bits(q)) for q in res["queries"][: fill_steps + timed_steps + 1]]
+    bits = [W.bf16_bits(L.host_kv[b:b + 1, h:h + 1]) for b, h in units]
+    uq = [[q[b:b + 1, :, h * G:(h + 1) * G] for q in qs_all] for b, h in units]
+    per_unit, n = time_oracle(w, bits, uq, fill_steps, timed_steps)
+    total_units = w.batch * w.n_kv_heads
+    return {"value": 1.0 / (per_unit * total_units), "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} unit-steps ({n_units} (sequence, KV head) units x {timed_steps} decode layer-steps "
+                      f"after {fill_steps} untimed fill steps): attention, scores, top-K, plan, gather; "
+                      f"per-unit mean scaled to the {total_units} units of the batch; numpy fp64, BLAS 1 thread"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle on this host, same workload, metric and
+    unit; each step is one (sequence, KV head) unit's decode layer-step,
+    scaled to the whole batch."""
+    import oracle as O
+    w = W.WORKLOADS[WORKLOAD]
+    wu = w.with_(batch=1, n_kv_heads=1, n_q_heads=w.group)
+    kv = W.make_host_kv(wu, 0, "cpu")
+    qs = W.QueryStream(wu, 0, "cpu")
+    fill = 8
+    queries = [O.bf16_bits_to_f64(W.bf16_bits(qs.next())) for _ in range(fill + args.warmup + args.steps + 1)]
+    per_unit, n = time_oracle(wu, [W.bf16_bits(kv)], [queries], fill + args.warmup, args.steps)
+    units = w.batch * w.n_kv_heads
+    value = 1.0 / (per_unit * units)
+    sample = (f"each step: one (sequence, KV head) unit's decode layer-step (attention, scores, top-K, plan, "
+              f"gather), scaled to the {units} units of the batch; numpy fp64, BLAS 1 thread")
+    line = {
+        "impl": "reference",
+        "metric": "sparse decode layer-steps/s (score+select+plan+prefetch+attn)",
+        "value": value, "unit": "layer-steps/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_unit * units * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: Llama-3.1-8B-shaped layer, 32K context", "batch": w.batch,
+                   "seq_len": w.context, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                   "budget_blocks": w.budget_blocks, "queries": w.n_queries, "fetch_cap": w.fetch_cap,
+                   "layers": w.layers},
+        "cpu_baseline": {"value": value, "unit": "layer-steps/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--query-ring", type=int, default=48)
+    ap.add_argument("--impl", default="oasis", choices=["oasis", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            args.steps = min(args.steps, 12)
+            args.warmup = min(args.warmup, 3)
+            run_reference(args)
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        res = run_gpu(args, rank, world, device)
+        if rank == 0:
+            emit_gpu(args, res, world)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

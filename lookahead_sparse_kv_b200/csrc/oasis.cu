@@ -1,0 +1,438 @@
+// oasis.cu - C ABI of the lookahead sparse-KV decode path (see include/oasis.h).
+//
+// Host side: argument validation before anything is enqueued, TMA tensor-map
+// encoding, workspace layout and kernel launches.  All kernels live in the
+// .cuh files included below so the library is one translation unit (the
+// device error word needs no relocatable device code).
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <algorithm>
+#include <mutex>
+
+#include "oasis.h"
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "plan.cuh"
+#include "prefetch.cuh"
+#include "score.cuh"
+#include "select.cuh"
+#include "summaries.cuh"
+
+namespace {
+
+using oasis::Dims;
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(OASIS_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int check_launch(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    g_msg[0] = '\0';
+    return OASIS_OK;
+}
+
+int validate(const oasis_dims* dp, Dims* out) {
+    if (dp == nullptr) return fail(OASIS_EINVAL, "dims is NULL");
+    const oasis_dims& d = *dp;
+    if (d.head_dim != oasis::kHeadDim) return fail(OASIS_EINVAL, "head_dim must be 128 (got %d)", d.head_dim);
+    if (d.block_tokens != oasis::kBlockTokens)
+        return fail(OASIS_EINVAL, "block_tokens must be 16 (got %d)", d.block_tokens);
+    if (d.batch < 1 || d.n_kv_heads < 1 || d.n_q_heads < 1)
+        return fail(OASIS_EINVAL, "batch, n_q_heads and n_kv_heads must be >= 1");
+    if (d.n_q_heads % d.n_kv_heads != 0)
+        return fail(OASIS_EINVAL, "n_q_heads (%d) must be a multiple of n_kv_heads (%d)", d.n_q_heads, d.n_kv_heads);
+    if (d.budget_blocks < 1 || d.budget_blocks > 1024)
+        return fail(OASIS_EINVAL, "budget_blocks must be in [1, 1024] (got %d)", d.budget_blocks);
+    if (d.max_blocks < d.budget_blocks || d.max_blocks > 32768)
+        return fail(OASIS_EINVAL, "max_blocks must be in [budget_blocks, 32768] (got %d)", d.max_blocks);
+    if (d.fetch_cap < 0 || d.fetch_cap > d.budget_blocks)
+        return fail(OASIS_EINVAL, "fetch_cap must be in [0, budget_blocks] (got %d)", d.fetch_cap);
+    if (d.n_queries < 1) return fail(OASIS_EINVAL, "n_queries must be >= 1");
+    const int G = d.n_q_heads / d.n_kv_heads;
+    if (static_cast<long long>(d.n_queries) * G > 64)
+        return fail(OASIS_EINVAL, "n_queries * G must be <= 64 (got %d)", d.n_queries * G);
+    const long long units = static_cast<long long>(d.batch) * d.n_kv_heads;
+    if (units > 65535) return fail(OASIS_EINVAL, "batch * n_kv_heads must be <= 65535");
+    if (units * d.max_blocks * 32 > 0x7FFFFFFFll || units * d.budget_blocks * 32 > 0x7FFFFFFFll)
+        return fail(OASIS_EINVAL, "tensor too large for 32-bit row coordinates");
+    if (out) *out = Dims{d.batch, d.n_q_heads, d.n_kv_heads, d.head_dim, d.block_tokens,
+                         d.max_blocks, d.budget_blocks, d.n_queries, d.fetch_cap};
+    return OASIS_OK;
+}
+
+int check_ptr(const void* p, const char* name, bool nullable = false) {
+    if (p == nullptr) return nullable ? OASIS_OK : fail(OASIS_EINVAL, "%s is NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return fail(OASIS_EINVAL, "%s is not 16-byte aligned", name);
+    return OASIS_OK;
+}
+
+// Resolves a pointer the device may read: device memory as is, pinned host
+// memory through its device mapping.  `allow_device` rejects device memory
+// when only mapped host memory makes sense.
+int device_view(const void* p, const char* name, bool allow_device, const void** out) {
+    cudaPointerAttributes a;
+    const cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(OASIS_ENOTMAPPED, "%s: cudaPointerGetAttributes failed (%s)", name, cudaGetErrorName(e));
+    }
+    if (a.type == cudaMemoryTypeHost) {
+        if (a.devicePointer == nullptr) return fail(OASIS_ENOTMAPPED, "%s: pinned host memory is not mapped", name);
+        *out = a.devicePointer;
+        return OASIS_OK;
+    }
+    if ((a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && allow_device) {
+        *out = p;
+        return OASIS_OK;
+    }
+    return fail(OASIS_ENOTMAPPED, "%s: not %s", name, allow_device ? "device or mapped pinned host memory"
+                                                                   : "mapped pinned host memory");
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// bf16 matrix [rows][128] with 256-B rows, boxes of 64 columns x box_rows,
+// 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned box_rows, const char* name) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(oasis::kHeadDim), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(oasis::kRowBytes)};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled(%s) failed: %d", name, static_cast<int>(r));
+    return OASIS_OK;
+}
+
+template <typename K>
+int set_smem(K kernel, int bytes, const char* what) {
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return OASIS_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Upper bound of attention streams the workspace is sized for: 148 SMs x 8
+// streams (two CTAs of four per SM), or more when ranges would exceed 256 slots.
+long long attn_max_streams(const Dims& d) {
+    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
+    const long long cap = 148ll * 8;
+    return std::max<long long>(1, std::min(T, std::max(cap, (T + 255) / 256)));
+}
+
+struct WsLayout {
+    size_t scores, lse, o, total;
+    long long partials;
+};
+
+WsLayout ws_layout(const Dims& d) {
+    WsLayout w;
+    const size_t units = static_cast<size_t>(d.B) * d.Hkv;
+    const size_t rows = static_cast<size_t>(d.Qn) * d.G();
+    w.partials = attn_max_streams(d) + static_cast<long long>(units);
+    w.scores = 0;
+    w.lse = align256(units * d.N * sizeof(float));
+    w.o = align256(w.lse + static_cast<size_t>(w.partials) * rows * sizeof(float));
+    w.total = align256(w.o + static_cast<size_t>(w.partials) * rows * oasis::kHeadDim * sizeof(float));
+    return w;
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
+                                                      cudaSuccess)
+            n = v;
+        else
+            n = 148;
+    }
+    return n;
+}
+
+// Streams for this launch: 8 per SM (4 with two-warp streams), at least 4
+// slots each, never more than the workspace holds.
+long long attn_streams(const Dims& d, int qg) {
+    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
+    long long ns = static_cast<long long>(sm_count()) * (qg == 1 ? 8 : 4);
+    ns = std::max(ns, (T + 255) / 256);
+    ns = std::min(ns, std::max(1ll, T / 4));
+    return std::min(ns, attn_max_streams(d));
+}
+
+template <int NTW, int QG>
+int launch_attn(const CUtensorMap& tm, const Dims& d, const uint16_t* q, const int32_t* st, const int32_t* ctx,
+                float scale_log2, float* out, float* lse, float* ws_o, float* ws_lse, cudaStream_t s) {
+    using Cfg = oasis::AttnCfg<NTW, QG>;
+    auto k = oasis::sparse_attn_kernel<NTW, QG>;
+    if (int rc = set_smem(k, Cfg::kSmem, "sparse_attn smem")) return rc;
+    const long long ns = attn_streams(d, QG);
+    const long long ctas = (ns + oasis::kAttnStreamsPerCta - 1) / oasis::kAttnStreamsPerCta;
+    k<<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmem, s>>>(tm, d, q, st, ctx, scale_log2,
+                                                                      static_cast<int>(ns), ws_o, ws_lse);
+    if (int rc = check_launch("sparse_attn launch")) return rc;
+    // merge: rows * (partials per unit + 1) floats of shared memory
+    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
+    const long long max_np = (static_cast<long long>(d.K) * ns + T - 1) / T + 1;
+    const int rows = d.Qn * d.G();
+    const int msmem = static_cast<int>(rows * (max_np + 1) * sizeof(float));
+    if (msmem > 200 * 1024) return fail(OASIS_EINVAL, "too many attention partials per unit");
+    if (int rc = set_smem(oasis::attn_merge_kernel, msmem, "attn_merge smem")) return rc;
+    oasis::attn_merge_kernel<<<d.B * d.Hkv, 256, msmem, s>>>(d, static_cast<int>(ns), ws_o, ws_lse, out, lse);
+    return check_launch("attn_merge launch");
+}
+
+template <int NPAD>
+int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
+                 const int32_t* ctx, float* scores, int rows, cudaStream_t s) {
+    using S = oasis::ScoreSmem<NPAD>;
+    auto k = oasis::lookahead_score_kernel<NPAD>;
+    if (int rc = set_smem(k, S::kBytes, "score smem")) return rc;
+    dim3 grid((d.N + oasis::kScoreTile - 1) / oasis::kScoreTile, d.B * d.Hkv);
+    k<<<grid, 128, S::kBytes, s>>>(tmax, tmin, d, q, ctx, scores, rows);
+    return check_launch("lookahead_score launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* oasis_last_error(void) { return g_msg; }
+
+const char* oasis_version(void) { return "oasis-b200 0.1 (sm_100a)"; }
+
+int oasis_check_dims(const oasis_dims* d) { return validate(d, nullptr); }
+
+size_t oasis_workspace_bytes(const oasis_dims* dp) {
+    Dims d;
+    if (validate(dp, &d) != OASIS_OK) return 0;
+    return ws_layout(d).total;
+}
+
+int oasis_build_summaries(const oasis_dims* dp, const void* kv, const int32_t* ctx_len, int32_t first_block,
+                          int32_t n_blocks, void* kmin, void* kmax, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(kv, "kv")) return rc;
+    if (int rc = check_ptr(ctx_len, "ctx_len", false)) return rc;
+    if (int rc = check_ptr(kmin, "kmin")) return rc;
+    if (int rc = check_ptr(kmax, "kmax")) return rc;
+    if (first_block < 0 || n_blocks < 0 || first_block + static_cast<long long>(n_blocks) > d.N)
+        return fail(OASIS_EINVAL, "block range [%d, %d) outside [0, %d)", first_block, first_block + n_blocks, d.N);
+    if (n_blocks == 0) return OASIS_OK;
+    const void* src = nullptr;
+    if (int rc = device_view(kv, "kv", true, &src)) return rc;
+    const long long items = static_cast<long long>(d.B) * d.Hkv * n_blocks;
+    const long long grid = (items + oasis::kSumGroups - 1) / oasis::kSumGroups;
+    if (grid > 0x7FFFFFFFll) return fail(OASIS_EINVAL, "too many blocks");
+    oasis::build_summaries_kernel<<<static_cast<unsigned>(grid), oasis::kSumThreads, 0,
+                                    static_cast<cudaStream_t>(stream)>>>(
+        d, static_cast<const uint4*>(src), ctx_len, first_block, n_blocks, static_cast<uint4*>(kmin),
+        static_cast<uint4*>(kmax));
+    return check_launch("build_summaries launch");
+}
+
+int oasis_append_kv(const oasis_dims* dp, const void* k_new, const void* v_new, const int32_t* ctx_len,
+                    int32_t* ctx_len_out, void* host_kv, void* kmin, void* kmax, const int32_t* slot_table,
+                    void* pool, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(k_new, "k_new")) return rc;
+    if (int rc = check_ptr(v_new, "v_new")) return rc;
+    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
+    if (int rc = check_ptr(ctx_len_out, "ctx_len_out", true)) return rc;
+    if (int rc = check_ptr(host_kv, "host_kv", true)) return rc;
+    if (int rc = check_ptr(kmin, "kmin")) return rc;
+    if (int rc = check_ptr(kmax, "kmax")) return rc;
+    if (int rc = check_ptr(pool, "pool", true)) return rc;
+    if (pool != nullptr)
+        if (int rc = check_ptr(slot_table, "slot_table")) return rc;
+    if (ctx_len_out != nullptr && ctx_len_out == ctx_len)
+        return fail(OASIS_EINVAL, "ctx_len_out must not alias ctx_len");
+    const void* hv = nullptr;
+    if (host_kv != nullptr)
+        if (int rc = device_view(host_kv, "host_kv", false, &hv)) return rc;
+    oasis::append_kv_kernel<<<d.B * d.Hkv, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        d, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), ctx_len, ctx_len_out,
+        static_cast<uint4*>(const_cast<void*>(hv)), static_cast<uint4*>(kmin), static_cast<uint4*>(kmax), slot_table,
+        static_cast<uint4*>(pool));
+    return check_launch("append_kv launch");
+}
+
+int oasis_lookahead_scores(const oasis_dims* dp, const void* q, const void* kmin, const void* kmax,
+                           const int32_t* ctx_len, float* scores, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(q, "q")) return rc;
+    if (int rc = check_ptr(kmin, "kmin")) return rc;
+    if (int rc = check_ptr(kmax, "kmax")) return rc;
+    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
+    if (int rc = check_ptr(scores, "scores")) return rc;
+    const int rows = (d.Qn > 1 ? d.Qn - 1 : 1) * d.G();
+    const unsigned long long total_rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.N;
+    CUtensorMap tmax, tmin;
+    if (int rc = make_map(&tmax, kmax, total_rows, oasis::kScoreTile, "kmax")) return rc;
+    if (int rc = make_map(&tmin, kmin, total_rows, oasis::kScoreTile, "kmin")) return rc;
+    const auto* qq = static_cast<const uint16_t*>(q);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rows <= 16) return launch_score<16>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
+    if (rows <= 32) return launch_score<32>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
+    if (rows <= 48) return launch_score<48>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
+    return launch_score<64>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
+}
+
+int oasis_select_topk(const oasis_dims* dp, const float* scores, const int32_t* ctx_len, int32_t* sel,
+                      float* sel_score, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(scores, "scores")) return rc;
+    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
+    if (int rc = check_ptr(sel, "sel")) return rc;
+    if (int rc = check_ptr(sel_score, "sel_score", true)) return rc;
+    const int smem = d.N * static_cast<int>(sizeof(uint32_t));
+    if (int rc = set_smem(oasis::select_topk_kernel, smem, "select smem")) return rc;
+    oasis::select_topk_kernel<<<d.B * d.Hkv, oasis::kSelThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+        d, scores, ctx_len, sel, sel_score);
+    return check_launch("select_topk launch");
+}
+
+int oasis_score_select(const oasis_dims* dp, const void* q, const void* kmin, const void* kmax,
+                       const int32_t* ctx_len, int32_t* sel, float* sel_score, void* ws, size_t ws_bytes,
+                       void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(ws, "ws")) return rc;
+    const WsLayout w = ws_layout(d);
+    if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
+    float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.scores);
+    if (int rc = oasis_lookahead_scores(dp, q, kmin, kmax, ctx_len, scores, stream)) return rc;
+    return oasis_select_topk(dp, scores, ctx_len, sel, sel_score, stream);
+}
+
+int oasis_plan_fetch(const oasis_dims* dp, const int32_t* sel, int32_t* slot_table, int32_t* last_used,
+                     int32_t step, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(sel, "sel")) return rc;
+    if (int rc = check_ptr(slot_table, "slot_table")) return rc;
+    if (int rc = check_ptr(last_used, "last_used")) return rc;
+    if (int rc = check_ptr(n_fetch, "n_fetch")) return rc;
+    if (d.C > 0) {
+        if (int rc = check_ptr(fetch_slot, "fetch_slot")) return rc;
+        if (int rc = check_ptr(fetch_block, "fetch_block")) return rc;
+    }
+    const int threads = (d.K + 31) / 32 * 32;
+    const int smem = 6 * d.K * static_cast<int>(sizeof(int32_t));
+    oasis::plan_fetch_kernel<<<d.B * d.Hkv, threads, smem, static_cast<cudaStream_t>(stream)>>>(
+        d, sel, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch);
+    return check_launch("plan_fetch launch");
+}
+
+int oasis_prefetch(const oasis_dims* dp, const void* host_kv, const int32_t* fetch_slot, const int32_t* fetch_block,
+                   const int32_t* n_fetch, void* pool, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(host_kv, "host_kv")) return rc;
+    if (int rc = check_ptr(n_fetch, "n_fetch")) return rc;
+    if (int rc = check_ptr(pool, "pool")) return rc;
+    if (d.C == 0) return OASIS_OK;
+    if (int rc = check_ptr(fetch_slot, "fetch_slot")) return rc;
+    if (int rc = check_ptr(fetch_block, "fetch_block")) return rc;
+    const void* hv = nullptr;
+    if (int rc = device_view(host_kv, "host_kv", false, &hv)) return rc;
+    const long long entries = static_cast<long long>(d.B) * d.Hkv * d.C;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(oasis::kPrefetchCtas, (entries + 1) / 2));
+    oasis::prefetch_kernel<<<grid, oasis::kPrefetchThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        d, static_cast<const uint4*>(hv), fetch_slot, fetch_block, n_fetch, static_cast<uint4*>(pool));
+    return check_launch("prefetch launch");
+}
+
+int oasis_sparse_attn(const oasis_dims* dp, const void* q, const void* pool, const int32_t* slot_table,
+                      const int32_t* ctx_len, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
+                      void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(q, "q")) return rc;
+    if (int rc = check_ptr(pool, "pool")) return rc;
+    if (int rc = check_ptr(slot_table, "slot_table")) return rc;
+    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
+    if (int rc = check_ptr(out, "out")) return rc;
+    if (int rc = check_ptr(lse, "lse")) return rc;
+    if (int rc = check_ptr(ws, "ws")) return rc;
+    const WsLayout w = ws_layout(d);
+    if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
+    CUtensorMap tm;
+    const unsigned long long rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.K * 2 * oasis::kBlockTokens;
+    if (int rc = make_map(&tm, pool, rows, 2 * oasis::kBlockTokens, "pool")) return rc;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* ws_lse = reinterpret_cast<float*>(base + w.lse);
+    float* ws_o = reinterpret_cast<float*>(base + w.o);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    const auto* qq = static_cast<const uint16_t*>(q);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int nt = (d.Qn * d.G() + 7) / 8;
+    switch (nt) {
+        case 1: return launch_attn<1, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
+        case 2: return launch_attn<2, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
+        case 3: return launch_attn<3, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
+        case 4: return launch_attn<4, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
+        case 5:
+        case 6: return launch_attn<3, 2>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
+        default: return launch_attn<4, 2>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
+    }
+}
+
+int oasis_read_device_error(uint32_t* out, int clear, void* stream) {
+    if (out == nullptr) return fail(OASIS_EINVAL, "out is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, oasis::g_oasis_dev_error, sizeof(v), 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error");
+    if (clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbolAsync(oasis::g_oasis_dev_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_fail(e, "clear device error");
+    }
+    *out = v;
+    return OASIS_OK;
+}
+
+}  // extern "C"

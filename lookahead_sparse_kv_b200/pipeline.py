@@ -1,0 +1,152 @@
+"""Per-layer device state and the stream / event order of a decode step.
+
+OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
+Prefetching, Figure 8: at step t each layer's draft queries drive top-K
+prediction, selection and the host-to-HBM transfer, which must land before
+that layer's attention at step t+1; the stages of different layers overlap.
+Figure 7 (right): attention at step t runs over the working set staged at
+step t-1.
+
+Streams (all work is in liboasis kernels; this module only orders them):
+
+* main  - [append] -> sparse attention -> plan        (per layer, in order)
+* score - lookahead scores + top-K, concurrent with the attention of the same
+          layer (they read disjoint buffers); waits for the layer's previous
+          plan before overwriting its selection
+* copy  - host-to-HBM gather, high priority, after the layer's plan; the next
+          step's append/attention of that layer waits for it
+
+Memory: the full KV of every layer lives in pinned host memory; HBM holds per
+layer the per-block summaries (N x 512 B per KV head), the fixed pool of K
+slots (8 KiB each) and a few small int tables.  One workspace serves all
+layers because each stream runs its layers in order and the two workspace
+regions (scores, attention partials) are disjoint.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import (append_kv, build_summaries, plan_fetch, prefetch, score_select, sparse_attn,
+               workspace_bytes)
+
+HEAD_DIM, BLOCK_TOKENS = 128, 16
+
+
+class LayerState:
+    """Device buffers of one attention layer."""
+
+    def __init__(self, d, host_kv: torch.Tensor, device="cuda"):
+        B, H, N, K = d.batch, d.n_kv_heads, d.max_blocks, d.budget_blocks
+        C, Qn, Hq, D, P = d.fetch_cap, d.n_queries, d.n_q_heads, HEAD_DIM, BLOCK_TOKENS
+        assert host_kv.is_pinned() and host_kv.shape == (B, H, N, 2, P, D)
+        self.d = d
+        self.host_kv = host_kv
+        self.kmin = torch.zeros((B, H, N, D), dtype=torch.bfloat16, device=device)
+        self.kmax = torch.zeros((B, H, N, D), dtype=torch.bfloat16, device=device)
+        self.pool = torch.zeros((B, H, K, 2, P, D), dtype=torch.bfloat16, device=device)
+        self.slot_table = torch.full((B, H, K), -1, dtype=torch.int32, device=device)
+        self.last_used = torch.full((B, H, K), -1, dtype=torch.int32, device=device)
+        self.sel = torch.full((B, H, K), -1, dtype=torch.int32, device=device)
+        self.sel_score = torch.empty((B, H, K), dtype=torch.float32, device=device)
+        cap = max(C, 1)
+        self.fetch_slot = torch.full((B, H, cap), -1, dtype=torch.int32, device=device)
+        self.fetch_block = torch.full((B, H, cap), -1, dtype=torch.int32, device=device)
+        self.n_fetch = torch.zeros((B, H), dtype=torch.int32, device=device)
+        self.out = torch.zeros((B, Qn, Hq, D), dtype=torch.float32, device=device)
+        self.lse = torch.zeros((B, Qn, Hq), dtype=torch.float32, device=device)
+        self.plan_ready = torch.cuda.Event()
+        self.fetch_done = torch.cuda.Event()
+
+    def device_bytes(self) -> int:
+        ts = [self.kmin, self.kmax, self.pool, self.slot_table, self.last_used, self.sel, self.sel_score,
+              self.fetch_slot, self.fetch_block, self.n_fetch, self.out, self.lse]
+        return sum(t.numel() * t.element_size() for t in ts)
+
+
+class DecodePipeline:
+    """Drives priming and decode steps over a list of layers."""
+
+    def __init__(self, d, layers, ctx_len: torch.Tensor, scale: float, device="cuda",
+                 overlap_score: bool = True):
+        self.d, self.layers, self.scale = d, layers, scale
+        self.ctx = [ctx_len, ctx_len.clone()]           # ping-pong when tokens are appended
+        self.cur = 0
+        self.ws = torch.zeros(workspace_bytes(d), dtype=torch.uint8, device=device)
+        self.main = torch.cuda.current_stream(device)
+        self.score_stream = torch.cuda.Stream(device) if overlap_score else self.main
+        lo, hi = torch.cuda.Stream.priority_range()
+        self.copy_stream = torch.cuda.Stream(device, priority=hi)
+        self.sel_ready = [torch.cuda.Event() for _ in layers]
+        self.timer = None        # optional: begin(name, stream) / end(name, stream) around each call
+
+    def _t(self, which, name, stream):
+        if self.timer is not None:
+            getattr(self.timer, which)(name, stream)
+
+    @property
+    def ctx_len(self) -> torch.Tensor:
+        return self.ctx[self.cur]
+
+    def build_summaries(self):
+        for L in self.layers:
+            build_summaries(self.d, L.host_kv, self.ctx_len, L.kmin, L.kmax, stream=self.main)
+
+    def _select_plan_fetch(self, i, L, q, step, ctx):
+        d, main = self.d, self.main
+        if self.score_stream is not main:
+            self.score_stream.wait_event(L.plan_ready)     # previous plan has read L.sel
+        self._t("begin", "score_select", self.score_stream)
+        score_select(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, self.ws, stream=self.score_stream)
+        self._t("end", "score_select", self.score_stream)
+        if self.score_stream is not main:
+            self.sel_ready[i].record(self.score_stream)
+            main.wait_event(self.sel_ready[i])
+        self._t("begin", "plan_fetch", main)
+        plan_fetch(d, L.sel, L.slot_table, L.last_used, step, L.fetch_slot, L.fetch_block, L.n_fetch, stream=main)
+        self._t("end", "plan_fetch", main)
+        L.plan_ready.record(main)
+        self.copy_stream.wait_event(L.plan_ready)
+        self._t("begin", "prefetch", self.copy_stream)
+        prefetch(d, L.host_kv, L.fetch_slot, L.fetch_block, L.n_fetch, L.pool, stream=self.copy_stream)
+        self._t("end", "prefetch", self.copy_stream)
+        L.fetch_done.record(self.copy_stream)
+
+    def prime(self, q_per_layer):
+        """Step 0: select, plan and fetch from the drafts before decoding starts."""
+        for i, (L, q) in enumerate(zip(self.layers, q_per_layer)):
+            L.plan_ready.record(self.main)
+            self._select_plan_fetch(i, L, q, 0, self.ctx_len)
+
+    def step(self, t, q_per_layer, appended=None):
+        """Decode step t >= 1: per layer [append] -> attention -> select/plan/fetch.
+
+        appended: optional list of (k_new, v_new) per layer, bf16 [B, Hkv, D],
+        the token accepted at the previous step; it is written at position
+        ctx_len[b] and the context is one token longer from this step on.
+        """
+        d, main = self.d, self.main
+        if appended is None:
+            ctx_in = ctx = self.ctx_len
+        else:
+            ctx_in, ctx = self.ctx[self.cur], self.ctx[1 - self.cur]
+        for i, (L, q) in enumerate(zip(self.layers, q_per_layer)):
+            main.wait_event(L.fetch_done)
+            if appended is not None:
+                k_new, v_new = appended[i]
+                append_kv(d, k_new, v_new, ctx_in, ctx if i == 0 else None, L.host_kv, L.kmin, L.kmax,
+                          L.slot_table, L.pool, stream=main)
+                if self.score_stream is not main:
+                    ev = torch.cuda.Event()
+                    ev.record(main)
+                    self.score_stream.wait_event(ev)       # grown summaries and context
+            self._t("begin", "sparse_attn", main)
+            sparse_attn(d, q, L.pool, L.slot_table, ctx, self.scale, L.out, L.lse, self.ws, stream=main)
+            self._t("end", "sparse_attn", main)
+            self._select_plan_fetch(i, L, q, t, ctx)
+        if appended is not None:
+            self.cur = 1 - self.cur
+
+    def wait_all(self):
+        for L in self.layers:
+            self.main.wait_event(L.fetch_done)

@@ -1,0 +1,79 @@
+"""The C ABI library loads, exports every entry point its header declares, and
+rejects bad arguments on the host before touching a device.  CPU only."""
+
+import ctypes
+import subprocess
+
+import pytest
+
+import lookahead_sparse_kv_b200 as lsk
+from lookahead_sparse_kv_b200 import build as lsk_build
+
+
+@pytest.fixture(scope="module")
+def L():
+    lsk_build.build()
+    return lsk.lib()
+
+
+def test_header_symbols_all_exported(L):
+    names = lsk.header_symbols()
+    assert len(names) >= 12
+    out = subprocess.run(["nm", "-D", "--defined-only", lsk.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(L, n)
+
+
+def _good():
+    return lsk.make_dims(batch=2, n_q_heads=8, n_kv_heads=2, max_blocks=64, budget_blocks=16,
+                         n_queries=5, fetch_cap=4)
+
+
+def test_check_dims_accepts_pages_shapes(L):
+    assert lsk.check_dims(_good()) == lsk.OK
+    from lookahead_sparse_kv_b200 import workloads as W
+    for w in W.WORKLOADS.values():
+        assert lsk.check_dims(lsk.dims_for(w)) == lsk.OK, w.name
+
+
+@pytest.mark.parametrize("field,value", [
+    ("head_dim", 64), ("block_tokens", 32), ("n_q_heads", 7), ("budget_blocks", 0),
+    ("budget_blocks", 2048), ("max_blocks", 8), ("fetch_cap", 17), ("fetch_cap", -1),
+    ("n_queries", 0), ("n_queries", 17), ("batch", 0), ("max_blocks", 40000),
+])
+def test_check_dims_rejects(L, field, value):
+    d = _good()
+    setattr(d, field, value)
+    assert lsk.check_dims(d) == lsk.EINVAL
+    assert lsk.workspace_bytes(d) == 0
+    assert lsk.last_error()
+
+
+def test_workspace_size_covers_scores_and_partials(L):
+    d = _good()
+    ws = lsk.workspace_bytes(d)
+    rows = d.n_queries * d.group
+    assert ws >= 4 * d.batch * d.n_kv_heads * d.max_blocks
+    assert ws >= 4 * d.batch * d.n_kv_heads * (d.budget_blocks // 8) * rows * 128
+
+
+def test_null_and_misaligned_pointers_rejected_on_host(L):
+    d = _good()
+    rc = L.oasis_build_summaries(ctypes.byref(d), None, None, 0, 4, None, None, None)
+    assert rc == lsk.EINVAL and "NULL" in lsk.last_error()
+    rc = L.oasis_plan_fetch(ctypes.byref(d), 16, 32, 48, 0, 64, 80, 97, None)
+    assert rc == lsk.EINVAL and "aligned" in lsk.last_error()
+    rc = L.oasis_build_summaries(ctypes.byref(d), 16, 32, 60, 8, 48, 64, None)
+    assert rc == lsk.EINVAL and "block range" in lsk.last_error()
+    rc = L.oasis_sparse_attn(ctypes.byref(d), 16, 32, 48, 64, 1.0, 80, 96, 112, 10, None)
+    assert rc == lsk.EINVAL and "workspace" in lsk.last_error()
+    with pytest.raises(lsk.OasisError):
+        lsk.plan_fetch(d, None, None, None, 0, None, None, None, stream=0)
+
+
+def test_version_string(L):
+    assert b"sm_100a" in L.oasis_version()

@@ -1,0 +1,234 @@
+"""Whole decode steps on the GPU against the oracle: the tiny planted workload
+stage by stage, the stream-ordered pipeline against the sequential order,
+a small multi-layer run with appended tokens, and the full-size 32K
+Llama-shaped layer (the benchmarked configuration) on sampled units."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import lookahead_sparse_kv_b200 as lsk
+import oracle as O
+from lookahead_sparse_kv_b200 import workloads as W
+from lookahead_sparse_kv_b200.pipeline import DecodePipeline, LayerState
+from tests.gpu_util import assert_attention_close, assert_selection_matches, f64, kv_split, np_i32
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from lookahead_sparse_kv_b200 import build
+    build.build()
+    lsk.lib()
+    yield
+    assert lsk.read_device_error(clear=True) == 0
+
+
+def _check_pool_holds_slot_blocks(pool, st, host_bits):
+    """Every occupied slot holds exactly the host bytes of its block."""
+    pb = W.bf16_bits(pool)
+    for b in range(st.shape[0]):
+        for h in range(st.shape[1]):
+            for s in np.nonzero(st[b, h] >= 0)[0]:
+                np.testing.assert_array_equal(pb[b, h, s], host_bits[b, h, st[b, h, s]])
+
+
+def test_tiny_decode_stage_by_stage():
+    w = W.WORKLOADS["tiny"]
+    d = lsk.dims_for(w)
+    host = W.make_host_kv(w).pin_memory()
+    host_bits = W.bf16_bits(host)
+    keys, vals = kv_split(host)
+    ctx = W.initial_ctx_len(w)
+    L = LayerState(d, host, DEV)
+    ws = torch.zeros(lsk.workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    ctx_d = ctx.to(DEV)
+    lsk.build_summaries(d, host, ctx_d, L.kmin, L.kmax)
+    omin, omax = O.block_summaries(keys, ctx.numpy())
+    qs = W.QueryStream(w)
+    planted = W.planted_positions(w, 0)[0].numpy()
+    scale = 1 / math.sqrt(128)
+    for t in range(w.steps + 1):
+        q = qs.next()
+        qd = q.to(DEV)
+        if t > 0:
+            st = np_i32(L.slot_table)
+            lsk.sparse_attn(d, qd, L.pool, L.slot_table, ctx_d, scale, L.out, L.lse, ws)
+            torch.cuda.synchronize()
+            pk, pv = kv_split(L.pool)
+            o_ref, lse_ref = O.sparse_attention(f64(q), pk, pv, st, ctx.numpy(), scale)
+            assert_attention_close(L.out, L.lse, o_ref, lse_ref)
+        lsk.score_select(d, qd, L.kmin, L.kmax, ctx_d, L.sel, L.sel_score, ws)
+        torch.cuda.synchronize()
+        sc = O.lookahead_scores(f64(q), omin, omax, ctx.numpy(), 16)
+        ref_sel, _ = O.select_topk(sc, ctx.numpy(), w.budget_blocks, 16)
+        sel = np_i32(L.sel)
+        assert_selection_matches(sel, ref_sel, sc, ctx.numpy(), w.budget_blocks)
+        for h in range(w.n_kv_heads):
+            assert set(planted[0, h].tolist()) <= set(sel[0, h].tolist())      # recall 1.0
+        st0, lu0 = np_i32(L.slot_table), np_i32(L.last_used)
+        lsk.plan_fetch(d, L.sel, L.slot_table, L.last_used, t, L.fetch_slot, L.fetch_block, L.n_fetch)
+        lsk.prefetch(d, host, L.fetch_slot, L.fetch_block, L.n_fetch, L.pool)
+        torch.cuda.synchronize()
+        plan = O.plan_fetch(sel, st0, lu0, t, w.fetch_cap)
+        np.testing.assert_array_equal(np_i32(L.slot_table), plan["slot_table"])
+        np.testing.assert_array_equal(np_i32(L.last_used), plan["last_used"])
+        np.testing.assert_array_equal(np_i32(L.n_fetch), plan["n_fetch"])
+        np.testing.assert_array_equal(np_i32(L.fetch_block), plan["fetch_block"])
+        _check_pool_holds_slot_blocks(L.pool, plan["slot_table"], host_bits)
+    # after priming + 8 steps with cap 8 the 32-slot pool is full
+    assert (np_i32(L.slot_table) >= 0).all()
+
+
+def _run(w, overlap, steps):
+    """Runs priming + steps with the stream pipeline; returns per-step outputs."""
+    d = lsk.dims_for(w)
+    host = W.make_host_kv(w).pin_memory()
+    L = LayerState(d, host, DEV)
+    pipe = DecodePipeline(d, [L], W.initial_ctx_len(w).to(DEV), 1 / math.sqrt(128), DEV,
+                          overlap_score=overlap)
+    pipe.build_summaries()
+    qs = W.QueryStream(w)
+    pipe.prime([qs.next().to(DEV)])
+    outs = []
+    for t in range(1, steps + 1):
+        pipe.step(t, [qs.next().to(DEV)])
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        outs.append((L.out.clone(), L.lse.clone(), L.slot_table.clone(), L.last_used.clone(), L.pool.clone()))
+    return outs
+
+
+def test_pipeline_streams_match_sequential_order():
+    w = W.WORKLOADS["llama8b_32k"].with_(batch=2, n_q_heads=8, n_kv_heads=2, context=8192,
+                                          max_blocks=512, budget_blocks=64, fetch_cap=8)
+    a = _run(w, overlap=True, steps=5)
+    b = _run(w, overlap=False, steps=5)
+    for x, y in zip(a, b):
+        for u, v in zip(x, y):
+            assert torch.equal(u, v)
+
+
+def test_multilayer_append_decode():
+    """Three layers, one appended token per step (context crosses block
+    boundaries), score overlapped with attention, gather on the copy stream."""
+    w = W.WORKLOADS["qwen8b_reasoning"].with_(batch=3, n_q_heads=8, n_kv_heads=2, context=16 * 40 - 2,
+                                              max_blocks=48, budget_blocks=16, fetch_cap=4, layers=3)
+    d = lsk.dims_for(w)
+    scale = 1 / math.sqrt(128)
+    hosts = [W.make_host_kv(w, l).pin_memory() for l in range(w.layers)]
+    layers = [LayerState(d, h, DEV) for h in hosts]
+    ctx = W.initial_ctx_len(w)
+    pipe = DecodePipeline(d, layers, ctx.to(DEV), scale, DEV, overlap_score=True)
+    pipe.build_summaries()
+    streams = [W.QueryStream(w, l) for l in range(w.layers)]
+    # oracle state per layer (float64 keys / values mirror the host KV)
+    ref = []
+    for l in range(w.layers):
+        k, v = kv_split(hosts[l])
+        kmin, kmax = O.block_summaries(k, ctx.numpy())
+        ref.append({"k": k, "v": v, "kmin": kmin, "kmax": kmax,
+                    "st": np.full((w.batch, w.n_kv_heads, w.budget_blocks), -1, np.int32),
+                    "lu": np.full((w.batch, w.n_kv_heads, w.budget_blocks), -1, np.int32)})
+    q0 = [s.next() for s in streams]
+    pipe.prime([q.to(DEV) for q in q0])
+    ctx_np = ctx.numpy().copy()
+
+    def check_select_plan(l, q, step):
+        r, L = ref[l], layers[l]
+        sc = O.lookahead_scores(f64(q), r["kmin"], r["kmax"], ctx_np, 16)
+        ref_sel, _ = O.select_topk(sc, ctx_np, w.budget_blocks, 16)
+        sel = np_i32(L.sel)
+        assert_selection_matches(sel, ref_sel, sc, ctx_np, w.budget_blocks)
+        plan = O.plan_fetch(sel, r["st"], r["lu"], step, w.fetch_cap)
+        np.testing.assert_array_equal(np_i32(L.slot_table), plan["slot_table"])
+        np.testing.assert_array_equal(np_i32(L.last_used), plan["last_used"])
+        r["st"], r["lu"] = plan["slot_table"], plan["last_used"]
+        _check_pool_holds_slot_blocks(L.pool, r["st"], W.bf16_bits(hosts[l]))
+
+    pipe.wait_all()
+    torch.cuda.synchronize()
+    for l in range(w.layers):
+        check_select_plan(l, q0[l], 0)
+    for t in range(1, 7):
+        qs = [s.next() for s in streams]
+        app = [W.append_rows(w, l, t) for l in range(w.layers)]
+        # the oracle's view of the pre-step pool: slots hold host blocks
+        pipe.step(t, [q.to(DEV) for q in qs], [(k.to(DEV), v.to(DEV)) for k, v in app])
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        for l in range(w.layers):
+            r, L = ref[l], layers[l]
+            k_new, v_new = f64(app[l][0]), f64(app[l][1])
+            for b in range(w.batch):
+                n, tt = divmod(int(ctx_np[b]), 16)
+                r["k"][b, :, n, tt] = k_new[b]
+                r["v"][b, :, n, tt] = v_new[b]
+            O.summary_append(r["kmin"], r["kmax"], k_new, ctx_np, 16)
+        ctx_np = ctx_np + 1
+        assert np_i32(pipe.ctx_len).tolist() == ctx_np.tolist()
+        for l in range(w.layers):
+            r, L = ref[l], layers[l]
+            np.testing.assert_array_equal(f64(L.kmin)[~np.isnan(r["kmin"])], r["kmin"][~np.isnan(r["kmin"])])
+            # attention ran over the slots as planned at step t-1
+            st_prev = r["st"]
+            pk = np.zeros((w.batch, w.n_kv_heads, w.budget_blocks, 16, 128))
+            pv = np.zeros_like(pk)
+            for b in range(w.batch):
+                for h in range(w.n_kv_heads):
+                    for s in range(w.budget_blocks):
+                        if st_prev[b, h, s] >= 0:
+                            pk[b, h, s] = r["k"][b, h, st_prev[b, h, s]]
+                            pv[b, h, s] = r["v"][b, h, st_prev[b, h, s]]
+            o_ref, lse_ref = O.sparse_attention(f64(qs[l]), pk, pv, st_prev, ctx_np, scale)
+            assert_attention_close(L.out, L.lse, o_ref, lse_ref)
+            check_select_plan(l, qs[l], t)
+
+
+def test_full_size_llama_layer_sampled():
+    """The benchmarked 32K Llama-3.1-8B-shaped layer (B=16, 32/8 heads,
+    2,048 blocks, budget 128, cap 16) in the bench's launch configuration;
+    outputs checked on sampled (sequence, KV head) units and plans in full."""
+    from bench import build_workload_state
+    w = W.WORKLOADS["llama8b_32k"]
+    st = build_workload_state(w, steps=3, device=DEV)
+    d, L, pipe, qs = st["dims"], st["layer"], st["pipe"], st["queries"]
+    host_bits = None
+    rng = np.random.default_rng(0)
+    units = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.batch, 4), rng.integers(0, w.n_kv_heads, 4))]
+    ctx = np_i32(pipe.ctx_len)
+    scale = 1 / math.sqrt(128)
+    pipe.prime([qs[0]])
+    pipe.wait_all()
+    torch.cuda.synchronize()
+    for t in range(1, 3):
+        st_prev, lu_prev = np_i32(L.slot_table), np_i32(L.last_used)
+        pool_prev = L.pool.clone()
+        pipe.step(t, [qs[t]])
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        sel = np_i32(L.sel)
+        plan = O.plan_fetch(sel, st_prev, lu_prev, t, w.fetch_cap)
+        np.testing.assert_array_equal(np_i32(L.slot_table), plan["slot_table"])
+        np.testing.assert_array_equal(np_i32(L.last_used), plan["last_used"])
+        q = f64(qs[t].cpu())
+        for b, h in units:
+            kv_unit = L.host_kv[b:b + 1, h:h + 1]
+            k, v = kv_split(kv_unit)
+            kmin, kmax = O.block_summaries(k, ctx[b:b + 1])
+            np.testing.assert_array_equal(f64(L.kmin[b:b + 1, h:h + 1].cpu()), kmin)
+            G = w.group
+            qu = q[b:b + 1, :, h * G:(h + 1) * G]
+            sc = O.lookahead_scores(qu, kmin, kmax, ctx[b:b + 1], 16)
+            ref_sel, _ = O.select_topk(sc, ctx[b:b + 1], w.budget_blocks, 16)
+            assert_selection_matches(sel[b:b + 1, h:h + 1], ref_sel, sc, ctx[b:b + 1], w.budget_blocks)
+            pk, pv = kv_split(pool_prev[b:b + 1, h:h + 1].cpu())
+            o_ref, lse_ref = O.sparse_attention(qu, pk, pv, st_prev[b:b + 1, h:h + 1], ctx[b:b + 1], scale)
+            assert_attention_close(L.out[b:b + 1, :, h * G:(h + 1) * G], L.lse[b:b + 1, :, h * G:(h + 1) * G],
+                                   o_ref, lse_ref)
+            hb = W.bf16_bits(kv_unit)
+            _check_pool_holds_slot_blocks(L.pool[b:b + 1, h:h + 1], plan["slot_table"][b:b + 1, h:h + 1], hb)
