@@ -173,7 +173,8 @@ int oasis_prefetch(const oasis_dims* d, const void* host_kv, const int32_t* fetc
  * every occupied slot of (b, h),
  *   out = sum softmax(scale * q.k) v,   lse = log sum exp(scale * q.k);
  * no occupied slot / no valid token gives out = 0, lse = -inf.  bf16 inputs,
- * fp32 accumulation.  q, pool, slot_table, ctx_len, out, lse, ws: device. */
+ * fp32 accumulation.  scale must be positive and finite (OASIS_EINVAL
+ * otherwise).  q, pool, slot_table, ctx_len, out, lse, ws: device. */
 int oasis_sparse_attn(const oasis_dims* d, const void* q, const void* pool,
                       const int32_t* slot_table, const int32_t* ctx_len, float scale,
                       float* out, float* lse, void* ws, size_t ws_bytes, void* stream);

@@ -14,8 +14,9 @@
 // blocks beyond the context.  Streams are independent - there is no CTA-wide
 // barrier anywhere in the kernel - so an SM keeps up to 8 streams x 24 KiB
 // of KV in flight.  A stream writes one normalised partial (output and
-// log-sum-exp) for every (sequence, KV head) unit its range touches; a small
-// second kernel merges the partials of each unit in a fixed order.
+// log-sum-exp) for every (sequence, KV head) unit its range touches; a second
+// kernel, launched as a programmatic dependent, merges the partials of each
+// unit in stream order (one warp per query row, every load in flight).
 //
 // Math per slot (16 tokens), per warp, on the warp-level tensor-core path
 // (mma.sync m16n8k16, bf16 in, fp32 accumulate), tokens as the M dimension
@@ -56,6 +57,84 @@ __host__ __device__ __forceinline__ void attn_unit_streams(long long u, long lon
     *last = ((u + 1) * K - 1) * NS / T;
 }
 
+// Merges the stream partials of each (unit, query row) in stream order:
+// lse = log sum_p exp(lse_p), out = sum_p exp(lse_p - lse) * o_p.  One warp
+// per (unit, row); lane j holds partial j's lse, lane c owns channels
+// 4c..4c+3 and keeps up to 8 partial loads in flight.
+constexpr int kMergeWarps = 4;
+
+__global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, int n_streams,
+                                                                      const float* __restrict__ ws_o,
+                                                                      const float* __restrict__ ws_lse,
+                                                                      float* __restrict__ out,
+                                                                      float* __restrict__ lse_out) {
+    const float kNegInf = -__int_as_float(0x7f800000);
+    const int lane = threadIdx.x & 31;
+    const int G = d.G();
+    const int rows = d.Qn * G;
+    const long long units = static_cast<long long>(d.B) * d.Hkv;
+    const long long gw = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
+    // partials are produced by the attention grid this kernel depends on
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (gw >= units * rows) return;
+    const long long u = gw / rows;
+    const int r = static_cast<int>(gw % rows);
+    const long long T = units * d.K;
+    long long first, last;
+    attn_unit_streams(u, d.K, n_streams, T, &first, &last);
+    const int np = static_cast<int>(last - first + 1);
+    const long long p0 = first + u;
+    float M = kNegInf;
+    for (int j0 = 0; j0 < np; j0 += 32) {
+        const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;
+        M = fmaxf(M, lj);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* src = reinterpret_cast<const float4*>(ws_o + (p0 * rows + r) * kHeadDim) + lane;
+    const long long pstride = static_cast<long long>(rows) * (kHeadDim / 4);
+    if (M != kNegInf) {
+        for (int j0 = 0; j0 < np; j0 += 32) {
+            const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;
+            const float wj = lj == kNegInf ? 0.f : __expf(lj - M);
+            float ws = wj;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xFFFFFFFFu, ws, o);
+            L += ws;
+            const int nj = min(32, np - j0);
+            for (int k0 = 0; k0 < nj; k0 += 8) {
+                float4 v[8];
+                float wk[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    wk[k] = __shfl_sync(0xFFFFFFFFu, wj, (k0 + k) & 31);
+                    v[k] = (k0 + k < nj && wk[k] > 0.f) ? src[(j0 + k0 + k) * pstride]
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float w = k0 + k < nj ? wk[k] : 0.f;
+                    acc.x += w * v[k].x;
+                    acc.y += w * v[k].y;
+                    acc.z += w * v[k].z;
+                    acc.w += w * v[k].w;
+                }
+            }
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+    const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
+    const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
+    reinterpret_cast<float4*>(out + orow * kHeadDim)[lane] = acc;
+    if (lane == 0) lse_out[orow] = L > 0.f ? M + logf(L) : kNegInf;
+}
+
 template <int NTW, int QG>
 __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_pool, Dims d, const uint16_t* __restrict__ q,
@@ -69,7 +148,6 @@ __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ls = warp / QG, qg = warp % QG;             // local stream, query group
     const long long gs = static_cast<long long>(blockIdx.x) * kAttnStreamsPerCta + ls;
-    if (gs >= n_streams) return;                           // the whole stream has no work
 
     uint8_t* ring = smem + ls * Cfg::kStreamStride;
     int* l_slot = reinterpret_cast<int*>(ring + kAttnStages * kBlockBytes);
@@ -82,10 +160,10 @@ __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
     const int rows = d.Qn * G;
     const long long K = d.K;
     const long long T = static_cast<long long>(d.B) * d.Hkv * K;
-    const long long s_begin = (gs * T + n_streams - 1) / n_streams;
-    const long long s_end = ((gs + 1) * T + n_streams - 1) / n_streams;
-    if (s_begin >= s_end) return;
+    const long long s_begin = gs < n_streams ? (gs * T + n_streams - 1) / n_streams : 0;
+    const long long s_end = gs < n_streams ? ((gs + 1) * T + n_streams - 1) / n_streams : 0;
     const long long u_first = s_begin / K, u_last = (s_end - 1) / K;
+    if (s_begin < s_end) {
 
     if (qg == 0) {
         if (lane < kAttnStages) {
@@ -254,24 +332,29 @@ __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
                     if (g + 8 >= nv) sacc[nt][2] = sacc[nt][3] = kNegInf;
                 }
             }
-            // online softmax over tokens, per query column (log2 domain)
+            // online softmax over tokens, per query column (log2 domain).  The
+            // reference max only moves when a tile's max exceeds it by more
+            // than 8 (weights stay <= 2^8), so O and l are rarely rescaled;
+            // lse = m + log2(l) is exact for any reference.  scale > 0.
             float alpha[NTW][2];
             bool rescale = false;
 #pragma unroll
             for (int nt = 0; nt < NTW; ++nt) {
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    const float x0 = sacc[nt][c] * scale_log2, x1 = sacc[nt][2 + c] * scale_log2;
-                    float mx = fmaxf(x0, x1);
+                    float mx = fmaxf(sacc[nt][c], sacc[nt][2 + c]);
                     mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
                     mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
                     mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-                    const float mnew = fmaxf(m_run[nt][c], mx);
-                    alpha[nt][c] = exp2f(m_run[nt][c] - mnew);
-                    rescale |= alpha[nt][c] != 1.f;
-                    m_run[nt][c] = mnew;
-                    sacc[nt][c] = exp2f(x0 - mnew);
-                    sacc[nt][2 + c] = exp2f(x1 - mnew);
+                    const float mx_s = mx * scale_log2;
+                    alpha[nt][c] = 1.f;
+                    if (mx_s > m_run[nt][c] + 8.f) {
+                        alpha[nt][c] = exp2f(m_run[nt][c] - mx_s);
+                        m_run[nt][c] = mx_s;
+                        rescale = true;
+                    }
+                    sacc[nt][c] = exp2f(fmaf(sacc[nt][c], scale_log2, -m_run[nt][c]));
+                    sacc[nt][2 + c] = exp2f(fmaf(sacc[nt][2 + c], scale_log2, -m_run[nt][c]));
                 }
             }
             if (__any_sync(0xFFFFFFFFu, rescale)) {
@@ -343,82 +426,9 @@ __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
     }
     if (u_cur >= 0) finalize(u_cur, any);
     for (long long uu = (u_cur < 0 ? u_first : u_cur + 1); uu <= u_last; ++uu) write_empty(uu);
-}
-
-// Merges the stream partials of each (sequence, KV head) unit in stream
-// order: lse = log sum_p exp(lse_p), out = sum_p exp(lse_p - lse) * o_p.
-// One CTA per unit; each thread owns (row, 4 channels) outputs and keeps 4
-// partial loads in flight.  Dynamic smem: rows * (partials + 1) floats.
-__global__ void __launch_bounds__(256) attn_merge_kernel(Dims d, int n_streams, const float* __restrict__ ws_o,
-                                                         const float* __restrict__ ws_lse, float* __restrict__ out,
-                                                         float* __restrict__ lse_out) {
-    extern __shared__ float s_w[];                         // [rows][np] weights, then [rows] lse
-    const float kNegInf = -__int_as_float(0x7f800000);
-    const long long u = blockIdx.x;
-    const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
-    const int G = d.G();
-    const int rows = d.Qn * G;
-    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
-    long long first, last;
-    attn_unit_streams(u, d.K, n_streams, T, &first, &last);
-    const int np = static_cast<int>(last - first + 1);
-    const long long p0 = first + u;                        // partial entry of stream `first`
-    float* s_lse = s_w + rows * np;
-    for (int i = threadIdx.x; i < rows * np; i += blockDim.x) {
-        const int j = i / rows, r = i % rows;
-        s_w[r * np + j] = ws_lse[(p0 + j) * rows + r];
-    }
-    __syncthreads();
-    for (int r = threadIdx.x; r < rows; r += blockDim.x) {
-        float* wr = s_w + r * np;
-        float M = kNegInf;
-        for (int j = 0; j < np; ++j) M = fmaxf(M, wr[j]);
-        float L = 0.f;
-        for (int j = 0; j < np; ++j) {
-            const float wj = (M == kNegInf || wr[j] == kNegInf) ? 0.f : __expf(wr[j] - M);
-            wr[j] = wj;
-            L += wj;
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        for (int j = 0; j < np; ++j) wr[j] *= inv;
-        s_lse[r] = L > 0.f ? M + logf(L) : kNegInf;
-    }
-    __syncthreads();
-    const long long pstride = static_cast<long long>(rows) * (kHeadDim / 4);
-    for (int i = threadIdx.x; i < rows * 32; i += blockDim.x) {
-        const int r = i >> 5, q4 = i & 31;
-        const float* wr = s_w + r * np;
-        const float4* src = reinterpret_cast<const float4*>(ws_o + (p0 * rows + r) * kHeadDim) + q4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        int j = 0;
-        for (; j + 4 <= np; j += 4) {
-            float4 v[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                v[k] = wr[j + k] > 0.f ? src[(j + k) * pstride] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float wk = wr[j + k];
-                acc.x += wk * v[k].x;
-                acc.y += wk * v[k].y;
-                acc.z += wk * v[k].z;
-                acc.w += wk * v[k].w;
-            }
-        }
-        for (; j < np; ++j) {
-            const float wk = wr[j];
-            if (wk > 0.f) {
-                const float4 v = src[j * pstride];
-                acc.x += wk * v.x;
-                acc.y += wk * v.y;
-                acc.z += wk * v.z;
-                acc.w += wk * v.w;
-            }
-        }
-        const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
-        reinterpret_cast<float4*>(out + orow * kHeadDim)[q4] = acc;
-        if (q4 == 0) lse_out[orow] = s_lse[r];
-    }
+    }   // s_begin < s_end
+    // let the merge kernel (launched as a programmatic dependent) start early
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 }  // namespace oasis

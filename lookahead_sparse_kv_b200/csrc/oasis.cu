@@ -207,14 +207,23 @@ int launch_attn(const CUtensorMap& tm, const Dims& d, const uint16_t* q, const i
     k<<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmem, s>>>(tm, d, q, st, ctx, scale_log2,
                                                                       static_cast<int>(ns), ws_o, ws_lse);
     if (int rc = check_launch("sparse_attn launch")) return rc;
-    // merge: rows * (partials per unit + 1) floats of shared memory
-    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
-    const long long max_np = (static_cast<long long>(d.K) * ns + T - 1) / T + 1;
-    const int rows = d.Qn * d.G();
-    const int msmem = static_cast<int>(rows * (max_np + 1) * sizeof(float));
-    if (msmem > 200 * 1024) return fail(OASIS_EINVAL, "too many attention partials per unit");
-    if (int rc = set_smem(oasis::attn_merge_kernel, msmem, "attn_merge smem")) return rc;
-    oasis::attn_merge_kernel<<<d.B * d.Hkv, 256, msmem, s>>>(d, static_cast<int>(ns), ws_o, ws_lse, out, lse);
+    // merge, as a programmatic dependent launch: its launch overlaps the
+    // attention tail and griddepcontrol.wait orders its reads after it
+    const long long warps = static_cast<long long>(d.B) * d.Hkv * d.Qn * d.G();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((warps + oasis::kMergeWarps - 1) / oasis::kMergeWarps));
+    cfg.blockDim = dim3(32 * oasis::kMergeWarps);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, oasis::attn_merge_kernel, d, static_cast<int>(ns),
+                                             static_cast<const float*>(ws_o), static_cast<const float*>(ws_lse),
+                                             out, lse);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_merge launch");
     return check_launch("attn_merge launch");
 }
 
@@ -395,6 +404,7 @@ int oasis_sparse_attn(const oasis_dims* dp, const void* q, const void* pool, con
     if (int rc = check_ptr(out, "out")) return rc;
     if (int rc = check_ptr(lse, "lse")) return rc;
     if (int rc = check_ptr(ws, "ws")) return rc;
+    if (!(scale > 0.f) || !(scale < 3.0e38f)) return fail(OASIS_EINVAL, "scale must be a positive finite float");
     const WsLayout w = ws_layout(d);
     if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
     CUtensorMap tm;
