@@ -57,6 +57,25 @@ def ring_index(t: int, n: int) -> int:
     return p if p < n else 2 * n - 2 - p
 
 
+def rank_workload(rank: int):
+    """Weak scaling: every rank runs the benchmarked workload on its own
+    seeded batch (no data is exchanged between ranks)."""
+    w = W.WORKLOADS[WORKLOAD]
+    return w.with_(seed=w.seed + 1000 * rank) if rank else w
+
+
+def max_over_ranks(x: float) -> float:
+    """Max of a per-rank value over all ranks (device time of the slowest
+    rank); identity without a process group."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def build_workload_state(w, steps: int, device="cuda", n_queries: int | None = None, layers: int = 1):
     """Pinned host KV, per-layer device state, pipeline and resident queries
     for `layers` layers of workload `w` (layer l draws its own KV and queries)."""
@@ -260,9 +279,7 @@ def isolated_kernel_ms(st, reps: int = 20) -> dict:
 
 
 def run_gpu(args, rank, world, device):
-    w = W.WORKLOADS[WORKLOAD]
-    if rank:
-        w = w.with_(seed=w.seed + 1000 * rank)
+    w = rank_workload(rank)
     st = build_workload_state(w, args.warmup + args.steps, device, n_queries=args.query_ring,
                               layers=args.layers)
     d, layers, pipe, qrings = st["dims"], st["layers"], st["pipe"], st["qrings"]
@@ -303,9 +320,7 @@ def run_gpu(args, rank, world, device):
     ms = ev0.elapsed_time(ev1)
     if world > 1:
         torch.distributed.barrier()
-        m = torch.tensor([ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(m, op=torch.distributed.ReduceOp.MAX)
-        ms = float(m.item())
+    ms = max_over_ranks(ms)
 
     # reuse of the selected set between consecutive steps (untimed)
     reuse = []
@@ -344,11 +359,7 @@ def run_gpu(args, rank, world, device):
     pipe.wait_all()
     e1.record(main)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        m = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(m, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(m.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
 
     iso = isolated_kernel_ms(st)
     h2d = measure_h2d_peak(device) if rank == 0 else None
@@ -446,7 +457,7 @@ def emit_gpu(args, res, world):
                 "d2h_bytes_per_step": nl * (L.out.numel() * 4 + L.lse.numel() * 4),
                 "note": "per step: every layer's queries copied in from pinned host memory and its outputs read "
                         "back, then synchronised; h2d bytes include the zero-copy gather of fetched blocks"},
-        "gpu_launches": 5 * layer_steps,
+        "gpu_launches": 6 * layer_steps,   # attention, merge, score, select, plan, gather
         "clocks": res["clocks"],
         "device_error_word": res["dev_err"],
     }
