@@ -144,6 +144,29 @@ int oasis_score_select(const oasis_dims* d, const void* q, const void* kmin,
                        const void* kmax, const int32_t* ctx_len, int32_t* sel,
                        float* sel_score, void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of oasis_score_select (no counterpart in the
+ * paper; it exists for callers that cannot provide device scratch memory).
+ * Some callers cannot allocate or pass a workspace: an attention backend
+ * behind an engine interface that hands over only input and output tensors,
+ * or a process that reserved its device memory up front, where a cudaMalloc
+ * would fail or stall the device in the middle of a decode step.  This entry
+ * point takes the same inputs and outputs as oasis_score_select and keeps the
+ * block scores in a fixed 4 MiB array compiled into the library instead:
+ *   - limit: batch * n_kv_heads * max_blocks <= 1048576 (4 MiB of fp32
+ *     scores); larger dims return OASIS_EINVAL with a message;
+ *   - it calls no cudaMalloc / cudaFree and no allocating library routine;
+ *   - the first call on each device looks up the array's device address
+ *     (with that device current) and caches it; make that first call before
+ *     any stream capture;
+ *   - every call on a device shares the one array, which keeps the last
+ *     call's scores; calls whose work overlaps on the GPU (for example on two
+ *     streams) race on it and must be serialised by the caller;
+ *   - each GPU that loads the library holds the 4 MiB until the process
+ *     exits. */
+int oasis_score_select_noalloc(const oasis_dims* d, const void* q, const void* kmin,
+                               const void* kmax, const int32_t* ctx_len, int32_t* sel,
+                               float* sel_score, void* stream);
+
 /* a4 - residency diff and capped fetch plan (OasisKV method sketch item 3;
  * Table 2: LRU eviction; Figure 9: per-head slot table).  Per (b, h), with
  * S* the blocks of sel: slots holding a block of S* get last_used = step;

@@ -68,6 +68,7 @@ _SIGS = {
     "oasis_select_topk": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V]),
     "oasis_score_select": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V,
                                           ctypes.c_size_t, _V]),
+    "oasis_score_select_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V]),
     "oasis_plan_fetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _I32, _V, _V, _V, _V]),
     "oasis_prefetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V]),
     "oasis_sparse_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, ctypes.c_float,
@@ -162,6 +163,14 @@ def score_select(d, q, kmin, kmax, ctx_len, sel, sel_score, ws, stream=None):
     _check(lib().oasis_score_select(ctypes.byref(d), _p(q), _p(kmin), _p(kmax), _p(ctx_len), _p(sel),
                                     _p(sel_score), _p(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)), "oasis_score_select")
+
+
+def score_select_noalloc(d, q, kmin, kmax, ctx_len, sel, sel_score=None, stream=None):
+    """oasis_score_select without a workspace: for callers that cannot
+    allocate or pass device scratch; the scores live in a fixed 4 MiB array
+    inside the library (see include/oasis.h for the limit and sharing rules)."""
+    _check(lib().oasis_score_select_noalloc(ctypes.byref(d), _p(q), _p(kmin), _p(kmax), _p(ctx_len), _p(sel),
+                                            _p(sel_score), _stream(stream)), "oasis_score_select_noalloc")
 
 
 def plan_fetch(d, sel, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream=None):

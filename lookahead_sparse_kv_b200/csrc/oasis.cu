@@ -240,6 +240,38 @@ int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d
 
 }  // namespace
 
+// Built-in scratch for oasis_score_select_noalloc: the fp32 block scores of
+// one call, at most kNoAllocScoreFloats of them.  Every device that loads the
+// library holds this array until the process exits.
+constexpr size_t kNoAllocScoreFloats = size_t(1) << 20;   // 4 MiB
+static __device__ __align__(256) float g_noalloc_scores[kNoAllocScoreFloats];
+
+namespace {
+
+// Device address of g_noalloc_scores on the current device.  In host code the
+// array's name is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+int noalloc_scores(float** out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static float* cached[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(OASIS_EINVAL, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scores);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+        cached[dev] = static_cast<float*>(p);
+    }
+    *out = cached[dev];
+    return OASIS_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* oasis_last_error(void) { return g_msg; }
@@ -443,6 +475,24 @@ int oasis_read_device_error(uint32_t* out, int clear, void* stream) {
     }
     *out = v;
     return OASIS_OK;
+}
+
+int oasis_score_select_noalloc(const oasis_dims* dp, const void* q, const void* kmin, const void* kmax,
+                               const int32_t* ctx_len, int32_t* sel, float* sel_score, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    const size_t n = static_cast<size_t>(d.B) * d.Hkv * d.N;
+    if (n > kNoAllocScoreFloats)
+        return fail(OASIS_EINVAL,
+                    "batch * n_kv_heads * max_blocks = %zu exceeds the built-in scratch of %zu block scores (4 MiB); "
+                    "use oasis_score_select with a workspace",
+                    n, kNoAllocScoreFloats);
+    float* scores = nullptr;
+    if (int rc = noalloc_scores(&scores)) return rc;
+    // No entry needs to start at zero: the scorer writes every valid block's
+    // score before the selector reads it, and nothing else is read.
+    if (int rc = oasis_lookahead_scores(dp, q, kmin, kmax, ctx_len, scores, stream)) return rc;
+    return oasis_select_topk(dp, scores, ctx_len, sel, sel_score, stream);
 }
 
 }  // extern "C"

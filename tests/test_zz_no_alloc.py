@@ -1,0 +1,54 @@
+"""The allocation-free scoring + selection entry point.
+
+Some callers cannot give this library device scratch memory: an attention
+backend plugged into an engine whose interface hands it only the input and
+output tensors, or a process that reserved its device memory at start-up, so
+that a cudaMalloc would fail or stall the device mid-step.  For them
+oasis_score_select_noalloc keeps the block scores in a fixed array inside the
+library.  This test checks, through the C ABI, that it returns what the
+workspace entry point returns on two calls in a row with different inputs
+(the array keeps the previous call's contents), and that sizes beyond the
+array are refused.  Kept in its own file, collected last."""
+
+import pytest
+import torch
+
+import lookahead_sparse_kv_b200 as lsk
+from lookahead_sparse_kv_b200 import build
+
+DEV = "cuda"
+
+
+@pytest.mark.gpu
+def test_noalloc_score_select_matches_workspace_version_twice():
+    build.build()
+    B, Hq, Hkv, N, K, Qn = 4, 32, 8, 1000, 64, 5
+    d = lsk.make_dims(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, max_blocks=N, budget_blocks=K,
+                      n_queries=Qn, fetch_cap=8)
+    g = torch.Generator()
+    g.manual_seed(77)
+    kv = torch.randn(B, Hkv, N, 2, 16, 128, generator=g).to(torch.bfloat16).to(DEV)
+    kmin = torch.empty((B, Hkv, N, 128), dtype=torch.bfloat16, device=DEV)
+    kmax = torch.empty_like(kmin)
+    ws = torch.zeros(lsk.workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    contexts = [torch.tensor([N * 16, 700 * 16 + 3, 37, 999 * 16], dtype=torch.int32, device=DEV),
+                torch.tensor([500 * 16, N * 16 - 1, 64 * 16, 5000], dtype=torch.int32, device=DEV)]
+    for call, ctx in enumerate(contexts):
+        lsk.build_summaries(d, kv, ctx, kmin, kmax)
+        q = torch.randn(B, Qn, Hq, 128, generator=g).to(torch.bfloat16).to(DEV)
+        sel_ws = torch.full((B, Hkv, K), -5, dtype=torch.int32, device=DEV)
+        sc_ws = torch.full((B, Hkv, K), 5.0, device=DEV)
+        sel_na = torch.full_like(sel_ws, -7)
+        sc_na = torch.full_like(sc_ws, 7.0)
+        lsk.score_select(d, q, kmin, kmax, ctx, sel_ws, sc_ws, ws)
+        lsk.score_select_noalloc(d, q, kmin, kmax, ctx, sel_na, sc_na)
+        torch.cuda.synchronize()
+        assert torch.equal(sel_na, sel_ws), f"call {call}: selections differ"
+        torch.testing.assert_close(sc_na, sc_ws, rtol=1e-5, atol=1e-4)
+    assert lsk.read_device_error(clear=True) == 0
+
+    too_big = lsk.make_dims(batch=64, n_q_heads=32, n_kv_heads=8, max_blocks=4096, budget_blocks=64,
+                            n_queries=Qn, fetch_cap=8)
+    with pytest.raises(lsk.OasisError) as e:
+        lsk.score_select_noalloc(too_big, q, kmin, kmax, contexts[0], sel_na, sc_na)
+    assert e.value.code == lsk.EINVAL and "scratch" in str(e.value)
