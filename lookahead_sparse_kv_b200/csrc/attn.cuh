@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
     const int tokV = (lane & 7) + ((lane >> 4) << 3), hiV = (lane >> 3) & 1;
     long long rp = 0;            // ring position of the next slot consumed
     long long u_cur = -1;
+    long long u_end = 0;         // first slot past the current unit
     bool any = false;            // the current unit has seen a slot
     bool failed = false;
 
@@ -274,7 +275,9 @@ __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
                     if (qg == 0) raise_dev_error(OASIS_DEVERR_ID_RANGE);
                     blk = -1;
                 }
-                if (blk >= 0) nv = min(kBlockTokens, ctx_len[(s / K) / d.Hkv] - blk * kBlockTokens);
+                // slot indices stay below 2^26 (host check): 32-bit division
+                const unsigned unit = static_cast<unsigned>(s) / static_cast<unsigned>(K);
+                if (blk >= 0) nv = min(kBlockTokens, ctx_len[unit / static_cast<unsigned>(d.Hkv)] - blk * kBlockTokens);
             }
             const unsigned m = __ballot_sync(0xFFFFFFFFu, nv > 0);
             if (nv > 0 && qg == 0) {
@@ -290,11 +293,13 @@ __global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
             for (int i = 0; i < kAttnStages && i < n_list; ++i) issue(i, rp + i);
 
         for (int i = 0; i < n_list; ++i, ++rp) {
-            const long long u = l_slot[i] / K;
-            if (u != u_cur) {
+            if (l_slot[i] >= u_end) {
+                // slots are listed in order: divide only when the unit changes
+                const long long u = l_slot[i] / K;
                 if (u_cur >= 0) finalize(u_cur, any);
                 for (long long uu = (u_cur < 0 ? u_first : u_cur + 1); uu < u; ++uu) write_empty(uu);
                 u_cur = u;
+                u_end = (u + 1) * K;
                 any = false;
                 load_unit(u);
             }
