@@ -63,7 +63,7 @@ __host__ __device__ __forceinline__ void attn_unit_streams(long long u, long lon
 // 4c..4c+3 and keeps up to 8 partial loads in flight.
 constexpr int kMergeWarps = 4;
 
-__global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, int n_streams, int per_stream,
+__global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, int n_streams,
                                                                       const float* __restrict__ ws_o,
                                                                       const float* __restrict__ ws_lse,
                                                                       float* __restrict__ out,
@@ -82,9 +82,8 @@ __global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, in
     const long long T = units * d.K;
     long long first, last;
     attn_unit_streams(u, d.K, n_streams, T, &first, &last);
-    // stream s leaves per_stream partials for unit u, at per_stream*(s+u)+i
-    const int np = static_cast<int>(per_stream * (last - first + 1));
-    const long long p0 = per_stream * (first + u);
+    const int np = static_cast<int>(last - first + 1);
+    const long long p0 = first + u;
     float M = kNegInf;
     for (int j0 = 0; j0 < np; j0 += 32) {
         const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;

@@ -18,7 +18,6 @@
 #include "oasis.h"
 
 #include "attn.cuh"
-#include "attn_tc.cuh"
 #include "common.cuh"
 #include "plan.cuh"
 #include "prefetch.cuh"
@@ -140,24 +139,6 @@ int make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned
     return OASIS_OK;
 }
 
-// The pool viewed as [slots][32 rows][128 columns] bf16, boxes of 8 slots x
-// 16 rows x 64 columns, 128-byte swizzle.
-int make_pool_map_3d(CUtensorMap* m, const void* base, unsigned long long slots) {
-    auto fn = encode_fn();
-    if (fn == nullptr) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled unavailable");
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(oasis::kHeadDim), 2ull * oasis::kBlockTokens,
-                                static_cast<cuuint64_t>(slots)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(oasis::kRowBytes),
-                                   static_cast<cuuint64_t>(oasis::kBlockBytes)};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(oasis::kBlockTokens), 8};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled(pool 3d) failed: %d", static_cast<int>(r));
-    return OASIS_OK;
-}
-
 template <typename K>
 int set_smem(K kernel, int bytes, const char* what) {
     const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -184,8 +165,7 @@ WsLayout ws_layout(const Dims& d) {
     WsLayout w;
     const size_t units = static_cast<size_t>(d.B) * d.Hkv;
     const size_t rows = static_cast<size_t>(d.Qn) * d.G();
-    // up to two partials (softmax groups) per stream and unit
-    w.partials = 2 * (attn_max_streams(d) + static_cast<long long>(units));
+    w.partials = attn_max_streams(d) + static_cast<long long>(units);
     w.scores = 0;
     w.lse = align256(units * d.N * sizeof(float));
     w.o = align256(w.lse + static_cast<size_t>(w.partials) * rows * sizeof(float));
@@ -240,8 +220,7 @@ int launch_attn(const CUtensorMap& tm, const Dims& d, const uint16_t* q, const i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int per_stream = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, oasis::attn_merge_kernel, d, static_cast<int>(ns), per_stream,
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, oasis::attn_merge_kernel, d, static_cast<int>(ns),
                                              static_cast<const float*>(ws_o), static_cast<const float*>(ws_lse),
                                              out, lse);
     if (e != cudaSuccess) return cuda_fail(e, "attn_merge launch");
@@ -514,68 +493,6 @@ int oasis_score_select_noalloc(const oasis_dims* dp, const void* q, const void* 
     // score before the selector reads it, and nothing else is read.
     if (int rc = oasis_lookahead_scores(dp, q, kmin, kmax, ctx_len, scores, stream)) return rc;
     return oasis_select_topk(dp, scores, ctx_len, sel, sel_score, stream);
-}
-
-// tcgen05 attention (same contract as oasis_sparse_attn); not yet in the
-// public header.
-int oasis_sparse_attn_tc(const oasis_dims* dp, const void* q, const void* pool, const int32_t* slot_table,
-                         const int32_t* ctx_len, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
-                         void* stream) {
-    Dims d;
-    if (int rc = validate(dp, &d)) return rc;
-    if (int rc = check_ptr(q, "q")) return rc;
-    if (int rc = check_ptr(pool, "pool")) return rc;
-    if (int rc = check_ptr(slot_table, "slot_table")) return rc;
-    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
-    if (int rc = check_ptr(out, "out")) return rc;
-    if (int rc = check_ptr(lse, "lse")) return rc;
-    if (int rc = check_ptr(ws, "ws")) return rc;
-    if (!(scale > 0.f) || !(scale < 3.0e38f)) return fail(OASIS_EINVAL, "scale must be a positive finite float");
-    const WsLayout w = ws_layout(d);
-    if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
-    CUtensorMap tm;
-    const unsigned long long prow = static_cast<unsigned long long>(d.B) * d.Hkv * d.K * 2 * oasis::kBlockTokens;
-    if (int rc = make_map(&tm, pool, prow, oasis::kBlockTokens, "pool")) return rc;
-    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
-    CUtensorMap tm3;
-    if (int rc = make_pool_map_3d(&tm3, pool, static_cast<unsigned long long>(T))) return rc;
-    long long ns = std::max<long long>(sm_count(), (T + oasis::kTcList - 1) / oasis::kTcList);
-    ns = std::min(ns, std::min(T, attn_max_streams(d)));
-    if ((T + ns - 1) / ns > oasis::kTcList) return fail(OASIS_EINVAL, "too many slots for the tcgen05 attention");
-    uint8_t* base = static_cast<uint8_t*>(ws);
-    float* ws_lse = reinterpret_cast<float*>(base + w.lse);
-    float* ws_o = reinterpret_cast<float*>(base + w.o);
-    const float scale_log2 = scale * 1.4426950408889634f;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int rows = d.Qn * d.G();
-    if (rows <= 32) {
-        const int bytes = oasis::TcSmem<32>::kAlloc;
-        if (int rc = set_smem(oasis::sparse_attn_tc_kernel<32>, bytes, "attn_tc smem")) return rc;
-        oasis::sparse_attn_tc_kernel<32><<<static_cast<unsigned>(ns), oasis::kTcThreads, bytes, s>>>(
-            tm, tm3, d, static_cast<const uint16_t*>(q), slot_table, ctx_len, scale_log2, ws_o, ws_lse);
-    } else {
-        const int bytes = oasis::TcSmem<64>::kAlloc;
-        if (int rc = set_smem(oasis::sparse_attn_tc_kernel<64>, bytes, "attn_tc smem")) return rc;
-        oasis::sparse_attn_tc_kernel<64><<<static_cast<unsigned>(ns), oasis::kTcThreads, bytes, s>>>(
-            tm, tm3, d, static_cast<const uint16_t*>(q), slot_table, ctx_len, scale_log2, ws_o, ws_lse);
-    }
-    if (int rc = check_launch("attn_tc launch")) return rc;
-    const int per_stream = rows <= 32 ? oasis::TcSmem<32>::kGroups : oasis::TcSmem<64>::kGroups;
-    const long long warps = static_cast<long long>(d.B) * d.Hkv * rows;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((warps + oasis::kMergeWarps - 1) / oasis::kMergeWarps));
-    cfg.blockDim = dim3(32 * oasis::kMergeWarps);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, oasis::attn_merge_kernel, d, static_cast<int>(ns), per_stream,
-                                             static_cast<const float*>(ws_o), static_cast<const float*>(ws_lse),
-                                             out, lse);
-    if (e != cudaSuccess) return cuda_fail(e, "attn_merge launch");
-    return check_launch("attn_merge launch");
 }
 
 }  // extern "C"
