@@ -59,6 +59,7 @@ class Workload:
     planted_key_scale: float = 0.5
     evict_prob: float = 0.0      # per-step probability that a resident slot is lost
     append: bool = False         # one new token per sequence per step
+    draft_lead: bool = False     # draft row j follows the query mean j steps ahead (see QueryStream)
     seed: int = 20260807
 
     @property
@@ -112,6 +113,12 @@ WORKLOADS = {
                             context=32768, max_blocks=_blocks(32768), budget_blocks=128,
                             n_queries=8, fetch_cap=16, layers=64, steps=16,
                             ar_rho=0.9, query_noise=0.05, evict_prob=0.1),
+    # The 32K Llama layer with drafts that lead the verification query (the
+    # prediction-quality and corrective-fetch measurements).
+    "llama8b_32k_lead": Workload("llama8b_32k_lead", batch=16, n_q_heads=32, n_kv_heads=8,
+                                 context=32768, max_blocks=_blocks(32768), budget_blocks=128,
+                                 n_queries=5, fetch_cap=16, steps=64, ar_rho=0.9,
+                                 query_noise=0.05, draft_lead=True),
     # 128K stress: heavy-tailed keys, planted groups hopping every 64 steps.
     "longctx_128k": Workload("longctx_128k", batch=8, n_q_heads=32, n_kv_heads=8,
                              context=131072, max_blocks=_blocks(131072), budget_blocks=128,
@@ -217,6 +224,14 @@ class QueryStream:
     d_t = rho * d_{t-1} + sqrt(1 - rho^2) * eta_t with unit stationary
     variance (absent when rho = 0).  Step 0 is the priming step (the drafts
     of the step before decoding starts).
+
+    With ``draft_lead`` the drafts look ahead: row j of step t is drawn around
+    m_{t+j}, the mean the verification row will have j steps later (the AR(1)
+    path is generated that far ahead), so draft j stands for a draft model
+    that proposes the token j positions on, whose query it carries (OasisKV
+    Figure 6: the propagated draft query approximates the true next-token
+    query).  Row 0 is drawn around m_t as before.  Without it every row of a
+    step shares m_t.
     """
 
     def __init__(self, w: Workload, layer: int = 0, device="cpu"):
@@ -225,9 +240,28 @@ class QueryStream:
         self.u = mean_directions(w, layer, device)          # [groups, B, H, D]
         self.d = torch.randn(self.u.shape[1:], generator=self.g, device=device)
         self.t = 0
+        if w.draft_lead:
+            # d_t .. d_{t+Qn-1}: the drift of the verification row and of each draft's target step
+            self.path = [self.d]
+            for _ in range(w.n_queries - 1):
+                self.path.append(self._ar_step(self.path[-1]))
+
+    def _ar_step(self, d):
+        eta = torch.randn(d.shape, generator=self.g, device=self.device)
+        return self.w.ar_rho * d + math.sqrt(1.0 - self.w.ar_rho ** 2) * eta
+
+    def _mean(self, t, d):
+        w = self.w
+        group = (t // w.hop_every) % self.u.shape[0] if w.hop_every else 0
+        m = self.u[group]
+        if w.ar_rho:
+            m = m + (w.drift_scale * w.query_mean_scale) * d
+        return m
 
     def next(self) -> torch.Tensor:
         w = self.w
+        if w.draft_lead:
+            return self._next_lead()
         group = (self.t // w.hop_every) % self.u.shape[0] if w.hop_every else 0
         m = self.u[group]
         if w.ar_rho:
@@ -238,6 +272,16 @@ class QueryStream:
         B, H, G, D, Qn = w.batch, w.n_kv_heads, w.group, w.head_dim, w.n_queries
         xi = torch.randn(B, Qn, H, G, D, generator=self.g, device=self.device)
         q = m.view(B, 1, H, 1, D) + w.query_noise * xi
+        self.t += 1
+        return q.reshape(B, Qn, H * G, D).to(torch.bfloat16)
+
+    def _next_lead(self) -> torch.Tensor:
+        w = self.w
+        B, H, G, D, Qn = w.batch, w.n_kv_heads, w.group, w.head_dim, w.n_queries
+        means = torch.stack([self._mean(self.t + j, self.path[j]) for j in range(Qn)], dim=1)   # [B, Qn, H, D]
+        xi = torch.randn(B, Qn, H, G, D, generator=self.g, device=self.device)
+        q = means.view(B, Qn, H, 1, D) + w.query_noise * xi
+        self.path = self.path[1:] + [self._ar_step(self.path[-1])]
         self.t += 1
         return q.reshape(B, Qn, H * G, D).to(torch.bfloat16)
 

@@ -50,6 +50,15 @@ Readings taken where the pages are silent (each also listed in the design doc):
 * R5 attention reads every occupied slot (the resident blocks), masking
   tokens at or beyond ``ctx_len``; all ``Qn`` rows see the same token set.
 * R6 empty token set: output 0, log-sum-exp -inf.
+* R7 exact set and corrective fetch ([OasisKV] Figure 6 and "What they did":
+  prediction misses need corrective fetches).  At decode step t the exact
+  set E_t is the top-K under the same scorer with the verification row
+  (row 0, the true query of step t) alone.  Agreement of a predicted set S
+  with E_t is |S & E_t| (reported over |E_t|); the lookahead prediction is
+  the selection made from the drafts of step t-1, the previous-token
+  prediction is E_{t-1}.  A corrective fetch brings every block of E_t that
+  is not resident before step t's attention, with the same planner and no
+  cap (C = K), as a use at step t.
 """
 
 from __future__ import annotations
@@ -70,6 +79,7 @@ __all__ = [
     "prefetch",
     "sparse_attention",
     "dense_attention",
+    "block_overlap",
     "decode_layer_steps",
 ]
 
@@ -151,7 +161,7 @@ def summary_append(kmin, kmax, k_new, ctx_len_before, block_tokens):
 
 
 # --------------------------------------------------- a2: lookahead scores
-def lookahead_scores(q, kmin, kmax, ctx_len, block_tokens):
+def lookahead_scores(q, kmin, kmax, ctx_len, block_tokens, rows=None):
     """Score every valid block of every (sequence, KV head) with the drafts.
 
     [OasisKV] Figure 7 (right): "the draft query then scans the compressed
@@ -163,12 +173,15 @@ def lookahead_scores(q, kmin, kmax, ctx_len, block_tokens):
     the G query heads sharing the KV head.
 
     q: float64 [B, Qn, Hq, D]; kmin/kmax float64 [B, Hkv, N, D].
+    rows: the query rows scored (default: the drafts 1..Qn-1, or row 0 when
+    Qn == 1); [0] scores with the verification query alone (R7).
     Returns float32 [B, Hkv, N]; blocks at or beyond n_valid are -inf.
     """
     B, Qn, Hq, D = q.shape
     _, H, N, _ = kmin.shape
     G = Hq // H
-    rows = list(range(1, Qn)) if Qn > 1 else [0]
+    if rows is None:
+        rows = list(range(1, Qn)) if Qn > 1 else [0]
     nv = n_valid_blocks(ctx_len, block_tokens)
     out = np.full((B, H, N), -np.inf, dtype=np.float32)
     for b in range(B):
@@ -365,9 +378,23 @@ def dense_attention(q, keys, values, ctx_len, scale):
     return o, lse
 
 
+# ------------------------------------- prediction quality (R7): set overlap
+def block_overlap(a, b):
+    """Per (sequence, KV head): how many distinct block ids of list ``b`` also
+    occur in list ``a`` (-1 entries are empty).  a, b: int [B, Hkv, *]."""
+    B, H = a.shape[:2]
+    out = np.zeros((B, H), dtype=np.int32)
+    for i in range(B):
+        for h in range(H):
+            sa = {int(x) for x in a[i, h] if x >= 0}
+            sb = {int(x) for x in b[i, h] if x >= 0}
+            out[i, h] = len(sa & sb)
+    return out
+
+
 # ------------------------------------------------ a7: per-step order
 def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
-                       budget_blocks, fetch_cap, scale, host_kv_bits=None):
+                       budget_blocks, fetch_cap, scale, host_kv_bits=None, corrective=False):
     """One layer through priming and T decode steps, in the pages' order.
 
     [OasisKV] Figure 8: at step t the draft queries drive top-K prediction,
@@ -381,6 +408,11 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
     keys/values: float64 [B, Hkv, N, P, D]; q_prime, q_steps[t]: float64
     [B, Qn, Hq, D].  Returns a list of per-step dicts (attention output,
     selection, plan) plus the final slot table.
+
+    With ``corrective`` each decode step first finds the exact set E_t from
+    the verification row, records the agreement counts of the lookahead and
+    previous-token predictions and the resident coverage of E_t, and fetches
+    E_t's missing blocks without a cap before the attention (R7).
     """
     B, H, N, P, D = keys.shape
     K = budget_blocks
@@ -400,13 +432,34 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
         st, lu = plan["slot_table"], plan["last_used"]
         return sc, sel, sel_score, plan
 
-    select_plan_fetch(q_prime, 0)
+    def corrective_fetch(qs, step, sel_lookahead, exact_prev):
+        nonlocal st, lu, pool_k, pool_v
+        exact, _ = select_topk(lookahead_scores(qs, kmin, kmax, ctx_len, P, rows=[0]), ctx_len, K, P)
+        rec = {"exact": exact,
+               "agree_lookahead": block_overlap(sel_lookahead, exact),
+               "agree_prev": block_overlap(exact_prev, exact) if exact_prev is not None else None,
+               "covered": block_overlap(st, exact)}
+        plan = plan_fetch(exact, st, lu, step, K)
+        pool_k = prefetch(keys, pool_k, plan["fetch_slot"], plan["fetch_block"], plan["n_fetch"])
+        pool_v = prefetch(values, pool_v, plan["fetch_slot"], plan["fetch_block"], plan["n_fetch"])
+        st, lu = plan["slot_table"], plan["last_used"]
+        rec["plan"] = plan
+        return rec
+
+    _, sel_prev, _, _ = select_plan_fetch(q_prime, 0)
+    exact_prev = None
     for t, qs in enumerate(q_steps, start=1):
+        corr = None
+        if corrective:
+            corr = corrective_fetch(qs, t, sel_prev, exact_prev)
+            exact_prev = corr["exact"]
         o, lse = sparse_attention(qs, pool_k, pool_v, st, ctx_len, scale)
         slot_table_used = st.copy()
         sc, sel, sel_score, plan = select_plan_fetch(qs, t)
+        sel_prev = sel
         records.append({"o": o, "lse": lse, "slot_table_attn": slot_table_used,
-                        "scores": sc, "sel": sel, "sel_score": sel_score, "plan": plan})
+                        "scores": sc, "sel": sel, "sel_score": sel_score, "plan": plan,
+                        "corrective": corr})
     return records, st, lu
 
 
