@@ -144,6 +144,28 @@ int oasis_score_select(const oasis_dims* d, const void* q, const void* kmin,
                        const void* kmax, const int32_t* ctx_len, int32_t* sel,
                        float* sel_score, void* ws, size_t ws_bytes, void* stream);
 
+/* a2 + a3 over a chosen range of query rows: the scores take the max over
+ * rows j in [row_begin, row_begin + row_count) (and the G heads) instead of
+ * the drafts, then top-K as oasis_select_topk.  row_begin = 0, row_count = 1
+ * ranks the blocks for the verification query alone: the exact top-K set of
+ * the true query (OasisKV Figure 6) and the previous-token prediction of
+ * Figure 4; a corrective fetch plans from it.  Same buffers and workspace as
+ * oasis_score_select; EINVAL if the rows fall outside [0, Qn). */
+int oasis_score_select_rows(const oasis_dims* d, const void* q, int32_t row_begin,
+                            int32_t row_count, const void* kmin, const void* kmax,
+                            const int32_t* ctx_len, int32_t* sel, float* sel_score,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Prediction quality (OasisKV Figure 4: top-K accuracy of the previous token
+ * vs a lookahead token; Figure 6: agreement of the predicted top-K with the
+ * exact set).  count[b][h] = number of distinct block ids in b[b][h][0..K)
+ * that also occur in a[b][h][0..K); -1 entries are empty.  a, b: device
+ * int32 [B][Hkv][K] (selections, exact sets or slot tables); count: device
+ * int32 [B][Hkv].  Ids outside [-1, N) are skipped and set
+ * OASIS_DEVERR_ID_RANGE. */
+int oasis_block_overlap(const oasis_dims* d, const int32_t* a, const int32_t* b,
+                        int32_t* count, void* stream);
+
 /* Allocation-free variant of oasis_score_select (no counterpart in the
  * paper; it exists for callers that cannot provide device scratch memory).
  * Some callers cannot allocate or pass a workspace: an attention backend

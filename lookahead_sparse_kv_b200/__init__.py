@@ -69,6 +69,9 @@ _SIGS = {
     "oasis_score_select": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V,
                                           ctypes.c_size_t, _V]),
     "oasis_score_select_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V]),
+    "oasis_score_select_rows": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _I32, _I32, _V, _V, _V, _V, _V, _V,
+                                               ctypes.c_size_t, _V]),
+    "oasis_block_overlap": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V]),
     "oasis_plan_fetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _I32, _V, _V, _V, _V]),
     "oasis_prefetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V]),
     "oasis_sparse_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, ctypes.c_float,
@@ -163,6 +166,21 @@ def score_select(d, q, kmin, kmax, ctx_len, sel, sel_score, ws, stream=None):
     _check(lib().oasis_score_select(ctypes.byref(d), _p(q), _p(kmin), _p(kmax), _p(ctx_len), _p(sel),
                                     _p(sel_score), _p(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)), "oasis_score_select")
+
+
+def score_select_rows(d, q, row_begin, row_count, kmin, kmax, ctx_len, sel, sel_score, ws, stream=None):
+    """Top-K for query rows [row_begin, row_begin + row_count); (0, 1) is the
+    verification query alone (exact set / previous-token prediction)."""
+    _check(lib().oasis_score_select_rows(ctypes.byref(d), _p(q), row_begin, row_count, _p(kmin), _p(kmax),
+                                         _p(ctx_len), _p(sel), _p(sel_score), _p(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)),
+           "oasis_score_select_rows")
+
+
+def block_overlap(d, a, b, count, stream=None):
+    """count[b][h] = distinct ids of list b also in list a (int32 [B][Hkv][K] each)."""
+    _check(lib().oasis_block_overlap(ctypes.byref(d), _p(a), _p(b), _p(count), _stream(stream)),
+           "oasis_block_overlap")
 
 
 def score_select_noalloc(d, q, kmin, kmax, ctx_len, sel, sel_score=None, stream=None):

@@ -19,6 +19,7 @@
 
 #include "attn.cuh"
 #include "common.cuh"
+#include "overlap.cuh"
 #include "plan.cuh"
 #include "prefetch.cuh"
 #include "score.cuh"
@@ -229,12 +230,12 @@ int launch_attn(const CUtensorMap& tm, const Dims& d, const uint16_t* q, const i
 
 template <int NPAD>
 int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
-                 const int32_t* ctx, float* scores, int rows, cudaStream_t s) {
+                 const int32_t* ctx, float* scores, int row0, int rows, cudaStream_t s) {
     using S = oasis::ScoreSmem<NPAD>;
     auto k = oasis::lookahead_score_kernel<NPAD>;
     if (int rc = set_smem(k, S::kBytes, "score smem")) return rc;
     dim3 grid((d.N + oasis::kScoreTile - 1) / oasis::kScoreTile, d.B * d.Hkv);
-    k<<<grid, 128, S::kBytes, s>>>(tmax, tmin, d, q, ctx, scores, rows);
+    k<<<grid, 128, S::kBytes, s>>>(tmax, tmin, d, q, ctx, scores, row0, rows);
     return check_launch("lookahead_score launch");
 }
 
@@ -268,6 +269,31 @@ int noalloc_scores(float** out) {
     }
     *out = cached[dev];
     return OASIS_OK;
+}
+
+// Scores with query rows [row_begin, row_begin + row_count) of each sequence.
+int scores_rows(const oasis_dims* dp, const void* q, int row_begin, int row_count, const void* kmin, const void* kmax,
+                const int32_t* ctx_len, float* scores, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(q, "q")) return rc;
+    if (int rc = check_ptr(kmin, "kmin")) return rc;
+    if (int rc = check_ptr(kmax, "kmax")) return rc;
+    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
+    if (int rc = check_ptr(scores, "scores")) return rc;
+    if (row_begin < 0 || row_count < 1 || row_begin + row_count > d.Qn)
+        return fail(OASIS_EINVAL, "query rows [%d, %d) outside [0, %d)", row_begin, row_begin + row_count, d.Qn);
+    const int rows = row_count * d.G();
+    const unsigned long long total_rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.N;
+    CUtensorMap tmax, tmin;
+    if (int rc = make_map(&tmax, kmax, total_rows, oasis::kScoreTile, "kmax")) return rc;
+    if (int rc = make_map(&tmin, kmin, total_rows, oasis::kScoreTile, "kmin")) return rc;
+    const auto* qq = static_cast<const uint16_t*>(q);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rows <= 16) return launch_score<16>(tmax, tmin, d, qq, ctx_len, scores, row_begin, rows, s);
+    if (rows <= 32) return launch_score<32>(tmax, tmin, d, qq, ctx_len, scores, row_begin, rows, s);
+    if (rows <= 48) return launch_score<48>(tmax, tmin, d, qq, ctx_len, scores, row_begin, rows, s);
+    return launch_score<64>(tmax, tmin, d, qq, ctx_len, scores, row_begin, rows, s);
 }
 
 }  // namespace
@@ -338,24 +364,9 @@ int oasis_append_kv(const oasis_dims* dp, const void* k_new, const void* v_new, 
 
 int oasis_lookahead_scores(const oasis_dims* dp, const void* q, const void* kmin, const void* kmax,
                            const int32_t* ctx_len, float* scores, void* stream) {
-    Dims d;
-    if (int rc = validate(dp, &d)) return rc;
-    if (int rc = check_ptr(q, "q")) return rc;
-    if (int rc = check_ptr(kmin, "kmin")) return rc;
-    if (int rc = check_ptr(kmax, "kmax")) return rc;
-    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
-    if (int rc = check_ptr(scores, "scores")) return rc;
-    const int rows = (d.Qn > 1 ? d.Qn - 1 : 1) * d.G();
-    const unsigned long long total_rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.N;
-    CUtensorMap tmax, tmin;
-    if (int rc = make_map(&tmax, kmax, total_rows, oasis::kScoreTile, "kmax")) return rc;
-    if (int rc = make_map(&tmin, kmin, total_rows, oasis::kScoreTile, "kmin")) return rc;
-    const auto* qq = static_cast<const uint16_t*>(q);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (rows <= 16) return launch_score<16>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
-    if (rows <= 32) return launch_score<32>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
-    if (rows <= 48) return launch_score<48>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
-    return launch_score<64>(tmax, tmin, d, qq, ctx_len, scores, rows, s);
+    if (dp == nullptr) return fail(OASIS_EINVAL, "dims is NULL");
+    const int qn = dp->n_queries;
+    return scores_rows(dp, q, qn > 1 ? 1 : 0, qn > 1 ? qn - 1 : 1, kmin, kmax, ctx_len, scores, stream);
 }
 
 int oasis_select_topk(const oasis_dims* dp, const float* scores, const int32_t* ctx_len, int32_t* sel,
@@ -384,6 +395,31 @@ int oasis_score_select(const oasis_dims* dp, const void* q, const void* kmin, co
     float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.scores);
     if (int rc = oasis_lookahead_scores(dp, q, kmin, kmax, ctx_len, scores, stream)) return rc;
     return oasis_select_topk(dp, scores, ctx_len, sel, sel_score, stream);
+}
+
+int oasis_score_select_rows(const oasis_dims* dp, const void* q, int32_t row_begin, int32_t row_count,
+                            const void* kmin, const void* kmax, const int32_t* ctx_len, int32_t* sel,
+                            float* sel_score, void* ws, size_t ws_bytes, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(ws, "ws")) return rc;
+    const WsLayout w = ws_layout(d);
+    if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
+    float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.scores);
+    if (int rc = scores_rows(dp, q, row_begin, row_count, kmin, kmax, ctx_len, scores, stream)) return rc;
+    return oasis_select_topk(dp, scores, ctx_len, sel, sel_score, stream);
+}
+
+int oasis_block_overlap(const oasis_dims* dp, const int32_t* a, const int32_t* b, int32_t* count, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(a, "a")) return rc;
+    if (int rc = check_ptr(b, "b")) return rc;
+    if (int rc = check_ptr(count, "count")) return rc;
+    const int smem = 2 * ((d.N + 31) / 32) * static_cast<int>(sizeof(uint32_t));
+    oasis::block_overlap_kernel<<<d.B * d.Hkv, oasis::kOverlapThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+        d, a, b, count);
+    return check_launch("block_overlap launch");
 }
 
 int oasis_plan_fetch(const oasis_dims* dp, const int32_t* sel, int32_t* slot_table, int32_t* last_used,

@@ -34,13 +34,14 @@ struct ScoreSmem {
     static constexpr int kTmemCols = NPAD <= 32 ? 32 : (NPAD <= 64 ? 64 : (NPAD <= 128 ? 128 : 256));
 };
 
-// rows = real query vectors (draft rows x G), NPAD = rows rounded up to 16.
+// rows = real query vectors (scored query rows x G), the scored rows being
+// row0, row0+1, ...; NPAD = rows rounded up to 16.
 template <int NPAD>
 __global__ void __launch_bounds__(128) lookahead_score_kernel(const __grid_constant__ CUtensorMap tm_kmax,
                                                               const __grid_constant__ CUtensorMap tm_kmin,
                                                               Dims d, const uint16_t* __restrict__ q,
                                                               const int32_t* __restrict__ ctx_len,
-                                                              float* __restrict__ scores, int rows) {
+                                                              float* __restrict__ scores, int row0, int rows) {
     using S = ScoreSmem<NPAD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,7 +85,7 @@ __global__ void __launch_bounds__(128) lookahead_score_kernel(const __grid_const
         const int r = it >> 4, c = it & 15;   // c: 8-channel chunk
         uint4 v = make_uint4(0, 0, 0, 0);
         if (r < rows) {
-            const int j = d.Qn > 1 ? 1 + r / G : 0;
+            const int j = row0 + r / G;
             const int g = r % G;
             v = *reinterpret_cast<const uint4*>(
                 q + ((static_cast<long long>(b) * d.Qn + j) * d.Hq + h * G + g) * kHeadDim + c * 8);

@@ -16,6 +16,13 @@ Streams (all work is in liboasis kernels; this module only orders them):
 * copy  - host-to-HBM gather, high priority, after the layer's plan; the next
           step's append/attention of that layer waits for it
 
+Exact-set mode (OasisKV Figures 4 and 6; prediction misses need corrective
+fetches): before a layer's attention at step t the main stream ranks the
+blocks for the verification query alone (the exact set E_t), counts how many
+of E_t the lookahead selection of step t-1, the previous step's exact set and
+the resident slots hold, and - with ``exact="correct"`` - plans and gathers
+the missing blocks of E_t with no cap, in stream order before the attention.
+
 Memory: the full KV of every layer lives in pinned host memory; HBM holds per
 layer the per-block summaries (N x 512 B per KV head), the fixed pool of K
 slots (8 KiB each) and a few small int tables.  One workspace serves all
@@ -27,8 +34,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (append_kv, build_summaries, plan_fetch, prefetch, score_select, sparse_attn,
-               workspace_bytes)
+from . import (append_kv, block_overlap, build_summaries, make_dims, plan_fetch, prefetch, score_select,
+               score_select_rows, sparse_attn, workspace_bytes)
 
 HEAD_DIM, BLOCK_TOKENS = 128, 16
 
@@ -57,6 +64,25 @@ class LayerState:
         self.lse = torch.zeros((B, Qn, Hq), dtype=torch.float32, device=device)
         self.plan_ready = torch.cuda.Event()
         self.fetch_done = torch.cuda.Event()
+        self.hist = None
+
+    def enable_exact(self, steps_cap: int, device="cuda"):
+        """Buffers of the exact-set mode: two exact sets (this step's and the
+        previous one), uncapped fetch lists, and per decode step t (slot
+        (t-1) % steps_cap) int32 [B, Hkv] counts: 0 lookahead agreement,
+        1 previous-token agreement, 2 resident coverage, 3 corrective fetches."""
+        d = self.d
+        B, H, K = d.batch, d.n_kv_heads, d.budget_blocks
+        self.exact = [torch.full((B, H, K), -1, dtype=torch.int32, device=device) for _ in range(2)]
+        self.cfetch_slot = torch.full((B, H, K), -1, dtype=torch.int32, device=device)
+        self.cfetch_block = torch.full((B, H, K), -1, dtype=torch.int32, device=device)
+        # each [B, Hkv] slice padded to 16 bytes (the library's pointer alignment)
+        self.hist = torch.zeros((4, steps_cap, (B * H + 3) // 4 * 4), dtype=torch.int32, device=device)
+        self.sel_read = torch.cuda.Event()
+
+    def hist_slot(self, k: int, slot: int) -> torch.Tensor:
+        d = self.d
+        return self.hist[k, slot, : d.batch * d.n_kv_heads].view(d.batch, d.n_kv_heads)
 
     def device_bytes(self) -> int:
         ts = [self.kmin, self.kmax, self.pool, self.slot_table, self.last_used, self.sel, self.sel_score,
@@ -68,8 +94,19 @@ class DecodePipeline:
     """Drives priming and decode steps over a list of layers."""
 
     def __init__(self, d, layers, ctx_len: torch.Tensor, scale: float, device="cuda",
-                 overlap_score: bool = True):
+                 overlap_score: bool = True, exact: str | None = None, steps_cap: int = 256):
+        assert exact in (None, "measure", "correct")
         self.d, self.layers, self.scale = d, layers, scale
+        self.exact = exact
+        self.steps_cap = steps_cap
+        if exact is not None:
+            # uncapped plan / gather for the corrective fetch; a workspace of its own
+            # because the score stream may be scoring the previous layer meanwhile
+            self.d_full = make_dims(d.batch, d.n_q_heads, d.n_kv_heads, d.max_blocks, d.budget_blocks,
+                                    d.n_queries, d.budget_blocks, d.head_dim, d.block_tokens)
+            self.ws_exact = torch.zeros(workspace_bytes(d), dtype=torch.uint8, device=device)
+            for L in layers:
+                L.enable_exact(steps_cap, device)
         self.ctx = [ctx_len, ctx_len.clone()]           # ping-pong when tokens are appended
         self.cur = 0
         self.ws = torch.zeros(workspace_bytes(d), dtype=torch.uint8, device=device)
@@ -96,6 +133,8 @@ class DecodePipeline:
         d, main = self.d, self.main
         if self.score_stream is not main:
             self.score_stream.wait_event(L.plan_ready)     # previous plan has read L.sel
+            if self.exact is not None and step > 0:
+                self.score_stream.wait_event(L.sel_read)   # so has the agreement count
         self._t("begin", "score_select", self.score_stream)
         score_select(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, self.ws, stream=self.score_stream)
         self._t("end", "score_select", self.score_stream)
@@ -111,6 +150,34 @@ class DecodePipeline:
         prefetch(d, L.host_kv, L.fetch_slot, L.fetch_block, L.n_fetch, L.pool, stream=self.copy_stream)
         self._t("end", "prefetch", self.copy_stream)
         L.fetch_done.record(self.copy_stream)
+
+    def _exact_step(self, L, q, t, ctx):
+        """Exact set of step t, agreement counts, optional corrective fetch (main stream)."""
+        d, main = self.d, self.main
+        cur, prev = L.exact[t % 2], L.exact[(t - 1) % 2]
+        h = [L.hist_slot(k, (t - 1) % self.steps_cap) for k in range(4)]
+        self._t("begin", "exact_set", main)
+        score_select_rows(d, q, 0, 1, L.kmin, L.kmax, ctx, cur, None, self.ws_exact, stream=main)
+        block_overlap(d, L.sel, cur, h[0], stream=main)
+        if t > 1:
+            block_overlap(d, prev, cur, h[1], stream=main)
+        block_overlap(d, L.slot_table, cur, h[2], stream=main)
+        L.sel_read.record(main)
+        self._t("end", "exact_set", main)
+        if self.exact == "correct":
+            self._t("begin", "corrective", main)
+            plan_fetch(self.d_full, cur, L.slot_table, L.last_used, t, L.cfetch_slot, L.cfetch_block, h[3],
+                       stream=main)
+            prefetch(self.d_full, L.host_kv, L.cfetch_slot, L.cfetch_block, h[3], L.pool, stream=main)
+            self._t("end", "corrective", main)
+
+    def prediction_counts(self):
+        """Host copies of the per-step counts, int64 [layers, 4, steps_cap, B, Hkv]
+        (see LayerState.enable_exact); synchronises."""
+        d = self.d
+        bh = d.batch * d.n_kv_heads
+        h = torch.stack([L.hist[:, :, :bh] for L in self.layers]).cpu().long()
+        return h.view(len(self.layers), 4, self.steps_cap, d.batch, d.n_kv_heads)
 
     def prime(self, q_per_layer):
         """Step 0: select, plan and fetch from the drafts before decoding starts."""
@@ -140,6 +207,8 @@ class DecodePipeline:
                     ev = torch.cuda.Event()
                     ev.record(main)
                     self.score_stream.wait_event(ev)       # grown summaries and context
+            if self.exact is not None:
+                self._exact_step(L, q, t, ctx)
             self._t("begin", "sparse_attn", main)
             sparse_attn(d, q, L.pool, L.slot_table, ctx, self.scale, L.out, L.lse, self.ws, stream=main)
             self._t("end", "sparse_attn", main)
