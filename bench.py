@@ -17,6 +17,15 @@ the data path).
 
 Prints one JSON line (rank 0).  With --impl reference the CPU oracle runs the
 same configuration on the host cores (rank 0 only).
+
+    python bench.py --prediction [--steps K] [--layers L]
+
+measures prediction quality and the corrective fetch instead (OasisKV
+Figures 4 and 6): the same layers with drafts that lead the verification
+query, each decode step ranking the blocks for the true query (the exact
+set), counting how much of it the lookahead selection and the previous
+step's exact set (the previous-token predictor) hold, and - in the third run
+- fetching the missing blocks before the attention.  One JSON line.
 """
 
 from __future__ import annotations
@@ -276,6 +285,106 @@ def isolated_kernel_ms(st, reps: int = 20) -> dict:
         out[name] = tot / reps
     out["_prefetch_blocks"] = fetched
     return out
+
+
+def run_prediction(args, device):
+    """Three runs over the same layers of the leading-draft workload: lookahead
+    prefetch only, plus the exact-set counts, plus the corrective fetch.  Each
+    is primed, warmed up until the pool is full and timed over --steps decode
+    steps; the queries are one unbroken AR(1) path (no ring)."""
+    w = W.WORKLOADS["llama8b_32k_lead"]
+    d = lsk.dims_for(w)
+    nl = args.layers
+    fill = w.budget_blocks // max(1, w.fetch_cap) + 4          # steps until the pool is full
+    total = 1 + fill + args.steps
+    layers, qpaths = [], []
+    for l in range(nl):
+        host = torch.empty((w.batch, w.n_kv_heads, w.max_blocks, 2, w.block_tokens, w.head_dim),
+                           dtype=torch.bfloat16, pin_memory=True)
+        W.make_host_kv(w, layer=l, device=device, out=host)
+        layers.append(LayerState(d, host, device))
+        qs = W.QueryStream(w, l, device)
+        qpaths.append([qs.next() for _ in range(total)])
+    torch.cuda.synchronize()
+    ctx = W.initial_ctx_len(w, device)
+    out = {}
+    for mode in (None, "measure", "correct"):
+        for L in layers:
+            L.slot_table.fill_(-1)
+            L.last_used.fill_(-1)
+            L.sel.fill_(-1)
+        pipe = DecodePipeline(d, layers, ctx, 1.0 / math.sqrt(w.head_dim), device, exact=mode,
+                              steps_cap=total)
+        pipe.build_summaries()
+        pipe.prime([p[0] for p in qpaths])
+        for t in range(1, 1 + fill):
+            pipe.step(t, [p[t] for p in qpaths])
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(pipe.main)
+        for t in range(1 + fill, total):
+            pipe.step(t, [p[t] for p in qpaths])
+        pipe.wait_all()
+        e1.record(pipe.main)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        res = {"layer_steps_per_s": nl * args.steps / (ms * 1e-3), "ms_per_step": ms / args.steps}
+        if mode is not None:
+            c = pipe.prediction_counts()[:, :, fill:total - 1].double()     # timed steps t = fill+1 .. total-1
+            k = float(w.budget_blocks)                                      # |exact set| (every context > K blocks)
+            per_layer = c.mean(dim=(2, 3, 4)) / k                           # [layers, 4]
+            res.update({
+                "lookahead_agreement": per_layer[:, 0].mean().item(),
+                "previous_token_agreement": per_layer[:, 1].mean().item(),
+                "resident_coverage": per_layer[:, 2].mean().item(),
+                "lookahead_agreement_per_layer": [round(x, 4) for x in per_layer[:, 0].tolist()],
+                "previous_token_agreement_per_layer": [round(x, 4) for x in per_layer[:, 1].tolist()],
+            })
+            if mode == "correct":
+                res["corrective_blocks_per_head_step"] = c[:, 3].mean().item()
+                res["corrective_mib_per_layer_step"] = (c[:, 3].sum(dim=(2, 3)).mean().item()
+                                                        * w.block_bytes / 2 ** 20)
+        out[mode or "lookahead_only"] = res
+        del pipe
+    # agreement only, on two of the layers, for faster-moving queries: the
+    # AR(1) coefficient and drift size set how far the true query moves per step
+    sweep = []
+    for rho, drift in ((0.9, 0.3), (0.9, 1.0), (0.7, 1.0), (0.5, 1.0), (0.2, 1.0)):
+        wq = w.with_(ar_rho=rho, drift_scale=drift)
+        sub = layers[:2]
+        paths = []
+        for l in range(len(sub)):
+            qs = W.QueryStream(wq, l, device)
+            paths.append([qs.next() for _ in range(total)])
+        for L in sub:
+            L.slot_table.fill_(-1)
+            L.last_used.fill_(-1)
+            L.sel.fill_(-1)
+        pipe = DecodePipeline(d, sub, ctx, 1.0 / math.sqrt(w.head_dim), device, exact="measure", steps_cap=total)
+        pipe.build_summaries()
+        pipe.prime([p[0] for p in paths])
+        for t in range(1, total):
+            pipe.step(t, [p[t] for p in paths])
+        pipe.wait_all()
+        c = pipe.prediction_counts()[:, :, fill:total - 1].double().mean(dim=(0, 2, 3, 4)) / float(w.budget_blocks)
+        sweep.append({"ar_rho": rho, "drift_scale": drift, "lookahead_agreement": c[0].item(),
+                      "previous_token_agreement": c[1].item(), "resident_coverage": c[2].item()})
+        del pipe
+    err = lsk.read_device_error(clear=True)
+    line = {
+        "metric": "top-K prediction agreement and corrective fetch (synthetic analog of OasisKV Figs. 4 and 6)",
+        "workload": f"llama8b_32k_lead: {nl} Llama-3.1-8B-shaped layers at 32K, batch {w.batch}, budget "
+                    f"{w.budget_blocks} blocks, cap {w.fetch_cap}, 1+{w.n_drafts} queries; draft j of step t "
+                    f"is drawn around the query mean of step t+j (AR(1) rho {w.ar_rho})",
+        "steps": args.steps, "warmup_steps": fill, "layers": nl,
+        "definitions": {"lookahead_agreement": "|lookahead top-K of step t-1 & exact top-K of step t| / K",
+                        "previous_token_agreement": "|exact top-K of step t-1 & exact top-K of step t| / K",
+                        "resident_coverage": "|resident blocks before step t & exact top-K of step t| / K",
+                        "exact top-K": "top-K under the same min/max bound with the verification query alone"},
+        "runs": out, "query_drift_sweep": sweep, "device_error_word": err,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def run_gpu(args, rank, world, device):
@@ -589,6 +698,8 @@ def main():
     ap.add_argument("--query-ring", type=int, default=48)
     ap.add_argument("--impl", default="oasis", choices=["oasis", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prediction", action="store_true",
+                    help="measure prediction agreement and the corrective fetch instead")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -603,6 +714,10 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.prediction:
+        if rank == 0:
+            run_prediction(args, device)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
