@@ -59,6 +59,10 @@ Readings taken where the pages are silent (each also listed in the design doc):
   prediction is E_{t-1}.  A corrective fetch brings every block of E_t that
   is not resident before step t's attention, with the same planner and no
   cap (C = K), as a use at step t.
+* R8 score-based victims (the alternative to Table 2's LRU in the eviction
+  ablation): stale slots are taken in order of their block's current
+  lookahead score, lowest first, ties to the lower block id (-0.0 == +0.0);
+  free slots still come first and a selected block is never evicted.
 """
 
 from __future__ import annotations
@@ -229,7 +233,7 @@ def select_topk(scores, ctx_len, budget_blocks, block_tokens):
 
 
 # ------------------------------------------ a4: residency diff + fetch plan
-def plan_fetch(sel, slot_table, last_used, step, fetch_cap):
+def plan_fetch(sel, slot_table, last_used, step, fetch_cap, scores=None):
     """Compare the selection with the resident set and plan a capped fetch.
 
     [OasisKV] method sketch item 3: predicted blocks are compared against the
@@ -243,7 +247,9 @@ def plan_fetch(sel, slot_table, last_used, step, fetch_cap):
       1. every slot holding a block of S* is stamped last_used = step;
       2. M = blocks of S* not resident, in rank order; F = first min(C, |M|);
       3. victims: free slots ascending, then slots whose block is not in S*
-         by (last_used, block id) ascending (R4);
+         by (last_used, block id) ascending (R4) - or, when ``scores``
+         (float32 [B, Hkv, N], this step's lookahead scores) is given, by
+         (score of the block, block id) ascending (R8);
       4. F[i] goes to victims[i], which is stamped last_used = step.
 
     Inputs are not modified.  Returns a dict with the new slot_table and
@@ -276,7 +282,10 @@ def plan_fetch(sel, slot_table, last_used, step, fetch_cap):
             free = [slot for slot in range(K) if st[b, h, slot] < 0]
             stale = [slot for slot in range(K)
                      if st[b, h, slot] >= 0 and int(st[b, h, slot]) not in in_sel]
-            stale.sort(key=lambda slot: (int(lu[b, h, slot]), int(st[b, h, slot])))
+            if scores is None:
+                stale.sort(key=lambda slot: (int(lu[b, h, slot]), int(st[b, h, slot])))
+            else:
+                stale.sort(key=lambda slot: (float(scores[b, h, st[b, h, slot]]), int(st[b, h, slot])))
             victims = free + stale
             assert len(victims) >= len(fetch)
             for i, blk in enumerate(fetch):
