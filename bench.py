@@ -26,6 +26,13 @@ query, each decode step ranking the blocks for the true query (the exact
 set), counting how much of it the lookahead selection and the previous
 step's exact set (the previous-token predictor) hold, and - in the third run
 - fetching the missing blocks before the attention.  One JSON line.
+
+    python bench.py --ablation [--steps K] [--layers L]
+
+is the synthetic analog of OasisKV Table 2: the fetch cap as a fraction of
+the budget K (0.01 .. 0.2 and uncapped) with LRU and score-ordered victims;
+per setting the fetch volume, the H2D rate, layer-steps/s and how much of the
+exact top-K of the true query and of the lookahead selection is resident.
 """
 
 from __future__ import annotations
@@ -387,6 +394,97 @@ def run_prediction(args, device):
     print(json.dumps(line), flush=True)
 
 
+def run_ablation(args, device):
+    """Fetch-ratio x victim-order sweep over the 32K Llama layers.  Every
+    setting starts from a pool primed with the full top-K (uncapped), runs
+    warm-up steps at its cap, then times --steps decode steps without the
+    exact-set stage; a second, untimed pass over the same steps measures the
+    coverage of the exact set (the residency decisions do not depend on it)."""
+    w = W.WORKLOADS["llama8b_32k"]
+    K = w.budget_blocks
+    d_full = lsk.dims_for(w.with_(fetch_cap=K))
+    nl = args.layers
+    warm = 8
+    total = 1 + warm + args.steps
+    layers, qpaths = [], []
+    for l in range(nl):
+        host = torch.empty((w.batch, w.n_kv_heads, w.max_blocks, 2, w.block_tokens, w.head_dim),
+                           dtype=torch.bfloat16, pin_memory=True)
+        W.make_host_kv(w, layer=l, device=device, out=host)
+        layers.append(LayerState(d_full, host, device))       # fetch lists sized for any cap <= K
+        qs = W.QueryStream(w, l, device)
+        qpaths.append([qs.next() for _ in range(total)])
+    torch.cuda.synchronize()
+    ctx = W.initial_ctx_len(w, device)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    cover = torch.zeros((w.batch, w.n_kv_heads), dtype=torch.int32, device=device)
+    rows = []
+    # the first setting runs once untimed first, so no row pays for the GPU's clock ramp
+    settings = [(0.10, "lru", False)] + [(r, v, True) for r in (0.01, 0.02, 0.05, 0.10, 0.20, 1.0)
+                                         for v in ("lru", "score")]
+    for ratio, victims, keep in settings:
+        cap = max(1, round(ratio * K))
+        d = lsk.dims_for(w.with_(fetch_cap=cap))
+        res = {"fetch_ratio": ratio, "cap": cap, "victims": victims}
+        for exact in ((None, "measure") if keep else (None,)):
+            for L in layers:
+                L.slot_table.fill_(-1)
+                L.last_used.fill_(-1)
+            primer = DecodePipeline(d_full, layers, ctx, scale, device, victims=victims)
+            primer.build_summaries()
+            primer.prime([p[0] for p in qpaths])
+            primer.wait_all()
+            torch.cuda.synchronize()
+            del primer
+            pipe = DecodePipeline(d, layers, ctx, scale, device, exact=exact, steps_cap=total, victims=victims)
+            for t in range(1, 1 + warm):
+                pipe.step(t, [p[t] for p in qpaths])
+            pipe.wait_all()
+            torch.cuda.synchronize()
+            fetched = torch.zeros((), dtype=torch.int64, device=device)
+            resident_sel = torch.zeros((), dtype=torch.int64, device=device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(pipe.main)
+            for t in range(1 + warm, total):
+                pipe.step(t, [p[t] for p in qpaths])
+                if exact is None:
+                    for L in layers:
+                        fetched += L.n_fetch.sum()
+            pipe.wait_all()
+            e1.record(pipe.main)
+            torch.cuda.synchronize()
+            if exact is None:
+                ms = e0.elapsed_time(e1)
+                nfetch = fetched.item() / (nl * args.steps)           # blocks per layer-step
+                for L in layers:                                       # final plan's fetches landed
+                    lsk.block_overlap(d, L.slot_table, L.sel, cover)
+                    resident_sel += cover.sum()
+                torch.cuda.synchronize()
+                res.update({"layer_steps_per_s": nl * args.steps / (ms * 1e-3),
+                            "fetch_mib_per_layer_step": nfetch * w.block_bytes / 2 ** 20,
+                            "h2d_gbs": nfetch * w.block_bytes * nl * args.steps / (ms * 1e-3) / 1e9,
+                            "selection_resident_after_fetch":
+                                resident_sel.item() / (nl * w.batch * w.n_kv_heads * K)})
+            else:
+                c = pipe.prediction_counts()[:, 2, warm:total - 1].double()
+                res["exact_coverage"] = c.mean().item() / K
+            del pipe
+        if keep:
+            rows.append(res)
+    line = {
+        "metric": "fetch-cap and victim-order ablation (synthetic analog of OasisKV Table 2)",
+        "workload": f"llama8b_32k: {nl} Llama-3.1-8B-shaped layers at 32K, batch {w.batch}, budget {K} blocks, "
+                    f"1+{w.n_drafts} queries, AR(1)-drifting queries",
+        "steps": args.steps, "warmup_steps": warm,
+        "definitions": {"cap": "max(1, round(fetch_ratio * K)) blocks per (sequence, KV head) per step",
+                        "exact_coverage": "|resident before step t & exact top-K of the true query| / K",
+                        "selection_resident_after_fetch": "|resident after the last fetch & last selection| / K",
+                        "victims": "lru = least recently used stale slot; score = lowest current lookahead score"},
+        "rows": rows, "device_error_word": lsk.read_device_error(clear=True),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_gpu(args, rank, world, device):
     w = rank_workload(rank)
     st = build_workload_state(w, args.warmup + args.steps, device, n_queries=args.query_ring,
@@ -700,6 +798,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prediction", action="store_true",
                     help="measure prediction agreement and the corrective fetch instead")
+    ap.add_argument("--ablation", action="store_true",
+                    help="fetch-cap x victim-order sweep (Table 2 analog) instead")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -714,9 +814,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if args.prediction:
+    if args.prediction or args.ablation:
         if rank == 0:
-            run_prediction(args, device)
+            (run_prediction if args.prediction else run_ablation)(args, device)
         return
     if world > 1:
         import datetime

@@ -202,6 +202,17 @@ int oasis_plan_fetch(const oasis_dims* d, const int32_t* sel, int32_t* slot_tabl
                      int32_t* last_used, int32_t step, int32_t* fetch_slot,
                      int32_t* fetch_block, int32_t* n_fetch, void* stream);
 
+/* a4 with score-ordered victims (the eviction ablation's alternative to the
+ * LRU order of OasisKV Table 2): as oasis_plan_fetch, except that stale slots
+ * are taken by (score of their block, block id) ascending, the lowest-scored
+ * block first (-0.0 == +0.0).  scores: device fp32 [B][Hkv][N], this step's
+ * lookahead scores (oasis_lookahead_scores); entries of resident blocks must
+ * be written (a resident block is always below n_valid). */
+int oasis_plan_fetch_scored(const oasis_dims* d, const int32_t* sel, const float* scores,
+                            int32_t* slot_table, int32_t* last_used, int32_t step,
+                            int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
+                            void* stream);
+
 /* a5 - host-to-HBM gather (OasisKV Figure 7: blocks "are prefetched from the
  * CPU cache"; Figure 8).  For i < n_fetch[b][h], copies the 8 KiB block
  * host_kv[b][h][fetch_block[b][h][i]] into pool[b][h][fetch_slot[b][h][i]]

@@ -73,6 +73,7 @@ _SIGS = {
                                                ctypes.c_size_t, _V]),
     "oasis_block_overlap": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V]),
     "oasis_plan_fetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _I32, _V, _V, _V, _V]),
+    "oasis_plan_fetch_scored": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _I32, _V, _V, _V, _V]),
     "oasis_prefetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V]),
     "oasis_sparse_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, ctypes.c_float,
                                          _V, _V, _V, ctypes.c_size_t, _V]),
@@ -195,6 +196,13 @@ def plan_fetch(d, sel, slot_table, last_used, step, fetch_slot, fetch_block, n_f
     _check(lib().oasis_plan_fetch(ctypes.byref(d), _p(sel), _p(slot_table), _p(last_used), int(step),
                                   _p(fetch_slot), _p(fetch_block), _p(n_fetch), _stream(stream)),
            "oasis_plan_fetch")
+
+
+def plan_fetch_scored(d, sel, scores, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream=None):
+    """oasis_plan_fetch with victims ordered by their block's score (lowest first)."""
+    _check(lib().oasis_plan_fetch_scored(ctypes.byref(d), _p(sel), _p(scores), _p(slot_table), _p(last_used),
+                                         int(step), _p(fetch_slot), _p(fetch_block), _p(n_fetch),
+                                         _stream(stream)), "oasis_plan_fetch_scored")
 
 
 def prefetch(d, host_kv, fetch_slot, fetch_block, n_fetch, pool, stream=None):

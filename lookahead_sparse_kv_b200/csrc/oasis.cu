@@ -296,6 +296,31 @@ int scores_rows(const oasis_dims* dp, const void* q, int row_begin, int row_coun
     return launch_score<64>(tmax, tmin, d, qq, ctx_len, scores, row_begin, rows, s);
 }
 
+// Residency diff + capped fetch plan; LRU victims, or by score if scores != NULL.
+int plan(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t* slot_table, int32_t* last_used,
+         int32_t step, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(sel, "sel")) return rc;
+    if (int rc = check_ptr(slot_table, "slot_table")) return rc;
+    if (int rc = check_ptr(last_used, "last_used")) return rc;
+    if (int rc = check_ptr(n_fetch, "n_fetch")) return rc;
+    if (d.C > 0) {
+        if (int rc = check_ptr(fetch_slot, "fetch_slot")) return rc;
+        if (int rc = check_ptr(fetch_block, "fetch_block")) return rc;
+    }
+    const int threads = (d.K + 31) / 32 * 32;
+    const int smem = 7 * d.K * static_cast<int>(sizeof(int32_t));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (scores != nullptr)
+        oasis::plan_fetch_kernel<true><<<d.B * d.Hkv, threads, smem, s>>>(d, sel, scores, slot_table, last_used,
+                                                                         step, fetch_slot, fetch_block, n_fetch);
+    else
+        oasis::plan_fetch_kernel<false><<<d.B * d.Hkv, threads, smem, s>>>(d, sel, scores, slot_table, last_used,
+                                                                          step, fetch_slot, fetch_block, n_fetch);
+    return check_launch("plan_fetch launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -424,21 +449,14 @@ int oasis_block_overlap(const oasis_dims* dp, const int32_t* a, const int32_t* b
 
 int oasis_plan_fetch(const oasis_dims* dp, const int32_t* sel, int32_t* slot_table, int32_t* last_used,
                      int32_t step, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch, void* stream) {
-    Dims d;
-    if (int rc = validate(dp, &d)) return rc;
-    if (int rc = check_ptr(sel, "sel")) return rc;
-    if (int rc = check_ptr(slot_table, "slot_table")) return rc;
-    if (int rc = check_ptr(last_used, "last_used")) return rc;
-    if (int rc = check_ptr(n_fetch, "n_fetch")) return rc;
-    if (d.C > 0) {
-        if (int rc = check_ptr(fetch_slot, "fetch_slot")) return rc;
-        if (int rc = check_ptr(fetch_block, "fetch_block")) return rc;
-    }
-    const int threads = (d.K + 31) / 32 * 32;
-    const int smem = 6 * d.K * static_cast<int>(sizeof(int32_t));
-    oasis::plan_fetch_kernel<<<d.B * d.Hkv, threads, smem, static_cast<cudaStream_t>(stream)>>>(
-        d, sel, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch);
-    return check_launch("plan_fetch launch");
+    return plan(dp, sel, nullptr, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream);
+}
+
+int oasis_plan_fetch_scored(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t* slot_table,
+                            int32_t* last_used, int32_t step, int32_t* fetch_slot, int32_t* fetch_block,
+                            int32_t* n_fetch, void* stream) {
+    if (int rc = check_ptr(scores, "scores")) return rc;
+    return plan(dp, sel, scores, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream);
 }
 
 int oasis_prefetch(const oasis_dims* dp, const void* host_kv, const int32_t* fetch_slot, const int32_t* fetch_block,

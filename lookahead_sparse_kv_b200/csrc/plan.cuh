@@ -12,9 +12,13 @@
 //   2. misses are numbered in rank order by a block-wide scan; the first
 //      min(C, |M|) are fetched;
 //   3. every unprotected slot j gets a 64-bit victim key - free slots
-//      (0, j), stale slots (1, last_used, block id) - and its rank among the
+//      (0, j), stale slots (1, order, block id) - and its rank among the
 //      candidates by counting smaller keys; rank r < nF receives fetch r.
-// Integer only, so the result is bit-exact against any correct planner.
+//      order = last_used (LRU, Table 2) or, for the score-based variant of
+//      the eviction ablation, the block's current lookahead score mapped to
+//      a monotone integer key (lowest score evicted first).
+// Integer only (the score enters as its order key), so the result is
+// bit-exact against any correct planner.
 #pragma once
 
 #include "common.cuh"
@@ -47,14 +51,18 @@ __device__ __forceinline__ int block_excl_sum_any(int v, int* tmp, int* total) {
     return incl - v;
 }
 
-__device__ __forceinline__ unsigned long long victim_key(int slot, int blk, int lu) {
+// order: an unsigned key, smaller = evicted earlier (blk < 15 bits, N <= 32768)
+__device__ __forceinline__ unsigned long long victim_key(int slot, int blk, uint32_t order) {
     if (blk < 0) return static_cast<unsigned long long>(slot);
-    return (1ull << 63) | (static_cast<unsigned long long>(static_cast<uint32_t>(lu) ^ 0x80000000u) << 31) |
+    return (1ull << 63) | (static_cast<unsigned long long>(order) << 31) |
            static_cast<unsigned long long>(static_cast<uint32_t>(blk));
 }
 
-// blockDim.x = K rounded up to a multiple of 32; dynamic smem 6*K ints.
+// blockDim.x = K rounded up to a multiple of 32; dynamic smem 7*K ints.
+// kScored: victims by the block's score (scores fp32 [B][Hkv][N]), else LRU.
+template <bool kScored>
 __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t* __restrict__ sel,
+                                                          const float* __restrict__ scores,
                                                           int32_t* __restrict__ slot_table,
                                                           int32_t* __restrict__ last_used, int step,
                                                           int32_t* __restrict__ fetch_slot,
@@ -68,6 +76,7 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
     int32_t* s_vict = sp + 3 * K;
     int32_t* s_nst = sp + 4 * K;
     int32_t* s_nlu = sp + 5 * K;
+    uint32_t* s_ord = reinterpret_cast<uint32_t*>(sp + 6 * K);
     __shared__ int tmp[32];
 
     const int i = threadIdx.x;
@@ -82,6 +91,10 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
         s_st[i] = st;
         s_lu[i] = last_used[base + i];
         s_prot[i] = 0;
+        if constexpr (kScored)
+            s_ord[i] = st >= 0 ? ordered_key(scores[static_cast<long long>(blockIdx.x) * N + st]) : 0u;
+        else
+            s_ord[i] = static_cast<uint32_t>(s_lu[i]) ^ 0x80000000u;   // signed order
         sv = sel[base + i];
         if (sv < -1 || sv >= N) {
             raise_dev_error(OASIS_DEVERR_ID_RANGE);
@@ -110,10 +123,10 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
         s_nst[i] = s_st[i];
         s_nlu[i] = prot ? step : s_lu[i];
         if (!prot) {
-            const unsigned long long mine = victim_key(i, s_st[i], s_lu[i]);
+            const unsigned long long mine = victim_key(i, s_st[i], s_ord[i]);
             int rank = 0;
             for (int j = 0; j < K; ++j)
-                if (!s_prot[j] && victim_key(j, s_st[j], s_lu[j]) < mine) ++rank;
+                if (!s_prot[j] && victim_key(j, s_st[j], s_ord[j]) < mine) ++rank;
             if (rank < nF) s_vict[rank] = i;
         }
     }

@@ -23,6 +23,11 @@ of E_t the lookahead selection of step t-1, the previous step's exact set and
 the resident slots hold, and - with ``exact="correct"`` - plans and gathers
 the missing blocks of E_t with no cap, in stream order before the attention.
 
+Victim order: LRU (OasisKV Table 2) or, with ``victims="score"``, the stale
+block with the lowest current lookahead score first; the scores of each
+layer then go to a buffer of its own so the plan on the main stream can
+read them while the score stream moves on to the next layer.
+
 Memory: the full KV of every layer lives in pinned host memory; HBM holds per
 layer the per-block summaries (N x 512 B per KV head), the fixed pool of K
 slots (8 KiB each) and a few small int tables.  One workspace serves all
@@ -34,8 +39,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (append_kv, block_overlap, build_summaries, make_dims, plan_fetch, prefetch, score_select,
-               score_select_rows, sparse_attn, workspace_bytes)
+from . import (append_kv, block_overlap, build_summaries, lookahead_scores, make_dims, plan_fetch,
+               plan_fetch_scored, prefetch, score_select, score_select_rows, select_topk, sparse_attn,
+               workspace_bytes)
 
 HEAD_DIM, BLOCK_TOKENS = 128, 16
 
@@ -65,6 +71,7 @@ class LayerState:
         self.plan_ready = torch.cuda.Event()
         self.fetch_done = torch.cuda.Event()
         self.hist = None
+        self.scores = None
 
     def enable_exact(self, steps_cap: int, device="cuda"):
         """Buffers of the exact-set mode: two exact sets (this step's and the
@@ -94,10 +101,17 @@ class DecodePipeline:
     """Drives priming and decode steps over a list of layers."""
 
     def __init__(self, d, layers, ctx_len: torch.Tensor, scale: float, device="cuda",
-                 overlap_score: bool = True, exact: str | None = None, steps_cap: int = 256):
-        assert exact in (None, "measure", "correct")
+                 overlap_score: bool = True, exact: str | None = None, steps_cap: int = 256,
+                 victims: str = "lru"):
+        assert exact in (None, "measure", "correct") and victims in ("lru", "score")
         self.d, self.layers, self.scale = d, layers, scale
         self.exact = exact
+        self.victims = victims
+        if victims == "score":
+            for L in layers:
+                if L.scores is None:
+                    L.scores = torch.empty((d.batch, d.n_kv_heads, d.max_blocks), dtype=torch.float32,
+                                           device=device)
         self.steps_cap = steps_cap
         if exact is not None:
             # uncapped plan / gather for the corrective fetch; a workspace of its own
@@ -136,13 +150,22 @@ class DecodePipeline:
             if self.exact is not None and step > 0:
                 self.score_stream.wait_event(L.sel_read)   # so has the agreement count
         self._t("begin", "score_select", self.score_stream)
-        score_select(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, self.ws, stream=self.score_stream)
+        if self.victims == "score":
+            lookahead_scores(d, q, L.kmin, L.kmax, ctx, L.scores, stream=self.score_stream)
+            select_topk(d, L.scores, ctx, L.sel, L.sel_score, stream=self.score_stream)
+        else:
+            score_select(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, self.ws, stream=self.score_stream)
         self._t("end", "score_select", self.score_stream)
         if self.score_stream is not main:
             self.sel_ready[i].record(self.score_stream)
             main.wait_event(self.sel_ready[i])
         self._t("begin", "plan_fetch", main)
-        plan_fetch(d, L.sel, L.slot_table, L.last_used, step, L.fetch_slot, L.fetch_block, L.n_fetch, stream=main)
+        if self.victims == "score":
+            plan_fetch_scored(d, L.sel, L.scores, L.slot_table, L.last_used, step, L.fetch_slot, L.fetch_block,
+                              L.n_fetch, stream=main)
+        else:
+            plan_fetch(d, L.sel, L.slot_table, L.last_used, step, L.fetch_slot, L.fetch_block, L.n_fetch,
+                       stream=main)
         self._t("end", "plan_fetch", main)
         L.plan_ready.record(main)
         self.copy_stream.wait_event(L.plan_ready)
