@@ -50,7 +50,7 @@ Readings taken where the pages are silent (each also listed in the design doc):
 * R5 attention reads every occupied slot (the resident blocks), masking
   tokens at or beyond ``ctx_len``; all ``Qn`` rows see the same token set.
 * R6 empty token set: output 0, log-sum-exp -inf.
-* R7 exact set and corrective fetch ([OasisKV] Figure 6 and "What they did":
+* R16 exact set and corrective fetch ([OasisKV] Figure 6 and "What they did":
   prediction misses need corrective fetches).  At decode step t the exact
   set E_t is the top-K under the same scorer with the verification row
   (row 0, the true query of step t) alone.  Agreement of a predicted set S
@@ -59,7 +59,7 @@ Readings taken where the pages are silent (each also listed in the design doc):
   prediction is E_{t-1}.  A corrective fetch brings every block of E_t that
   is not resident before step t's attention, with the same planner and no
   cap (C = K), as a use at step t.
-* R8 score-based victims (the alternative to Table 2's LRU in the eviction
+* R17 score-based victims (the alternative to Table 2's LRU in the eviction
   ablation): stale slots are taken in order of their block's current
   lookahead score, lowest first, ties to the lower block id (-0.0 == +0.0);
   free slots still come first and a selected block is never evicted.
@@ -178,7 +178,7 @@ def lookahead_scores(q, kmin, kmax, ctx_len, block_tokens, rows=None):
 
     q: float64 [B, Qn, Hq, D]; kmin/kmax float64 [B, Hkv, N, D].
     rows: the query rows scored (default: the drafts 1..Qn-1, or row 0 when
-    Qn == 1); [0] scores with the verification query alone (R7).
+    Qn == 1); [0] scores with the verification query alone (R16).
     Returns float32 [B, Hkv, N]; blocks at or beyond n_valid are -inf.
     """
     B, Qn, Hq, D = q.shape
@@ -249,7 +249,7 @@ def plan_fetch(sel, slot_table, last_used, step, fetch_cap, scores=None):
       3. victims: free slots ascending, then slots whose block is not in S*
          by (last_used, block id) ascending (R4) - or, when ``scores``
          (float32 [B, Hkv, N], this step's lookahead scores) is given, by
-         (score of the block, block id) ascending (R8);
+         (score of the block, block id) ascending (R17);
       4. F[i] goes to victims[i], which is stamped last_used = step.
 
     Inputs are not modified.  Returns a dict with the new slot_table and
@@ -387,7 +387,7 @@ def dense_attention(q, keys, values, ctx_len, scale):
     return o, lse
 
 
-# ------------------------------------- prediction quality (R7): set overlap
+# ------------------------------------ prediction quality (R16): set overlap
 def block_overlap(a, b):
     """Per (sequence, KV head): how many distinct block ids of list ``b`` also
     occur in list ``a`` (-1 entries are empty).  a, b: int [B, Hkv, *]."""
@@ -421,7 +421,7 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
     With ``corrective`` each decode step first finds the exact set E_t from
     the verification row, records the agreement counts of the lookahead and
     previous-token predictions and the resident coverage of E_t, and fetches
-    E_t's missing blocks without a cap before the attention (R7).
+    E_t's missing blocks without a cap before the attention (R16).
     """
     B, H, N, P, D = keys.shape
     K = budget_blocks

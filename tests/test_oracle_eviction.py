@@ -20,7 +20,7 @@ def _state():
 def test_hand_worked_lru_vs_score_victims():
     """Worked by hand: the free slot 3 goes first; the second victim is the
     least recently used stale slot (slot 2, last used at 2) under LRU, but the
-    lowest-scored stale block (block 10 in slot 0, score -5) under R8."""
+    lowest-scored stale block (block 10 in slot 0, score -5) under R17."""
     st, lu, sel, scores = _state()
     lru = O.plan_fetch(sel, st, lu, 5, 2)
     assert lru["fetch_slot"][0, 0].tolist() == [3, 2]
