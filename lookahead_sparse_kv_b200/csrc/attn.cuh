@@ -57,11 +57,22 @@ __host__ __device__ __forceinline__ void attn_unit_streams(long long u, long lon
     *last = ((u + 1) * K - 1) * NS / T;
 }
 
+// floor(x / t) for x < 2^53, t < 2^31 without the 64-bit integer division
+// routine: a double quotient, then an exact integer correction.
+__device__ __forceinline__ long long floor_div_small(long long x, long long t) {
+    long long q = static_cast<long long>(static_cast<double>(x) / static_cast<double>(t));
+    if (q * t > x) --q;
+    else if ((q + 1) * t <= x) ++q;
+    return q;
+}
+
 // Merges the stream partials of each (unit, query row) in stream order:
 // lse = log sum_p exp(lse_p), out = sum_p exp(lse_p - lse) * o_p.  One warp
 // per (unit, row); lane j holds partial j's lse, lane c owns channels
-// 4c..4c+3 and keeps up to 8 partial loads in flight.
-constexpr int kMergeWarps = 4;
+// 4c..4c+3.  Up to 16 partials (the usual case) are read in one round trip:
+// every lse and output load is issued before any of them is used.
+constexpr int kMergeWarps = 2;                   // small CTAs: the whole grid fits in one wave
+constexpr int kMergeFast = 16;
 
 __global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, int n_streams,
                                                                       const float* __restrict__ ws_o,
@@ -72,54 +83,78 @@ __global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, in
     const int lane = threadIdx.x & 31;
     const int G = d.G();
     const int rows = d.Qn * G;
-    const long long units = static_cast<long long>(d.B) * d.Hkv;
-    const long long gw = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
+    const int units = d.B * d.Hkv;
+    const int gw = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);   // < units * rows <= 2^22
     // partials are produced by the attention grid this kernel depends on
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (gw >= units * rows) return;
-    const long long u = gw / rows;
-    const int r = static_cast<int>(gw % rows);
-    const long long T = units * d.K;
-    long long first, last;
-    attn_unit_streams(u, d.K, n_streams, T, &first, &last);
+    const int u = gw / rows;
+    const int r = gw - u * rows;
+    // streams whose ranges touch unit u (attn_unit_streams): slot s is in stream floor(s*NS/T)
+    const long long T = static_cast<long long>(units) * d.K;
+    const long long first = floor_div_small(static_cast<long long>(u) * d.K * n_streams, T);
+    const long long last = floor_div_small((static_cast<long long>(u + 1) * d.K - 1) * n_streams, T);
     const int np = static_cast<int>(last - first + 1);
     const long long p0 = first + u;
-    float M = kNegInf;
-    for (int j0 = 0; j0 < np; j0 += 32) {
-        const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;
-        M = fmaxf(M, lj);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     const float4* src = reinterpret_cast<const float4*>(ws_o + (p0 * rows + r) * kHeadDim) + lane;
     const long long pstride = static_cast<long long>(rows) * (kHeadDim / 4);
-    if (M != kNegInf) {
+    float M = kNegInf, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (np <= kMergeFast) {
+        const float lj = lane < np ? ws_lse[(p0 + lane) * rows + r] : kNegInf;
+        float4 v[kMergeFast];
+#pragma unroll
+        for (int k = 0; k < kMergeFast; ++k) v[k] = k < np ? src[k * pstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+        M = lj;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+        const float wj = (lj == kNegInf) ? 0.f : __expf(lj - M);
+        L = wj;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+#pragma unroll
+        for (int k = 0; k < kMergeFast; ++k) {
+            const float w = __shfl_sync(0xFFFFFFFFu, wj, k);
+            if (w > 0.f) {                      // empty partials may hold stale outputs
+                acc.x += w * v[k].x;
+                acc.y += w * v[k].y;
+                acc.z += w * v[k].z;
+                acc.w += w * v[k].w;
+            }
+        }
+    } else {
         for (int j0 = 0; j0 < np; j0 += 32) {
             const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;
-            const float wj = lj == kNegInf ? 0.f : __expf(lj - M);
-            float ws = wj;
+            M = fmaxf(M, lj);
+        }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xFFFFFFFFu, ws, o);
-            L += ws;
-            const int nj = min(32, np - j0);
-            for (int k0 = 0; k0 < nj; k0 += 8) {
-                float4 v[8];
-                float wk[8];
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+        if (M != kNegInf) {
+            for (int j0 = 0; j0 < np; j0 += 32) {
+                const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;
+                const float wj = lj == kNegInf ? 0.f : __expf(lj - M);
+                float ws = wj;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    wk[k] = __shfl_sync(0xFFFFFFFFu, wj, (k0 + k) & 31);
-                    v[k] = (k0 + k < nj && wk[k] > 0.f) ? src[(j0 + k0 + k) * pstride]
-                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
+                for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xFFFFFFFFu, ws, o);
+                L += ws;
+                const int nj = min(32, np - j0);
+                for (int k0 = 0; k0 < nj; k0 += 8) {
+                    float4 v[8];
+                    float wk[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float w = k0 + k < nj ? wk[k] : 0.f;
-                    acc.x += w * v[k].x;
-                    acc.y += w * v[k].y;
-                    acc.z += w * v[k].z;
-                    acc.w += w * v[k].w;
+                    for (int k = 0; k < 8; ++k) {
+                        wk[k] = __shfl_sync(0xFFFFFFFFu, wj, (k0 + k) & 31);
+                        v[k] = (k0 + k < nj && wk[k] > 0.f) ? src[(j0 + k0 + k) * pstride]
+                                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float w = k0 + k < nj ? wk[k] : 0.f;
+                        acc.x += w * v[k].x;
+                        acc.y += w * v[k].y;
+                        acc.z += w * v[k].z;
+                        acc.w += w * v[k].w;
+                    }
                 }
             }
         }
@@ -129,7 +164,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, in
     acc.y *= inv;
     acc.z *= inv;
     acc.w *= inv;
-    const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
+    const int b = u / d.Hkv, h = u - b * d.Hkv;
     const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
     reinterpret_cast<float4*>(out + orow * kHeadDim)[lane] = acc;
     if (lane == 0) lse_out[orow] = L > 0.f ? M + logf(L) : kNegInf;
