@@ -33,6 +33,14 @@ is the synthetic analog of OasisKV Table 2: the fetch cap as a fraction of
 the budget K (0.01 .. 0.2 and uncapped) with LRU and score-ordered victims;
 per setting the fetch volume, the H2D rate, layer-steps/s and how much of the
 exact top-K of the true query and of the lookahead selection is resident.
+
+    python bench.py --deep [--steps K]
+
+compares the eager stream pipeline with the same decode step captured once as
+a CUDA graph and replayed, on a 64-layer stack shaped like Qwen3-32B at 32K
+(64/8 heads, 1+7 queries), at batch 16 (transfer-bound) and batch 2 (launch-
+bound).  Host KV is shared by layers l and l+8 (8 distinct layers, as the
+host-memory fallback allows); queries differ per layer.
 """
 
 from __future__ import annotations
@@ -485,6 +493,89 @@ def run_ablation(args, device):
     print(json.dumps(line), flush=True)
 
 
+def run_deep(args, device):
+    """Eager vs graph-replayed decode steps of a 64-layer stack."""
+    base = W.WORKLOADS["qwen32b_32k"]
+    nl, distinct, ring = 64, 8, 16
+    steps = min(args.steps, 48)
+    rows = []
+    for batch in (16, 2):
+        w = base.with_(batch=batch, evict_prob=0.0)
+        d = lsk.dims_for(w)
+        hosts = []
+        for l in range(distinct):
+            h = torch.empty((w.batch, w.n_kv_heads, w.max_blocks, 2, w.block_tokens, w.head_dim),
+                            dtype=torch.bfloat16, pin_memory=True)
+            W.make_host_kv(w, layer=l, device=device, out=h)
+            hosts.append(h)
+        layers = [LayerState(d, hosts[l % distinct], device) for l in range(nl)]
+        # queries of all layers for one step in one tensor, so a step costs one copy
+        streams = [W.QueryStream(w, l, device) for l in range(nl)]
+        qring = [torch.stack([qs.next() for qs in streams]) for _ in range(ring)]     # [ring][layers, B, Qn, Hq, D]
+        q_all = torch.empty_like(qring[0])
+        q_static = list(q_all)
+        ctx = W.initial_ctx_len(w, device)
+        torch.cuda.synchronize()
+        built = False
+        for mode in ("eager", "graph"):
+            for L in layers:
+                L.slot_table.fill_(-1)
+                L.last_used.fill_(-1)
+            pipe = DecodePipeline(d, layers, ctx, 1.0 / math.sqrt(w.head_dim), device, device_step=(mode == "graph"))
+            with torch.cuda.stream(pipe.main):
+                if not built:
+                    pipe.build_summaries()
+                    built = True
+                pipe.prime(list(qring[0]))
+            t = 1
+
+            def load_queries(t):
+                with torch.cuda.stream(pipe.main):
+                    q_all.copy_(qring[ring_index(t, ring)], non_blocking=True)
+
+            for _ in range(4):                         # warm-up, eager in both modes
+                load_queries(t)
+                with torch.cuda.stream(pipe.main):
+                    pipe.step(t, q_static)
+                t += 1
+            with torch.cuda.stream(pipe.main):
+                pipe.wait_all()
+            torch.cuda.synchronize()
+            if mode == "graph":
+                pipe.capture(q_static)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            h0 = time.perf_counter()
+            e0.record(pipe.main)
+            for _ in range(steps):
+                load_queries(t)
+                if mode == "graph":
+                    pipe.replay()
+                else:
+                    with torch.cuda.stream(pipe.main):
+                        pipe.step(t, q_static)
+                t += 1
+            with torch.cuda.stream(pipe.main):
+                pipe.wait_all()
+            e1.record(pipe.main)
+            host_ms = (time.perf_counter() - h0) * 1e3
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            rows.append({"batch": batch, "mode": mode, "layer_steps_per_s": nl * steps / (ms * 1e-3),
+                         "ms_per_step": ms / steps, "host_enqueue_ms_per_step": host_ms / steps,
+                         "gpu_launches_per_step": 1 if mode == "graph" else None})
+            del pipe
+        del layers, hosts, qring, q_all, q_static
+        torch.cuda.empty_cache()
+    line = {
+        "metric": "decode step of a 64-layer stack: eager stream pipeline vs one CUDA graph replay per step",
+        "workload": f"qwen32b_32k shape: {nl} layers (host KV of 8 distinct layers, l -> l mod 8), 64/8 heads, "
+                    f"32K context, budget 128 blocks, cap 16, 1+7 queries; batch 16 and 2; "
+                    f"every step copies all layers' queries into fixed buffers (one copy) in both modes",
+        "steps": steps, "rows": rows, "device_error_word": lsk.read_device_error(clear=True),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_gpu(args, rank, world, device):
     w = rank_workload(rank)
     st = build_workload_state(w, args.warmup + args.steps, device, n_queries=args.query_ring,
@@ -800,6 +891,8 @@ def main():
                     help="measure prediction agreement and the corrective fetch instead")
     ap.add_argument("--ablation", action="store_true",
                     help="fetch-cap x victim-order sweep (Table 2 analog) instead")
+    ap.add_argument("--deep", action="store_true",
+                    help="64-layer stack, eager vs CUDA-graph replay, instead")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -814,9 +907,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if args.prediction or args.ablation:
+    if args.prediction or args.ablation or args.deep:
         if rank == 0:
-            (run_prediction if args.prediction else run_ablation)(args, device)
+            (run_prediction if args.prediction else run_ablation if args.ablation else run_deep)(args, device)
         return
     if world > 1:
         import datetime

@@ -213,6 +213,21 @@ int oasis_plan_fetch_scored(const oasis_dims* d, const int32_t* sel, const float
                             int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
                             void* stream);
 
+/* a4 with the step number in device memory (a7 graph capture: the planner is
+ * the only call of a decode step that takes a per-step scalar, so a captured
+ * multi-layer step reads it from here and replays unchanged).  As
+ * oasis_plan_fetch (scores == NULL) or oasis_plan_fetch_scored (scores
+ * given), with step = *step read on the device when the kernel runs.
+ * step: device int32, 16-byte aligned. */
+int oasis_plan_fetch_at(const oasis_dims* d, const int32_t* sel, const float* scores,
+                        int32_t* slot_table, int32_t* last_used, const int32_t* step,
+                        int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
+                        void* stream);
+
+/* *step += 1 on the device (one thread), stream-ordered: the first call of a
+ * captured decode step. */
+int oasis_step_advance(int32_t* step, void* stream);
+
 /* a5 - host-to-HBM gather (OasisKV Figure 7: blocks "are prefetched from the
  * CPU cache"; Figure 8).  For i < n_fetch[b][h], copies the 8 KiB block
  * host_kv[b][h][fetch_block[b][h][i]] into pool[b][h][fetch_slot[b][h][i]]

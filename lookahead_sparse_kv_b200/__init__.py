@@ -74,6 +74,8 @@ _SIGS = {
     "oasis_block_overlap": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V]),
     "oasis_plan_fetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _I32, _V, _V, _V, _V]),
     "oasis_plan_fetch_scored": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _I32, _V, _V, _V, _V]),
+    "oasis_plan_fetch_at": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V, _V, _V]),
+    "oasis_step_advance": (ctypes.c_int, [_V, _V]),
     "oasis_prefetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V]),
     "oasis_sparse_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, ctypes.c_float,
                                          _V, _V, _V, ctypes.c_size_t, _V]),
@@ -203,6 +205,19 @@ def plan_fetch_scored(d, sel, scores, slot_table, last_used, step, fetch_slot, f
     _check(lib().oasis_plan_fetch_scored(ctypes.byref(d), _p(sel), _p(scores), _p(slot_table), _p(last_used),
                                          int(step), _p(fetch_slot), _p(fetch_block), _p(n_fetch),
                                          _stream(stream)), "oasis_plan_fetch_scored")
+
+
+def plan_fetch_at(d, sel, scores, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream=None):
+    """Plan with the step number read on the device from ``step`` (int32
+    tensor); LRU victims when ``scores`` is None, score-ordered otherwise."""
+    _check(lib().oasis_plan_fetch_at(ctypes.byref(d), _p(sel), _p(scores), _p(slot_table), _p(last_used), _p(step),
+                                     _p(fetch_slot), _p(fetch_block), _p(n_fetch), _stream(stream)),
+           "oasis_plan_fetch_at")
+
+
+def step_advance(step, stream=None):
+    """step[0] += 1 on the device, in stream order."""
+    _check(lib().oasis_step_advance(_p(step), _stream(stream)), "oasis_step_advance")
 
 
 def prefetch(d, host_kv, fetch_slot, fetch_block, n_fetch, pool, stream=None):

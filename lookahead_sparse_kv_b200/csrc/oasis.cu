@@ -296,9 +296,11 @@ int scores_rows(const oasis_dims* dp, const void* q, int row_begin, int row_coun
     return launch_score<64>(tmax, tmin, d, qq, ctx_len, scores, row_begin, rows, s);
 }
 
-// Residency diff + capped fetch plan; LRU victims, or by score if scores != NULL.
+// Residency diff + capped fetch plan; LRU victims, or by score if scores != NULL;
+// the step from step_dev (device) if that is not NULL.
 int plan(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t* slot_table, int32_t* last_used,
-         int32_t step, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch, void* stream) {
+         int32_t step, const int32_t* step_dev, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
+         void* stream) {
     Dims d;
     if (int rc = validate(dp, &d)) return rc;
     if (int rc = check_ptr(sel, "sel")) return rc;
@@ -313,11 +315,11 @@ int plan(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t*
     const int smem = 7 * d.K * static_cast<int>(sizeof(int32_t));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (scores != nullptr)
-        oasis::plan_fetch_kernel<true><<<d.B * d.Hkv, threads, smem, s>>>(d, sel, scores, slot_table, last_used,
-                                                                         step, fetch_slot, fetch_block, n_fetch);
+        oasis::plan_fetch_kernel<true><<<d.B * d.Hkv, threads, smem, s>>>(
+            d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
     else
-        oasis::plan_fetch_kernel<false><<<d.B * d.Hkv, threads, smem, s>>>(d, sel, scores, slot_table, last_used,
-                                                                          step, fetch_slot, fetch_block, n_fetch);
+        oasis::plan_fetch_kernel<false><<<d.B * d.Hkv, threads, smem, s>>>(
+            d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
     return check_launch("plan_fetch launch");
 }
 
@@ -449,14 +451,28 @@ int oasis_block_overlap(const oasis_dims* dp, const int32_t* a, const int32_t* b
 
 int oasis_plan_fetch(const oasis_dims* dp, const int32_t* sel, int32_t* slot_table, int32_t* last_used,
                      int32_t step, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch, void* stream) {
-    return plan(dp, sel, nullptr, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream);
+    return plan(dp, sel, nullptr, slot_table, last_used, step, nullptr, fetch_slot, fetch_block, n_fetch, stream);
 }
 
 int oasis_plan_fetch_scored(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t* slot_table,
                             int32_t* last_used, int32_t step, int32_t* fetch_slot, int32_t* fetch_block,
                             int32_t* n_fetch, void* stream) {
     if (int rc = check_ptr(scores, "scores")) return rc;
-    return plan(dp, sel, scores, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream);
+    return plan(dp, sel, scores, slot_table, last_used, step, nullptr, fetch_slot, fetch_block, n_fetch, stream);
+}
+
+int oasis_plan_fetch_at(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t* slot_table,
+                        int32_t* last_used, const int32_t* step, int32_t* fetch_slot, int32_t* fetch_block,
+                        int32_t* n_fetch, void* stream) {
+    if (int rc = check_ptr(step, "step")) return rc;
+    if (int rc = check_ptr(scores, "scores", true)) return rc;
+    return plan(dp, sel, scores, slot_table, last_used, 0, step, fetch_slot, fetch_block, n_fetch, stream);
+}
+
+int oasis_step_advance(int32_t* step, void* stream) {
+    if (int rc = check_ptr(step, "step")) return rc;
+    oasis::step_advance_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(step);
+    return check_launch("step_advance launch");
 }
 
 int oasis_prefetch(const oasis_dims* dp, const void* host_kv, const int32_t* fetch_slot, const int32_t* fetch_block,

@@ -60,11 +60,14 @@ __device__ __forceinline__ unsigned long long victim_key(int slot, int blk, uint
 
 // blockDim.x = K rounded up to a multiple of 32; dynamic smem 7*K ints.
 // kScored: victims by the block's score (scores fp32 [B][Hkv][N]), else LRU.
+// step_dev (nullable): the step number is read from device memory instead of
+// `step`, so a captured graph can replay the plan at every step.
 template <bool kScored>
 __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t* __restrict__ sel,
                                                           const float* __restrict__ scores,
                                                           int32_t* __restrict__ slot_table,
                                                           int32_t* __restrict__ last_used, int step,
+                                                          const int32_t* __restrict__ step_dev,
                                                           int32_t* __restrict__ fetch_slot,
                                                           int32_t* __restrict__ fetch_block,
                                                           int32_t* __restrict__ n_fetch) {
@@ -81,6 +84,7 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
 
     const int i = threadIdx.x;
     const long long base = static_cast<long long>(blockIdx.x) * K;
+    if (step_dev != nullptr) step = *step_dev;
     int sv = -1;
     if (i < K) {
         int st = slot_table[base + i];
@@ -149,5 +153,8 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
     }
     if (i == 0) n_fetch[blockIdx.x] = nF;
 }
+
+// Advances a device-resident step counter by one (one thread).
+__global__ void step_advance_kernel(int32_t* step) { *step += 1; }
 
 }  // namespace oasis

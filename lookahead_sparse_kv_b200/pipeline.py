@@ -28,6 +28,16 @@ block with the lowest current lookahead score first; the scores of each
 layer then go to a buffer of its own so the plan on the main stream can
 read them while the score stream moves on to the next layer.
 
+Graph mode (``device_step=True``): the step number lives in device memory
+(advanced by a kernel at the start of each step, read by the planner), so a
+whole multi-layer decode step can be captured once as a CUDA graph
+(``capture``) and replayed (``replay``) with one launch per step.  Inside
+the graph the score stream forks from the main stream at each layer and all
+gathers join the main stream at the end, so a replay is self-contained; the
+price is that the last layers' gathers no longer overlap the next step's
+first layers, which matters little for deep stacks.  Appends and the
+exact-set stage take per-step host values and are not captured.
+
 Memory: the full KV of every layer lives in pinned host memory; HBM holds per
 layer the per-block summaries (N x 512 B per KV head), the fixed pool of K
 slots (8 KiB each) and a few small int tables.  One workspace serves all
@@ -40,8 +50,8 @@ from __future__ import annotations
 import torch
 
 from . import (append_kv, block_overlap, build_summaries, lookahead_scores, make_dims, plan_fetch,
-               plan_fetch_scored, prefetch, score_select, score_select_rows, select_topk, sparse_attn,
-               workspace_bytes)
+               plan_fetch_at, plan_fetch_scored, prefetch, score_select, score_select_rows, select_topk,
+               sparse_attn, step_advance, workspace_bytes)
 
 HEAD_DIM, BLOCK_TOKENS = 128, 16
 
@@ -102,9 +112,13 @@ class DecodePipeline:
 
     def __init__(self, d, layers, ctx_len: torch.Tensor, scale: float, device="cuda",
                  overlap_score: bool = True, exact: str | None = None, steps_cap: int = 256,
-                 victims: str = "lru"):
+                 victims: str = "lru", device_step: bool = False):
         assert exact in (None, "measure", "correct") and victims in ("lru", "score")
+        assert not (device_step and exact is not None), "the exact-set stage is not graph-capturable"
         self.d, self.layers, self.scale = d, layers, scale
+        self.step_dev = torch.zeros(4, dtype=torch.int32, device=device) if device_step else None
+        self.graph = None
+        self._step_host = 0
         self.exact = exact
         self.victims = victims
         if victims == "score":
@@ -124,11 +138,15 @@ class DecodePipeline:
         self.ctx = [ctx_len, ctx_len.clone()]           # ping-pong when tokens are appended
         self.cur = 0
         self.ws = torch.zeros(workspace_bytes(d), dtype=torch.uint8, device=device)
-        self.main = torch.cuda.current_stream(device)
+        # a stream of its own in graph mode: capture cannot start on the default stream
+        self.main = torch.cuda.Stream(device) if device_step else torch.cuda.current_stream(device)
+        if device_step:
+            self.main.wait_stream(torch.cuda.current_stream(device))
         self.score_stream = torch.cuda.Stream(device) if overlap_score else self.main
         lo, hi = torch.cuda.Stream.priority_range()
         self.copy_stream = torch.cuda.Stream(device, priority=hi)
         self.sel_ready = [torch.cuda.Event() for _ in layers]
+        self.fork = [torch.cuda.Event() for _ in layers]
         self.timer = None        # optional: begin(name, stream) / end(name, stream) around each call
 
     def _t(self, which, name, stream):
@@ -143,10 +161,25 @@ class DecodePipeline:
         for L in self.layers:
             build_summaries(self.d, L.host_kv, self.ctx_len, L.kmin, L.kmax, stream=self.main)
 
-    def _select_plan_fetch(self, i, L, q, step, ctx):
+    def _plan(self, d, sel, scores, L, step, fetch_slot, fetch_block, n_fetch):
+        if self.step_dev is not None:
+            plan_fetch_at(d, sel, scores, L.slot_table, L.last_used, self.step_dev, fetch_slot, fetch_block,
+                          n_fetch, stream=self.main)
+        elif scores is not None:
+            plan_fetch_scored(d, sel, scores, L.slot_table, L.last_used, step, fetch_slot, fetch_block, n_fetch,
+                              stream=self.main)
+        else:
+            plan_fetch(d, sel, L.slot_table, L.last_used, step, fetch_slot, fetch_block, n_fetch, stream=self.main)
+
+    def _select_plan_fetch(self, i, L, q, step, ctx, in_graph=False):
         d, main = self.d, self.main
         if self.score_stream is not main:
-            self.score_stream.wait_event(L.plan_ready)     # previous plan has read L.sel
+            if in_graph:
+                # fork from this replay's main stream; the previous plan ran in the previous replay
+                self.fork[i].record(main)
+                self.score_stream.wait_event(self.fork[i])
+            else:
+                self.score_stream.wait_event(L.plan_ready)     # previous plan has read L.sel
             if self.exact is not None and step > 0:
                 self.score_stream.wait_event(L.sel_read)   # so has the agreement count
         self._t("begin", "score_select", self.score_stream)
@@ -160,12 +193,8 @@ class DecodePipeline:
             self.sel_ready[i].record(self.score_stream)
             main.wait_event(self.sel_ready[i])
         self._t("begin", "plan_fetch", main)
-        if self.victims == "score":
-            plan_fetch_scored(d, L.sel, L.scores, L.slot_table, L.last_used, step, L.fetch_slot, L.fetch_block,
-                              L.n_fetch, stream=main)
-        else:
-            plan_fetch(d, L.sel, L.slot_table, L.last_used, step, L.fetch_slot, L.fetch_block, L.n_fetch,
-                       stream=main)
+        self._plan(d, L.sel, L.scores if self.victims == "score" else None, L, step, L.fetch_slot, L.fetch_block,
+                   L.n_fetch)
         self._t("end", "plan_fetch", main)
         L.plan_ready.record(main)
         self.copy_stream.wait_event(L.plan_ready)
@@ -189,8 +218,7 @@ class DecodePipeline:
         self._t("end", "exact_set", main)
         if self.exact == "correct":
             self._t("begin", "corrective", main)
-            plan_fetch(self.d_full, cur, L.slot_table, L.last_used, t, L.cfetch_slot, L.cfetch_block, h[3],
-                       stream=main)
+            self._plan(self.d_full, cur, None, L, t, L.cfetch_slot, L.cfetch_block, h[3])
             prefetch(self.d_full, L.host_kv, L.cfetch_slot, L.cfetch_block, h[3], L.pool, stream=main)
             self._t("end", "corrective", main)
 
@@ -215,13 +243,23 @@ class DecodePipeline:
         the token accepted at the previous step; it is written at position
         ctx_len[b] and the context is one token longer from this step on.
         """
+        assert self.graph is None, "a captured pipeline advances by replay()"
+        self._step_body(t, q_per_layer, appended, in_graph=False)
+
+    def _step_body(self, t, q_per_layer, appended, in_graph):
         d, main = self.d, self.main
+        if self.step_dev is not None:
+            if not in_graph:
+                assert t == self._step_host + 1, "device-step pipelines take consecutive steps"
+                self._step_host = t
+            step_advance(self.step_dev, stream=main)
         if appended is None:
             ctx_in = ctx = self.ctx_len
         else:
             ctx_in, ctx = self.ctx[self.cur], self.ctx[1 - self.cur]
         for i, (L, q) in enumerate(zip(self.layers, q_per_layer)):
-            main.wait_event(L.fetch_done)
+            if not in_graph:
+                main.wait_event(L.fetch_done)
             if appended is not None:
                 k_new, v_new = appended[i]
                 append_kv(d, k_new, v_new, ctx_in, ctx if i == 0 else None, L.host_kv, L.kmin, L.kmax,
@@ -235,10 +273,33 @@ class DecodePipeline:
             self._t("begin", "sparse_attn", main)
             sparse_attn(d, q, L.pool, L.slot_table, ctx, self.scale, L.out, L.lse, self.ws, stream=main)
             self._t("end", "sparse_attn", main)
-            self._select_plan_fetch(i, L, q, t, ctx)
+            self._select_plan_fetch(i, L, q, t, ctx, in_graph)
         if appended is not None:
             self.cur = 1 - self.cur
+        if in_graph:
+            for L in self.layers:                      # every gather joins before the step ends
+                main.wait_event(L.fetch_done)
+
+    def capture(self, q_static):
+        """Captures one decode step over fixed query buffers as a CUDA graph
+        (device-step pipelines only, after prime()); later steps run by
+        copying their queries into q_static and calling replay()."""
+        assert self.step_dev is not None and self.exact is None and self.timer is None
+        self.wait_all()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.main):
+            self._step_body(None, q_static, None, in_graph=True)
+        self.graph = g
+        # capture only records the work: the counter is where prime() left it
+
+    def replay(self):
+        """One decode step (step counter + every layer), as one graph launch on the main stream."""
+        with torch.cuda.stream(self.main):
+            self.graph.replay()
 
     def wait_all(self):
+        if self.graph is not None:      # a replay ends with every gather joined to the main stream
+            return
         for L in self.layers:
             self.main.wait_event(L.fetch_done)
