@@ -63,6 +63,11 @@ Readings taken where the pages are silent (each also listed in the design doc):
   ablation): stale slots are taken in order of their block's current
   lookahead score, lowest first, ties to the lower block id (-0.0 == +0.0);
   free slots still come first and a selected block is never evicted.
+* R19 residency loss (the 32K Qwen3-32B configuration: a seeded share of
+  the attended KV misses residency each step): at decode step t, after the
+  layer's attention and before its selection / plan, every slot the step's
+  mask marks is freed (slot -> -1); a lost block that is selected again is
+  a miss and is fetched again.
 """
 
 from __future__ import annotations
@@ -84,6 +89,7 @@ __all__ = [
     "sparse_attention",
     "dense_attention",
     "block_overlap",
+    "evict_slots",
     "decode_layer_steps",
 ]
 
@@ -401,9 +407,18 @@ def block_overlap(a, b):
     return out
 
 
+# ---------------------------------------------- residency loss (R19)
+def evict_slots(slot_table, mask):
+    """Frees every slot whose mask entry is set (R19).  Returns a new table."""
+    st = slot_table.copy()
+    st[np.asarray(mask, dtype=bool)] = -1
+    return st
+
+
 # ------------------------------------------------ a7: per-step order
 def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
-                       budget_blocks, fetch_cap, scale, host_kv_bits=None, corrective=False):
+                       budget_blocks, fetch_cap, scale, host_kv_bits=None, corrective=False,
+                       evict_masks=None):
     """One layer through priming and T decode steps, in the pages' order.
 
     [OasisKV] Figure 8: at step t the draft queries drive top-K prediction,
@@ -422,6 +437,8 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
     the verification row, records the agreement counts of the lookahead and
     previous-token predictions and the resident coverage of E_t, and fetches
     E_t's missing blocks without a cap before the attention (R16).
+    ``evict_masks[t-1]`` (bool [B, Hkv, K]), when given, frees slots after the
+    attention of decode step t and before its plan (R19).
     """
     B, H, N, P, D = keys.shape
     K = budget_blocks
@@ -464,6 +481,8 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
             exact_prev = corr["exact"]
         o, lse = sparse_attention(qs, pool_k, pool_v, st, ctx_len, scale)
         slot_table_used = st.copy()
+        if evict_masks is not None:
+            st = evict_slots(st, evict_masks[t - 1])
         sc, sel, sel_score, plan = select_plan_fetch(qs, t)
         sel_prev = sel
         records.append({"o": o, "lse": lse, "slot_table_attn": slot_table_used,

@@ -76,3 +76,42 @@ def test_score_victims_keep_the_planner_invariants(seed):
             for s in range(K):
                 if st[b, h, s] in chosen:
                     assert p["slot_table"][b, h, s] == st[b, h, s]
+
+
+def test_residency_loss_frees_slots_and_forces_refetch():
+    """R19: a lost slot is free at the next plan; its block, if selected
+    again, is a miss and lands in a free slot (free slots come first)."""
+    st = np.array([[[10, 11, 12, 13]]], dtype=np.int32)
+    lu = np.array([[[4, 4, 4, 4]]], dtype=np.int32)
+    mask = np.array([[[False, True, False, True]]])
+    st2 = O.evict_slots(st, mask)
+    assert st2[0, 0].tolist() == [10, -1, 12, -1]
+    assert st[0, 0].tolist() == [10, 11, 12, 13]                 # input untouched
+    sel = np.array([[[11, 10, 12, 13]]], dtype=np.int32)
+    p = O.plan_fetch(sel, st2, lu, 5, 4)
+    assert p["n_fetch"][0, 0] == 2
+    assert p["fetch_block"][0, 0, :2].tolist() == [11, 13]       # rank order
+    assert p["fetch_slot"][0, 0, :2].tolist() == [1, 3]          # the freed slots, ascending
+
+
+def test_decode_with_residency_loss_refetches_what_was_lost():
+    """Over a few decode steps with a loss mask, the fetch count is at least the
+    number of lost blocks the next selection wants back (up to the cap)."""
+    r = np.random.default_rng(9)
+    B, Qn, Hq, H, N, P, D, K = 1, 3, 4, 2, 20, 16, 8, 6
+    keys = r.standard_normal((B, H, N, P, D)).astype(np.float32).astype(np.float64)
+    vals = r.standard_normal((B, H, N, P, D))
+    ctx = np.array([N * P])
+    kmin, kmax = O.block_summaries(keys, ctx)
+    qp = r.standard_normal((B, Qn, Hq, D))
+    qsteps = [qp + 0.01 * r.standard_normal((B, Qn, Hq, D)) for _ in range(4)]   # nearly the same selection
+    masks = [r.random((B, H, K)) < 0.5 for _ in range(4)]
+    recs, _, _ = O.decode_layer_steps(keys, vals, kmin, kmax, ctx, qp, qsteps, budget_blocks=K, fetch_cap=K,
+                                      scale=0.3, evict_masks=masks)
+    for t, rec in enumerate(recs):
+        before = O.evict_slots(rec["slot_table_attn"], masks[t])
+        lost = set(rec["slot_table_attn"][0, 0][masks[t][0, 0]].tolist()) - {-1}
+        wanted_back = lost & set(rec["sel"][0, 0].tolist())
+        assert rec["plan"]["n_fetch"][0, 0] >= len(wanted_back)
+        assert set(rec["plan"]["fetch_block"][0, 0].tolist()) >= wanted_back
+        assert (before[0, 0][masks[t][0, 0]] == -1).all()
