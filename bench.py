@@ -500,7 +500,7 @@ def run_deep(args, device):
     steps = min(args.steps, 48)
     rows = []
     for batch in (16, 2):
-        w = base.with_(batch=batch, evict_prob=0.0)
+        w = base.with_(batch=batch)
         d = lsk.dims_for(w)
         hosts = []
         for l in range(distinct):
@@ -514,6 +514,11 @@ def run_deep(args, device):
         qring = [torch.stack([qs.next() for qs in streams]) for _ in range(ring)]     # [ring][layers, B, Qn, Hq, D]
         q_all = torch.empty_like(qring[0])
         q_static = list(q_all)
+        # the configuration's seeded residency loss, one mask per layer and step (ring like the queries)
+        mring = [torch.stack([W.eviction_mask(w, l, r, device) for l in range(nl)]).to(torch.uint8)
+                 for r in range(ring)]
+        m_all = torch.empty_like(mring[0])
+        m_static = list(m_all)
         ctx = W.initial_ctx_len(w, device)
         torch.cuda.synchronize()
         built = False
@@ -532,17 +537,18 @@ def run_deep(args, device):
             def load_queries(t):
                 with torch.cuda.stream(pipe.main):
                     q_all.copy_(qring[ring_index(t, ring)], non_blocking=True)
+                    m_all.copy_(mring[ring_index(t, ring)], non_blocking=True)
 
             for _ in range(4):                         # warm-up, eager in both modes
                 load_queries(t)
                 with torch.cuda.stream(pipe.main):
-                    pipe.step(t, q_static)
+                    pipe.step(t, q_static, evict=m_static)
                 t += 1
             with torch.cuda.stream(pipe.main):
                 pipe.wait_all()
             torch.cuda.synchronize()
             if mode == "graph":
-                pipe.capture(q_static)
+                pipe.capture(q_static, evict_static=m_static)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             h0 = time.perf_counter()
             e0.record(pipe.main)
@@ -552,7 +558,7 @@ def run_deep(args, device):
                     pipe.replay()
                 else:
                     with torch.cuda.stream(pipe.main):
-                        pipe.step(t, q_static)
+                        pipe.step(t, q_static, evict=m_static)
                 t += 1
             with torch.cuda.stream(pipe.main):
                 pipe.wait_all()
@@ -564,13 +570,14 @@ def run_deep(args, device):
                          "ms_per_step": ms / steps, "host_enqueue_ms_per_step": host_ms / steps,
                          "gpu_launches_per_step": 1 if mode == "graph" else None})
             del pipe
-        del layers, hosts, qring, q_all, q_static
+        del layers, hosts, qring, q_all, q_static, mring, m_all, m_static
         torch.cuda.empty_cache()
     line = {
         "metric": "decode step of a 64-layer stack: eager stream pipeline vs one CUDA graph replay per step",
         "workload": f"qwen32b_32k shape: {nl} layers (host KV of 8 distinct layers, l -> l mod 8), 64/8 heads, "
                     f"32K context, budget 128 blocks, cap 16, 1+7 queries; batch 16 and 2; "
-                    f"every step copies all layers' queries into fixed buffers (one copy) in both modes",
+                    f"seeded 10 % residency loss per step; every step copies all layers' queries and loss masks "
+                    f"into fixed buffers (one copy each) in both modes",
         "steps": steps, "rows": rows, "device_error_word": lsk.read_device_error(clear=True),
     }
     print(json.dumps(line), flush=True)

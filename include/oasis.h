@@ -224,6 +224,15 @@ int oasis_plan_fetch_at(const oasis_dims* d, const int32_t* sel, const float* sc
                         int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
                         void* stream);
 
+/* Residency loss (the 32K Qwen3-32B configuration: a seeded share of the
+ * attended KV misses residency each step; no counterpart in the method
+ * itself, it models blocks lost to memory pressure): slot_table[i] = -1
+ * wherever mask[i] != 0.  mask: device uint8 [B][Hkv][K]; slot_table:
+ * device int32 [B][Hkv][K], updated in place.  Call it after a layer's
+ * attention and before its plan, so a lost block that is selected again is
+ * fetched again. */
+int oasis_evict_slots(const oasis_dims* d, const uint8_t* mask, int32_t* slot_table, void* stream);
+
 /* *step += 1 on the device (one thread), stream-ordered: the first call of a
  * captured decode step. */
 int oasis_step_advance(int32_t* step, void* stream);

@@ -76,6 +76,7 @@ _SIGS = {
     "oasis_plan_fetch_scored": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _I32, _V, _V, _V, _V]),
     "oasis_plan_fetch_at": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V, _V, _V]),
     "oasis_step_advance": (ctypes.c_int, [_V, _V]),
+    "oasis_evict_slots": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V]),
     "oasis_prefetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V]),
     "oasis_sparse_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, ctypes.c_float,
                                          _V, _V, _V, ctypes.c_size_t, _V]),
@@ -213,6 +214,11 @@ def plan_fetch_at(d, sel, scores, slot_table, last_used, step, fetch_slot, fetch
     _check(lib().oasis_plan_fetch_at(ctypes.byref(d), _p(sel), _p(scores), _p(slot_table), _p(last_used), _p(step),
                                      _p(fetch_slot), _p(fetch_block), _p(n_fetch), _stream(stream)),
            "oasis_plan_fetch_at")
+
+
+def evict_slots(d, mask, slot_table, stream=None):
+    """Frees the slots whose mask byte (uint8 [B][Hkv][K]) is set."""
+    _check(lib().oasis_evict_slots(ctypes.byref(d), _p(mask), _p(slot_table), _stream(stream)), "oasis_evict_slots")
 
 
 def step_advance(step, stream=None):

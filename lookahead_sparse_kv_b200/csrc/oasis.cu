@@ -469,6 +469,17 @@ int oasis_plan_fetch_at(const oasis_dims* dp, const int32_t* sel, const float* s
     return plan(dp, sel, scores, slot_table, last_used, 0, step, fetch_slot, fetch_block, n_fetch, stream);
 }
 
+int oasis_evict_slots(const oasis_dims* dp, const uint8_t* mask, int32_t* slot_table, void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(mask, "mask")) return rc;
+    if (int rc = check_ptr(slot_table, "slot_table")) return rc;
+    const long long n = static_cast<long long>(d.B) * d.Hkv * d.K;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>((n + 255) / 256, 4 * 148));
+    oasis::evict_slots_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(n, mask, slot_table);
+    return check_launch("evict_slots launch");
+}
+
 int oasis_step_advance(int32_t* step, void* stream) {
     if (int rc = check_ptr(step, "step")) return rc;
     oasis::step_advance_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(step);

@@ -154,6 +154,13 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
     if (i == 0) n_fetch[blockIdx.x] = nF;
 }
 
+// Residency loss: frees every slot whose mask byte is set (n = B*Hkv*K).
+__global__ void evict_slots_kernel(long long n, const uint8_t* __restrict__ mask, int32_t* __restrict__ slot_table) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        if (mask[i]) slot_table[i] = -1;
+}
+
 // Advances a device-resident step counter by one (one thread).
 __global__ void step_advance_kernel(int32_t* step) { *step += 1; }
 

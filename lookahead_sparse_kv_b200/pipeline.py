@@ -49,7 +49,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (append_kv, block_overlap, build_summaries, lookahead_scores, make_dims, plan_fetch,
+from . import (append_kv, block_overlap, build_summaries, evict_slots, lookahead_scores, make_dims, plan_fetch,
                plan_fetch_at, plan_fetch_scored, prefetch, score_select, score_select_rows, select_topk,
                sparse_attn, step_advance, workspace_bytes)
 
@@ -236,17 +236,19 @@ class DecodePipeline:
             L.plan_ready.record(self.main)
             self._select_plan_fetch(i, L, q, 0, self.ctx_len)
 
-    def step(self, t, q_per_layer, appended=None):
-        """Decode step t >= 1: per layer [append] -> attention -> select/plan/fetch.
+    def step(self, t, q_per_layer, appended=None, evict=None):
+        """Decode step t >= 1: per layer [append] -> attention -> [loss] -> select/plan/fetch.
 
         appended: optional list of (k_new, v_new) per layer, bf16 [B, Hkv, D],
         the token accepted at the previous step; it is written at position
         ctx_len[b] and the context is one token longer from this step on.
+        evict: optional list of uint8 masks [B, Hkv, K] per layer; the marked
+        slots are freed after the layer's attention (residency loss).
         """
         assert self.graph is None, "a captured pipeline advances by replay()"
-        self._step_body(t, q_per_layer, appended, in_graph=False)
+        self._step_body(t, q_per_layer, appended, in_graph=False, evict=evict)
 
-    def _step_body(self, t, q_per_layer, appended, in_graph):
+    def _step_body(self, t, q_per_layer, appended, in_graph, evict=None):
         d, main = self.d, self.main
         if self.step_dev is not None:
             if not in_graph:
@@ -273,6 +275,8 @@ class DecodePipeline:
             self._t("begin", "sparse_attn", main)
             sparse_attn(d, q, L.pool, L.slot_table, ctx, self.scale, L.out, L.lse, self.ws, stream=main)
             self._t("end", "sparse_attn", main)
+            if evict is not None:
+                evict_slots(d, evict[i], L.slot_table, stream=main)
             self._select_plan_fetch(i, L, q, t, ctx, in_graph)
         if appended is not None:
             self.cur = 1 - self.cur
@@ -280,16 +284,17 @@ class DecodePipeline:
             for L in self.layers:                      # every gather joins before the step ends
                 main.wait_event(L.fetch_done)
 
-    def capture(self, q_static):
-        """Captures one decode step over fixed query buffers as a CUDA graph
-        (device-step pipelines only, after prime()); later steps run by
-        copying their queries into q_static and calling replay()."""
+    def capture(self, q_static, evict_static=None):
+        """Captures one decode step over fixed query (and, optionally, loss
+        mask) buffers as a CUDA graph (device-step pipelines only, after
+        prime()); later steps run by copying their inputs into those buffers
+        and calling replay()."""
         assert self.step_dev is not None and self.exact is None and self.timer is None
         self.wait_all()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=self.main):
-            self._step_body(None, q_static, None, in_graph=True)
+            self._step_body(None, q_static, None, in_graph=True, evict=evict_static)
         self.graph = g
         # capture only records the work: the counter is where prime() left it
 

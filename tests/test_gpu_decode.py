@@ -189,12 +189,15 @@ def test_multilayer_append_decode():
             check_select_plan(l, qs[l], t)
 
 
-def test_full_size_llama_layer_sampled():
-    """The benchmarked 32K Llama-3.1-8B-shaped layer (B=16, 32/8 heads,
-    2,048 blocks, budget 128, cap 16) in the bench's launch configuration;
-    outputs checked on sampled (sequence, KV head) units and plans in full."""
+@pytest.mark.parametrize("name", ["llama8b_32k", "qwen32b_32k", "longctx_128k"])
+def test_full_size_layer_sampled(name):
+    """One layer of a configuration at full size, built as the bench builds it
+    (the 32K Llama layer is the benchmarked one): outputs checked on sampled
+    (sequence, KV head) units and plans in full.  The 32K Qwen3-32B layer
+    (64/8 heads, 1+7 queries) runs with its seeded 10 % residency loss; the
+    128K layer has heavy-tailed keys and 8,192 blocks per head."""
     from bench import build_workload_state
-    w = W.WORKLOADS["llama8b_32k"]
+    w = W.WORKLOADS[name]
     st = build_workload_state(w, steps=3, device=DEV)
     d, L, pipe, qs = st["dims"], st["layer"], st["pipe"], st["queries"]
     host_bits = None
@@ -208,11 +211,13 @@ def test_full_size_llama_layer_sampled():
     for t in range(1, 3):
         st_prev, lu_prev = np_i32(L.slot_table), np_i32(L.last_used)
         pool_prev = L.pool.clone()
-        pipe.step(t, [qs[t]])
+        mask = W.eviction_mask(w, 0, t, DEV) if w.evict_prob > 0 else None
+        pipe.step(t, [qs[t]], evict=None if mask is None else [mask.to(torch.uint8)])
         pipe.wait_all()
         torch.cuda.synchronize()
         sel = np_i32(L.sel)
-        plan = O.plan_fetch(sel, st_prev, lu_prev, t, w.fetch_cap)
+        st_plan = st_prev if mask is None else O.evict_slots(st_prev, mask.cpu().numpy())
+        plan = O.plan_fetch(sel, st_plan, lu_prev, t, w.fetch_cap)
         np.testing.assert_array_equal(np_i32(L.slot_table), plan["slot_table"])
         np.testing.assert_array_equal(np_i32(L.last_used), plan["last_used"])
         q = f64(qs[t].cpu())
@@ -232,3 +237,57 @@ def test_full_size_llama_layer_sampled():
                                    o_ref, lse_ref)
             hb = W.bf16_bits(kv_unit)
             _check_pool_holds_slot_blocks(L.pool[b:b + 1, h:h + 1], plan["slot_table"][b:b + 1, h:h + 1], hb)
+
+
+def test_pipeline_with_residency_loss_step_by_step():
+    """Reduced 32K Qwen3-32B-shaped layer (G = 8, 1+7 queries: 64 query rows)
+    with a seeded residency-loss mask every step: attention over the slots
+    before the loss, selection, and the plan over the table after it."""
+    w = W.WORKLOADS["qwen32b_32k"].with_(batch=2, n_q_heads=16, n_kv_heads=2, context=6000, max_blocks=400,
+                                          budget_blocks=32, fetch_cap=4, evict_prob=0.2)
+    d = lsk.dims_for(w)
+    K, C = w.budget_blocks, w.fetch_cap
+    host = W.make_host_kv(w).pin_memory()
+    host_bits = W.bf16_bits(host)
+    keys, vals = kv_split(host)
+    ctx = W.initial_ctx_len(w)
+    cnp = ctx.numpy()
+    L = LayerState(d, host, DEV)
+    scale = 1 / math.sqrt(128)
+    pipe = DecodePipeline(d, [L], ctx.to(DEV), scale, DEV)
+    pipe.build_summaries()
+    kmin, kmax = O.block_summaries(keys, cnp)
+    qs = W.QueryStream(w)
+    pipe.prime([qs.next().to(DEV)])
+    pipe.wait_all()
+    torch.cuda.synchronize()
+    st, lu = np_i32(L.slot_table), np_i32(L.last_used)
+    lost_total = 0
+    for t in range(1, 15):
+        q = qs.next()
+        mask = W.eviction_mask(w, 0, t)
+        pipe.step(t, [q.to(DEV)], evict=[mask.to(torch.uint8).to(DEV)])
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        pk = np.zeros((w.batch, w.n_kv_heads, K, 16, 128))
+        pv = np.zeros_like(pk)
+        for b in range(w.batch):
+            for h in range(w.n_kv_heads):
+                for s in range(K):
+                    if st[b, h, s] >= 0:
+                        pk[b, h, s], pv[b, h, s] = keys[b, h, st[b, h, s]], vals[b, h, st[b, h, s]]
+        o_ref, lse_ref = O.sparse_attention(f64(q), pk, pv, st, cnp, scale)
+        assert_attention_close(L.out, L.lse, o_ref, lse_ref)
+        lost_total += int(((st >= 0) & mask.numpy()).sum())
+        st = O.evict_slots(st, mask.numpy())
+        sc = O.lookahead_scores(f64(q), kmin, kmax, cnp, 16)
+        ref_sel, _ = O.select_topk(sc, cnp, K, 16)
+        sel = np_i32(L.sel)
+        assert_selection_matches(sel, ref_sel, sc, cnp, K)
+        plan = O.plan_fetch(sel, st, lu, t, C)
+        np.testing.assert_array_equal(np_i32(L.slot_table), plan["slot_table"])
+        np.testing.assert_array_equal(np_i32(L.last_used), plan["last_used"])
+        st, lu = plan["slot_table"], plan["last_used"]
+        _check_pool_holds_slot_blocks(L.pool, st, host_bits)
+    assert lost_total > 0
+
