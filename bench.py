@@ -694,6 +694,33 @@ def algorithmic_bytes(w, fetched_blocks_per_layer_step):
     }
 
 
+def overlap_efficiency(iso_ms, pipeline_ms_per_layer_step):
+    """eta = (T_compute + T_fetch - T_pipeline) / min(T_compute, T_fetch) per
+    layer-step: 1 when the gather hides completely behind (or hides) the
+    compute, 0 when they run back to back.  T_compute and T_fetch are the
+    isolated times of the layer's device work without and with only the
+    gather; T_pipeline the measured per-layer-step time of the pipeline."""
+    t_c = iso_ms["sparse_attn"] + iso_ms["score_select"] + iso_ms["plan_fetch"]
+    t_f = iso_ms["prefetch"]
+    return {"value": (t_c + t_f - pipeline_ms_per_layer_step) / min(t_c, t_f),
+            "compute_ms": t_c, "fetch_ms": t_f, "pipeline_ms": pipeline_ms_per_layer_step}
+
+
+def token_kv_intensity(w, fetched_blocks_per_layer_step):
+    """OasisKV Figure 1: tokens generated per decode pass per KV-cache byte
+    moved, per memory tier; one token per sequence per layer-step."""
+    units = w.batch * w.n_kv_heads
+    nv = math.ceil(w.context / w.block_tokens)
+    hbm = units * w.budget_blocks * w.block_bytes + units * nv * 2 * w.head_dim * 2   # resident KV + summaries
+    io = fetched_blocks_per_layer_step * w.block_bytes
+    dense = units * nv * w.block_bytes
+    mib = float(2 ** 20)
+    return {"hbm_tokens_per_mib": w.batch / (hbm / mib), "pcie_tokens_per_mib": w.batch / (io / mib) if io else None,
+            "dense_hbm_tokens_per_mib": w.batch / (dense / mib),
+            "definition": "batch tokens per MiB of KV-cache bytes per layer-step: HBM = resident KV + block summaries "
+                          "read; PCIe = fetched blocks; dense = the whole KV read by dense attention"}
+
+
 def emit_gpu(args, res, world):
     w, timer = res["w"], res["timer"]
     nl = len(res["layers"])
@@ -756,6 +783,8 @@ def emit_gpu(args, res, world):
         "fetched_blocks_per_layer_step": fetched,
         "h2d_gbs_avg": ab["prefetch"] * layer_steps / (res["ms"] * 1e-3) / 1e9,
         "reuse": sum(res["reuse"]) / len(res["reuse"]),
+        "overlap_efficiency": overlap_efficiency(iso, res["ms"] / layer_steps),
+        "token_kv_intensity": token_kv_intensity(w, fetched),
         "h2d_peak": res["h2d"],
         "e2e": {"value": e2e_value, "unit": "layer-steps/s",
                 "h2d_bytes_per_step": nl * (q_bytes + int(ab["prefetch"])),
