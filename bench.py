@@ -128,8 +128,25 @@ class KernelTimer:
     def __init__(self, n):
         self.ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                        for _ in range(n)] for k in KERNELS}
+        for pairs in self.ev.values():                 # create them now (torch does on first record),
+            for a, b in pairs:                         # not inside the timed region
+                a.record()
+                b.record()
         self.i = {k: 0 for k in KERNELS}
         self.on = False
+
+    def native_handles(self):
+        """Raw begin / end event handles of the next launch of each kernel, in
+        the order the native layer step records them (0 = not recorded)."""
+        out = []
+        for name in KERNELS:
+            if self.on and self.i[name] < len(self.ev[name]):
+                a, b = self.ev[name][self.i[name]]
+                out += [a.cuda_event, b.cuda_event]
+                self.i[name] += 1
+            else:
+                out += [0, 0]
+        return out
 
     def begin(self, name, stream):
         if self.on and self.i[name] < len(self.ev[name]):
@@ -613,6 +630,7 @@ def run_gpu(args, rank, world, device):
     timer.on = True
     with ClockSampler(torch.cuda.current_device()) as clk:
         ev0.record(main)
+        h0 = time.perf_counter()
         for i in range(args.steps):
             pipe.step(t, qs_at(t))
             for l, L in enumerate(layers):
@@ -620,6 +638,7 @@ def run_gpu(args, rank, world, device):
             t += 1
         pipe.wait_all()
         ev1.record(main)
+        host_ms = (time.perf_counter() - h0) * 1e3
         torch.cuda.synchronize()
     timer.on = False
     ms = ev0.elapsed_time(ev1)
@@ -669,7 +688,7 @@ def run_gpu(args, rank, world, device):
     iso = isolated_kernel_ms(st)
     h2d = measure_h2d_peak(device) if rank == 0 else None
     err = lsk.read_device_error(clear=True)
-    return {"w": w, "d": d, "ms": ms, "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
+    return {"w": w, "d": d, "ms": ms, "host_ms": host_ms, "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
             "e2e_ms": e2e_ms, "e2e_steps": e2e_steps, "h2d": h2d, "clocks": clk.summary(), "dev_err": err,
             "layer": layers[0], "layers": layers, "queries": qrings[0], "iso": iso}
 
@@ -792,6 +811,7 @@ def emit_gpu(args, res, world):
                 "note": "per step: every layer's queries copied in from pinned host memory and its outputs read "
                         "back, then synchronised; h2d bytes include the zero-copy gather of fetched blocks"},
         "gpu_launches": 6 * layer_steps,   # attention, merge, score, select, plan, gather
+        "host_enqueue_ms_per_step": res["host_ms"] / args.steps,
         "clocks": res["clocks"],
         "device_error_word": res["dev_err"],
     }

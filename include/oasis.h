@@ -237,6 +237,65 @@ int oasis_evict_slots(const oasis_dims* d, const uint8_t* mask, int32_t* slot_ta
  * captured decode step. */
 int oasis_step_advance(int32_t* step, void* stream);
 
+/* ---- a7: one layer's decode step in a single call ------------------------
+ * OasisKV Figure 8: per layer, attention over the resident blocks on the main
+ * stream; lookahead scoring and top-K on a second stream concurrent with it;
+ * the plan on the main stream once the selection is ready; the gather on a
+ * third (high-priority) stream once the plan is ready, landing before that
+ * layer's attention at the next step.  This entry point enqueues all of it
+ * with the stream / event order done natively (cudaStreamWaitEvent /
+ * cudaEventRecord), so a whole layer-step costs the host one call. */
+
+/* One attention layer's buffers; every pointer is device memory unless noted. */
+typedef struct oasis_layer {
+    const void* host_kv;    /* pinned, mapped host KV [B][Hkv][N][2][P][D] bf16 */
+    const void* kmin;       /* [B][Hkv][N][D] bf16 */
+    const void* kmax;
+    void* pool;             /* [B][Hkv][K][2][P][D] bf16 */
+    int32_t* slot_table;    /* [B][Hkv][K] */
+    int32_t* last_used;     /* [B][Hkv][K] */
+    int32_t* sel;           /* [B][Hkv][K] */
+    float* sel_score;       /* [B][Hkv][K], may be NULL */
+    float* scores;          /* NULL: scores in the workspace, LRU victims (oasis_plan_fetch);
+                               [B][Hkv][N] of this layer: scores kept here, score-ordered
+                               victims (oasis_plan_fetch_scored) */
+    int32_t* fetch_slot;    /* [B][Hkv][C] */
+    int32_t* fetch_block;   /* [B][Hkv][C] */
+    int32_t* n_fetch;       /* [B][Hkv] */
+    float* out;             /* [B][Qn][Hq][D] fp32 */
+    float* lse;             /* [B][Qn][Hq] fp32 */
+} oasis_layer;
+
+/* Streams (cudaStream_t; NULL is the default stream) and this layer's events
+ * (cudaEvent_t, created by the caller) of a layer-step.  score may equal main
+ * (no overlap).  With in_graph
+ * set (inside a capture of a whole step) the main stream does not wait for
+ * fetch_done and the score stream forks from main through `fork` instead of
+ * waiting for plan_ready.  timing: optional begin / end events recorded
+ * around attention (main), score+select (score), plan (main) and gather (copy),
+ * in that order; NULL entries are skipped. */
+typedef struct oasis_step_sync {
+    void* main;
+    void* score;
+    void* copy;
+    void* fetch_done;       /* recorded on copy after the gather */
+    void* plan_ready;       /* recorded on main after the plan */
+    void* sel_ready;        /* recorded on score after the selection */
+    void* fork;             /* in_graph only */
+    int32_t in_graph;
+    void* timing[8];
+} oasis_step_sync;
+
+/* Decode step `step` of one layer, in the order above: [wait fetch_done] ->
+ * attention(q, scale) -> [residency loss: evict_mask, may be NULL] -> scores +
+ * top-K -> plan (step number `step`, or *step_dev when step_dev != NULL) ->
+ * gather.  Same buffers, workspace and results as the individual calls; the
+ * first error returns before anything after it is enqueued. */
+int oasis_decode_layer_step(const oasis_dims* d, const oasis_layer* layer, const void* q,
+                            const int32_t* ctx_len, const uint8_t* evict_mask, int32_t step,
+                            const int32_t* step_dev, float scale, void* ws, size_t ws_bytes,
+                            const oasis_step_sync* sync);
+
 /* a5 - host-to-HBM gather (OasisKV Figure 7: blocks "are prefetched from the
  * CPU cache"; Figure 8).  For i < n_fetch[b][h], copies the 8 KiB block
  * host_kv[b][h][fetch_block[b][h][i]] into pool[b][h][fetch_slot[b][h][i]]

@@ -57,6 +57,20 @@ def dims_for(w) -> Dims:
                      w.n_queries, w.fetch_cap, w.head_dim, w.block_tokens)
 
 
+class Layer(ctypes.Structure):
+    """oasis_layer: one attention layer's buffers (device addresses)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "host_kv", "kmin", "kmax", "pool", "slot_table", "last_used", "sel", "sel_score", "scores",
+        "fetch_slot", "fetch_block", "n_fetch", "out", "lse")]
+
+
+class StepSync(ctypes.Structure):
+    """oasis_step_sync: streams, this layer's events, graph flag, timing events."""
+    _fields_ = [("main", ctypes.c_void_p), ("score", ctypes.c_void_p), ("copy", ctypes.c_void_p),
+                ("fetch_done", ctypes.c_void_p), ("plan_ready", ctypes.c_void_p), ("sel_ready", ctypes.c_void_p),
+                ("fork", ctypes.c_void_p), ("in_graph", ctypes.c_int32), ("timing", ctypes.c_void_p * 8)]
+
+
 _LIB = None
 _V = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -77,6 +91,8 @@ _SIGS = {
     "oasis_plan_fetch_at": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V, _V, _V]),
     "oasis_step_advance": (ctypes.c_int, [_V, _V]),
     "oasis_evict_slots": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V]),
+    "oasis_decode_layer_step": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Layer), _V, _V, _V, _I32, _V,
+                                               ctypes.c_float, _V, ctypes.c_size_t, ctypes.POINTER(StepSync)]),
     "oasis_prefetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V]),
     "oasis_sparse_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, ctypes.c_float,
                                          _V, _V, _V, ctypes.c_size_t, _V]),
@@ -219,6 +235,21 @@ def plan_fetch_at(d, sel, scores, slot_table, last_used, step, fetch_slot, fetch
 def evict_slots(d, mask, slot_table, stream=None):
     """Frees the slots whose mask byte (uint8 [B][Hkv][K]) is set."""
     _check(lib().oasis_evict_slots(ctypes.byref(d), _p(mask), _p(slot_table), _stream(stream)), "oasis_evict_slots")
+
+
+def make_layer(host_kv, kmin, kmax, pool, slot_table, last_used, sel, sel_score, scores, fetch_slot, fetch_block,
+               n_fetch, out, lse) -> Layer:
+    """oasis_layer from tensors (None for the nullable sel_score / scores)."""
+    return Layer(*[_p(t) for t in (host_kv, kmin, kmax, pool, slot_table, last_used, sel, sel_score, scores,
+                                    fetch_slot, fetch_block, n_fetch, out, lse)])
+
+
+def decode_layer_step(d, layer: Layer, q, ctx_len, evict_mask, step, step_dev, scale, ws, sync: StepSync):
+    """One layer's decode step (attention, [loss], scores + top-K, plan, gather) in one call."""
+    _check(lib().oasis_decode_layer_step(ctypes.byref(d), ctypes.byref(layer), _p(q), _p(ctx_len), _p(evict_mask),
+                                         int(step), _p(step_dev), float(scale), _p(ws),
+                                         ws.numel() * ws.element_size(), ctypes.byref(sync)),
+           "oasis_decode_layer_step")
 
 
 def step_advance(step, stream=None):

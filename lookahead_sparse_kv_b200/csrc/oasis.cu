@@ -480,6 +480,83 @@ int oasis_evict_slots(const oasis_dims* dp, const uint8_t* mask, int32_t* slot_t
     return check_launch("evict_slots launch");
 }
 
+namespace {
+
+int ev_record(void* ev, void* stream, const char* what) {
+    if (ev == nullptr) return OASIS_OK;
+    const cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(ev), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? OASIS_OK : cuda_fail(e, what);
+}
+
+int ev_wait(void* stream, void* ev, const char* what) {
+    const cudaError_t e = cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), static_cast<cudaEvent_t>(ev), 0);
+    return e == cudaSuccess ? OASIS_OK : cuda_fail(e, what);
+}
+
+}  // namespace
+
+int oasis_decode_layer_step(const oasis_dims* dp, const oasis_layer* L, const void* q, const int32_t* ctx_len,
+                            const uint8_t* evict_mask, int32_t step, const int32_t* step_dev, float scale, void* ws,
+                            size_t ws_bytes, const oasis_step_sync* S) {
+    if (L == nullptr || S == nullptr) return fail(OASIS_EINVAL, "layer and sync must not be NULL");
+    if (S->fetch_done == nullptr || S->plan_ready == nullptr || S->sel_ready == nullptr)
+        return fail(OASIS_EINVAL, "fetch_done, plan_ready and sel_ready events must be given");
+    if (S->in_graph && S->fork == nullptr) return fail(OASIS_EINVAL, "in_graph needs the fork event");
+    const bool overlap = S->score != S->main;
+    int rc;
+    if (!S->in_graph && (rc = ev_wait(S->main, S->fetch_done, "wait fetch_done"))) return rc;
+    // attention over the working set staged by the previous step
+    if ((rc = ev_record(S->timing[0], S->main, "timing"))) return rc;
+    if ((rc = oasis_sparse_attn(dp, q, L->pool, L->slot_table, ctx_len, scale, L->out, L->lse, ws, ws_bytes,
+                                S->main)))
+        return rc;
+    if ((rc = ev_record(S->timing[1], S->main, "timing"))) return rc;
+    if (evict_mask != nullptr && (rc = oasis_evict_slots(dp, evict_mask, L->slot_table, S->main))) return rc;
+    // lookahead scores + top-K, concurrent with the attention
+    if (overlap) {
+        if (S->in_graph) {
+            if ((rc = ev_record(S->fork, S->main, "record fork")) || (rc = ev_wait(S->score, S->fork, "wait fork")))
+                return rc;
+        } else if ((rc = ev_wait(S->score, S->plan_ready, "wait plan_ready"))) {   // previous plan read sel
+            return rc;
+        }
+    }
+    if ((rc = ev_record(S->timing[2], S->score, "timing"))) return rc;
+    if (L->scores != nullptr) {
+        if ((rc = oasis_lookahead_scores(dp, q, L->kmin, L->kmax, ctx_len, L->scores, S->score)) ||
+            (rc = oasis_select_topk(dp, L->scores, ctx_len, L->sel, L->sel_score, S->score)))
+            return rc;
+    } else if ((rc = oasis_score_select(dp, q, L->kmin, L->kmax, ctx_len, L->sel, L->sel_score, ws, ws_bytes,
+                                        S->score))) {
+        return rc;
+    }
+    if ((rc = ev_record(S->timing[3], S->score, "timing"))) return rc;
+    if (overlap && ((rc = ev_record(S->sel_ready, S->score, "record sel_ready")) ||
+                    (rc = ev_wait(S->main, S->sel_ready, "wait sel_ready"))))
+        return rc;
+    // residency diff + capped plan
+    if ((rc = ev_record(S->timing[4], S->main, "timing"))) return rc;
+    if (step_dev != nullptr)
+        rc = oasis_plan_fetch_at(dp, L->sel, L->scores, L->slot_table, L->last_used, step_dev, L->fetch_slot,
+                                 L->fetch_block, L->n_fetch, S->main);
+    else if (L->scores != nullptr)
+        rc = oasis_plan_fetch_scored(dp, L->sel, L->scores, L->slot_table, L->last_used, step, L->fetch_slot,
+                                     L->fetch_block, L->n_fetch, S->main);
+    else
+        rc = oasis_plan_fetch(dp, L->sel, L->slot_table, L->last_used, step, L->fetch_slot, L->fetch_block,
+                              L->n_fetch, S->main);
+    if (rc) return rc;
+    if ((rc = ev_record(S->timing[5], S->main, "timing"))) return rc;
+    if ((rc = ev_record(S->plan_ready, S->main, "record plan_ready")) ||
+        (rc = ev_wait(S->copy, S->plan_ready, "wait plan_ready")))
+        return rc;
+    // the gather of the missing blocks, on the copy stream
+    if ((rc = ev_record(S->timing[6], S->copy, "timing"))) return rc;
+    if ((rc = oasis_prefetch(dp, L->host_kv, L->fetch_slot, L->fetch_block, L->n_fetch, L->pool, S->copy))) return rc;
+    if ((rc = ev_record(S->timing[7], S->copy, "timing"))) return rc;
+    return ev_record(S->fetch_done, S->copy, "record fetch_done");
+}
+
 int oasis_step_advance(int32_t* step, void* stream) {
     if (int rc = check_ptr(step, "step")) return rc;
     oasis::step_advance_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(step);

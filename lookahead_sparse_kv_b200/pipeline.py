@@ -28,6 +28,11 @@ block with the lowest current lookahead score first; the scores of each
 layer then go to a buffer of its own so the plan on the main stream can
 read them while the score stream moves on to the next layer.
 
+Native steps: unless the exact-set stage is on, a layer's decode step is one
+call into the library (``oasis_decode_layer_step``), which enqueues the
+kernels and does the stream / event order above in C, so the host cost per
+layer-step is one call instead of a dozen.
+
 Graph mode (``device_step=True``): the step number lives in device memory
 (advanced by a kernel at the start of each step, read by the planner), so a
 whole multi-layer decode step can be captured once as a CUDA graph
@@ -49,9 +54,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (append_kv, block_overlap, build_summaries, evict_slots, lookahead_scores, make_dims, plan_fetch,
-               plan_fetch_at, plan_fetch_scored, prefetch, score_select, score_select_rows, select_topk,
-               sparse_attn, step_advance, workspace_bytes)
+from . import (StepSync, append_kv, block_overlap, build_summaries, decode_layer_step, evict_slots,
+               lookahead_scores, make_dims, make_layer, plan_fetch, plan_fetch_at, plan_fetch_scored, prefetch,
+               score_select, score_select_rows, select_topk, sparse_attn, step_advance, workspace_bytes)
 
 HEAD_DIM, BLOCK_TOKENS = 128, 16
 
@@ -147,6 +152,12 @@ class DecodePipeline:
         self.copy_stream = torch.cuda.Stream(device, priority=hi)
         self.sel_ready = [torch.cuda.Event() for _ in layers]
         self.fork = [torch.cuda.Event() for _ in layers]
+        # the native step takes raw event handles: create every event now (torch creates them
+        # on first record; recording on an idle stream completes at once)
+        for i, L in enumerate(layers):
+            for ev in (L.plan_ready, L.fetch_done, self.sel_ready[i], self.fork[i]):
+                ev.record(self.main)
+        self._native = [None] * len(layers)
         self.timer = None        # optional: begin(name, stream) / end(name, stream) around each call
 
     def _t(self, which, name, stream):
@@ -202,6 +213,22 @@ class DecodePipeline:
         prefetch(d, L.host_kv, L.fetch_slot, L.fetch_block, L.n_fetch, L.pool, stream=self.copy_stream)
         self._t("end", "prefetch", self.copy_stream)
         L.fetch_done.record(self.copy_stream)
+
+    def _native_layer(self, i, L):
+        if self._native[i] is None:
+            self._native[i] = make_layer(L.host_kv, L.kmin, L.kmax, L.pool, L.slot_table, L.last_used, L.sel,
+                                         L.sel_score, L.scores if self.victims == "score" else None, L.fetch_slot,
+                                         L.fetch_block, L.n_fetch, L.out, L.lse)
+        return self._native[i]
+
+    def _native_sync(self, i, L, in_graph):
+        sync = StepSync(self.main.cuda_stream, self.score_stream.cuda_stream, self.copy_stream.cuda_stream,
+                        L.fetch_done.cuda_event, L.plan_ready.cuda_event, self.sel_ready[i].cuda_event,
+                        self.fork[i].cuda_event, 1 if in_graph else 0)
+        if self.timer is not None and hasattr(self.timer, "native_handles"):
+            for k, h in enumerate(self.timer.native_handles()):
+                sync.timing[k] = h
+        return sync
 
     def _exact_step(self, L, q, t, ctx):
         """Exact set of step t, agreement counts, optional corrective fetch (main stream)."""
@@ -260,8 +287,8 @@ class DecodePipeline:
         else:
             ctx_in, ctx = self.ctx[self.cur], self.ctx[1 - self.cur]
         for i, (L, q) in enumerate(zip(self.layers, q_per_layer)):
-            if not in_graph:
-                main.wait_event(L.fetch_done)
+            if not in_graph and (self.exact is not None or appended is not None):
+                main.wait_event(L.fetch_done)          # (the native step waits for it itself)
             if appended is not None:
                 k_new, v_new = appended[i]
                 append_kv(d, k_new, v_new, ctx_in, ctx if i == 0 else None, L.host_kv, L.kmin, L.kmax,
@@ -270,8 +297,12 @@ class DecodePipeline:
                     ev = torch.cuda.Event()
                     ev.record(main)
                     self.score_stream.wait_event(ev)       # grown summaries and context
-            if self.exact is not None:
-                self._exact_step(L, q, t, ctx)
+            if self.exact is None:
+                decode_layer_step(d, self._native_layer(i, L), q, ctx, None if evict is None else evict[i],
+                                  0 if t is None else t, self.step_dev, self.scale, self.ws,
+                                  self._native_sync(i, L, in_graph))
+                continue
+            self._exact_step(L, q, t, ctx)
             self._t("begin", "sparse_attn", main)
             sparse_attn(d, q, L.pool, L.slot_table, ctx, self.scale, L.out, L.lse, self.ws, stream=main)
             self._t("end", "sparse_attn", main)

@@ -77,3 +77,23 @@ def test_null_and_misaligned_pointers_rejected_on_host(L):
 
 def test_version_string(L):
     assert b"sm_100a" in L.oasis_version()
+
+
+def test_native_layer_step_rejects_missing_streams_and_events(L):
+    """oasis_decode_layer_step checks its layer / sync arguments before any
+    CUDA call: no sync, no events, or a graph step without its fork event
+    are EINVAL."""
+    d = lsk.make_dims(batch=1, n_q_heads=8, n_kv_heads=2, max_blocks=64, budget_blocks=16, n_queries=5,
+                      fetch_cap=4)
+    layer = lsk.Layer()
+
+    def call(sync):
+        return L.oasis_decode_layer_step(ctypes.byref(d), ctypes.byref(layer), None, None, None, 1, None,
+                                         ctypes.c_float(0.1), None, 0, sync)
+
+    assert call(None) == lsk.EINVAL
+    s = lsk.StepSync()                                   # NULL streams are the default stream
+    assert call(ctypes.byref(s)) == lsk.EINVAL and "events" in lsk.last_error()
+    s.fetch_done = s.plan_ready = s.sel_ready = 2
+    s.in_graph = 1
+    assert call(ctypes.byref(s)) == lsk.EINVAL and "fork" in lsk.last_error()
