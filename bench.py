@@ -646,6 +646,19 @@ def run_gpu(args, rank, world, device):
         torch.distributed.barrier()
     ms = max_over_ranks(ms)
 
+    # host cost of a step: a few steps enqueued right after a synchronize, so the
+    # launch queue has room and the host never waits on the device
+    host_cost = []
+    for _ in range(3):
+        torch.cuda.synchronize()
+        h0 = time.perf_counter()
+        for _ in range(4):
+            pipe.step(t, qs_at(t))
+            t += 1
+        host_cost.append((time.perf_counter() - h0) * 1e3 / 4)
+    pipe.wait_all()
+    torch.cuda.synchronize()
+
     # reuse of the selected set between consecutive steps (untimed)
     reuse = []
     prev = [L.sel.clone() for L in layers]
@@ -688,7 +701,7 @@ def run_gpu(args, rank, world, device):
     iso = isolated_kernel_ms(st)
     h2d = measure_h2d_peak(device) if rank == 0 else None
     err = lsk.read_device_error(clear=True)
-    return {"w": w, "d": d, "ms": ms, "host_ms": host_ms, "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
+    return {"w": w, "d": d, "ms": ms, "host_ms": host_ms, "host_cost_ms": min(host_cost), "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
             "e2e_ms": e2e_ms, "e2e_steps": e2e_steps, "h2d": h2d, "clocks": clk.summary(), "dev_err": err,
             "layer": layers[0], "layers": layers, "queries": qrings[0], "iso": iso}
 
@@ -812,6 +825,7 @@ def emit_gpu(args, res, world):
                         "back, then synchronised; h2d bytes include the zero-copy gather of fetched blocks"},
         "gpu_launches": 6 * layer_steps,   # attention, merge, score, select, plan, gather
         "host_enqueue_ms_per_step": res["host_ms"] / args.steps,
+        "host_cost_ms_per_step": res["host_cost_ms"],
         "clocks": res["clocks"],
         "device_error_word": res["dev_err"],
     }
