@@ -69,12 +69,14 @@ __device__ __forceinline__ long long floor_div_small(long long x, long long t) {
 // Merges the stream partials of each (unit, query row) in stream order:
 // lse = log sum_p exp(lse_p), out = sum_p exp(lse_p - lse) * o_p.  One warp
 // per (unit, row); lane j holds partial j's lse, lane c owns channels
-// 4c..4c+3.  Up to 16 partials (the usual case) are read in one round trip:
-// every lse and output load is issued before any of them is used.
-constexpr int kMergeWarps = 2;                   // small CTAs: the whole grid fits in one wave
-constexpr int kMergeFast = 16;
+// 4c..4c+3.  Up to 12 partials (the usual case: 8 streams per SM give about
+// 10 per unit on the 32K Llama layer) are read in one round trip: every lse
+// and output load is issued before any of them is used.  Small CTAs, and at
+// most 80 registers so that 12 CTAs fit an SM and the grid runs in one wave.
+constexpr int kMergeWarps = 2;
+constexpr int kMergeFast = 12;
 
-__global__ void __launch_bounds__(32 * kMergeWarps) attn_merge_kernel(Dims d, int n_streams,
+__global__ void __launch_bounds__(32 * kMergeWarps, 12) attn_merge_kernel(Dims d, int n_streams,
                                                                       const float* __restrict__ ws_o,
                                                                       const float* __restrict__ ws_lse,
                                                                       float* __restrict__ out,
