@@ -21,8 +21,8 @@ Sources, cited by page title plus figure / table / section:
   Inference" (in the reference list of the mlsanity.com index page of the
   same paper): the per-channel min/max upper bound used as the block scorer.
   The OasisKV pages say the draft query scans keys compressed by per-block
-  min/max pooling (Figure 7) but do not print the scoring formula; this build
-  fixes it as Quest's bound.
+  min/max pooling (Figure 7) but do not print the scoring formula; the
+  scorer here is Quest's bound.
 
 Data conventions (all arrays numpy):
 
@@ -37,7 +37,7 @@ Data conventions (all arrays numpy):
   right).  When ``Qn == 1`` there are no drafts and row 0 is used for scoring
   (a degenerate previous-token predictor; see the readings below).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
 
 * R1 scorer: ``s[n] = max_{j>=1, g<G} sum_c max(q_c*kmin_c, q_c*kmax_c)``,
   no 1/sqrt(D) factor, summed in fp64 and rounded once to fp32.
