@@ -262,13 +262,39 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def strip_comments(src: str) -> str:
+    """C/CUDA source without comments and with whitespace collapsed, so that
+    a comment edit does not count as a kernel change (string literals kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"':                                   # string literal (inline PTX)
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the CUDA sources as the compiler sees them (comments and
+    whitespace removed); the ncu traffic file is valid while it matches."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "lookahead_sparse_kv_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -739,8 +765,9 @@ def overlap_efficiency(iso_ms, pipeline_ms_per_layer_step):
 
 
 def token_kv_intensity(w, fetched_blocks_per_layer_step):
-    """OasisKV Figure 1: tokens generated per decode pass per KV-cache byte
-    moved, per memory tier; one token per sequence per layer-step."""
+    """OasisKV Figure 1: how many new tokens a decode pass yields for each
+    KV-cache byte it moves, per memory tier (HBM, PCIe); one token per
+    sequence per layer-step."""
     units = w.batch * w.n_kv_heads
     nv = math.ceil(w.context / w.block_tokens)
     hbm = units * w.budget_blocks * w.block_bytes + units * nv * 2 * w.head_dim * 2   # resident KV + summaries

@@ -130,7 +130,7 @@ int oasis_lookahead_scores(const oasis_dims* d, const void* q, const void* kmin,
                            const void* kmax, const int32_t* ctx_len, float* scores,
                            void* stream);
 
-/* a3 - top-K selection (OasisKV Figure 7: "the next step's top-K blocks").
+/* a3 - top-K selection (OasisKV Figure 7: the K blocks the next step uses).
  * Per (b, h): ranks the valid blocks by (score descending, block id
  * ascending; -0.0 == +0.0) and writes the first min(K, n_valid) ids to sel in
  * rank order, -1 padded; sel_score (nullable) gets their scores, -inf padded.
@@ -296,8 +296,8 @@ int oasis_decode_layer_step(const oasis_dims* d, const oasis_layer* layer, const
                             const int32_t* step_dev, float scale, void* ws, size_t ws_bytes,
                             const oasis_step_sync* sync);
 
-/* a5 - host-to-HBM gather (OasisKV Figure 7: blocks "are prefetched from the
- * CPU cache"; Figure 8).  For i < n_fetch[b][h], copies the 8 KiB block
+/* a5 - host-to-HBM gather (OasisKV Figure 7: the chosen blocks come in from
+ * the CPU-side KV cache ahead of use; Figure 8).  For i < n_fetch[b][h], copies the 8 KiB block
  * host_kv[b][h][fetch_block[b][h][i]] into pool[b][h][fetch_slot[b][h][i]]
  * with a kernel that reads the mapped pinned host memory directly over PCIe
  * (no copy-engine call, so it stays stream-ordered after the planner).
@@ -306,8 +306,8 @@ int oasis_prefetch(const oasis_dims* d, const void* host_kv, const int32_t* fetc
                    const int32_t* fetch_block, const int32_t* n_fetch, void* pool,
                    void* stream);
 
-/* a6 - sparse GQA decode attention (OasisKV Figure 7, right: normal and
- * draft queries together over the sparse KV working set).  For every b,
+/* a6 - sparse GQA decode attention (OasisKV Figure 7, right: the verification
+ * query and the drafts attended in one pass over the resident working set).  For every b,
  * row j < Qn and query head hq (KV head h = hq / G): over the valid tokens of
  * every occupied slot of (b, h),
  *   out = sum softmax(scale * q.k) v,   lse = log sum exp(scale * q.k);

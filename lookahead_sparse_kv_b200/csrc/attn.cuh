@@ -1,10 +1,9 @@
 // attn.cuh - sparse GQA decode attention over the resident pool slots.
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
-// Prefetching, Figure 7 (right): one attention kernel processes the normal
-// (verification) query and the draft queries together over the sparse KV
-// working set; Figure 9: the per-head slot table says which block each
-// pool slot holds.
+// Prefetching, Figure 7 (right): the verification query and the drafts are
+// attended in one pass over the resident sparse working set; Figure 9: the
+// per-head slot table says which block each pool slot holds.
 //
 // Work split (stream-K): the T = B*Hkv*K pool slots, in (sequence, KV head,
 // slot) order, are cut into NS contiguous ranges, one per "stream".  A

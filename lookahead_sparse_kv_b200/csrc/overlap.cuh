@@ -1,9 +1,9 @@
 // overlap.cuh - agreement of two block-id lists per (sequence, KV head).
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
-// Prefetching, Figure 4 (top-K block prediction accuracy with the previous
-// token vs a lookahead token) and Figure 6 (agreement of the top-K set the
-// draft query predicts with the exact set of the true next-token query):
+// Prefetching, Figure 4 (how well the previous token and a lookahead token
+// each predict the top-K blocks) and Figure 6 (overlap between the top-K set
+// predicted from the draft query and the one the real next query yields):
 // count[b][h] = number of distinct block ids of list b[b][h][*] that also
 // occur in list a[b][h][*].  -1 entries are empty.
 //

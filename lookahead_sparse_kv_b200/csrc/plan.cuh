@@ -1,9 +1,9 @@
 // plan.cuh - residency diff, capped fetch list and LRU victims.
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
-// Prefetching: method sketch item 3 (predicted blocks are compared against
-// the resident GPU blocks and only the missing ones are fetched, capped per
-// step), Table 2 (LRU eviction), Figure 9 (a per-KV-head table maps each GPU
+// Prefetching: method sketch item 3 (the prediction is diffed against the
+// GPU-resident blocks; only the difference is copied, under a per-step cap),
+// Table 2 (LRU eviction), Figure 9 (a per-KV-head table maps each GPU
 // block slot to a CPU block), "Terms in this paper" (capped eviction).
 //
 // One CTA per (b, h) with one thread per slot / rank (K <= 1024):

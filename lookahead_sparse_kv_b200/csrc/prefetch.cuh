@@ -1,9 +1,9 @@
 // prefetch.cuh - host-to-HBM block gather through mapped pinned memory.
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
-// Prefetching, Figure 7 (selected blocks are prefetched from the CPU cache)
-// and Figure 8 (the transfer for step t+1 runs in the background after step
-// t's selection).
+// Prefetching, Figure 7 (the chosen blocks come in from the CPU-side KV cache
+// ahead of use) and Figure 8 (the copy for step t+1 runs in the background
+// once step t has selected).
 //
 // The kernel reads the pinned host KV directly over PCIe (zero-copy) and
 // writes each 8 KiB block into its pool slot, so the gather stays ordered on

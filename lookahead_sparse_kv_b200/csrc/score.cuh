@@ -1,8 +1,8 @@
 // score.cuh - lookahead block scores on the 5th-generation tensor cores.
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
-// Prefetching, Figure 7 (right): the draft queries scan the min/max
-// compressed keys to predict the next step's top-K blocks.  The per-block
+// Prefetching, Figure 7 (right): the drafts are run against the min/max
+// compressed keys, and the result ranks the blocks for the next step.  The per-block
 // bound is Quest's (Quest: Query-Aware Sparsity for Efficient Long-Context LLM
 // Inference): sum_c max(q_c*kmin_c, q_c*kmax_c), maxed over the draft rows
 // and the G query heads of the KV head.

@@ -1,7 +1,7 @@
 // select.cuh - per-(sequence, KV head) top-K block selection.
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
-// Prefetching, Figure 7: the scan predicts "the next step's top-K blocks";
+// Prefetching, Figure 7: the scores pick the K blocks the next step uses;
 // "What they did", item 4: a fixed token budget (K = budget / P blocks).
 // Ranking: score descending, ties to the lower block id, -0.0 == +0.0.
 //

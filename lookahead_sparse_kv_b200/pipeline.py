@@ -1,9 +1,10 @@
 """Per-layer device state and the stream / event order of a decode step.
 
 OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
-Prefetching, Figure 8: at step t each layer's draft queries drive top-K
-prediction, selection and the host-to-HBM transfer, which must land before
-that layer's attention at step t+1; the stages of different layers overlap.
+Prefetching, Figure 8: at step t each layer's drafts drive the top-K
+prediction, the selection and the host-to-HBM copy, and the copy has to
+complete before the same layer attends at step t+1; the stages of different
+layers overlap.
 Figure 7 (right): attention at step t runs over the working set staged at
 step t-1.
 

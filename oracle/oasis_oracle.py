@@ -174,9 +174,10 @@ def summary_append(kmin, kmax, k_new, ctx_len_before, block_tokens):
 def lookahead_scores(q, kmin, kmax, ctx_len, block_tokens, rows=None):
     """Score every valid block of every (sequence, KV head) with the drafts.
 
-    [OasisKV] Figure 7 (right): "the draft query then scans the compressed
-    keys to predict the next step's top-K blocks"; method sketch item 2:
-    draft tokens rank the KV blocks the next step will need.  The bound is
+    [OasisKV] Figure 7 (right): the draft query is run against the min/max
+    compressed keys, and its result ranks the blocks for the next step;
+    method sketch item 2: draft tokens rank the KV blocks the next step will
+    need.  The bound is
     Quest's: for one query q and one block, sum over channels of the larger
     of q_c*kmin_c and q_c*kmax_c, an upper bound on q.k for every key of the
     block.  The block's score is the largest bound over the draft rows and
@@ -212,8 +213,9 @@ def lookahead_scores(q, kmin, kmax, ctx_len, block_tokens, rows=None):
 def select_topk(scores, ctx_len, budget_blocks, block_tokens):
     """Per (sequence, KV head): the K best blocks under the token budget.
 
-    [OasisKV] Figure 7: predict "the next step's top-K blocks"; "What they
-    did" item 4: a 2,048-token KV budget, i.e. K = budget / P blocks.
+    [OasisKV] Figure 7: the ranking yields the K blocks the next step uses;
+    "What they did" item 4: a 2,048-token KV budget, i.e. K = budget / P
+    blocks.
     Ranking: fp32 score descending, ties to the lower block index (R2).  If
     a sequence has no more than K valid blocks, all of them are selected.
 
@@ -242,9 +244,9 @@ def select_topk(scores, ctx_len, budget_blocks, block_tokens):
 def plan_fetch(sel, slot_table, last_used, step, fetch_cap, scores=None):
     """Compare the selection with the resident set and plan a capped fetch.
 
-    [OasisKV] method sketch item 3: predicted blocks are compared against the
-    resident GPU blocks and only the missing ones are fetched, capped per
-    step so the transfer fits the PCIe budget; "What they did" item 3 and
+    [OasisKV] method sketch item 3: the prediction is diffed against what is
+    already resident on the GPU, only the difference crosses PCIe, and a
+    per-step cap keeps that transfer within the link's budget; "What they did" item 3 and
     "Terms in this paper" (capped eviction); Table 2 (LRU eviction);
     Figure 9 (a per-KV-head table mapping each GPU block slot to a CPU
     block).
@@ -309,8 +311,9 @@ def plan_fetch(sel, slot_table, last_used, step, fetch_cap, scores=None):
 def prefetch(host_kv, pool, fetch_slot, fetch_block, n_fetch):
     """Copy each planned block from the host KV cache into its pool slot.
 
-    [OasisKV] Figure 7: selected blocks "are prefetched from the CPU cache";
-    Figure 8: the transfer lands before that layer's attention at step t+1.
+    [OasisKV] Figure 7: the chosen blocks come in from the CPU-side KV cache
+    ahead of use; Figure 8: the copy completes before the same layer attends
+    at step t+1.
     host_kv: [B, Hkv, N, ...]; pool: [B, Hkv, K, ...] (same trailing shape,
     any dtype: the copy is bytewise).  Returns a new pool array.
     """
@@ -327,9 +330,9 @@ def prefetch(host_kv, pool, fetch_slot, fetch_block, n_fetch):
 def sparse_attention(q, pool_k, pool_v, slot_table, ctx_len, scale):
     """GQA decode attention of all Qn query rows over the resident blocks.
 
-    [OasisKV] Figure 7 (right): the attention kernel processes the normal and
-    draft queries together over the sparse KV working set; Figure 9: slot
-    table entries name the CPU block each GPU slot holds.
+    [OasisKV] Figure 7 (right): the verification query and the drafts are
+    attended in one pass over the resident sparse working set; Figure 9:
+    slot table entries name the CPU block each GPU slot holds.
 
     q: float64 [B, Qn, Hq, D]; pool_k / pool_v: float64 [B, Hkv, K, P, D];
     slot_table int32 [B, Hkv, K].  Returns o float64 [B, Qn, Hq, D] and
@@ -421,9 +424,9 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
                        evict_masks=None):
     """One layer through priming and T decode steps, in the pages' order.
 
-    [OasisKV] Figure 8: at step t the draft queries drive top-K prediction,
-    selection and transfer, all finished before that layer's attention at
-    step t+1; Figure 7 (right): attention at step t runs over the working set
+    [OasisKV] Figure 8: at step t the drafts drive the top-K prediction,
+    the selection and the copy, and all of it completes before the same
+    layer attends at step t+1; Figure 7 (right): attention at step t runs over the working set
     staged by step t-1.  Priming (a cold pool) runs one
     select / plan / fetch from ``q_prime`` at step 0; decode step t
     (t = 1..T) runs attention over the working set, then select / plan /
