@@ -32,7 +32,7 @@ def test_kernel_hash_ignores_comment_edits_only(tmp_path, monkeypatch):
 
 def test_overlap_efficiency_bounds():
     iso = {"sparse_attn": 0.04, "score_select": 0.05, "plan_fetch": 0.01, "prefetch": 0.25}
-    t_c, t_f = 0.10, 0.25
+    t_c, t_f = 0.06, 0.25                 # max(attention, scores + top-K) + plan
     full = bench.overlap_efficiency(iso, max(t_c, t_f))          # perfect overlap
     none = bench.overlap_efficiency(iso, t_c + t_f)              # back to back
     assert math.isclose(full["value"], 1.0) and math.isclose(none["value"], 0.0, abs_tol=1e-12)
