@@ -34,12 +34,30 @@ MUTATIONS = {
         "reshape(G, Qn, D).transpose(1, 0, 2)\n"
         "            lse[b, :, h * G:(h + 1) * G] = (m + np.log(l)).reshape(Qn, G)\n"
         "    return o, lse\n\n\ndef dense_attention"),
+    # prediction quality, corrective fetch, victim order, residency loss: their own pin files
+    "overlap counts repeated ids": (
+        "out[i, h] = len(sa & sb)", "out[i, h] = sum(1 for x in b[i, h] if x >= 0 and int(x) in sa)",
+        ["test_oracle_prediction.py"]),
+    "exact set scored from the drafts": (
+        "select_topk(lookahead_scores(qs, kmin, kmax, ctx_len, P, rows=[0]), ctx_len, K, P)",
+        "select_topk(lookahead_scores(qs, kmin, kmax, ctx_len, P), ctx_len, K, P)",
+        ["test_oracle_prediction.py"]),
+    "corrective fetch capped": (
+        "plan = plan_fetch(exact, st, lu, step, K)", "plan = plan_fetch(exact, st, lu, step, fetch_cap)",
+        ["test_oracle_prediction.py"]),
+    "highest-scored stale block evicted": (
+        "stale.sort(key=lambda slot: (float(scores[b, h, st[b, h, slot]]), int(st[b, h, slot])))",
+        "stale.sort(key=lambda slot: (-float(scores[b, h, st[b, h, slot]]), int(st[b, h, slot])))",
+        ["test_oracle_eviction.py"]),
+    "lost slots kept": (
+        "st[np.asarray(mask, dtype=bool)] = -1", "st = st", ["test_oracle_eviction.py"]),
 }
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_planted_mistake(name, tmp_path):
-    old, new = MUTATIONS[name]
+    old, new, *pins = MUTATIONS[name]
+    pins = pins[0] if pins else ["test_oracle.py"]
     for sub in ("oracle", "tests", "lookahead_sparse_kv_b200"):
         shutil.copytree(os.path.join(ROOT, sub), tmp_path / sub,
                         ignore=shutil.ignore_patterns("*.so", "__pycache__", "_build"))
@@ -47,7 +65,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     src = src_path.read_text()
     assert src.count(old) == 1, f"mutation anchor not found once: {name}"
     src_path.write_text(src.replace(old, new))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        str(tmp_path / "tests" / "test_oracle.py")],
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider"] +
+                       [str(tmp_path / "tests" / f) for f in pins],
                        cwd=tmp_path, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"no pin failed for planted mistake: {name}\n{r.stdout[-2000:]}"
