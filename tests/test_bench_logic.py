@@ -47,3 +47,58 @@ def test_token_kv_intensity_of_the_32k_layer():
     # dense reads the whole 2 GiB of KV
     assert math.isclose(r["dense_hbm_tokens_per_mib"], 16 / 2048)
     assert math.isclose(r["pcie_tokens_per_mib"], 16 / (1583 * 8192 / 2 ** 20))
+
+
+class _FakeTimer:
+    def __init__(self, ms):
+        self.ms = ms
+
+    def mean_ms(self, name):
+        return self.ms.get(name)
+
+
+class _FakeLayer:
+    def __init__(self, w):
+        import torch
+        self.out = torch.empty(w.batch, w.n_queries, w.n_q_heads, w.head_dim)
+        self.lse = torch.empty(w.batch, w.n_queries, w.n_q_heads)
+
+
+def test_gpu_line_keeps_the_contract(capsys):
+    """The GPU arm's JSON line, built from fake timings: every key of the
+    contract, the shared metric/config, and the roofline of the dominant kernel."""
+    import argparse
+    import json
+
+    import torch
+    w = W.WORKLOADS[bench.WORKLOAD]
+    nl, steps = 8, 10
+    ms_pipe = {"sparse_attn": 0.16, "score_select": 0.16, "plan_fetch": 0.01, "prefetch": 0.277}
+    res = {
+        "w": w, "timer": _FakeTimer(ms_pipe), "layers": [None] * nl,
+        "fetch_hist": torch.full((steps * nl,), 1583.0),
+        "h2d": {"memcpy_gbs": 55.6, "zero_copy_gbs": 51.1, "peak_gbs": 55.6},
+        "iso": {"sparse_attn": 0.043, "score_select": 0.046, "plan_fetch": 0.012, "prefetch": 0.26,
+                "select_only": 0.016, "build_summaries": 20.9, "_prefetch_blocks": 1572},
+        "ms": 2.25 * steps, "e2e_steps": steps, "e2e_ms": 2.4 * steps, "layer": _FakeLayer(w),
+        "reuse": [0.9, 0.89], "host_ms": 2.1 * steps, "host_cost_ms": 0.19,
+        "clocks": {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 10}, "dev_err": 0,
+    }
+    args = argparse.Namespace(steps=steps, warmup=3, no_cpu_baseline=True)
+    bench.emit_gpu(args, res, 1)
+    d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in d, k
+    assert d["metric"] == bench.METRIC and d["config"] == bench.headline_config(w, nl, 1)
+    assert math.isclose(d["value"], nl / (d["ms_per_step"] * 1e-3))
+    assert d["steps"] == steps and d["warmup"] == 3 and d["n_gpus"] == 1 and d["scaling"] == "weak"
+    r = d["roofline"]
+    assert r["kernel"] == "prefetch" and r["bound"] == "h2d" and r["unit"] == "GB/s" and r["peak"] == 55.6
+    assert math.isclose(r["achieved"], 1583 * w.block_bytes / 0.277e-3 / 1e9)
+    assert math.isclose(r["frac"], r["achieved"] / r["peak"])
+    e = d["e2e"]
+    assert e["unit"] == d["unit"] and e["h2d_bytes_per_step"] > nl * 1583 * w.block_bytes
+    assert e["d2h_bytes_per_step"] == nl * (w.batch * w.n_queries * w.n_q_heads * (w.head_dim + 1) * 4)
+    assert d["gpu_launches"] == 6 * steps * nl
+    assert d["kernels_isolated"]["sparse_attn"]["bound"] == "hbm"
