@@ -435,3 +435,23 @@ def test_decode_steps_with_full_budget_are_dense():
         np.testing.assert_allclose(rec["o"], od, rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(rec["lse"], lsed, rtol=1e-12)
     assert sorted(st[0, 0].tolist()) == list(range(N))
+
+
+def test_bf16_widening_matches_torch_on_every_bit_pattern():
+    """Every one of the 65,536 bf16 patterns widens to the value torch's own
+    bf16 -> float64 conversion gives (NaNs stay NaN); narrowing inverts it
+    on the non-NaN patterns and refuses values that would need rounding."""
+    import torch
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):                # signalling-NaN patterns
+        ours = O.bf16_bits_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))      # -0.0 kept
+    back = O.f64_to_bf16_bits(ours[~nan])
+    assert np.array_equal(back, bits[~nan])
+    for x in (1.0 + 2.0 ** -8, 1.0 / 3.0, 2.0 ** -140 * 1.5):
+        with pytest.raises(ValueError):
+            O.f64_to_bf16_bits(np.array([x]))
