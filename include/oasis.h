@@ -290,7 +290,11 @@ typedef struct oasis_step_sync {
  * attention(q, scale) -> [residency loss: evict_mask, may be NULL] -> scores +
  * top-K -> plan (step number `step`, or *step_dev when step_dev != NULL) ->
  * gather.  Same buffers, workspace and results as the individual calls; the
- * first error returns before anything after it is enqueued. */
+ * first error returns before anything after it is enqueued.  q is read on
+ * main (attention) and on score (scores + top-K); outside a graph the score
+ * stream follows earlier main-stream work only through plan_ready, so a
+ * caller that writes q on main must also order score after that write (an
+ * event recorded on main and waited on by score). */
 int oasis_decode_layer_step(const oasis_dims* d, const oasis_layer* layer, const void* q,
                             const int32_t* ctx_len, const uint8_t* evict_mask, int32_t step,
                             const int32_t* step_dev, float scale, void* ws, size_t ws_bytes,

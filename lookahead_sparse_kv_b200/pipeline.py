@@ -151,6 +151,7 @@ class DecodePipeline:
         self.score_stream = torch.cuda.Stream(device) if overlap_score else self.main
         lo, hi = torch.cuda.Stream.priority_range()
         self.copy_stream = torch.cuda.Stream(device, priority=hi)
+        self.step_start = torch.cuda.Event()
         self.sel_ready = [torch.cuda.Event() for _ in layers]
         self.fork = [torch.cuda.Event() for _ in layers]
         # the native step takes raw event handles: create every event now (torch creates them
@@ -264,19 +265,30 @@ class DecodePipeline:
             L.plan_ready.record(self.main)
             self._select_plan_fetch(i, L, q, 0, self.ctx_len)
 
-    def step(self, t, q_per_layer, appended=None, evict=None):
+    def step(self, t, q_per_layer, appended=None, evict=None, inputs_ready=None, layer_done=None):
         """Decode step t >= 1: per layer [append] -> attention -> [loss] -> select/plan/fetch.
 
+        Each layer's queries are read on the main stream (attention) and on the
+        score stream (scores); the score stream starts the step after all work
+        enqueued on the main stream before this call, so queries written there
+        (a non-blocking copy, say) are seen by both.
         appended: optional list of (k_new, v_new) per layer, bf16 [B, Hkv, D],
         the token accepted at the previous step; it is written at position
         ctx_len[b] and the context is one token longer from this step on.
         evict: optional list of uint8 masks [B, Hkv, K] per layer; the marked
         slots are freed after the layer's attention (residency loss).
+        inputs_ready: optional list of CUDA events, one per layer; layer i's
+        work on both streams waits for event i first, so a caller can bring
+        each layer's queries in on a stream of its own.
+        layer_done: optional list of CUDA events, one per layer; event i is
+        recorded on the main stream once layer i's attention and plan are
+        enqueued (its out and lse are final from there on).
         """
         assert self.graph is None, "a captured pipeline advances by replay()"
-        self._step_body(t, q_per_layer, appended, in_graph=False, evict=evict)
+        self._step_body(t, q_per_layer, appended, in_graph=False, evict=evict, inputs_ready=inputs_ready,
+                        layer_done=layer_done)
 
-    def _step_body(self, t, q_per_layer, appended, in_graph, evict=None):
+    def _step_body(self, t, q_per_layer, appended, in_graph, evict=None, inputs_ready=None, layer_done=None):
         d, main = self.d, self.main
         if self.step_dev is not None:
             if not in_graph:
@@ -287,7 +299,15 @@ class DecodePipeline:
             ctx_in = ctx = self.ctx_len
         else:
             ctx_in, ctx = self.ctx[self.cur], self.ctx[1 - self.cur]
+        if not in_graph and self.score_stream is not main:
+            # the queries may have been written on main just before this step
+            self.step_start.record(main)
+            self.score_stream.wait_event(self.step_start)
         for i, (L, q) in enumerate(zip(self.layers, q_per_layer)):
+            if inputs_ready is not None and inputs_ready[i] is not None:
+                main.wait_event(inputs_ready[i])
+                if self.score_stream is not main:
+                    self.score_stream.wait_event(inputs_ready[i])
             if not in_graph and (self.exact is not None or appended is not None):
                 main.wait_event(L.fetch_done)          # (the native step waits for it itself)
             if appended is not None:
@@ -302,14 +322,16 @@ class DecodePipeline:
                 decode_layer_step(d, self._native_layer(i, L), q, ctx, None if evict is None else evict[i],
                                   0 if t is None else t, self.step_dev, self.scale, self.ws,
                                   self._native_sync(i, L, in_graph))
-                continue
-            self._exact_step(L, q, t, ctx)
-            self._t("begin", "sparse_attn", main)
-            sparse_attn(d, q, L.pool, L.slot_table, ctx, self.scale, L.out, L.lse, self.ws, stream=main)
-            self._t("end", "sparse_attn", main)
-            if evict is not None:
-                evict_slots(d, evict[i], L.slot_table, stream=main)
-            self._select_plan_fetch(i, L, q, t, ctx, in_graph)
+            else:
+                self._exact_step(L, q, t, ctx)
+                self._t("begin", "sparse_attn", main)
+                sparse_attn(d, q, L.pool, L.slot_table, ctx, self.scale, L.out, L.lse, self.ws, stream=main)
+                self._t("end", "sparse_attn", main)
+                if evict is not None:
+                    evict_slots(d, evict[i], L.slot_table, stream=main)
+                self._select_plan_fetch(i, L, q, t, ctx, in_graph)
+            if layer_done is not None and layer_done[i] is not None:
+                layer_done[i].record(main)
         if appended is not None:
             self.cur = 1 - self.cur
         if in_graph:

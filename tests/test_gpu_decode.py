@@ -113,6 +113,73 @@ def test_pipeline_streams_match_sequential_order():
             assert torch.equal(u, v)
 
 
+def _run_fed(w, mode, steps):
+    """Two pipelined layers fed three ways: queries copied synchronously
+    ("sync"), copied non-blocking from pinned memory on the main stream into
+    one reused buffer right before each step ("main"), or copied per layer on
+    an input stream with inputs_ready / layer_done events and read back on an
+    output stream ("events").  Returns per-step results."""
+    w = w.with_(layers=2)
+    d = lsk.dims_for(w)
+    layers = [LayerState(d, W.make_host_kv(w, l).pin_memory(), DEV) for l in range(2)]
+    pipe = DecodePipeline(d, layers, W.initial_ctx_len(w).to(DEV), 1 / math.sqrt(128), DEV, overlap_score=True)
+    pipe.build_summaries()
+    streams = [W.QueryStream(w, l) for l in range(2)]
+    pipe.prime([s.next().to(DEV) for s in streams])
+    qbuf = [torch.empty((w.batch, w.n_queries, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=DEV)
+            for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ev = [torch.cuda.Event() for _ in range(2)]
+    out_ev = [torch.cuda.Event() for _ in range(2)]
+    outs = []
+    for t in range(1, steps + 1):
+        hq = [s.next().pin_memory() for s in streams]
+        if mode == "sync":
+            pipe.step(t, [q.to(DEV) for q in hq])
+            torch.cuda.synchronize()
+            res = [(L.out.cpu(), L.lse.cpu()) for L in layers]
+        elif mode == "main":
+            for l in range(2):
+                qbuf[l].copy_(hq[l], non_blocking=True)
+            pipe.step(t, qbuf)
+            res = [(L.out.to("cpu", non_blocking=True), L.lse.to("cpu", non_blocking=True)) for L in layers]
+            torch.cuda.synchronize()
+        else:
+            with torch.cuda.stream(s_in):
+                for l in range(2):
+                    qbuf[l].copy_(hq[l], non_blocking=True)
+                    in_ev[l].record(s_in)
+            pipe.step(t, qbuf, inputs_ready=in_ev, layer_done=out_ev)
+            hout = [(torch.empty_like(L.out, device="cpu").pin_memory(),
+                     torch.empty_like(L.lse, device="cpu").pin_memory()) for L in layers]
+            with torch.cuda.stream(s_out):
+                for l, L in enumerate(layers):
+                    s_out.wait_event(out_ev[l])
+                    hout[l][0].copy_(L.out, non_blocking=True)
+                    hout[l][1].copy_(L.lse, non_blocking=True)
+            s_out.synchronize()
+            res = hout
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        outs.append([(o, s, L.slot_table.cpu(), L.pool.cpu()) for (o, s), L in zip(res, layers)])
+    return outs
+
+
+@pytest.mark.parametrize("mode", ["main", "events"])
+def test_queries_fed_on_other_streams_match_synchronous_feed(mode):
+    """Scoring reads the queries on its own stream: copies enqueued on the
+    main stream right before step(), or on an input stream announced by
+    per-layer events, give bit-identical outputs, plans and pools."""
+    w = W.WORKLOADS["llama8b_32k"].with_(batch=2, n_q_heads=8, n_kv_heads=2, context=8192,
+                                          max_blocks=512, budget_blocks=64, fetch_cap=8)
+    ref = _run_fed(w, "sync", 5)
+    got = _run_fed(w, mode, 5)
+    for a, b in zip(ref, got):
+        for x, y in zip(a, b):
+            for u, v in zip(x, y):
+                assert torch.equal(u, v)
+
+
 def test_multilayer_append_decode():
     """Three layers, one appended token per step (context crosses block
     boundaries), score overlapped with attention, gather on the copy stream."""
