@@ -6,6 +6,15 @@ raises ``OasisError`` on a non-zero return.  No computation happens in
 Python and there is no fallback: if the library is not built, the first call
 raises.
 
+The C ABI sees plain pointers, so it cannot tell a short buffer from a long
+one.  Before a call, each tensor argument is checked against the dims: its
+dtype, that it is contiguous, that it holds at least the elements the call
+touches, and that device buffers are on a CUDA device.  A failed check raises
+``OasisError`` (EINVAL) before anything is enqueued.  Raw integer addresses
+are passed through unchecked: they are the caller's responsibility.  Where
+host KV lives (device memory or mapped pinned host memory) is checked by the
+library itself.
+
 The operations follow the page "OasisKV: Scaling In-Decode KV Cache Beyond
 HBM with Lookahead Sparse Prefetching" (Figures 7-9, Table 2); see the header
 for the exact contract of each call.
@@ -129,13 +138,67 @@ def last_error() -> str:
     return lib().oasis_last_error().decode()
 
 
-def _p(x):
-    """Address of a tensor / int / None for a void* argument."""
+_BF16, _I32_T, _F32 = "bfloat16", "int32", "float32"
+_U8 = ("uint8", "bool")          # byte masks: torch's bool is one byte holding 0 or 1
+
+
+def _arg(x, what: str, name: str, dtype, numel: int, device: bool = True, nullable: bool = False):
+    """Address of tensor argument `name` after checking it against the call:
+    dtype, contiguity, at least `numel` elements, and a CUDA device when
+    `device` (host KV may be either; the library checks its mapping)."""
     if x is None:
-        return None
+        if nullable:
+            return None
+        raise OasisError(EINVAL, what, f"{name} is None")
     if isinstance(x, int):
         return x
+    names = (dtype,) if isinstance(dtype, str) else dtype
+    if str(x.dtype)[len("torch."):] not in names:
+        raise OasisError(EINVAL, what, f"{name} must be {' or '.join(names)}, got {x.dtype}")
+    if not x.is_contiguous():
+        raise OasisError(EINVAL, what, f"{name} must be contiguous")
+    if x.numel() < numel:
+        raise OasisError(EINVAL, what, f"{name} holds {x.numel()} elements, the call needs {numel}")
+    if device and not x.is_cuda:
+        raise OasisError(EINVAL, what, f"{name} must be on a CUDA device, got {x.device}")
     return x.data_ptr()
+
+
+def _ws(x, what: str):
+    """Address and byte size of a workspace tensor (any dtype, on the device)."""
+    if isinstance(x, int) or x is None:
+        raise OasisError(EINVAL, what, "ws must be a tensor (its size is taken from it)")
+    if not x.is_contiguous() or not x.is_cuda:
+        raise OasisError(EINVAL, what, "ws must be a contiguous CUDA tensor")
+    return x.data_ptr(), x.numel() * x.element_size()
+
+
+class _Sizes:
+    """Element counts of every buffer the calls take, from valid dims."""
+
+    def __init__(self, d, what: str):
+        rc = lib().oasis_check_dims(ctypes.byref(d))
+        if rc != OK:
+            raise OasisError(rc, what, last_error())
+        B, Hq, Hkv, N, K = d.batch, d.n_q_heads, d.n_kv_heads, d.max_blocks, d.budget_blocks
+        D, P, Qn, C = d.head_dim, d.block_tokens, d.n_queries, d.fetch_cap
+        self.what = what
+        self.b = B
+        self.units = B * Hkv
+        self.kv = B * Hkv * N * 2 * P * D          # host KV / pool-shaped blocks [B][Hkv][N][2][P][D]
+        self.summary = B * Hkv * N * D             # kmin, kmax
+        self.q = B * Qn * Hq * D
+        self.row = B * Hkv * D                     # one appended K or V row per (b, h)
+        self.scores = B * Hkv * N
+        self.k = B * Hkv * K                       # sel, sel_score, slot_table, last_used, masks
+        self.c = B * Hkv * C                       # fetch_slot, fetch_block
+        self.cap = C
+        self.pool = B * Hkv * K * 2 * P * D
+        self.out = B * Qn * Hq * D
+        self.lse = B * Qn * Hq
+
+    def fetch_list(self, x, name):
+        return _arg(x, self.what, name, _I32_T, self.c, nullable=self.cap == 0)
 
 
 def _stream(stream):
@@ -161,111 +224,184 @@ def workspace_bytes(d: Dims) -> int:
 
 
 def build_summaries(d, kv, ctx_len, kmin, kmax, first_block=0, n_blocks=None, stream=None):
+    w = "oasis_build_summaries"
+    z = _Sizes(d, w)
     n = d.max_blocks - first_block if n_blocks is None else n_blocks
-    _check(lib().oasis_build_summaries(ctypes.byref(d), _p(kv), _p(ctx_len), first_block, n,
-                                       _p(kmin), _p(kmax), _stream(stream)), "oasis_build_summaries")
+    _check(lib().oasis_build_summaries(ctypes.byref(d), _arg(kv, w, "kv", _BF16, z.kv, device=False),
+                                       _arg(ctx_len, w, "ctx_len", _I32_T, z.b), first_block, n,
+                                       _arg(kmin, w, "kmin", _BF16, z.summary),
+                                       _arg(kmax, w, "kmax", _BF16, z.summary), _stream(stream)), w)
 
 
 def append_kv(d, k_new, v_new, ctx_len, ctx_len_out, host_kv, kmin, kmax, slot_table, pool, stream=None):
-    _check(lib().oasis_append_kv(ctypes.byref(d), _p(k_new), _p(v_new), _p(ctx_len), _p(ctx_len_out),
-                                 _p(host_kv), _p(kmin), _p(kmax), _p(slot_table), _p(pool),
-                                 _stream(stream)), "oasis_append_kv")
+    w = "oasis_append_kv"
+    z = _Sizes(d, w)
+    _check(lib().oasis_append_kv(ctypes.byref(d), _arg(k_new, w, "k_new", _BF16, z.row),
+                                 _arg(v_new, w, "v_new", _BF16, z.row), _arg(ctx_len, w, "ctx_len", _I32_T, z.b),
+                                 _arg(ctx_len_out, w, "ctx_len_out", _I32_T, z.b, nullable=True),
+                                 _arg(host_kv, w, "host_kv", _BF16, z.kv, device=False),
+                                 _arg(kmin, w, "kmin", _BF16, z.summary), _arg(kmax, w, "kmax", _BF16, z.summary),
+                                 _arg(slot_table, w, "slot_table", _I32_T, z.k), _arg(pool, w, "pool", _BF16, z.pool),
+                                 _stream(stream)), w)
 
 
 def lookahead_scores(d, q, kmin, kmax, ctx_len, scores, stream=None):
-    _check(lib().oasis_lookahead_scores(ctypes.byref(d), _p(q), _p(kmin), _p(kmax), _p(ctx_len),
-                                        _p(scores), _stream(stream)), "oasis_lookahead_scores")
+    w = "oasis_lookahead_scores"
+    z = _Sizes(d, w)
+    _check(lib().oasis_lookahead_scores(ctypes.byref(d), _arg(q, w, "q", _BF16, z.q),
+                                        _arg(kmin, w, "kmin", _BF16, z.summary),
+                                        _arg(kmax, w, "kmax", _BF16, z.summary),
+                                        _arg(ctx_len, w, "ctx_len", _I32_T, z.b),
+                                        _arg(scores, w, "scores", _F32, z.scores), _stream(stream)), w)
 
 
 def select_topk(d, scores, ctx_len, sel, sel_score=None, stream=None):
-    _check(lib().oasis_select_topk(ctypes.byref(d), _p(scores), _p(ctx_len), _p(sel), _p(sel_score),
-                                   _stream(stream)), "oasis_select_topk")
+    w = "oasis_select_topk"
+    z = _Sizes(d, w)
+    _check(lib().oasis_select_topk(ctypes.byref(d), _arg(scores, w, "scores", _F32, z.scores),
+                                   _arg(ctx_len, w, "ctx_len", _I32_T, z.b), _arg(sel, w, "sel", _I32_T, z.k),
+                                   _arg(sel_score, w, "sel_score", _F32, z.k, nullable=True), _stream(stream)), w)
 
 
 def score_select(d, q, kmin, kmax, ctx_len, sel, sel_score, ws, stream=None):
-    _check(lib().oasis_score_select(ctypes.byref(d), _p(q), _p(kmin), _p(kmax), _p(ctx_len), _p(sel),
-                                    _p(sel_score), _p(ws), ws.numel() * ws.element_size(),
-                                    _stream(stream)), "oasis_score_select")
+    w = "oasis_score_select"
+    z = _Sizes(d, w)
+    _check(lib().oasis_score_select(ctypes.byref(d), _arg(q, w, "q", _BF16, z.q),
+                                    _arg(kmin, w, "kmin", _BF16, z.summary), _arg(kmax, w, "kmax", _BF16, z.summary),
+                                    _arg(ctx_len, w, "ctx_len", _I32_T, z.b), _arg(sel, w, "sel", _I32_T, z.k),
+                                    _arg(sel_score, w, "sel_score", _F32, z.k, nullable=True), *_ws(ws, w),
+                                    _stream(stream)), w)
 
 
 def score_select_rows(d, q, row_begin, row_count, kmin, kmax, ctx_len, sel, sel_score, ws, stream=None):
     """Top-K for query rows [row_begin, row_begin + row_count); (0, 1) is the
     verification query alone (exact set / previous-token prediction)."""
-    _check(lib().oasis_score_select_rows(ctypes.byref(d), _p(q), row_begin, row_count, _p(kmin), _p(kmax),
-                                         _p(ctx_len), _p(sel), _p(sel_score), _p(ws),
-                                         ws.numel() * ws.element_size(), _stream(stream)),
-           "oasis_score_select_rows")
+    w = "oasis_score_select_rows"
+    z = _Sizes(d, w)
+    _check(lib().oasis_score_select_rows(ctypes.byref(d), _arg(q, w, "q", _BF16, z.q), row_begin, row_count,
+                                         _arg(kmin, w, "kmin", _BF16, z.summary),
+                                         _arg(kmax, w, "kmax", _BF16, z.summary),
+                                         _arg(ctx_len, w, "ctx_len", _I32_T, z.b), _arg(sel, w, "sel", _I32_T, z.k),
+                                         _arg(sel_score, w, "sel_score", _F32, z.k, nullable=True), *_ws(ws, w),
+                                         _stream(stream)), w)
 
 
 def block_overlap(d, a, b, count, stream=None):
     """count[b][h] = distinct ids of list b also in list a (int32 [B][Hkv][K] each)."""
-    _check(lib().oasis_block_overlap(ctypes.byref(d), _p(a), _p(b), _p(count), _stream(stream)),
-           "oasis_block_overlap")
+    w = "oasis_block_overlap"
+    z = _Sizes(d, w)
+    _check(lib().oasis_block_overlap(ctypes.byref(d), _arg(a, w, "a", _I32_T, z.k), _arg(b, w, "b", _I32_T, z.k),
+                                     _arg(count, w, "count", _I32_T, z.units), _stream(stream)), w)
 
 
 def score_select_noalloc(d, q, kmin, kmax, ctx_len, sel, sel_score=None, stream=None):
     """oasis_score_select without a workspace: for callers that cannot
     allocate or pass device scratch; the scores live in a fixed 4 MiB array
     inside the library (see include/oasis.h for the limit and sharing rules)."""
-    _check(lib().oasis_score_select_noalloc(ctypes.byref(d), _p(q), _p(kmin), _p(kmax), _p(ctx_len), _p(sel),
-                                            _p(sel_score), _stream(stream)), "oasis_score_select_noalloc")
+    w = "oasis_score_select_noalloc"
+    z = _Sizes(d, w)
+    _check(lib().oasis_score_select_noalloc(ctypes.byref(d), _arg(q, w, "q", _BF16, z.q),
+                                            _arg(kmin, w, "kmin", _BF16, z.summary),
+                                            _arg(kmax, w, "kmax", _BF16, z.summary),
+                                            _arg(ctx_len, w, "ctx_len", _I32_T, z.b), _arg(sel, w, "sel", _I32_T, z.k),
+                                            _arg(sel_score, w, "sel_score", _F32, z.k, nullable=True),
+                                            _stream(stream)), w)
 
 
 def plan_fetch(d, sel, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream=None):
-    _check(lib().oasis_plan_fetch(ctypes.byref(d), _p(sel), _p(slot_table), _p(last_used), int(step),
-                                  _p(fetch_slot), _p(fetch_block), _p(n_fetch), _stream(stream)),
-           "oasis_plan_fetch")
+    w = "oasis_plan_fetch"
+    z = _Sizes(d, w)
+    _check(lib().oasis_plan_fetch(ctypes.byref(d), _arg(sel, w, "sel", _I32_T, z.k),
+                                  _arg(slot_table, w, "slot_table", _I32_T, z.k),
+                                  _arg(last_used, w, "last_used", _I32_T, z.k), int(step),
+                                  z.fetch_list(fetch_slot, "fetch_slot"), z.fetch_list(fetch_block, "fetch_block"),
+                                  _arg(n_fetch, w, "n_fetch", _I32_T, z.units), _stream(stream)), w)
 
 
 def plan_fetch_scored(d, sel, scores, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream=None):
     """oasis_plan_fetch with victims ordered by their block's score (lowest first)."""
-    _check(lib().oasis_plan_fetch_scored(ctypes.byref(d), _p(sel), _p(scores), _p(slot_table), _p(last_used),
-                                         int(step), _p(fetch_slot), _p(fetch_block), _p(n_fetch),
-                                         _stream(stream)), "oasis_plan_fetch_scored")
+    w = "oasis_plan_fetch_scored"
+    z = _Sizes(d, w)
+    _check(lib().oasis_plan_fetch_scored(ctypes.byref(d), _arg(sel, w, "sel", _I32_T, z.k),
+                                         _arg(scores, w, "scores", _F32, z.scores),
+                                         _arg(slot_table, w, "slot_table", _I32_T, z.k),
+                                         _arg(last_used, w, "last_used", _I32_T, z.k), int(step),
+                                         z.fetch_list(fetch_slot, "fetch_slot"),
+                                         z.fetch_list(fetch_block, "fetch_block"),
+                                         _arg(n_fetch, w, "n_fetch", _I32_T, z.units), _stream(stream)), w)
 
 
 def plan_fetch_at(d, sel, scores, slot_table, last_used, step, fetch_slot, fetch_block, n_fetch, stream=None):
     """Plan with the step number read on the device from ``step`` (int32
     tensor); LRU victims when ``scores`` is None, score-ordered otherwise."""
-    _check(lib().oasis_plan_fetch_at(ctypes.byref(d), _p(sel), _p(scores), _p(slot_table), _p(last_used), _p(step),
-                                     _p(fetch_slot), _p(fetch_block), _p(n_fetch), _stream(stream)),
-           "oasis_plan_fetch_at")
+    w = "oasis_plan_fetch_at"
+    z = _Sizes(d, w)
+    _check(lib().oasis_plan_fetch_at(ctypes.byref(d), _arg(sel, w, "sel", _I32_T, z.k),
+                                     _arg(scores, w, "scores", _F32, z.scores, nullable=True),
+                                     _arg(slot_table, w, "slot_table", _I32_T, z.k),
+                                     _arg(last_used, w, "last_used", _I32_T, z.k), _arg(step, w, "step", _I32_T, 1),
+                                     z.fetch_list(fetch_slot, "fetch_slot"), z.fetch_list(fetch_block, "fetch_block"),
+                                     _arg(n_fetch, w, "n_fetch", _I32_T, z.units), _stream(stream)), w)
 
 
 def evict_slots(d, mask, slot_table, stream=None):
     """Frees the slots whose mask byte (uint8 [B][Hkv][K]) is set."""
-    _check(lib().oasis_evict_slots(ctypes.byref(d), _p(mask), _p(slot_table), _stream(stream)), "oasis_evict_slots")
+    w = "oasis_evict_slots"
+    z = _Sizes(d, w)
+    _check(lib().oasis_evict_slots(ctypes.byref(d), _arg(mask, w, "mask", _U8, z.k),
+                                   _arg(slot_table, w, "slot_table", _I32_T, z.k), _stream(stream)), w)
 
 
-def make_layer(host_kv, kmin, kmax, pool, slot_table, last_used, sel, sel_score, scores, fetch_slot, fetch_block,
-               n_fetch, out, lse) -> Layer:
-    """oasis_layer from tensors (None for the nullable sel_score / scores)."""
-    return Layer(*[_p(t) for t in (host_kv, kmin, kmax, pool, slot_table, last_used, sel, sel_score, scores,
-                                    fetch_slot, fetch_block, n_fetch, out, lse)])
+def make_layer(d, host_kv, kmin, kmax, pool, slot_table, last_used, sel, sel_score, scores, fetch_slot,
+               fetch_block, n_fetch, out, lse) -> Layer:
+    """oasis_layer from tensors checked against dims `d` (None for the
+    nullable sel_score / scores)."""
+    w = "make_layer"
+    z = _Sizes(d, w)
+    return Layer(_arg(host_kv, w, "host_kv", _BF16, z.kv, device=False), _arg(kmin, w, "kmin", _BF16, z.summary),
+                 _arg(kmax, w, "kmax", _BF16, z.summary), _arg(pool, w, "pool", _BF16, z.pool),
+                 _arg(slot_table, w, "slot_table", _I32_T, z.k), _arg(last_used, w, "last_used", _I32_T, z.k),
+                 _arg(sel, w, "sel", _I32_T, z.k), _arg(sel_score, w, "sel_score", _F32, z.k, nullable=True),
+                 _arg(scores, w, "scores", _F32, z.scores, nullable=True), z.fetch_list(fetch_slot, "fetch_slot"),
+                 z.fetch_list(fetch_block, "fetch_block"), _arg(n_fetch, w, "n_fetch", _I32_T, z.units),
+                 _arg(out, w, "out", _F32, z.out), _arg(lse, w, "lse", _F32, z.lse))
 
 
 def decode_layer_step(d, layer: Layer, q, ctx_len, evict_mask, step, step_dev, scale, ws, sync: StepSync):
-    """One layer's decode step (attention, [loss], scores + top-K, plan, gather) in one call."""
-    _check(lib().oasis_decode_layer_step(ctypes.byref(d), ctypes.byref(layer), _p(q), _p(ctx_len), _p(evict_mask),
-                                         int(step), _p(step_dev), float(scale), _p(ws),
-                                         ws.numel() * ws.element_size(), ctypes.byref(sync)),
-           "oasis_decode_layer_step")
+    """One layer's decode step (attention, [loss], scores + top-K, plan, gather) in one call;
+    `layer` comes from make_layer, which checked its buffers."""
+    w = "oasis_decode_layer_step"
+    z = _Sizes(d, w)
+    _check(lib().oasis_decode_layer_step(ctypes.byref(d), ctypes.byref(layer), _arg(q, w, "q", _BF16, z.q),
+                                         _arg(ctx_len, w, "ctx_len", _I32_T, z.b),
+                                         _arg(evict_mask, w, "evict_mask", _U8, z.k, nullable=True), int(step),
+                                         _arg(step_dev, w, "step_dev", _I32_T, 1, nullable=True), float(scale),
+                                         *_ws(ws, w), ctypes.byref(sync)), w)
 
 
 def step_advance(step, stream=None):
     """step[0] += 1 on the device, in stream order."""
-    _check(lib().oasis_step_advance(_p(step), _stream(stream)), "oasis_step_advance")
+    w = "oasis_step_advance"
+    _check(lib().oasis_step_advance(_arg(step, w, "step", _I32_T, 1), _stream(stream)), w)
 
 
 def prefetch(d, host_kv, fetch_slot, fetch_block, n_fetch, pool, stream=None):
-    _check(lib().oasis_prefetch(ctypes.byref(d), _p(host_kv), _p(fetch_slot), _p(fetch_block),
-                                _p(n_fetch), _p(pool), _stream(stream)), "oasis_prefetch")
+    w = "oasis_prefetch"
+    z = _Sizes(d, w)
+    _check(lib().oasis_prefetch(ctypes.byref(d), _arg(host_kv, w, "host_kv", _BF16, z.kv, device=False),
+                                z.fetch_list(fetch_slot, "fetch_slot"), z.fetch_list(fetch_block, "fetch_block"),
+                                _arg(n_fetch, w, "n_fetch", _I32_T, z.units), _arg(pool, w, "pool", _BF16, z.pool),
+                                _stream(stream)), w)
 
 
 def sparse_attn(d, q, pool, slot_table, ctx_len, scale, out, lse, ws, stream=None):
-    _check(lib().oasis_sparse_attn(ctypes.byref(d), _p(q), _p(pool), _p(slot_table), _p(ctx_len),
-                                   float(scale), _p(out), _p(lse), _p(ws), ws.numel() * ws.element_size(),
-                                   _stream(stream)), "oasis_sparse_attn")
+    w = "oasis_sparse_attn"
+    z = _Sizes(d, w)
+    _check(lib().oasis_sparse_attn(ctypes.byref(d), _arg(q, w, "q", _BF16, z.q), _arg(pool, w, "pool", _BF16, z.pool),
+                                   _arg(slot_table, w, "slot_table", _I32_T, z.k),
+                                   _arg(ctx_len, w, "ctx_len", _I32_T, z.b), float(scale),
+                                   _arg(out, w, "out", _F32, z.out), _arg(lse, w, "lse", _F32, z.lse), *_ws(ws, w),
+                                   _stream(stream)), w)
 
 
 def read_device_error(clear: bool = True, stream=None) -> int:

@@ -218,7 +218,7 @@ class DecodePipeline:
 
     def _native_layer(self, i, L):
         if self._native[i] is None:
-            self._native[i] = make_layer(L.host_kv, L.kmin, L.kmax, L.pool, L.slot_table, L.last_used, L.sel,
+            self._native[i] = make_layer(self.d, L.host_kv, L.kmin, L.kmax, L.pool, L.slot_table, L.last_used, L.sel,
                                          L.sel_score, L.scores if self.victims == "score" else None, L.fetch_slot,
                                          L.fetch_block, L.n_fetch, L.out, L.lse)
         return self._native[i]

@@ -97,3 +97,34 @@ def test_native_layer_step_rejects_missing_streams_and_events(L):
     s.fetch_done = s.plan_ready = s.sel_ready = 2
     s.in_graph = 1
     assert call(ctypes.byref(s)) == lsk.EINVAL and "fork" in lsk.last_error()
+
+
+def test_binding_checks_tensors_before_calling():
+    """The Python binding rejects a tensor that does not fit the call (dtype,
+    layout, size, device) with EINVAL before the library sees a pointer;
+    raw integer addresses are passed through unchecked."""
+    import torch
+    d = _good()
+    B, H, K = d.batch, d.n_kv_heads, d.budget_blocks
+    good = torch.zeros(B * H * K, dtype=torch.int32)
+
+    def err(fn):
+        with pytest.raises(lsk.OasisError) as e:
+            fn()
+        assert e.value.code == lsk.EINVAL
+        return str(e.value)
+
+    # the mask goes in as a raw address (unchecked), so the slot table is the argument under test
+    assert "slot_table must be int32" in err(lambda: lsk.evict_slots(d, 16, good.float()))
+    assert "slot_table must be contiguous" in err(lambda: lsk.evict_slots(d, 16, good.view(B * H, K).t()))
+    assert "slot_table holds" in err(lambda: lsk.evict_slots(d, 16, good[1:]))
+    assert "slot_table must be on a CUDA device" in err(lambda: lsk.evict_slots(d, 16, good))
+    assert "mask holds" in err(lambda: lsk.evict_slots(d, torch.zeros(B * H * K - 1, dtype=torch.uint8), 16))
+    assert "mask is None" in err(lambda: lsk.evict_slots(d, None, good))
+    bad = _good()
+    bad.head_dim = 64
+    assert "head_dim" in err(lambda: lsk.evict_slots(bad, None, None))
+    # a raw address skips the tensor checks; the library then answers for it (NULL slot table)
+    with pytest.raises(lsk.OasisError) as e:
+        lsk.evict_slots(d, 16, 0)
+    assert e.value.code == lsk.EINVAL and "slot_table" in str(e.value)

@@ -62,12 +62,15 @@ def test_score_select_rows_matches_oracle(B, Hq, Hkv, Qn, N, K, rows):
 def test_score_select_rows_rejects_rows_outside_the_step():
     d = lsk.make_dims(batch=1, n_q_heads=8, n_kv_heads=2, max_blocks=64, budget_blocks=16,
                       n_queries=5, fetch_cap=4)
-    t = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    q = torch.zeros((1, 5, 8, 128), dtype=torch.bfloat16, device=DEV)
+    summ = torch.zeros((1, 2, 64, 128), dtype=torch.bfloat16, device=DEV)
+    ctx = torch.full((1,), 64 * 16, dtype=torch.int32, device=DEV)
+    sel = torch.zeros((1, 2, 16), dtype=torch.int32, device=DEV)
     ws = torch.zeros(lsk.workspace_bytes(d), dtype=torch.uint8, device=DEV)
     for rb, rc in [(-1, 1), (0, 0), (4, 2), (5, 1)]:
         with pytest.raises(lsk.OasisError) as e:
-            lsk.score_select_rows(d, t, rb, rc, t, t, t, t, None, ws)
-        assert e.value.code == lsk.EINVAL
+            lsk.score_select_rows(d, q, rb, rc, summ, summ, ctx, sel, None, ws)
+        assert e.value.code == lsk.EINVAL and "query rows" in str(e.value)
 
 
 @pytest.mark.parametrize("B,Hkv,N,K,seed", [(2, 3, 50, 20, 0), (4, 8, 2048, 128, 1), (1, 2, 32768, 1024, 2),

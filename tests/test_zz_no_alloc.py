@@ -49,6 +49,7 @@ def test_noalloc_score_select_matches_workspace_version_twice():
 
     too_big = lsk.make_dims(batch=64, n_q_heads=32, n_kv_heads=8, max_blocks=4096, budget_blocks=64,
                             n_queries=Qn, fetch_cap=8)
-    with pytest.raises(lsk.OasisError) as e:
-        lsk.score_select_noalloc(too_big, q, kmin, kmax, contexts[0], sel_na, sc_na)
+    with pytest.raises(lsk.OasisError) as e:     # raw addresses: the library's own size check answers
+        lsk.score_select_noalloc(too_big, q.data_ptr(), kmin.data_ptr(), kmax.data_ptr(), contexts[0].data_ptr(),
+                                 sel_na.data_ptr(), sc_na.data_ptr())
     assert e.value.code == lsk.EINVAL and "scratch" in str(e.value)
