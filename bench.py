@@ -975,112 +975,108 @@ def emit_gpu(args, res, world):
 
 
 # -------------------------------------------------------------- oracle
-class OracleUnit:
-    """The CPU oracle driving one (sequence, KV head) unit through decode
-    layer-steps: attention over its pool, scores, top-K, plan, gather."""
-
-    def __init__(self, w, host_bits):
-        import numpy as np
-
-        import oracle as O
-        self.O, self.np, self.w = O, np, w
-        self.host_bits = host_bits                          # uint16 [1, 1, N, 2, P, D]
-        kv = O.bf16_bits_to_f64(host_bits)
-        self.keys, self.vals = kv[:, :, :, 0], kv[:, :, :, 1]
-        self.ctx = np.array([w.context], dtype=np.int64)
-        self.kmin, self.kmax = O.block_summaries(self.keys, self.ctx)   # admission, not timed
-        K, P, D = w.budget_blocks, w.block_tokens, w.head_dim
-        self.st = np.full((1, 1, K), -1, np.int32)
-        self.lu = np.full((1, 1, K), -1, np.int32)
-        self.pool_k = np.zeros((1, 1, K, P, D))
-        self.pool_v = np.zeros((1, 1, K, P, D))
-        self.scale = 1.0 / math.sqrt(D)
-
-    def step(self, q, t, attend=True):
-        O, w = self.O, self.w
-        if attend:
-            O.sparse_attention(q, self.pool_k, self.pool_v, self.st, self.ctx, self.scale)
-        sc = O.lookahead_scores(q, self.kmin, self.kmax, self.ctx, w.block_tokens)
-        sel, _ = O.select_topk(sc, self.ctx, w.budget_blocks, w.block_tokens)
-        plan = O.plan_fetch(sel, self.st, self.lu, t, w.fetch_cap)
-        self.pool_k = O.prefetch(self.keys, self.pool_k, plan["fetch_slot"], plan["fetch_block"], plan["n_fetch"])
-        self.pool_v = O.prefetch(self.vals, self.pool_v, plan["fetch_slot"], plan["fetch_block"], plan["n_fetch"])
-        self.st, self.lu = plan["slot_table"], plan["last_used"]
+def oracle_cfg(w) -> dict:
+    """The workload fields the oracle's per-unit driver needs."""
+    return {"context": w.context, "block_tokens": w.block_tokens, "budget_blocks": w.budget_blocks,
+            "head_dim": w.head_dim, "fetch_cap": w.fetch_cap}
 
 
-def time_oracle(w, unit_bits, unit_queries, fill_steps, timed_steps):
-    """Seconds per decode layer-step per unit, BLAS limited to one thread.
-    unit_bits: list of host-KV bit arrays of single units; unit_queries:
-    list (per unit) of per-step float64 queries [1, Qn, G, D]."""
-    try:
-        from threadpoolctl import threadpool_limits
-        lim = threadpool_limits(limits=1)
-    except ImportError:                       # pragma: no cover
-        lim = None
-    times = []
-    try:
-        for bits, qs in zip(unit_bits, unit_queries):
-            u = OracleUnit(w, bits)
-            u.step(qs[0], 0, attend=False)                  # priming
-            for i in range(1, fill_steps + 1):
-                u.step(qs[i % len(qs)], i)
-            for i in range(fill_steps + 1, fill_steps + 1 + timed_steps):
-                t0 = time.perf_counter()
-                u.step(qs[i % len(qs)], i)
-                times.append(time.perf_counter() - t0)
-    finally:
-        if lim is not None:
-            lim.__exit__(None, None, None)
-    return sum(times) / len(times), len(times)
-
-
-def cpu_baseline(w, res, n_units=6, fill_steps=8, timed_steps=24):
+def cpu_baseline(w, res, n_units=6, fill_steps=8, timed_steps=24, par_fill=4, par_timed=8):
     """The oracle, as it stands, on this host's cores, on a sample of the
-    benchmarked workload: a few (sequence, KV head) units of the same KV and
-    queries, layer-steps/s scaled to the whole batch."""
+    benchmarked workload (the same KV and queries), in layer-steps/s of the
+    whole batch: on one core (a few units one after another) and on all
+    usable cores (one unit per core, all at once).  `value` is the all-cores
+    figure when that run succeeds, else the one-core figure."""
     import numpy as np
 
     import oracle as O
+    from oracle import decode_timing as T
     L = res["layer"]
     G = w.group
-    rng = np.random.default_rng(0)
-    units = [(int(rng.integers(w.batch)), int(rng.integers(w.n_kv_heads))) for _ in range(n_units)]
-    qs_all = [O.bf16_bits_to_f64(W.bf16_bits(q)) for q in res["queries"][: fill_steps + timed_steps + 1]]
-    bits = [W.bf16_bits(L.host_kv[b:b + 1, h:h + 1]) for b, h in units]
-    uq = [[q[b:b + 1, :, h * G:(h + 1) * G] for q in qs_all] for b, h in units]
-    per_unit, n = time_oracle(w, bits, uq, fill_steps, timed_steps)
     total_units = w.batch * w.n_kv_heads
-    return {"value": 1.0 / (per_unit * total_units), "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} unit-steps ({n_units} (sequence, KV head) units x {timed_steps} decode layer-steps "
-                      f"after {fill_steps} untimed fill steps): attention, scores, top-K, plan, gather; "
-                      f"per-unit mean scaled to the {total_units} units of the batch; numpy fp64, BLAS 1 thread"}
+    qs_all = [O.bf16_bits_to_f64(W.bf16_bits(q)) for q in res["queries"][: fill_steps + timed_steps + 1]]
+
+    def unit(b, h, steps):
+        return W.bf16_bits(L.host_kv[b:b + 1, h:h + 1]), [q[b:b + 1, :, h * G:(h + 1) * G] for q in qs_all[:steps]]
+
+    rng = np.random.default_rng(0)
+    picks = [(int(rng.integers(w.batch)), int(rng.integers(w.n_kv_heads))) for _ in range(n_units)]
+    times = []
+    for b, h in picks:
+        bits, qs = unit(b, h, fill_steps + timed_steps + 1)
+        times += T.run_unit(oracle_cfg(w), bits, qs, fill_steps, timed_steps)
+    one = 1.0 / (sum(times) / len(times) * total_units)
+    single = {"value": one, "unit": "layer-steps/s", "cores": 1,
+              "sample": f"{len(times)} unit-steps ({n_units} (sequence, KV head) units x {timed_steps} decode "
+                        f"layer-steps after {fill_steps} untimed fill steps) one after another; per-unit mean "
+                        f"scaled to the {total_units} units of the batch"}
+    line = {"value": one, "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
+            "sample": single["sample"] + "; numpy fp64, BLAS 1 thread", "single_core": single,
+            "nproc": os.cpu_count(), "usable_cores": T.usable_cores(), "cpu_model": T.cpu_model()}
+    workers = max(1, min(T.usable_cores(), 64, total_units))          # one process (≈0.2 GB) per unit
+    try:
+        flat = [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+        order = rng.permutation(len(flat))[:workers]
+        units = [unit(*flat[i], par_fill + par_timed + 1) for i in order]
+        per_unit = T.run_units_parallel(oracle_cfg(w), units, par_fill, par_timed, workers, timeout_s=300.0)
+        rate = sum(len(t) / sum(t) for t in per_unit)                 # unit-steps/s, all cores together
+        line.update({"value": rate / total_units, "cores": workers,
+                     "sample": f"{workers} (sequence, KV head) units, one per core, started together, each "
+                               f"{par_timed} timed decode layer-steps after {par_fill} untimed fill steps; the "
+                               f"sum of the units' step rates scaled to the {total_units} units of the batch; "
+                               f"numpy fp64, BLAS 1 thread per process"})
+    except Exception as e:                                            # one core stays the baseline
+        line["all_cores_error"] = f"{type(e).__name__}: {e}"[:200]
+    return line
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle on this host, same workload, metric and
-    unit; each step is one (sequence, KV head) unit's decode layer-step,
-    scaled to the whole batch."""
+    """--impl reference: the CPU oracle on this host's cores, same workload,
+    metric and unit.  Each step is one decode layer-step of P (sequence, KV
+    head) units of the benchmarked workload at once, one per core (P = the
+    usable cores, at most 64), timed by the wall clock and scaled to the
+    whole batch and the layers of a step; one core if that cannot run."""
     import oracle as O
+    from oracle import decode_timing as T
     w = W.WORKLOADS[WORKLOAD]
-    wu = w.with_(batch=1, n_kv_heads=1, n_q_heads=w.group)
+    total_units = w.batch * w.n_kv_heads
+    P = max(1, min(T.usable_cores(), 64, total_units))
+    wu = w.with_(batch=-(-P // w.n_kv_heads))
     kv = W.make_host_kv(wu, 0, "cpu")
     qs = W.QueryStream(wu, 0, "cpu")
-    fill = 8
-    queries = [O.bf16_bits_to_f64(W.bf16_bits(qs.next())) for _ in range(fill + args.warmup + args.steps + 1)]
-    per_unit, n = time_oracle(wu, [W.bf16_bits(kv)], [queries], fill + args.warmup, args.steps)
-    units = w.batch * w.n_kv_heads
-    value = 1.0 / (per_unit * units)
-    sample = (f"each step: one (sequence, KV head) unit's decode layer-step (attention, scores, top-K, plan, "
-              f"gather), scaled to the {units} units of the batch and the {args.layers} layers of a step; "
-              f"numpy fp64, BLAS 1 thread")
+    ring = [O.bf16_bits_to_f64(W.bf16_bits(qs.next())) for _ in range(48)]   # walked in order, then again
+    G, fill = w.group, 8
+    units = []
+    for k in range(P):
+        b, h = divmod(k, w.n_kv_heads)
+        units.append((W.bf16_bits(kv[b:b + 1, h:h + 1]), [q[b:b + 1, :, h * G:(h + 1) * G] for q in ring]))
+    what = ("decode layer-step (attention, scores, top-K, plan, gather) of the 32K Llama-shaped layer, scaled to "
+            f"the {total_units} units of the batch and the {args.layers} layers of a step; numpy fp64, BLAS 1 "
+            "thread per process")
+    try:
+        with T.UnitPool(oracle_cfg(wu), units, fill, timeout_s=300.0) as pool:
+            for _ in range(args.warmup):
+                pool.step()
+            walls = [pool.step()[0] for _ in range(args.steps)]
+        unit_steps_per_s = P / (sum(walls) / len(walls))
+        cores = P
+        sample = (f"each step: {P} (sequence, KV head) units, one process per core, each doing one " + what +
+                  "; wall clock per step")
+    except Exception as e:                                            # one core
+        times = T.run_unit(oracle_cfg(wu), units[0][0], units[0][1], fill + args.warmup, args.steps)
+        unit_steps_per_s = len(times) / sum(times)
+        cores = 1
+        sample = (f"each step: one (sequence, KV head) unit's " + what +
+                  f" (the all-cores run failed: {type(e).__name__})")
+    value = unit_steps_per_s / total_units
     line = {
         "impl": "reference",
         "metric": METRIC,
         "value": value, "unit": "layer-steps/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_unit * units * args.layers * 1e3, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": args.layers / value * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
         "config": headline_config(w, args.layers, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "layer-steps/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "layer-steps/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

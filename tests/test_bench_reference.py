@@ -37,3 +37,26 @@ def test_reference_on_nonzero_ranks_prints_nothing():
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2"], cwd=ROOT,
                        capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_cpu_baseline_times_one_core_and_all_cores():
+    """The GPU arm's cpu_baseline on a small workload, driven on the CPU:
+    a one-core figure, an all-cores figure from spawned processes (one unit
+    per usable core), and the host it ran on."""
+    from oracle import decode_timing as T
+    W = bench.W
+    w = W.WORKLOADS["llama8b_32k"].with_(batch=2, n_q_heads=8, n_kv_heads=2, context=1024, max_blocks=64,
+                                          budget_blocks=16, fetch_cap=4)
+
+    class _Layer:
+        host_kv = W.make_host_kv(w, 0, "cpu")
+
+    qs = W.QueryStream(w, 0, "cpu")
+    res = {"layer": _Layer(), "queries": [qs.next() for _ in range(12)]}
+    line = bench.cpu_baseline(w, res, n_units=2, fill_steps=2, timed_steps=3, par_fill=1, par_timed=2)
+    assert "all_cores_error" not in line, line.get("all_cores_error")
+    assert line["kind"] == "oracle" and line["unit"] == "layer-steps/s" and line["value"] > 0
+    workers = min(T.usable_cores(), 64, w.batch * w.n_kv_heads)
+    assert line["cores"] == workers and line["usable_cores"] == T.usable_cores()
+    assert line["single_core"]["cores"] == 1 and line["single_core"]["value"] > 0
+    assert line["nproc"] >= 1 and line["cpu_model"]
