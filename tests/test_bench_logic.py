@@ -102,3 +102,24 @@ def test_gpu_line_keeps_the_contract(capsys):
     assert e["d2h_bytes_per_step"] == nl * (w.batch * w.n_queries * w.n_q_heads * (w.head_dim + 1) * 4)
     assert d["gpu_launches"] == 6 * steps * nl
     assert d["kernels_isolated"]["sparse_attn"]["bound"] == "hbm"
+
+
+def test_clock_summary_from_sampled_lines():
+    """The clocks record of the bench line, from nvidia-smi rows as
+    `--format=csv,noheader,nounits` prints them: median and max SM clock, and
+    every throttle reason seen Active in any row; malformed rows are skipped."""
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "1965, 1965, 250.31, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1950, 1965, 612.02, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1965, 1965, 640.77, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "[N/A], 1965, 600.00, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage",
+        "",
+    ]
+    s = c.summary()
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    c.lines = ["1200, 1965, 900.0, 0x8, Active, Not Active, Active, Not Active"]
+    assert c.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    c.lines = []
+    assert c.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
