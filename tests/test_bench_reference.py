@@ -60,3 +60,34 @@ def test_cpu_baseline_times_one_core_and_all_cores():
     assert line["cores"] == workers and line["usable_cores"] == T.usable_cores()
     assert line["single_core"]["cores"] == 1 and line["single_core"]["value"] > 0
     assert line["nproc"] >= 1 and line["cpu_model"]
+
+
+def test_timing_harness_runs_the_oracles_decode_path():
+    """The unit driver the CPU baseline and the reference arm time walks the
+    same decode path as the oracle's own multi-step function: after priming
+    and 5 steps its slot table, recency and pool are identical."""
+    import numpy as np
+
+    import oracle as O
+    from oracle import decode_timing as T
+    W = bench.W
+    w = W.WORKLOADS["llama8b_32k"].with_(batch=1, n_q_heads=4, n_kv_heads=1, context=64 * 16 - 7, max_blocks=64,
+                                          budget_blocks=16, fetch_cap=4)
+    bits = W.bf16_bits(W.make_host_kv(w, 0, "cpu"))
+    qs = W.QueryStream(w, 0, "cpu")
+    queries = [O.bf16_bits_to_f64(W.bf16_bits(qs.next())) for _ in range(6)]
+    u = T.OracleUnit(bench.oracle_cfg(w), bits)
+    u.step(queries[0], 0, attend=False)
+    for t in range(1, 6):
+        u.step(queries[t], t)
+    kv = O.bf16_bits_to_f64(bits)
+    keys, vals = kv[:, :, :, 0], kv[:, :, :, 1]
+    ctx = np.array([w.context])
+    kmin, kmax = O.block_summaries(keys, ctx)
+    _, st, lu = O.decode_layer_steps(keys, vals, kmin, kmax, ctx, queries[0], queries[1:], w.budget_blocks,
+                                     w.fetch_cap, 1 / np.sqrt(128))
+    np.testing.assert_array_equal(u.st, st)
+    np.testing.assert_array_equal(u.lu, lu)
+    assert (st >= 0).sum() == w.budget_blocks                      # the pool filled up
+    for s in range(w.budget_blocks):
+        np.testing.assert_array_equal(u.pool_k[0, 0, s], keys[0, 0, st[0, 0, s]])
