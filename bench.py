@@ -121,17 +121,64 @@ def max_over_ranks(x: float) -> float:
     return float(t.item())
 
 
-def build_workload_state(w, steps: int, device="cuda", n_queries: int | None = None, layers: int = 1):
+def _available_host_bytes():
+    """Bytes this process may still take: MemAvailable, capped by the
+    container's cgroup memory limit (v2 or v1) when one is set; None if
+    neither can be read."""
+    vals = []
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    vals.append(int(line.split()[1]) * 1024)
+    except (OSError, ValueError, IndexError):
+        pass
+    for lim_p, cur_p in (("/sys/fs/cgroup/memory.max", "/sys/fs/cgroup/memory.current"),
+                         ("/sys/fs/cgroup/memory/memory.limit_in_bytes", "/sys/fs/cgroup/memory/memory.usage_in_bytes")):
+        try:
+            with open(lim_p) as f:
+                lim = f.read().strip()
+            with open(cur_p) as f:
+                cur = int(f.read().strip())
+            if lim.isdigit() and int(lim) < (1 << 60):
+                vals.append(int(lim) - cur)
+        except (OSError, ValueError):
+            pass
+    return min(vals) if vals else None
+
+
+def host_kv_layers(w, layers: int, local_ranks: int, reserve_gib: float = 4.0, avail=None) -> int:
+    """Distinct host-KV layers one rank pins: all `layers` when the host's
+    available memory holds them for every rank on the node plus a reserve,
+    else as many as fit (at least one).  Layer l then reads the host KV of
+    layer l mod that number: the same bytes cross PCIe per layer-step, only
+    fewer distinct gigabytes sit in host memory."""
+    per_layer = w.batch * w.n_kv_heads * w.max_blocks * w.block_bytes
+    if avail is None:
+        avail = _available_host_bytes()
+    if avail is None:
+        return layers
+    per_rank = avail / max(1, local_ranks) - reserve_gib * (1 << 30)
+    return max(1, min(layers, int(per_rank // per_layer)))
+
+
+def build_workload_state(w, steps: int, device="cuda", n_queries: int | None = None, layers: int = 1,
+                         host_layers: int | None = None):
     """Pinned host KV, per-layer device state, pipeline and resident queries
-    for `layers` layers of workload `w` (layer l draws its own KV and queries)."""
+    for `layers` layers of workload `w` (layer l draws its own queries; its KV
+    is its own when l < host_layers, else layer l mod host_layers's)."""
     d = lsk.dims_for(w)
     states, qrings, hosts = [], [], []
     nq = n_queries if n_queries is not None else min(QUERY_RING, max(steps, 1))
+    host_layers = layers if host_layers is None else max(1, min(layers, host_layers))
     for l in range(layers):
-        host = torch.empty((w.batch, w.n_kv_heads, w.max_blocks, 2, w.block_tokens, w.head_dim),
-                           dtype=torch.bfloat16, pin_memory=True)
-        W.make_host_kv(w, layer=l, device=device, out=host)
-        torch.cuda.synchronize()
+        if l < host_layers:
+            host = torch.empty((w.batch, w.n_kv_heads, w.max_blocks, 2, w.block_tokens, w.head_dim),
+                               dtype=torch.bfloat16, pin_memory=True)
+            W.make_host_kv(w, layer=l, device=device, out=host)
+            torch.cuda.synchronize()
+        else:
+            host = hosts[l % host_layers]
         states.append(LayerState(d, host, device))
         qs = W.QueryStream(w, l, device)
         qrings.append([qs.next() for _ in range(max(nq, 1))])
@@ -731,8 +778,13 @@ def run_deep(args, device):
 
 def run_gpu(args, rank, world, device):
     w = rank_workload(rank)
+    try:
+        host_layers = host_kv_layers(w, args.layers, int(os.environ.get("LOCAL_WORLD_SIZE", world)))
+    except Exception:                                   # no estimate: one host KV per layer, as asked
+        host_layers = args.layers
     st = build_workload_state(w, args.warmup + args.steps, device, n_queries=args.query_ring,
-                              layers=args.layers)
+                              layers=args.layers, host_layers=host_layers)
+    st["host_layers"] = host_layers
     d, layers, pipe, qrings = st["dims"], st["layers"], st["pipe"], st["qrings"]
     nl, nq = len(layers), len(qrings[0])
     timer = KernelTimer(args.steps * nl)
@@ -842,7 +894,8 @@ def run_gpu(args, rank, world, device):
     err = lsk.read_device_error(clear=True)
     return {"w": w, "d": d, "ms": ms, "host_ms": host_ms, "host_cost_ms": min(host_cost), "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
             "e2e_ms": e2e_ms, "e2e_steps": e2e_steps, "h2d": h2d, "clocks": clk.summary(), "dev_err": err,
-            "layer": layers[0], "layers": layers, "queries": qrings[0], "iso": iso}
+            "layer": layers[0], "layers": layers, "queries": qrings[0], "iso": iso,
+            "host_layers": st["host_layers"]}
 
 
 def algorithmic_bytes(w, fetched_blocks_per_layer_step):
@@ -964,6 +1017,7 @@ def emit_gpu(args, res, world):
                         "back as soon as that layer is done, the host waiting for the last read-back before the "
                         "next step; h2d bytes include the zero-copy gather of fetched blocks"},
         "gpu_launches": 6 * layer_steps,   # attention, merge, score, select, plan, gather
+        "host_kv_layers": res.get("host_layers", nl),   # distinct pinned host KV per rank (layer l -> l mod this)
         "host_enqueue_ms_per_step": res["host_ms"] / args.steps,
         "host_cost_ms_per_step": res["host_cost_ms"],
         "clocks": res["clocks"],

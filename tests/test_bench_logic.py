@@ -101,6 +101,7 @@ def test_gpu_line_keeps_the_contract(capsys):
     assert e["unit"] == d["unit"] and e["h2d_bytes_per_step"] > nl * 1583 * w.block_bytes
     assert e["d2h_bytes_per_step"] == nl * (w.batch * w.n_queries * w.n_q_heads * (w.head_dim + 1) * 4)
     assert d["gpu_launches"] == 6 * steps * nl
+    assert d["host_kv_layers"] == nl
     assert d["kernels_isolated"]["sparse_attn"]["bound"] == "hbm"
 
 
@@ -123,3 +124,21 @@ def test_clock_summary_from_sampled_lines():
     assert c.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     c.lines = []
     assert c.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_host_kv_layers_fit_the_node(monkeypatch):
+    """Distinct pinned host-KV layers per rank (2 GiB each for the 32K Llama
+    layer): all of them when memory allows, fewer on a tight node, never 0,
+    and all of them when the host's memory cannot be read."""
+    w = W.WORKLOADS["llama8b_32k"]
+    gib = 1 << 30
+    assert w.batch * w.n_kv_heads * w.max_blocks * w.block_bytes == 2 * gib
+    assert bench.host_kv_layers(w, 8, 1, avail=64 * gib) == 8
+    assert bench.host_kv_layers(w, 8, 8, avail=1024 * gib) == 8
+    assert bench.host_kv_layers(w, 8, 8, avail=100 * gib) == 4          # 12.5 - 4 GiB per rank
+    assert bench.host_kv_layers(w, 8, 8, avail=10 * gib) == 1
+    monkeypatch.setattr(bench, "_available_host_bytes", lambda: None)
+    assert bench.host_kv_layers(w, 8, 8) == 8
+    monkeypatch.undo()
+    got = bench._available_host_bytes()
+    assert got is None or got > 0
