@@ -142,3 +142,44 @@ def test_host_kv_layers_fit_the_node(monkeypatch):
     monkeypatch.undo()
     got = bench._available_host_bytes()
     assert got is None or got > 0
+
+
+def test_workload_state_aliases_host_kv_past_the_distinct_layers(monkeypatch):
+    """build_workload_state with fewer distinct host-KV layers than layers:
+    only that many pinned buffers are made, layer l holds buffer l mod L, and
+    every layer keeps queries of its own (device parts stubbed)."""
+    import torch
+    pinned = []
+    real_empty = torch.empty
+
+    def empty(*a, pin_memory=False, **k):
+        t = real_empty(*a, **k)
+        if pin_memory:
+            pinned.append(t)
+        return t
+
+    class Layer:
+        def __init__(self, d, host, device):
+            self.host_kv = host
+
+    class Pipe:
+        def __init__(self, d, states, ctx, scale, device):
+            self.states = states
+
+        def build_summaries(self):
+            pass
+
+    monkeypatch.setattr(bench, "LayerState", Layer)
+    monkeypatch.setattr(bench, "DecodePipeline", Pipe)
+    monkeypatch.setattr(bench.torch, "empty", empty)
+    monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda *a, **k: None)
+    w = W.WORKLOADS["llama8b_32k"].with_(batch=1, n_q_heads=8, n_kv_heads=2, context=256, max_blocks=16,
+                                          budget_blocks=8, fetch_cap=2)
+    st = bench.build_workload_state(w, 3, device="cpu", n_queries=2, layers=5, host_layers=2)
+    hosts = [L.host_kv for L in st["layers"]]
+    assert len(pinned) == 2
+    assert all(hosts[l] is pinned[l % 2] for l in range(5))
+    assert not torch.equal(pinned[0], pinned[1])                       # distinct layers draw distinct KV
+    assert len(st["qrings"]) == 5 and not torch.equal(st["qrings"][0][0], st["qrings"][2][0])
+    st = bench.build_workload_state(w, 3, device="cpu", n_queries=2, layers=3)
+    assert len(pinned) == 5                                            # default: one host KV per layer
