@@ -147,6 +147,43 @@ def _available_host_bytes():
     return min(vals) if vals else None
 
 
+def parse_cpulist(text: str) -> set:
+    """CPU numbers of a Linux cpulist string such as "0-31,64-95"."""
+    cpus = set()
+    for part in text.strip().split(","):
+        if not part:
+            continue
+        lo, _, hi = part.partition("-")
+        cpus.update(range(int(lo), int(hi or lo) + 1))
+    return cpus
+
+
+def gpu_local_cpus(domain: int, bus: int, dev: int, sysfs: str = "/sys/bus/pci/devices"):
+    """The CPUs the kernel lists as local to the PCI device domain:bus:dev.0
+    (its NUMA node's), or None when sysfs does not say."""
+    try:
+        with open(os.path.join(sysfs, f"{domain:04x}:{bus:02x}:{dev:02x}.0", "local_cpulist")) as f:
+            return parse_cpulist(f.read())
+    except (OSError, ValueError):
+        return None
+
+
+def bind_near_gpu(device):
+    """Restricts this process to the allowed CPUs local to its GPU, so that
+    the pinned host KV it allocates next lands in that GPU's NUMA node (first
+    touch) and its gathers do not cross the socket interconnect.  Returns the
+    number of CPUs kept, or None when nothing was changed."""
+    try:
+        p = torch.cuda.get_device_properties(device)
+        cpus = (gpu_local_cpus(p.pci_domain_id, p.pci_bus_id, p.pci_device_id) or set()) & os.sched_getaffinity(0)
+        if not cpus:
+            return None
+        os.sched_setaffinity(0, cpus)
+        return len(cpus)
+    except Exception:
+        return None
+
+
 def host_kv_layers(w, layers: int, local_ranks: int, reserve_gib: float = 4.0, avail=None) -> int:
     """Distinct host-KV layers one rank pins: all `layers` when the host's
     available memory holds them for every rank on the node plus a reserve,
@@ -1018,6 +1055,7 @@ def emit_gpu(args, res, world):
                         "next step; h2d bytes include the zero-copy gather of fetched blocks"},
         "gpu_launches": 6 * layer_steps,   # attention, merge, score, select, plan, gather
         "host_kv_layers": res.get("host_layers", nl),   # distinct pinned host KV per rank (layer l -> l mod this)
+        "cpus_bound": res.get("cpus_bound"),   # rank 0's CPUs local to its GPU (multi-rank runs), else null
         "host_enqueue_ms_per_step": res["host_ms"] / args.steps,
         "host_cost_ms_per_step": res["host_cost_ms"],
         "clocks": res["clocks"],
@@ -1172,11 +1210,14 @@ def main():
             if rank == 0:
                 fn(args, device)
             return
+    bound = None
     if world > 1:
         import datetime
+        bound = bind_near_gpu(device)                    # before any pinned host memory is allocated
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     try:
         res = run_gpu(args, rank, world, device)
+        res["cpus_bound"] = bound
         if rank == 0:
             emit_gpu(args, res, world)
     finally:

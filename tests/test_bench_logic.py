@@ -101,7 +101,7 @@ def test_gpu_line_keeps_the_contract(capsys):
     assert e["unit"] == d["unit"] and e["h2d_bytes_per_step"] > nl * 1583 * w.block_bytes
     assert e["d2h_bytes_per_step"] == nl * (w.batch * w.n_queries * w.n_q_heads * (w.head_dim + 1) * 4)
     assert d["gpu_launches"] == 6 * steps * nl
-    assert d["host_kv_layers"] == nl
+    assert d["host_kv_layers"] == nl and d["cpus_bound"] is None
     assert d["kernels_isolated"]["sparse_attn"]["bound"] == "hbm"
 
 
@@ -183,3 +183,14 @@ def test_workload_state_aliases_host_kv_past_the_distinct_layers(monkeypatch):
     assert len(st["qrings"]) == 5 and not torch.equal(st["qrings"][0][0], st["qrings"][2][0])
     st = bench.build_workload_state(w, 3, device="cpu", n_queries=2, layers=3)
     assert len(pinned) == 5                                            # default: one host KV per layer
+
+
+def test_cpulist_and_gpu_local_cpus(tmp_path):
+    """The CPUs local to a GPU, from a sysfs-shaped tree."""
+    assert bench.parse_cpulist("0-3,8,10-11\n") == {0, 1, 2, 3, 8, 10, 11}
+    assert bench.parse_cpulist("5") == {5}
+    dev = tmp_path / "0000:1b:00.0"
+    dev.mkdir()
+    (dev / "local_cpulist").write_text("0-27,56-83\n")
+    assert bench.gpu_local_cpus(0, 0x1B, 0, str(tmp_path)) == set(range(28)) | set(range(56, 84))
+    assert bench.gpu_local_cpus(0, 0x1C, 0, str(tmp_path)) is None
