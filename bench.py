@@ -121,27 +121,42 @@ def max_over_ranks(x: float) -> float:
     return float(t.item())
 
 
+MEMINFO = "/proc/meminfo"
+CGROUP_V2, CGROUP_V1 = "/sys/fs/cgroup", "/sys/fs/cgroup/memory"
+
+
 def _available_host_bytes():
     """Bytes this process may still take: MemAvailable, capped by the
     container's cgroup memory limit (v2 or v1) when one is set; None if
     neither can be read."""
     vals = []
     try:
-        with open("/proc/meminfo") as f:
+        with open(MEMINFO) as f:
             for line in f:
                 if line.startswith("MemAvailable:"):
                     vals.append(int(line.split()[1]) * 1024)
     except (OSError, ValueError, IndexError):
         pass
-    for lim_p, cur_p in (("/sys/fs/cgroup/memory.max", "/sys/fs/cgroup/memory.current"),
-                         ("/sys/fs/cgroup/memory/memory.limit_in_bytes", "/sys/fs/cgroup/memory/memory.usage_in_bytes")):
+    for base, lim_f, cur_f, cache_key in ((CGROUP_V2, "memory.max", "memory.current", "inactive_file"),
+                                          (CGROUP_V1, "memory.limit_in_bytes", "memory.usage_in_bytes",
+                                           "total_inactive_file")):
         try:
-            with open(lim_p) as f:
+            with open(os.path.join(base, lim_f)) as f:
                 lim = f.read().strip()
-            with open(cur_p) as f:
+            with open(os.path.join(base, cur_f)) as f:
                 cur = int(f.read().strip())
-            if lim.isdigit() and int(lim) < (1 << 60):
-                vals.append(int(lim) - cur)
+            if not (lim.isdigit() and int(lim) < (1 << 60)):
+                continue
+            cache = 0                                   # reclaimable page cache counts as free
+            try:
+                with open(os.path.join(base, "memory.stat")) as f:
+                    for line in f:
+                        k, _, v = line.partition(" ")
+                        if k == cache_key:
+                            cache = int(v)
+            except (OSError, ValueError):
+                pass
+            vals.append(int(lim) - max(0, cur - cache))
         except (OSError, ValueError):
             pass
     return min(vals) if vals else None

@@ -194,3 +194,31 @@ def test_cpulist_and_gpu_local_cpus(tmp_path):
     (dev / "local_cpulist").write_text("0-27,56-83\n")
     assert bench.gpu_local_cpus(0, 0x1B, 0, str(tmp_path)) == set(range(28)) | set(range(56, 84))
     assert bench.gpu_local_cpus(0, 0x1C, 0, str(tmp_path)) is None
+
+
+def test_available_host_bytes_reads_meminfo_and_cgroup_limits(tmp_path, monkeypatch):
+    """MemAvailable, capped by a cgroup limit less the cgroup's use without
+    its reclaimable page cache; an unlimited cgroup does not cap."""
+    gib = 1 << 30
+    mi = tmp_path / "meminfo"
+    mi.write_text(f"MemTotal: {512 * gib // 1024} kB\nMemAvailable:   {400 * gib // 1024} kB\n")
+    v2, v1 = tmp_path / "v2", tmp_path / "v1"
+    v2.mkdir()
+    v1.mkdir()
+    monkeypatch.setattr(bench, "MEMINFO", str(mi))
+    monkeypatch.setattr(bench, "CGROUP_V2", str(v2))
+    monkeypatch.setattr(bench, "CGROUP_V1", str(v1))
+    assert bench._available_host_bytes() == 400 * gib                   # no cgroup files
+    (v2 / "memory.max").write_text("max\n")
+    (v2 / "memory.current").write_text(f"{10 * gib}\n")
+    assert bench._available_host_bytes() == 400 * gib                   # unlimited
+    (v2 / "memory.max").write_text(f"{64 * gib}\n")
+    (v2 / "memory.stat").write_text(f"anon {6 * gib}\ninactive_file {4 * gib}\nactive_file 0\n")
+    assert bench._available_host_bytes() == 64 * gib - 6 * gib          # 10 used, 4 of it reclaimable
+    (v1 / "memory.limit_in_bytes").write_text(f"{32 * gib}\n")
+    (v1 / "memory.usage_in_bytes").write_text(f"{2 * gib}\n")
+    assert bench._available_host_bytes() == 30 * gib                    # the tightest limit wins
+    monkeypatch.setattr(bench, "MEMINFO", str(tmp_path / "missing"))
+    (v1 / "memory.limit_in_bytes").unlink()
+    (v2 / "memory.max").unlink()
+    assert bench._available_host_bytes() is None
