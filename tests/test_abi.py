@@ -128,3 +128,35 @@ def test_binding_checks_tensors_before_calling():
     with pytest.raises(lsk.OasisError) as e:
         lsk.evict_slots(d, 16, 0)
     assert e.value.code == lsk.EINVAL and "slot_table" in str(e.value)
+
+
+@pytest.mark.parametrize("dims", ["null", "valid"])
+def test_every_entry_point_rejects_null_arguments(L, dims):
+    """Each int-returning entry point, called with NULL pointers (and NULL or
+    valid dims), returns EINVAL with a message: host-side checks come before
+    any device work, so this holds on a machine without a GPU."""
+    d = _good()
+    for name, (res, args) in lsk._SIGS.items():
+        if res is not ctypes.c_int or not args:
+            continue
+        vals = []
+        for a in args:
+            if a in (ctypes.c_int32, ctypes.c_int, ctypes.c_size_t):
+                vals.append(0)
+            elif a is ctypes.c_float:
+                vals.append(1.0)
+            elif dims == "valid" and a is not None and getattr(a, "_type_", None) is lsk.Dims:
+                vals.append(ctypes.byref(d))
+            else:
+                vals.append(None)
+        rc = getattr(L, name)(*vals)
+        expect = lsk.EINVAL
+        if name == "oasis_score_select_noalloc" and dims == "valid" and not _has_gpu():
+            expect = lsk.ECUDA        # it looks up its device-resident scratch first: no device, no scratch
+        assert rc == expect, f"{name} returned {rc}"
+        assert lsk.last_error(), name
+
+
+def _has_gpu():
+    import torch
+    return torch.cuda.is_available()
