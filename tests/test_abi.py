@@ -137,8 +137,8 @@ def test_every_entry_point_rejects_null_arguments(L, dims):
     any device work, so this holds on a machine without a GPU."""
     d = _good()
     for name, (res, args) in lsk._SIGS.items():
-        if res is not ctypes.c_int or not args:
-            continue
+        if res is not ctypes.c_int or not args or (dims == "valid" and name == "oasis_check_dims"):
+            continue                  # (valid dims are all oasis_check_dims takes)
         vals = []
         for a in args:
             if a in (ctypes.c_int32, ctypes.c_int, ctypes.c_size_t):
