@@ -184,7 +184,10 @@ int oasis_block_overlap(const oasis_dims* d, const int32_t* a, const int32_t* b,
  *     call's scores; calls whose work overlaps on the GPU (for example on two
  *     streams) race on it and must be serialised by the caller;
  *   - each GPU that loads the library holds the 4 MiB until the process
- *     exits. */
+ *     exits;
+ *   - errors: the dims and the scratch limit are checked first, then the
+ *     array's address is looked up (OASIS_ECUDA when no device is usable),
+ *     then the buffers, as in oasis_lookahead_scores / oasis_select_topk. */
 int oasis_score_select_noalloc(const oasis_dims* d, const void* q, const void* kmin,
                                const void* kmax, const int32_t* ctx_len, int32_t* sel,
                                float* sel_score, void* stream);
