@@ -239,9 +239,10 @@ def append_kv(d, k_new, v_new, ctx_len, ctx_len_out, host_kv, kmin, kmax, slot_t
     _check(lib().oasis_append_kv(ctypes.byref(d), _arg(k_new, w, "k_new", _BF16, z.row),
                                  _arg(v_new, w, "v_new", _BF16, z.row), _arg(ctx_len, w, "ctx_len", _I32_T, z.b),
                                  _arg(ctx_len_out, w, "ctx_len_out", _I32_T, z.b, nullable=True),
-                                 _arg(host_kv, w, "host_kv", _BF16, z.kv, device=False),
+                                 _arg(host_kv, w, "host_kv", _BF16, z.kv, device=False, nullable=True),
                                  _arg(kmin, w, "kmin", _BF16, z.summary), _arg(kmax, w, "kmax", _BF16, z.summary),
-                                 _arg(slot_table, w, "slot_table", _I32_T, z.k), _arg(pool, w, "pool", _BF16, z.pool),
+                                 _arg(slot_table, w, "slot_table", _I32_T, z.k, nullable=True),
+                                 _arg(pool, w, "pool", _BF16, z.pool, nullable=True),
                                  _stream(stream)), w)
 
 

@@ -160,3 +160,17 @@ def test_every_entry_point_rejects_null_arguments(L, dims):
 def _has_gpu():
     import torch
     return torch.cuda.is_available()
+
+
+def test_binding_passes_optional_buffers_through_as_null():
+    """Arguments the header documents as optional (here the append's host KV,
+    slot table and pool) reach the library as NULL: the error below is the
+    library's own host-side check of a required pointer given as a raw NULL
+    address, raised before any device work, not the binding's None check."""
+    d = _good()
+    with pytest.raises(lsk.OasisError) as e:
+        lsk.append_kv(d, 16, 32, 48, None, None, 0, 80, None, None)
+    assert e.value.code == lsk.EINVAL and "kmin is NULL" in str(e.value)
+    with pytest.raises(lsk.OasisError) as e:
+        lsk.append_kv(d, 16, 32, 48, None, None, None, 80, None, None)
+    assert "kmin is None" in str(e.value)                  # required: the binding stops it
