@@ -91,3 +91,35 @@ def test_timing_harness_runs_the_oracles_decode_path():
     assert (st >= 0).sum() == w.budget_blocks                      # the pool filled up
     for s in range(w.budget_blocks):
         np.testing.assert_array_equal(u.pool_k[0, 0, s], keys[0, 0, st[0, 0, s]])
+
+
+def test_oracle_worker_pool_fails_fast_and_never_hangs():
+    """A worker that dies while setting up, and a pool that outlives its time
+    limit, both end in an exception within seconds (the benchmark then
+    reports the one-core figure); no process is left behind."""
+    import time
+
+    import numpy as np
+    import pytest as _pytest
+
+    from oracle import decode_timing as T
+    W = bench.W
+    w = W.WORKLOADS["llama8b_32k"].with_(batch=1, n_q_heads=4, n_kv_heads=1, context=1024, max_blocks=64,
+                                          budget_blocks=16, fetch_cap=4)
+    cfg = bench.oracle_cfg(w)
+    bits = W.bf16_bits(W.make_host_kv(w, 0, "cpu"))
+    qs = W.QueryStream(w, 0, "cpu")
+    import oracle as O
+    queries = [O.bf16_bits_to_f64(W.bf16_bits(qs.next())) for _ in range(4)]
+    t0 = time.monotonic()
+    with _pytest.raises(Exception):
+        T.run_units_parallel(cfg, [(bits, queries), (np.zeros(3, np.uint16), queries)], 1, 2, 2, timeout_s=60)
+    assert time.monotonic() - t0 < 30
+    t0 = time.monotonic()
+    pool = None
+    with _pytest.raises(Exception):
+        with T.UnitPool(cfg, [(bits, queries)], 5000, timeout_s=1.0) as pool:  # ≈10 s of set-up: killed at 1 s
+            pool.step()
+    assert time.monotonic() - t0 < 20
+    if pool is not None:
+        assert all(p.poll() is not None for p in pool.procs)
