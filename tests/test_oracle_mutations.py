@@ -51,6 +51,19 @@ MUTATIONS = {
         ["test_oracle_eviction.py"]),
     "lost slots kept": (
         "st[np.asarray(mask, dtype=bool)] = -1", "st = st", ["test_oracle_eviction.py"]),
+    # Figure 8: attention at step t reads the working set staged at step t-1, not this step's fetch
+    "attention over this step's fetch": (
+        "        o, lse = sparse_attention(qs, pool_k, pool_v, st, ctx_len, scale)\n"
+        "        slot_table_used = st.copy()\n"
+        "        if evict_masks is not None:\n"
+        "            st = evict_slots(st, evict_masks[t - 1])\n"
+        "        sc, sel, sel_score, plan = select_plan_fetch(qs, t)\n",
+        "        if evict_masks is not None:\n"
+        "            st = evict_slots(st, evict_masks[t - 1])\n"
+        "        sc, sel, sel_score, plan = select_plan_fetch(qs, t)\n"
+        "        o, lse = sparse_attention(qs, pool_k, pool_v, st, ctx_len, scale)\n"
+        "        slot_table_used = st.copy()\n",
+        ["test_oracle.py", "test_oracle_prediction.py", "test_oracle_eviction.py"]),
 }
 
 
