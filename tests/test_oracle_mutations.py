@@ -51,6 +51,18 @@ MUTATIONS = {
         ["test_oracle_eviction.py"]),
     "lost slots kept": (
         "st[np.asarray(mask, dtype=bool)] = -1", "st = st", ["test_oracle_eviction.py"]),
+    # Quest's bound carries no 1/sqrt(D) and takes the max over the query heads (R1)
+    "bound scaled by 1/sqrt(D)": ("bound = term.sum(axis=2)                             # [R, n], fp64",
+                                  "bound = term.sum(axis=2) / math.sqrt(D)"),
+    "bound summed over query heads": ("out[b, h, n0:n1] = bound.max(axis=0).astype(np.float32)",
+                                      "out[b, h, n0:n1] = bound.sum(axis=0).astype(np.float32)"),
+    "valid blocks rounded down": ("return (ctx + block_tokens - 1) // block_tokens", "return ctx // block_tokens"),
+    "gather slot and block swapped": (
+        "out[b, h, int(fetch_slot[b, h, i])] = host_kv[b, h, int(fetch_block[b, h, i])]",
+        "out[b, h, int(fetch_block[b, h, i]) % out.shape[2]] = host_kv[b, h, int(fetch_slot[b, h, i])]"),
+    "append never reopens a block": ("        if t == 0:\n            kmin[b, :, n, :] = k_new[b]",
+                                     "        if False:\n            kmin[b, :, n, :] = k_new[b]"),
+    "attention sees one token past the context": ("valid = min(P, ctx - blk * P)", "valid = min(P, ctx + 1 - blk * P)"),
     # Figure 8: attention at step t reads the working set staged at step t-1, not this step's fetch
     "attention over this step's fetch": (
         "        o, lse = sparse_attention(qs, pool_k, pool_v, st, ctx_len, scale)\n"
