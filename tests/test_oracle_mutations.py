@@ -63,6 +63,13 @@ MUTATIONS = {
     "append never reopens a block": ("        if t == 0:\n            kmin[b, :, n, :] = k_new[b]",
                                      "        if False:\n            kmin[b, :, n, :] = k_new[b]"),
     "attention sees one token past the context": ("valid = min(P, ctx - blk * P)", "valid = min(P, ctx + 1 - blk * P)"),
+    "one block short of the budget": ("            take = order[:K]\n", "            take = order[:K - 1]\n"),
+    "one fetch over the cap": ("fetch = missing[:min(C, len(missing))]", "fetch = missing[:min(C + 1, len(missing))]"),
+    # under LRU a just-stamped selected resident never sorts first, so only score-ordered victims show it
+    "selected residents not protected": (
+        "                     if st[b, h, slot] >= 0 and int(st[b, h, slot]) not in in_sel]",
+        "                     if st[b, h, slot] >= 0]",
+        ["test_oracle.py", "test_oracle_eviction.py"]),
     # Figure 8: attention at step t reads the working set staged at step t-1, not this step's fetch
     "attention over this step's fetch": (
         "        o, lse = sparse_attention(qs, pool_k, pool_v, st, ctx_len, scale)\n"
