@@ -1,8 +1,9 @@
 """Plain CPU oracle for the OasisKV lookahead sparse-KV decode path.
 
 TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the tests, the smoke check in
-``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import or run
-anything in this package.  The CUDA library never calls into it and shares no
+``__graft_entry__``, and the CPU-baseline leg and ``--impl reference`` arm of
+``bench.py`` (through ``oracle/decode_timing.py``) may import or run anything
+in this package.  The CUDA library never calls into it and shares no
 code, header, table or helper with it; the only thing both sides share is the
 seeded input generator, which holds none of the method's arithmetic.
 
