@@ -1191,13 +1191,14 @@ def run_reference(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--layers", type=int, default=8)
-    ap.add_argument("--query-ring", type=int, default=48)
-    ap.add_argument("--impl", default="oasis", choices=["oasis", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gpus", type=int, default=1, help="GPUs (one rank each under torchrun; weak scaling)")
+    ap.add_argument("--steps", type=int, default=400, help="timed decode steps (each runs every layer)")
+    ap.add_argument("--warmup", type=int, default=10, help="untimed steps before them (at least 3)")
+    ap.add_argument("--layers", type=int, default=8, help="pipelined attention layers per step")
+    ap.add_argument("--query-ring", type=int, default=48, help="pre-generated query steps, walked back and forth")
+    ap.add_argument("--impl", default="oasis", choices=["oasis", "reference"],
+                    help="reference: the CPU oracle on the host cores, same metric and config")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing in the GPU line")
     ap.add_argument("--prediction", action="store_true",
                     help="measure prediction agreement and the corrective fetch instead")
     ap.add_argument("--ablation", action="store_true",
