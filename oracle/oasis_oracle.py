@@ -64,6 +64,14 @@ Readings taken where the pages are silent:
   ablation): stale slots are taken in order of their block's current
   lookahead score, lowest first, ties to the lower block id (-0.0 == +0.0);
   free slots still come first and a selected block is never evicted.
+* R9 appended tokens (the long-output reasoning configuration: one new
+  token per sequence per step): the token accepted at step t-1 is written at
+  the start of step t, before that layer's attention, at position
+  ``ctx_len[b]`` of the host KV, folded into the block summaries, and copied
+  into the pool slot that holds its block if that block is resident; the
+  context is one token longer from then on.  A token that opens a new block
+  is therefore not attended at the step it arrives: its block becomes
+  resident only once a plan selects and fetches it (Figure 8 order).
 * R19 residency loss (the 32K Qwen3-32B configuration: a seeded share of
   the attended KV misses residency each step): at decode step t, after the
   layer's attention and before its selection / plan, every slot the step's
@@ -83,6 +91,7 @@ __all__ = [
     "n_valid_blocks",
     "block_summaries",
     "summary_append",
+    "append_token",
     "lookahead_scores",
     "select_topk",
     "plan_fetch",
@@ -169,6 +178,38 @@ def summary_append(kmin, kmax, k_new, ctx_len_before, block_tokens):
             kmin[b, :, n, :] = np.minimum(kmin[b, :, n, :], k_new[b])
             kmax[b, :, n, :] = np.maximum(kmax[b, :, n, :], k_new[b])
     return kmin, kmax
+
+
+def append_token(keys, values, kmin, kmax, pool_k, pool_v, slot_table, ctx_len, k_new, v_new):
+    """Write one new token per sequence (R9), in place, and return the grown
+    context lengths.
+
+    The row goes to position ``ctx_len[b]`` of every KV head's host keys and
+    values, into the summaries (``summary_append``: the compressed keys of
+    [OasisKV] Figure 7 stay current while decoding grows the context), and
+    into the pool slot holding its block when that block is resident
+    ([OasisKV] Figure 9: the slot table names the CPU block each GPU slot
+    holds), so that the resident copy keeps matching the host copy.
+
+    keys/values: float64 [B, Hkv, N, P, D]; pool_k/pool_v: float64
+    [B, Hkv, K, P, D]; slot_table int [B, Hkv, K]; k_new/v_new: float64
+    [B, Hkv, D].
+    """
+    B, H, N, P, D = keys.shape
+    for b in range(B):
+        pos = int(ctx_len[b])
+        if pos >= N * P:
+            raise ValueError(f"sequence {b} is full ({N * P} tokens)")
+        n, t = divmod(pos, P)
+        keys[b, :, n, t] = k_new[b]
+        values[b, :, n, t] = v_new[b]
+        for h in range(H):
+            for slot in range(slot_table.shape[2]):
+                if int(slot_table[b, h, slot]) == n:
+                    pool_k[b, h, slot, t] = k_new[b, h]
+                    pool_v[b, h, slot, t] = v_new[b, h]
+    summary_append(kmin, kmax, k_new, ctx_len, P)
+    return np.asarray(ctx_len, dtype=np.int64) + 1
 
 
 # --------------------------------------------------- a2: lookahead scores
@@ -422,7 +463,7 @@ def evict_slots(slot_table, mask):
 # ------------------------------------------------ a7: per-step order
 def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
                        budget_blocks, fetch_cap, scale, host_kv_bits=None, corrective=False,
-                       evict_masks=None):
+                       evict_masks=None, appends=None):
     """One layer through priming and T decode steps, in the pages' order.
 
     [OasisKV] Figure 8: at step t the drafts drive the top-K prediction,
@@ -443,8 +484,16 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
     E_t's missing blocks without a cap before the attention (R16).
     ``evict_masks[t-1]`` (bool [B, Hkv, K]), when given, frees slots after the
     attention of decode step t and before its plan (R19).
+    ``appends[t-1]`` = (k_new, v_new), float64 [B, Hkv, D], when given, is the
+    token written at the start of decode step t, before anything else of that
+    step (R9); the caller's arrays are left as they were (the grown keys,
+    values and summaries are copies) and each record carries the context
+    length its step used as ``ctx_len``.
     """
     B, H, N, P, D = keys.shape
+    if appends is not None:
+        keys, values, kmin, kmax = keys.copy(), values.copy(), kmin.copy(), kmax.copy()
+    ctx_len = np.asarray(ctx_len, dtype=np.int64).copy()
     K = budget_blocks
     st = np.full((B, H, K), -1, dtype=np.int32)
     lu = np.full((B, H, K), -1, dtype=np.int32)
@@ -479,6 +528,9 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
     _, sel_prev, _, _ = select_plan_fetch(q_prime, 0)
     exact_prev = None
     for t, qs in enumerate(q_steps, start=1):
+        if appends is not None:
+            k_new, v_new = appends[t - 1]
+            ctx_len = append_token(keys, values, kmin, kmax, pool_k, pool_v, st, ctx_len, k_new, v_new)
         corr = None
         if corrective:
             corr = corrective_fetch(qs, t, sel_prev, exact_prev)
@@ -491,7 +543,7 @@ def decode_layer_steps(keys, values, kmin, kmax, ctx_len, q_prime, q_steps,
         sel_prev = sel
         records.append({"o": o, "lse": lse, "slot_table_attn": slot_table_used,
                         "scores": sc, "sel": sel, "sel_score": sel_score, "plan": plan,
-                        "corrective": corr})
+                        "corrective": corr, "ctx_len": ctx_len.copy()})
     return records, st, lu
 
 

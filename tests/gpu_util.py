@@ -66,3 +66,18 @@ def assert_attention_close(o_gpu, lse_gpu, o_or, lse_or, atol=ATOL, rtol=RTOL):
     fin = np.isfinite(lse_or)
     assert (np.isfinite(lse_gpu) == fin).all()
     np.testing.assert_allclose(lse_gpu[fin], lse_or[fin], atol=atol, rtol=rtol)
+
+
+def sampled_units(w, n, seed=0):
+    """n distinct (sequence, KV head) units of workload w for sampled checks:
+    the first and the last unit of the batch (the last sequence's last KV
+    head, where an off-by-one in a unit index would show), the rest seeded."""
+    rng = np.random.default_rng(seed)
+    total = w.batch * w.n_kv_heads
+    picks = [0, total - 1]
+    for u in rng.permutation(total):
+        if len(picks) >= min(n, total):
+            break
+        if int(u) not in picks:
+            picks.append(int(u))
+    return [divmod(u, w.n_kv_heads) for u in picks]

@@ -13,7 +13,7 @@ import lookahead_sparse_kv_b200 as lsk
 import oracle as O
 from lookahead_sparse_kv_b200 import workloads as W
 from lookahead_sparse_kv_b200.pipeline import DecodePipeline, LayerState
-from tests.gpu_util import assert_attention_close, assert_selection_matches, f64, kv_split, np_i32
+from tests.gpu_util import assert_attention_close, assert_selection_matches, f64, kv_split, np_i32, sampled_units
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -268,8 +268,7 @@ def test_full_size_layer_sampled(name):
     st = build_workload_state(w, steps=3, device=DEV)
     d, L, pipe, qs = st["dims"], st["layer"], st["pipe"], st["queries"]
     host_bits = None
-    rng = np.random.default_rng(0)
-    units = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.batch, 4), rng.integers(0, w.n_kv_heads, 4))]
+    units = sampled_units(w, 16)
     ctx = np_i32(pipe.ctx_len)
     scale = 1 / math.sqrt(128)
     pipe.prime([qs[0]])

@@ -437,6 +437,94 @@ def test_decode_steps_with_full_budget_are_dense():
     assert sorted(st[0, 0].tolist()) == list(range(N))
 
 
+def test_append_token_writes_host_summary_and_resident_slot():
+    """Three appended tokens, the second opening a new block: the host rows
+    hold the new values, the summaries equal a rebuild of the grown context,
+    the slot that holds the block gets the row and no other slot changes."""
+    r = _rng(41)
+    B, H, N, P, D, K = 2, 2, 4, 4, 8, 3
+    keys = _bf16_round(r.standard_normal((B, H, N, P, D)))
+    vals = _bf16_round(r.standard_normal((B, H, N, P, D)))
+    ctx = np.array([2 * P - 1, P])                        # one token short of a block / a fresh block
+    kmin, kmax = O.block_summaries(keys, ctx)
+    st = np.array([[[1, -1, 0], [-1, 2, -1]], [[1, 0, -1], [3, -1, 1]]], dtype=np.int32)
+    pool_k = np.zeros((B, H, K, P, D))
+    pool_v = np.zeros((B, H, K, P, D))
+    for b in range(B):
+        for h in range(H):
+            for slot in range(K):
+                if st[b, h, slot] >= 0:
+                    pool_k[b, h, slot] = keys[b, h, st[b, h, slot]]
+                    pool_v[b, h, slot] = vals[b, h, st[b, h, slot]]
+    k0, v0 = keys.copy(), vals.copy()
+    for step in range(3):
+        pk_before, pv_before = pool_k.copy(), pool_v.copy()
+        k_new = _bf16_round(r.standard_normal((B, H, D)))
+        v_new = _bf16_round(r.standard_normal((B, H, D)))
+        pos = ctx.copy()
+        ctx = O.append_token(keys, vals, kmin, kmax, pool_k, pool_v, st, ctx, k_new, v_new)
+        for b in range(B):
+            n, t = divmod(int(pos[b]), P)
+            k0[b, :, n, t], v0[b, :, n, t] = k_new[b], v_new[b]
+            for h in range(H):
+                for slot in range(K):
+                    if st[b, h, slot] == n:
+                        pk_before[b, h, slot, t] = k_new[b, h]
+                        pv_before[b, h, slot, t] = v_new[b, h]
+        np.testing.assert_array_equal(ctx, pos + 1)
+        np.testing.assert_array_equal(keys, k0)
+        np.testing.assert_array_equal(vals, v0)
+        np.testing.assert_array_equal(pool_k, pk_before)
+        np.testing.assert_array_equal(pool_v, pv_before)
+        rmin, rmax = O.block_summaries(keys, ctx)
+        np.testing.assert_array_equal(kmin, rmin)
+        np.testing.assert_array_equal(kmax, rmax)
+    # the resident slot of sequence 1's second block got all three rows
+    np.testing.assert_array_equal(pool_k[1, 0, 0, :3], keys[1, 0, 1, :3])
+
+
+def test_decode_steps_with_appends_and_full_budget_are_dense():
+    """Full budget with one appended token per step (the context crosses a
+    block boundary): each step's attention equals dense attention over the
+    grown context, so the new token is visible to the step it was appended
+    at and the resident copy of its block stays current.  The one exception
+    is a token that opens a new block: that block is not resident yet (the
+    step's own plan fetches it, Figure 8), so at that step it is the one
+    token dense attention must leave out."""
+    r = _rng(42)
+    B, Qn, Hq, H, N, P, D = 2, 3, 4, 2, 6, 16, 16
+    keys = _bf16_round(r.standard_normal((B, H, N, P, D)))
+    vals = _bf16_round(r.standard_normal((B, H, N, P, D)))
+    ctx = np.array([4 * P - 2, 5 * P - 1])
+    kmin, kmax = O.block_summaries(keys, ctx)
+    qp = _bf16_round(r.standard_normal((B, Qn, Hq, D)))
+    steps = 5
+    qsteps = [_bf16_round(r.standard_normal((B, Qn, Hq, D))) for _ in range(steps)]
+    apps = [(_bf16_round(r.standard_normal((B, H, D))), _bf16_round(r.standard_normal((B, H, D))))
+            for _ in range(steps)]
+    k_in, v_in = keys.copy(), vals.copy()
+    recs, st, _ = O.decode_layer_steps(keys, vals, kmin, kmax, ctx, qp, qsteps, budget_blocks=N, fetch_cap=N,
+                                       scale=0.25, appends=apps)
+    np.testing.assert_array_equal(keys, k_in)               # the caller's arrays are not grown
+    grown_k, grown_v, c = keys.copy(), vals.copy(), ctx.copy()
+    opened = 0
+    for t, (rec, qs) in enumerate(zip(recs, qsteps)):
+        visible = c + 1
+        for b in range(B):
+            n, tok = divmod(int(c[b]), P)
+            grown_k[b, :, n, tok] = apps[t][0][b]
+            grown_v[b, :, n, tok] = apps[t][1][b]
+            if tok == 0:
+                visible[b] -= 1
+                opened += 1
+        c = c + 1
+        np.testing.assert_array_equal(rec["ctx_len"], c)
+        od, lsed = O.dense_attention(qs, grown_k, grown_v, visible, 0.25)
+        np.testing.assert_allclose(rec["o"], od, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(rec["lse"], lsed, rtol=1e-12)
+    assert opened == 2                                      # both sequences crossed a block boundary
+
+
 def test_bf16_widening_matches_torch_on_every_bit_pattern():
     """Every one of the 65,536 bf16 patterns widens to the value torch's own
     bf16 -> float64 conversion gives (NaNs stay NaN); narrowing inverts it

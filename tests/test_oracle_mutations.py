@@ -70,6 +70,11 @@ MUTATIONS = {
         "                     if st[b, h, slot] >= 0 and int(st[b, h, slot]) not in in_sel]",
         "                     if st[b, h, slot] >= 0]",
         ["test_oracle.py", "test_oracle_eviction.py"]),
+    # R9: the appended row reaches the resident copy of its block, and the context grows
+    "appended row not copied into the resident slot": (
+        "                    pool_k[b, h, slot, t] = k_new[b, h]\n", "                    pass\n"),
+    "context not grown by an append": ("    return np.asarray(ctx_len, dtype=np.int64) + 1\n",
+                                       "    return np.asarray(ctx_len, dtype=np.int64)\n"),
     # Figure 8: attention at step t reads the working set staged at step t-1, not this step's fetch
     "attention over this step's fetch": (
         "        o, lse = sparse_attention(qs, pool_k, pool_v, st, ctx_len, scale)\n"

@@ -44,7 +44,8 @@ def test_noalloc_score_select_matches_workspace_version_twice():
         lsk.score_select_noalloc(d, q, kmin, kmax, ctx, sel_na, sc_na)
         torch.cuda.synchronize()
         assert torch.equal(sel_na, sel_ws), f"call {call}: selections differ"
-        torch.testing.assert_close(sc_na, sc_ws, rtol=1e-5, atol=1e-4)
+        # the same scorer and selector kernels on the same inputs: identical bits
+        assert torch.equal(sc_na, sc_ws), f"call {call}: selected scores differ"
     assert lsk.read_device_error(clear=True) == 0
 
     too_big = lsk.make_dims(batch=64, n_q_heads=32, n_kv_heads=8, max_blocks=4096, budget_blocks=64,
