@@ -1,22 +1,28 @@
 """Benchmark of the lookahead sparse-KV decode path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload qwen32b_32k|llama8b_32k]
 
-Workload: Llama-3.1-8B-shaped attention layers at 32K context (batch 16,
-32 query / 8 KV heads, head dim 128, 2,048 blocks of 16 tokens per KV head,
-budget 2,048 tokens = 128 blocks, 1 verification + 4 draft queries, fetch cap
-16 blocks per head per step, AR(1)-drifting queries), synthetic bf16 data,
-stacked --layers deep (default 8, each layer with its own 2 GiB host KV) so
-that a layer's host-to-HBM transfer overlaps the other layers' work as in
-the OasisKV pipeline (Figure 8).  One step = one decode step through every
-layer: per layer, sparse attention over the resident pool, lookahead scores,
-top-K selection, the capped fetch plan and the gather of the missing blocks
-from pinned host memory.  Metric: layer-steps/s = layers x steps / time
-(whole job; weak scaling - every rank runs its own batch, no collective on
-the data path).
+Default workload (the largest configuration that fits one GPU): a 64-layer
+stack shaped like Qwen3-32B at 32K context - batch 16, 64 query / 8 KV
+heads, head dim 128, 2,048 blocks of 16 tokens per KV head (about 128 GB of
+bf16 KV in pinned host memory), budget 2,048 tokens = 128 blocks, 1
+verification + 7 draft queries, fetch cap 16 blocks per head per step, AR(1)
+drifting queries, and every step a seeded 10 % of the resident slots lost
+from residency before the plan.  Layers beyond the host-KV layers the node
+can pin read the host KV of layer l mod that number (the line reports it as
+``host_kv_layers``).  ``--workload llama8b_32k`` runs the 8-layer Llama-3.1-8B
+stack at 32K (32/8 heads, 1+4 queries) instead.  One step = one decode step
+through every layer: per layer, sparse attention over the resident pool,
+the residency loss, lookahead scores, top-K selection, the capped fetch plan
+and the gather of the missing blocks from pinned host memory, stages of
+different layers overlapping as in the OasisKV pipeline (Figure 8).
+Metric: layer-steps/s = layers x steps / time (whole job; weak scaling -
+every rank runs its own batch, no collective on the data path).
 
 Prints one JSON line (rank 0).  With --impl reference the CPU oracle runs the
-same configuration on the host cores (rank 0 only).
+same configuration on the host cores (rank 0 only): each timed step is one
+decode layer-step of the whole batch.
 
     python bench.py --prediction [--steps K] [--layers L]
 
@@ -72,18 +78,30 @@ import lookahead_sparse_kv_b200 as lsk                                    # noqa
 from lookahead_sparse_kv_b200 import workloads as W                        # noqa: E402
 from lookahead_sparse_kv_b200.pipeline import DecodePipeline, LayerState  # noqa: E402
 
-WORKLOAD = "llama8b_32k"
+WORKLOAD = "qwen32b_32k"            # the default (headline) workload
 METRIC = "sparse decode layer-steps/s (score+select+plan+prefetch+attn)"
-DATA = "synthetic (seeded bf16 KV ~N(0,1) with 4 outlier channels x8, AR(1)-drifting queries)"
+# per benchmarked workload: default layers, pre-generated query steps, description
+BENCH_WORKLOADS = {
+    "qwen32b_32k": {"layers": 64, "ring": 16, "host_kv_cap": 16,
+                    "desc": "Qwen3-32B-shaped attention layers at 32K context (64/8 heads, 1+7 queries), "
+                            "a seeded 10 % residency loss every step, pipelined across layers"},
+    "llama8b_32k": {"layers": 8, "ring": 48, "host_kv_cap": 0,
+                    "desc": "Llama-3.1-8B-shaped attention layers at 32K context, pipelined across layers"},
+}
 
 
-def headline_config(w, nl: int, world: int) -> dict:
-    """The `config` of the headline line, shared by both arms."""
-    return {"workload": f"{WORKLOAD}: {nl} Llama-3.1-8B-shaped attention layers at 32K context, "
-                        f"pipelined across layers",
+def data_label(w) -> str:
+    loss = f", seeded Bernoulli({w.evict_prob:g}) residency-loss masks" if w.evict_prob > 0 else ""
+    return f"synthetic (seeded bf16 KV ~N(0,1) with 4 outlier channels x8, AR(1)-drifting queries{loss})"
+
+
+def headline_config(w, nl: int, world: int, name: str = WORKLOAD) -> dict:
+    """The `config` of the benchmark line, shared by both arms."""
+    return {"workload": f"{name}: {nl} {BENCH_WORKLOADS[name]['desc']}",
             "batch": w.batch, "seq_len": w.context, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
             "head_dim": w.head_dim, "block_tokens": w.block_tokens, "budget_blocks": w.budget_blocks,
             "queries": w.n_queries, "fetch_cap": w.fetch_cap, "layers": nl,
+            "evict_prob": w.evict_prob,
             "parallelism": f"dp{world} (independent replicas)",
             "l2": "inputs larger than L2: per layer-step 128 MiB summaries + 128 MiB pool read"}
 QUERY_RING = 256
@@ -102,10 +120,10 @@ def ring_index(t: int, n: int) -> int:
     return p if p < n else 2 * n - 2 - p
 
 
-def rank_workload(rank: int):
+def rank_workload(rank: int, name: str = WORKLOAD):
     """Weak scaling: every rank runs the benchmarked workload on its own
     seeded batch (no data is exchanged between ranks)."""
-    w = W.WORKLOADS[WORKLOAD]
+    w = W.WORKLOADS[name]
     return w.with_(seed=w.seed + 1000 * rank) if rank else w
 
 
@@ -218,7 +236,9 @@ def build_workload_state(w, steps: int, device="cuda", n_queries: int | None = N
                          host_layers: int | None = None):
     """Pinned host KV, per-layer device state, pipeline and resident queries
     for `layers` layers of workload `w` (layer l draws its own queries; its KV
-    is its own when l < host_layers, else layer l mod host_layers's)."""
+    is its own when l < host_layers, else layer l mod host_layers's).  With a
+    residency loss (w.evict_prob > 0) each layer also gets a ring of its
+    seeded per-step loss masks (uint8 [B, Hkv, K]) as ``mrings``."""
     d = lsk.dims_for(w)
     states, qrings, hosts = [], [], []
     nq = n_queries if n_queries is not None else min(QUERY_RING, max(steps, 1))
@@ -235,11 +255,15 @@ def build_workload_state(w, steps: int, device="cuda", n_queries: int | None = N
         qs = W.QueryStream(w, l, device)
         qrings.append([qs.next() for _ in range(max(nq, 1))])
         hosts.append(host)
+    mrings = None
+    if w.evict_prob > 0:
+        mrings = [[W.eviction_mask(w, l, i, device).to(torch.uint8) for i in range(max(nq, 1))]
+                  for l in range(layers)]
     pipe = DecodePipeline(d, states, W.initial_ctx_len(w, device), 1.0 / math.sqrt(w.head_dim), device)
     pipe.build_summaries()
     torch.cuda.synchronize()
     return {"dims": d, "layers": states, "layer": states[0], "pipe": pipe, "qrings": qrings,
-            "queries": qrings[0], "host": hosts[0]}
+            "queries": qrings[0], "host": hosts[0], "mrings": mrings}
 
 
 class KernelTimer:
@@ -738,6 +762,114 @@ def run_longctx(args, device):
     print(json.dumps(line), flush=True)
 
 
+def run_reasoning(args, device):
+    """Long-output reasoning decode: 36 layers shaped like Qwen3-8B (batch 64,
+    32/8 heads, budget 128 blocks, cap 8, 1+4 queries), one new token per
+    sequence appended every step (host KV, summaries and the resident slot of
+    its block updated in place).  The context is measured in four windows
+    that start at 1K (the whole context fits the budget), 4K, 8K and just
+    below 17K tokens: each window resets the pool, rebuilds the summaries of
+    its starting context, primes, fills the pool over warm-up steps and times
+    --steps (at most 32) decode steps.  Host KV: layers share the pinned KV of
+    layer l mod L (L distinct layers, 4.6 GB each); the rows appended at a
+    step are drawn per distinct layer, so layers that share host KV append
+    identical rows and every layer's summaries and pool stay consistent with
+    it."""
+    base = W.WORKLOADS["qwen8b_reasoning"]
+    nl = args.layers if args.layers_given else base.layers
+    steps = min(args.steps, 32)
+    warm = base.budget_blocks // max(1, base.fetch_cap) + 2
+    total = 1 + warm + steps
+    ring = 16
+    cap_tokens = base.max_blocks * base.block_tokens                   # 17,408
+    starts = [1024, 4096, 8192, cap_tokens - total - 8]
+    try:
+        distinct = host_kv_layers(base, nl, 1)
+    except Exception:
+        distinct = nl
+    distinct = max(1, min(distinct, args.host_kv_layers or 4))
+    d = lsk.dims_for(base)
+    hosts = []
+    for l in range(distinct):
+        h = torch.empty((base.batch, base.n_kv_heads, base.max_blocks, 2, base.block_tokens, base.head_dim),
+                        dtype=torch.bfloat16, pin_memory=True)
+        W.make_host_kv(base, layer=l, device=device, out=h)
+        hosts.append(h)
+    layers = [LayerState(d, hosts[l % distinct], device) for l in range(nl)]
+    qrings = []
+    for l in range(nl):
+        qs = W.QueryStream(base, l, device)
+        qrings.append([qs.next() for _ in range(ring)])
+    torch.cuda.synchronize()
+    h2d = measure_h2d_peak(device)
+    scale = 1.0 / math.sqrt(base.head_dim)
+    rows = []
+    for c0 in starts:
+        # rows appended at decode steps 1 .. total-1, per distinct host layer
+        apps = [[W.append_rows(base, l, c0 + t, device) for l in range(distinct)] for t in range(total)]
+        for L in layers:
+            L.slot_table.fill_(-1)
+            L.last_used.fill_(-1)
+        ctx = torch.full((base.batch,), c0, dtype=torch.int32, device=device)
+        pipe = DecodePipeline(d, layers, ctx, scale, device)
+        pipe.build_summaries()
+
+        def qs_at(t):
+            return [r[ring_index(t, ring)] for r in qrings]
+
+        def app_at(t):
+            return [apps[t][l % distinct] for l in range(nl)]
+
+        pipe.prime(qs_at(0))
+        for t in range(1, 1 + warm):
+            pipe.step(t, qs_at(t), appended=app_at(t))
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        fetched = torch.zeros((), dtype=torch.int64, device=device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(pipe.main)
+        h0 = time.perf_counter()
+        for t in range(1 + warm, total):
+            pipe.step(t, qs_at(t), appended=app_at(t))
+            for L in layers:
+                fetched += L.n_fetch.sum()
+        pipe.wait_all()
+        e1.record(pipe.main)
+        host_ms = (time.perf_counter() - h0) * 1e3
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        ctx_end = int(pipe.ctx_len[0].item())
+        per_ls = ms / (nl * steps)
+        fetched_ls = fetched.item() / (nl * steps)
+        gbs = fetched_ls * base.block_bytes / (per_ls * 1e-3) / 1e9
+        w_now = base.with_(context=ctx_end)
+        iso = isolated_kernel_ms({"pipe": pipe, "layers": layers, "dims": d, "qrings": [[qs_at(total - 1)[0]]]},
+                                 reps=5)
+        iso.pop("_prefetch_blocks")
+        ab = algorithmic_bytes(w_now, fetched_ls)
+        attn_gbs = ab["sparse_attn"] / (iso["sparse_attn"] * 1e-3) / 1e9
+        rows.append({
+            "context_start": c0, "context_end": ctx_end,
+            "layer_steps_per_s": 1.0 / (per_ls * 1e-3), "tokens_per_s": 1.0 / (per_ls * 1e-3) / nl * base.batch,
+            "fetched_blocks_per_layer_step": fetched_ls, "h2d_gbs": gbs, "h2d_frac": gbs / h2d["peak_gbs"],
+            "overlap_efficiency": overlap_efficiency(iso, per_ls)["value"],
+            "compute_ms": overlap_efficiency(iso, per_ls)["compute_ms"],
+            "attention_hbm_gbs": attn_gbs, "host_enqueue_ms_per_step": host_ms / steps,
+            "isolated_ms": {k: iso[k] for k in ("sparse_attn", "score_select", "plan_fetch", "prefetch")}})
+        del pipe
+    line = {
+        "metric": "long-output reasoning decode with appends: layer-steps/s, tokens/s, H2D vs PCIe roof, "
+                  "overlap efficiency, per context window",
+        "workload": f"qwen8b_reasoning: {nl} Qwen3-8B-shaped layers, batch 64, 32/8 heads, budget "
+                    f"{base.budget_blocks} blocks, cap {base.fetch_cap}, 1+4 queries, one appended token per "
+                    f"sequence per step; host KV of {distinct} distinct layers (l -> l mod {distinct})",
+        "steps_per_window": steps, "warmup_steps": warm, "h2d_peak": h2d, "windows": rows,
+        "gpu_launches_per_layer_step": launches_per_layer_step(base) + 1,     # + the append
+        "device_error_word": lsk.read_device_error(clear=True),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_deep(args, device):
     """Eager vs graph-replayed decode steps of a 64-layer stack."""
     base = W.WORKLOADS["qwen32b_32k"]
@@ -829,16 +961,22 @@ def run_deep(args, device):
 
 
 def run_gpu(args, rank, world, device):
-    w = rank_workload(rank)
+    w = rank_workload(rank, args.workload)
+    nl = args.layers
     try:
-        host_layers = host_kv_layers(w, args.layers, int(os.environ.get("LOCAL_WORLD_SIZE", world)))
+        host_layers = host_kv_layers(w, nl, int(os.environ.get("LOCAL_WORLD_SIZE", world)))
     except Exception:                                   # no estimate: one host KV per layer, as asked
-        host_layers = args.layers
+        host_layers = nl
+    # the 64-layer stack's 128 GiB of host KV would pin most of a GPU node's
+    # memory: by default 16 distinct layers (32 GiB) are pinned and shared
+    cap = args.host_kv_layers or BENCH_WORKLOADS[args.workload]["host_kv_cap"]
+    if cap:
+        host_layers = min(host_layers, cap)
     st = build_workload_state(w, args.warmup + args.steps, device, n_queries=args.query_ring,
-                              layers=args.layers, host_layers=host_layers)
+                              layers=nl, host_layers=host_layers)
     st["host_layers"] = host_layers
-    d, layers, pipe, qrings = st["dims"], st["layers"], st["pipe"], st["qrings"]
-    nl, nq = len(layers), len(qrings[0])
+    d, layers, pipe, qrings, mrings = st["dims"], st["layers"], st["pipe"], st["qrings"], st["mrings"]
+    nq = len(qrings[0])
     timer = KernelTimer(args.steps * nl)
     pipe.timer = timer
     main = pipe.main
@@ -848,10 +986,16 @@ def run_gpu(args, rank, world, device):
         i = ring_index(t, nq)
         return [r[i] for r in qrings]
 
+    def ms_at(t):                                       # the step's residency-loss masks, or None
+        if mrings is None:
+            return None
+        i = ring_index(t, nq)
+        return [r[i] for r in mrings]
+
     pipe.prime(qs_at(0))
     t = 1
     for _ in range(args.warmup):
-        pipe.step(t, qs_at(t))
+        pipe.step(t, qs_at(t), evict=ms_at(t))
         t += 1
     pipe.wait_all()
     torch.cuda.synchronize()
@@ -865,7 +1009,7 @@ def run_gpu(args, rank, world, device):
         ev0.record(main)
         h0 = time.perf_counter()
         for i in range(args.steps):
-            pipe.step(t, qs_at(t))
+            pipe.step(t, qs_at(t), evict=ms_at(t))
             for l, L in enumerate(layers):
                 fetch_hist[i, l].copy_(L.n_fetch, non_blocking=True)
             t += 1
@@ -886,7 +1030,7 @@ def run_gpu(args, rank, world, device):
         torch.cuda.synchronize()
         h0 = time.perf_counter()
         for _ in range(4):
-            pipe.step(t, qs_at(t))
+            pipe.step(t, qs_at(t), evict=ms_at(t))
             t += 1
         host_cost.append((time.perf_counter() - h0) * 1e3 / 4)
     pipe.wait_all()
@@ -895,8 +1039,8 @@ def run_gpu(args, rank, world, device):
     # reuse of the selected set between consecutive steps (untimed)
     reuse = []
     prev = [L.sel.clone() for L in layers]
-    for _ in range(16):
-        pipe.step(t, qs_at(t))
+    for _ in range(8):
+        pipe.step(t, qs_at(t), evict=ms_at(t))
         t += 1
         pipe.wait_all()
         for l, L in enumerate(layers):
@@ -909,7 +1053,9 @@ def run_gpu(args, rank, world, device):
     # end-to-end through the API: every step copies each layer's queries in
     # from pinned host memory (input stream, one event per layer) and reads
     # each layer's outputs back once that layer is done (output stream); the
-    # host waits for the last read-back before it starts the next step
+    # host waits for the last read-back before it starts the next step.  The
+    # residency-loss masks stand for the memory system, not for a caller's
+    # input, and stay on the device.
     e2e_steps = min(args.steps, 200)
     hq = [[q.cpu().pin_memory() for q in r[: min(nq, 32)]] for r in qrings]
     qdev = [torch.empty_like(r[0]) for r in qrings]
@@ -928,7 +1074,7 @@ def run_gpu(args, rank, world, device):
             for l in range(nl):
                 qdev[l].copy_(hq[l][j], non_blocking=True)
                 in_ev[l].record(s_in)
-        pipe.step(t, qdev, inputs_ready=in_ev, layer_done=out_ev)
+        pipe.step(t, qdev, evict=ms_at(t), inputs_ready=in_ev, layer_done=out_ev)
         t += 1
         with torch.cuda.stream(s_out):
             for l, L in enumerate(layers):
@@ -940,13 +1086,16 @@ def run_gpu(args, rank, world, device):
     e1.record(main)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    del hq, hout, hlse
 
     iso = isolated_kernel_ms(st)
     h2d = measure_h2d_peak(device) if rank == 0 else None
     err = lsk.read_device_error(clear=True)
-    return {"w": w, "d": d, "ms": ms, "host_ms": host_ms, "host_cost_ms": min(host_cost), "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
+    return {"w": w, "name": args.workload, "d": d, "ms": ms, "host_ms": host_ms, "host_cost_ms": min(host_cost),
+            "timer": timer, "fetch_hist": fetch_hist, "reuse": reuse,
             "e2e_ms": e2e_ms, "e2e_steps": e2e_steps, "h2d": h2d, "clocks": clk.summary(), "dev_err": err,
-            "layer": layers[0], "layers": layers, "queries": qrings[0], "iso": iso,
+            "layer": layers[0], "layers": layers, "queries": qrings[0],
+            "masks": None if mrings is None else mrings[0], "iso": iso,
             "host_layers": st["host_layers"]}
 
 
@@ -1003,6 +1152,12 @@ def token_kv_intensity(w, fetched_blocks_per_layer_step):
                           "read; PCIe = fetched blocks; dense = the whole KV read by dense attention"}
 
 
+def launches_per_layer_step(w) -> int:
+    """Kernels of one layer-step: attention and its merge, scores, top-K,
+    plan and gather, plus the residency loss when the workload has one."""
+    return 6 + (1 if w.evict_prob > 0 else 0)
+
+
 def emit_gpu(args, res, world):
     w, timer = res["w"], res["timer"]
     nl = len(res["layers"])
@@ -1048,8 +1203,8 @@ def emit_gpu(args, res, world):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": DATA,
-        "config": headline_config(w, nl, world),
+        "data": data_label(w),
+        "config": headline_config(w, nl, world, res.get("name", WORKLOAD)),
         "roofline": {"kernel": dominant, "bound": kd["bound"], "achieved": kd["achieved_gbs"],
                      "peak": kd["peak_gbs"], "unit": "GB/s", "frac": kd["frac"], "traffic": kd["traffic"],
                      "peak_source": kd["peak_source"]},
@@ -1068,7 +1223,7 @@ def emit_gpu(args, res, world):
                 "note": "per step: every layer's queries copied in from pinned host memory and its outputs read "
                         "back as soon as that layer is done, the host waiting for the last read-back before the "
                         "next step; h2d bytes include the zero-copy gather of fetched blocks"},
-        "gpu_launches": 6 * layer_steps,   # attention, merge, score, select, plan, gather
+        "gpu_launches": launches_per_layer_step(w) * layer_steps,
         "host_kv_layers": res.get("host_layers", nl),   # distinct pinned host KV per rank (layer l -> l mod this)
         "cpus_bound": res.get("cpus_bound"),   # rank 0's CPUs local to its GPU (multi-rank runs), else null
         "host_enqueue_ms_per_step": res["host_ms"] / args.steps,
@@ -1102,16 +1257,21 @@ def cpu_baseline(w, res, n_units=6, fill_steps=8, timed_steps=24, par_fill=4, pa
     G = w.group
     total_units = w.batch * w.n_kv_heads
     qs_all = [O.bf16_bits_to_f64(W.bf16_bits(q)) for q in res["queries"][: fill_steps + timed_steps + 1]]
+    ms_all = None
+    if res.get("masks") is not None:                   # the same loss masks the GPU run used
+        ms_all = [m.cpu().numpy().astype(bool) for m in res["masks"][: fill_steps + timed_steps + 1]]
 
     def unit(b, h, steps):
-        return W.bf16_bits(L.host_kv[b:b + 1, h:h + 1]), [q[b:b + 1, :, h * G:(h + 1) * G] for q in qs_all[:steps]]
+        masks = None if ms_all is None else [m[b:b + 1, h:h + 1] for m in ms_all[:steps]]
+        return (W.bf16_bits(L.host_kv[b:b + 1, h:h + 1]), [q[b:b + 1, :, h * G:(h + 1) * G] for q in qs_all[:steps]],
+                masks)
 
     rng = np.random.default_rng(0)
     picks = [(int(rng.integers(w.batch)), int(rng.integers(w.n_kv_heads))) for _ in range(n_units)]
     times = []
     for b, h in picks:
-        bits, qs = unit(b, h, fill_steps + timed_steps + 1)
-        times += T.run_unit(oracle_cfg(w), bits, qs, fill_steps, timed_steps)
+        bits, qs, masks = unit(b, h, fill_steps + timed_steps + 1)
+        times += T.run_unit(oracle_cfg(w), bits, qs, fill_steps, timed_steps, masks=masks)
     one = 1.0 / (sum(times) / len(times) * total_units)
     single = {"value": one, "unit": "layer-steps/s", "cores": 1,
               "sample": f"{len(times)} unit-steps ({n_units} (sequence, KV head) units x {timed_steps} decode "
@@ -1139,50 +1299,69 @@ def cpu_baseline(w, res, n_units=6, fill_steps=8, timed_steps=24, par_fill=4, pa
 
 def run_reference(args):
     """--impl reference: the CPU oracle on this host's cores, same workload,
-    metric and unit.  Each step is one decode layer-step of P (sequence, KV
-    head) units of the benchmarked workload at once, one per core (P = the
-    usable cores, at most 64), timed by the wall clock and scaled to the
-    whole batch and the layers of a step; one core if that cannot run."""
+    metric, unit and config as the GPU arm.  Each timed step is one decode
+    layer-step (attention, residency loss, scores, top-K, plan, gather) of
+    the whole batch at one layer: every (sequence, KV head) unit of the batch,
+    spread over one process per usable core (at most 64), timed by the wall
+    clock from the start of the step to the last process's reply.  Every
+    layer of the stack has the same shape and work, so layer-steps/s is the
+    number of timed layer-steps over their time, with no scaling; a step of
+    this arm is one layer-step, and ms_per_step is its time.  --ref-units U
+    (quick checks only) times the first U units and scales to the batch, and
+    says so in its sample."""
     import oracle as O
     from oracle import decode_timing as T
-    w = W.WORKLOADS[WORKLOAD]
+    w = W.WORKLOADS[args.workload]
     total_units = w.batch * w.n_kv_heads
-    P = max(1, min(T.usable_cores(), 64, total_units))
-    wu = w.with_(batch=-(-P // w.n_kv_heads))
+    n_units = total_units if not args.ref_units else max(1, min(args.ref_units, total_units))
+    P = max(1, min(T.usable_cores(), 64, n_units))
+    wu = w.with_(batch=-(-n_units // w.n_kv_heads))
     kv = W.make_host_kv(wu, 0, "cpu")
     qs = W.QueryStream(wu, 0, "cpu")
-    ring = [O.bf16_bits_to_f64(W.bf16_bits(qs.next())) for _ in range(48)]   # walked in order, then again
-    G, fill = w.group, 8
+    ring_n = 16
+    ring = [O.bf16_bits_to_f64(W.bf16_bits(qs.next())) for _ in range(ring_n)]   # walked in order, then again
+    masks = None
+    if w.evict_prob > 0:
+        masks = [W.eviction_mask(wu, 0, i, "cpu").numpy() for i in range(ring_n)]
+    G, fill = w.group, 4
     units = []
-    for k in range(P):
+    for k in range(n_units):
         b, h = divmod(k, w.n_kv_heads)
-        units.append((W.bf16_bits(kv[b:b + 1, h:h + 1]), [q[b:b + 1, :, h * G:(h + 1) * G] for q in ring]))
-    what = ("decode layer-step (attention, scores, top-K, plan, gather) of the 32K Llama-shaped layer, scaled to "
-            f"the {total_units} units of the batch and the {args.layers} layers of a step; numpy fp64, BLAS 1 "
-            "thread per process")
+        units.append((W.bf16_bits(kv[b:b + 1, h:h + 1]), [q[b:b + 1, :, h * G:(h + 1) * G] for q in ring],
+                      None if masks is None else [m[b:b + 1, h:h + 1] for m in masks]))
+    del kv
+    loss = ", residency loss," if masks is not None else ""
+    what = (f"decode layer-step (attention{loss} scores, top-K, plan, gather) of {n_units} (sequence, KV head) units "
+            f"of {args.workload} at one layer; numpy fp64, BLAS 1 thread per process")
+    scaled = n_units != total_units
     try:
-        with T.UnitPool(oracle_cfg(wu), units, fill, timeout_s=300.0) as pool:
+        with T.UnitPool(oracle_cfg(wu), units, fill, timeout_s=1500.0, workers=P) as pool:
             for _ in range(args.warmup):
                 pool.step()
             walls = [pool.step()[0] for _ in range(args.steps)]
-        unit_steps_per_s = P / (sum(walls) / len(walls))
         cores = P
-        sample = (f"each step: {P} (sequence, KV head) units, one process per core, each doing one " + what +
-                  "; wall clock per step")
+        sample = (f"each step: one {what}, the units spread over {P} processes (one per core) and stepped "
+                  f"together, wall clock from start to the last reply")
     except Exception as e:                                            # one core
-        times = T.run_unit(oracle_cfg(wu), units[0][0], units[0][1], fill + args.warmup, args.steps)
-        unit_steps_per_s = len(times) / sum(times)
+        walls = []
+        times = [T.run_unit(oracle_cfg(wu), *u[:2], fill + args.warmup, args.steps, masks=u[2])
+                 for u in units[: max(1, min(4, n_units))]]
+        per_step = [sum(t[i] for t in times) / len(times) for i in range(args.steps)]
+        walls = [x * n_units for x in per_step]
         cores = 1
-        sample = (f"each step: one (sequence, KV head) unit's " + what +
-                  f" (the all-cores run failed: {type(e).__name__})")
-    value = unit_steps_per_s / total_units
+        sample = (f"each step: {len(times)} units' {what.split(' of ', 1)[0]} on one core, the mean scaled to "
+                  f"{n_units} units (the all-cores run failed: {type(e).__name__})")
+    ms = sum(walls) / len(walls) * 1e3 * (total_units / n_units)
+    if scaled:
+        sample += f"; scaled from {n_units} to the {total_units} units of the batch"
+    value = 1e3 / ms
     line = {
         "impl": "reference",
         "metric": METRIC,
         "value": value, "unit": "layer-steps/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": args.layers / value * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
-        "config": headline_config(w, args.layers, args.gpus),
+        "warmup": args.warmup, "ms_per_step": ms, "step_layers": 1, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": data_label(w),
+        "config": headline_config(w, args.layers, args.gpus, args.workload),
         "cpu_baseline": {"value": value, "unit": "layer-steps/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -1192,10 +1371,19 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1, help="GPUs (one rank each under torchrun; weak scaling)")
-    ap.add_argument("--steps", type=int, default=400, help="timed decode steps (each runs every layer)")
+    ap.add_argument("--steps", type=int, default=50, help="timed decode steps (each runs every layer)")
     ap.add_argument("--warmup", type=int, default=10, help="untimed steps before them (at least 3)")
-    ap.add_argument("--layers", type=int, default=8, help="pipelined attention layers per step")
-    ap.add_argument("--query-ring", type=int, default=48, help="pre-generated query steps, walked back and forth")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(BENCH_WORKLOADS),
+                    help="benchmarked stack (default: the 64-layer Qwen3-32B-shaped one with residency loss)")
+    ap.add_argument("--layers", type=int, default=None, help="pipelined attention layers per step "
+                    "(default: the workload's, 64 or 8)")
+    ap.add_argument("--host-kv-layers", type=int, default=0,
+                    help="most distinct pinned host-KV layers (0: the workload's default cap, 16 for the "
+                         "64-layer stack, within what the node's memory holds)")
+    ap.add_argument("--query-ring", type=int, default=None,
+                    help="pre-generated query steps, walked back and forth (default: the workload's)")
+    ap.add_argument("--ref-units", type=int, default=0,
+                    help="reference arm, quick checks only: time this many units and scale to the batch")
     ap.add_argument("--impl", default="oasis", choices=["oasis", "reference"],
                     help="reference: the CPU oracle on the host cores, same metric and config")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing in the GPU line")
@@ -1207,8 +1395,16 @@ def main():
                     help="64-layer stack, eager vs CUDA-graph replay, instead")
     ap.add_argument("--longctx", action="store_true",
                     help="128K layer: budget x cap sweep with overlap efficiency, instead")
+    ap.add_argument("--reasoning", action="store_true",
+                    help="36-layer Qwen3-8B reasoning decode with appends, context windows 1K-17K, instead")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    spec = BENCH_WORKLOADS[args.workload]
+    args.layers_given = args.layers is not None
+    side_mode = args.prediction or args.ablation or args.deep or args.longctx or args.reasoning
+    # the side modes run their own workloads; their stacks default to 8 layers
+    args.layers = args.layers or (8 if side_mode else spec["layers"])
+    args.query_ring = args.query_ring or spec["ring"]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -1220,7 +1416,7 @@ def main():
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     modes = [(args.prediction, run_prediction), (args.ablation, run_ablation), (args.deep, run_deep),
-             (args.longctx, run_longctx)]
+             (args.longctx, run_longctx), (args.reasoning, run_reasoning)]
     for on, fn in modes:
         if on:
             if rank == 0:

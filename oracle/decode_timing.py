@@ -9,8 +9,10 @@ so they start quickly and are safe to start from a process that already
 uses a GPU.
 
 A unit is described by a plain dict (context, block_tokens, budget_blocks,
-head_dim, fetch_cap), its host-KV bit pattern (uint16 [1, 1, N, 2, P, D])
-and a list of float64 queries per step ([1, Qn, G, D]).
+head_dim, fetch_cap), its host-KV bit pattern (uint16 [1, 1, N, 2, P, D]),
+a list of float64 queries per step ([1, Qn, G, D]) and, for workloads with a
+residency loss, a list of bool masks per step ([1, 1, K]); both lists are
+walked cyclically.
 """
 
 from __future__ import annotations
@@ -45,10 +47,14 @@ class OracleUnit:
         self.pool_v = np.zeros((1, 1, K, P, D))
         self.scale = 1.0 / math.sqrt(D)
 
-    def step(self, q, t, attend=True):
+    def step(self, q, t, attend=True, mask=None):
+        """One decode layer-step (priming when attend is False); `mask`, when
+        given, frees slots after the attention and before the plan (R19)."""
         c = self.cfg
         if attend:
             O.sparse_attention(q, self.pool_k, self.pool_v, self.st, self.ctx, self.scale)
+        if mask is not None:
+            self.st = O.evict_slots(self.st, mask)
         sc = O.lookahead_scores(q, self.kmin, self.kmax, self.ctx, c["block_tokens"])
         sel, _ = O.select_topk(sc, self.ctx, c["budget_blocks"], c["block_tokens"])
         plan = O.plan_fetch(sel, self.st, self.lu, t, c["fetch_cap"])
@@ -65,29 +71,40 @@ def _one_blas_thread():
         return None
 
 
-def _prepare(cfg: dict, host_bits: np.ndarray, queries: list, fill_steps: int) -> OracleUnit:
-    u = OracleUnit(cfg, host_bits)
+def _unit_inputs(spec):
+    """(bits, queries, masks or None) of a unit given as (bits, queries) or
+    (bits, queries, masks)."""
+    bits, queries = spec[0], spec[1]
+    return bits, queries, (spec[2] if len(spec) > 2 else None)
+
+
+def _step_unit(u: OracleUnit, queries: list, masks, i: int):
+    u.step(queries[i % len(queries)], i, mask=None if masks is None else masks[i % len(masks)])
+
+
+def _prepare(cfg: dict, spec, fill_steps: int) -> OracleUnit:
+    bits, queries, masks = _unit_inputs(spec)
+    u = OracleUnit(cfg, bits)
     u.step(queries[0], 0, attend=False)                   # priming
     for i in range(1, fill_steps + 1):
-        u.step(queries[i % len(queries)], i)
+        _step_unit(u, queries, masks, i)
     return u
 
 
-def _timed(u: OracleUnit, queries: list, fill_steps: int, timed_steps: int) -> list:
-    times = []
-    for i in range(fill_steps + 1, fill_steps + 1 + timed_steps):
-        t0 = time.perf_counter()
-        u.step(queries[i % len(queries)], i)
-        times.append(time.perf_counter() - t0)
-    return times
-
-
-def run_unit(cfg: dict, host_bits: np.ndarray, queries: list, fill_steps: int, timed_steps: int) -> list:
+def run_unit(cfg: dict, host_bits: np.ndarray, queries: list, fill_steps: int, timed_steps: int,
+             masks: list | None = None) -> list:
     """Seconds of each timed decode layer-step of one unit (BLAS on one
     thread): priming, `fill_steps` untimed steps, then `timed_steps` timed."""
     lim = _one_blas_thread()
     try:
-        return _timed(_prepare(cfg, host_bits, queries, fill_steps), queries, fill_steps, timed_steps)
+        spec = (host_bits, queries, masks)
+        u = _prepare(cfg, spec, fill_steps)
+        times = []
+        for i in range(fill_steps + 1, fill_steps + 1 + timed_steps):
+            t0 = time.perf_counter()
+            _step_unit(u, queries, masks, i)
+            times.append(time.perf_counter() - t0)
+        return times
     finally:
         if lim is not None:
             lim.__exit__(None, None, None)
@@ -130,13 +147,14 @@ def _recv(stream):
 
 
 def _worker() -> int:
-    """One unit in a process of its own: receive it, prime and fill, say
-    ready; then one timed step per start byte (its seconds sent back as a
-    float64), until the end byte."""
+    """A group of units in a process of its own: receive them, prime and
+    fill each, say ready; then, per start byte, one timed decode layer-step of
+    every unit of the group in turn (the seconds of the whole group sent back
+    as a float64), until the end byte."""
     inp, out = sys.stdin.buffer, sys.stdout.buffer
-    cfg, bits, queries, fill_steps = _recv(inp)
+    cfg, specs, fill_steps = _recv(inp)
     _one_blas_thread()
-    u = _prepare(cfg, bits, queries, fill_steps)
+    units = [(_prepare(cfg, spec, fill_steps), _unit_inputs(spec)) for spec in specs]
     out.write(b"R")
     out.flush()
     i = fill_steps + 1
@@ -145,20 +163,23 @@ def _worker() -> int:
         if c != b"G":
             return 0 if c == b"E" else 1
         t0 = time.perf_counter()
-        u.step(queries[i % len(queries)], i)
+        for u, (_, queries, masks) in units:
+            _step_unit(u, queries, masks, i)
         out.write(np.float64(time.perf_counter() - t0).tobytes())
         out.flush()
         i += 1
 
 
 class UnitPool:
-    """Units, one per worker process, stepped together: `step()` runs one
-    timed decode layer-step on every unit at once and returns the wall time
-    (seconds, the parent's clock from start to the last reply) and each
-    unit's own step time.  A watchdog ends the workers if `timeout_s` passes,
-    so no call blocks for longer."""
+    """Units spread over worker processes (one unit per process, or
+    `workers` processes taking the units in turn), stepped together:
+    `step()` runs one timed decode layer-step on every unit at once and
+    returns the wall time (seconds, the parent's clock from start to the last
+    reply) and each process's own time.  A watchdog ends the workers if
+    `timeout_s` passes, so no call blocks for longer."""
 
-    def __init__(self, cfg: dict, units: list, fill_steps: int, timeout_s: float = 600.0):
+    def __init__(self, cfg: dict, units: list, fill_steps: int, timeout_s: float = 600.0,
+                 workers: int | None = None):
         import subprocess
         import threading
         root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -167,12 +188,14 @@ class UnitPool:
         self._watchdog = threading.Timer(timeout_s, self._kill)
         self._watchdog.daemon = True
         self._watchdog.start()
+        n = len(units) if workers is None else max(1, min(workers, len(units)))
+        groups = [units[k::n] for k in range(n)]
         try:
-            for _ in units:
+            for _ in groups:
                 self.procs.append(subprocess.Popen([sys.executable, "-m", "oracle.decode_timing"], cwd=root,
                                                    env=env, stdin=subprocess.PIPE, stdout=subprocess.PIPE))
-            for p, (bits, queries) in zip(self.procs, units):
-                _send(p.stdin, (cfg, bits, queries, fill_steps))
+            for p, group in zip(self.procs, groups):
+                _send(p.stdin, (cfg, group, fill_steps))
             for p in self.procs:
                 if p.stdout.read(1) != b"R":
                     raise RuntimeError("an oracle worker did not get ready")
@@ -222,7 +245,7 @@ class UnitPool:
 
 def run_units_parallel(cfg: dict, units: list, fill_steps: int, timed_steps: int, workers: int,
                        timeout_s: float = 600.0) -> list:
-    """The timed steps of every (host_bits, queries) unit of `units`, run
+    """The timed steps of every (host_bits, queries[, masks]) unit of `units`, run
     `workers` processes at a time, the processes of a wave stepping together.
     Returns each unit's list of step seconds."""
     results = []

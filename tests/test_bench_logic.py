@@ -100,7 +100,7 @@ def test_gpu_line_keeps_the_contract(capsys):
     e = d["e2e"]
     assert e["unit"] == d["unit"] and e["h2d_bytes_per_step"] > nl * 1583 * w.block_bytes
     assert e["d2h_bytes_per_step"] == nl * (w.batch * w.n_queries * w.n_q_heads * (w.head_dim + 1) * 4)
-    assert d["gpu_launches"] == 6 * steps * nl
+    assert d["gpu_launches"] == bench.launches_per_layer_step(w) * steps * nl
     assert d["host_kv_layers"] == nl and d["cpus_bound"] is None
     assert d["kernels_isolated"]["sparse_attn"]["bound"] == "hbm"
 

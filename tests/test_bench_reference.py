@@ -13,7 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_reference_line_keeps_the_contract():
-    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "4", "--warmup", "3"],
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "4", "--warmup", "3",
+                        "--ref-units", "8"],
                        cwd=ROOT, capture_output=True, text=True, timeout=600,
                        env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
     assert r.returncode == 0, r.stderr[-2000:]
@@ -23,10 +24,13 @@ def test_reference_line_keeps_the_contract():
     assert d["impl"] == "reference"
     assert d["metric"] == bench.METRIC and d["unit"] == "layer-steps/s" and d["higher_is_better"] is True
     assert d["steps"] == 4 and d["warmup"] == 3 and d["n_gpus"] == 1
-    assert d["config"] == bench.headline_config(bench.W.WORKLOADS[bench.WORKLOAD], 8, 1)
+    nl = bench.BENCH_WORKLOADS[bench.WORKLOAD]["layers"]
+    assert d["config"] == bench.headline_config(bench.W.WORKLOADS[bench.WORKLOAD], nl, 1)
     assert d["value"] > 0 and d["vs_baseline"] is None and d["scaling"] == "weak"
-    # value and ms_per_step describe the same 8-layer step, as on the GPU arm
-    assert abs(d["value"] - 8 / (d["ms_per_step"] * 1e-3)) <= 1e-9 * d["value"]
+    # a timed step of this arm is one layer-step of the whole batch: value needs no layer scaling
+    assert d["step_layers"] == 1
+    assert abs(d["value"] - 1 / (d["ms_per_step"] * 1e-3)) <= 1e-9 * d["value"]
+    assert "scaled from 8 to the 128 units" in d["cpu_baseline"]["sample"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

@@ -357,3 +357,70 @@ def test_pipeline_with_residency_loss_step_by_step():
         _check_pool_holds_slot_blocks(L.pool, st, host_bits)
     assert lost_total > 0
 
+
+
+def test_full_size_reasoning_layer_with_appends():
+    """One layer of the long-output reasoning configuration at full size
+    (batch 64, 32/8 heads: 512 units, 1,088 blocks per head, budget 128,
+    cap 8) near the end of its 17K context, built as the bench builds it, run
+    for five decode steps with one appended token per sequence per step; the
+    context crosses a block boundary on the way.  Plans are checked in full;
+    on 16 sampled units (the first and last included) the host rows the
+    append wrote through the mapping, the grown summaries, the selection, the
+    attention over the working set of the previous step with the new token in
+    place, and the bytes of every occupied slot."""
+    from bench import build_workload_state
+    w = W.WORKLOADS["qwen8b_reasoning"]
+    c0 = w.max_blocks * w.block_tokens - 16 - 3          # 17,389: three appends to the block boundary
+    w = w.with_(context=c0)
+    st = build_workload_state(w, steps=6, device=DEV)
+    d, L, pipe, qs = st["dims"], st["layer"], st["pipe"], st["queries"]
+    units = sampled_units(w, 16)
+    scale = 1 / math.sqrt(128)
+    G, K = w.group, w.budget_blocks
+    before = {(b, h): L.host_kv[b:b + 1, h:h + 1].clone() for b, h in units}   # host bytes before any append
+    pipe.prime([qs[0]])
+    pipe.wait_all()
+    torch.cuda.synchronize()
+    grown = {u: kv_split(before[u]) for u in units}                           # f64 keys / values per unit
+    for t in range(1, 6):
+        st_prev, lu_prev = np_i32(L.slot_table), np_i32(L.last_used)
+        ctx_before = np_i32(pipe.ctx_len)
+        k_new, v_new = W.append_rows(w, 0, t, DEV)
+        pipe.step(t, [qs[t]], appended=[(k_new, v_new)])
+        pipe.wait_all()
+        torch.cuda.synchronize()
+        ctx = np_i32(pipe.ctx_len)
+        np.testing.assert_array_equal(ctx, ctx_before + 1)
+        sel = np_i32(L.sel)
+        plan = O.plan_fetch(sel, st_prev, lu_prev, t, w.fetch_cap)
+        np.testing.assert_array_equal(np_i32(L.slot_table), plan["slot_table"])
+        np.testing.assert_array_equal(np_i32(L.last_used), plan["last_used"])
+        kn, vn = f64(k_new.cpu()), f64(v_new.cpu())
+        q = f64(qs[t].cpu())
+        for b, h in units:
+            k, v = grown[(b, h)]
+            n, tok = divmod(int(ctx_before[b]), 16)
+            k[0, 0, n, tok], v[0, 0, n, tok] = kn[b, h], vn[b, h]
+            kf, vf = kv_split(L.host_kv[b:b + 1, h:h + 1])
+            np.testing.assert_array_equal(kf, k)                             # the append reached host KV
+            np.testing.assert_array_equal(vf, v)
+            kmin, kmax = O.block_summaries(k, ctx[b:b + 1])
+            valid = ~np.isnan(kmin)
+            np.testing.assert_array_equal(f64(L.kmin[b:b + 1, h:h + 1].cpu())[valid], kmin[valid])
+            np.testing.assert_array_equal(f64(L.kmax[b:b + 1, h:h + 1].cpu())[valid], kmax[valid])
+            qu = q[b:b + 1, :, h * G:(h + 1) * G]
+            sc = O.lookahead_scores(qu, kmin, kmax, ctx[b:b + 1], 16)
+            ref_sel, _ = O.select_topk(sc, ctx[b:b + 1], K, 16)
+            assert_selection_matches(sel[b:b + 1, h:h + 1], ref_sel, sc, ctx[b:b + 1], K)
+            stu = st_prev[b:b + 1, h:h + 1]
+            pk = np.zeros((1, 1, K, 16, 128))
+            pv = np.zeros_like(pk)
+            for s in np.nonzero(stu[0, 0] >= 0)[0]:
+                pk[0, 0, s], pv[0, 0, s] = k[0, 0, stu[0, 0, s]], v[0, 0, stu[0, 0, s]]
+            o_ref, lse_ref = O.sparse_attention(qu, pk, pv, stu, ctx[b:b + 1], scale)
+            assert_attention_close(L.out[b:b + 1, :, h * G:(h + 1) * G], L.lse[b:b + 1, :, h * G:(h + 1) * G],
+                                   o_ref, lse_ref)
+            hb = W.bf16_bits(L.host_kv[b:b + 1, h:h + 1])
+            _check_pool_holds_slot_blocks(L.pool[b:b + 1, h:h + 1], plan["slot_table"][b:b + 1, h:h + 1], hb)
+    assert int(np_i32(pipe.ctx_len)[0]) == c0 + 5                           # crossed 17,392

@@ -89,7 +89,7 @@ def test_pipeline_with_score_victims_step_by_step():
         sc = O.lookahead_scores(f64(q), kmin, kmax, cnp, 16)
         gsc = L.scores.cpu().numpy()
         nv = int(O.n_valid_blocks(cnp, 16).min())
-        np.testing.assert_allclose(gsc[:, :, :nv], sc[:, :, :nv], rtol=SCORE_REL, atol=1e-3)
+        np.testing.assert_allclose(gsc[:, :, :nv], sc[:, :, :nv], rtol=SCORE_REL, atol=0)
         ref_sel, _ = O.select_topk(sc, cnp, K, 16)
         sel = np_i32(L.sel)
         assert_selection_matches(sel, ref_sel, sc, cnp, K)
