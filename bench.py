@@ -107,7 +107,7 @@ def headline_config(w, nl: int, world: int, name: str = WORKLOAD) -> dict:
 QUERY_RING = 256
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic_llama8b_32k.json")
-KERNELS = ("sparse_attn", "score_select", "plan_fetch", "prefetch")
+KERNELS = ("sparse_attn", "score_select_plan", "prefetch")
 
 
 # ------------------------------------------------------------------ setup
@@ -460,15 +460,17 @@ def isolated_kernel_ms(st, reps: int = 20) -> dict:
     s = torch.cuda.current_stream()
     ctx = pipe.ctx_len
     st_c, lu_c = L.slot_table.clone(), L.last_used.clone()
+    fs_c, fb_c, nf_c = L.fetch_slot.clone(), L.fetch_block.clone(), L.n_fetch.clone()
     calls = {
         "sparse_attn": lambda: lsk.sparse_attn(d, q, L.pool, L.slot_table, ctx, pipe.scale, L.out, L.lse, pipe.ws,
                                                stream=s),
         # the gather of the last plan of the timed run (re-copies the same blocks)
         "prefetch": lambda: lsk.prefetch(d, L.host_kv, L.fetch_slot, L.fetch_block, L.n_fetch, L.pool, stream=s),
-        "score_select": lambda: lsk.score_select(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, pipe.ws, stream=s),
+        # scores + top-K + plan in one launch, on copies of the slot table and recency
+        "score_select_plan": lambda: lsk.score_select_plan(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, None, st_c,
+                                                           lu_c, 10 ** 6, None, fs_c, fb_c, nf_c, pipe.ws, stream=s),
         "select_only": lambda: lsk.select_topk(d, pipe.ws.view(torch.float32), ctx, L.sel, L.sel_score, stream=s),
-        "plan_fetch": lambda: lsk.plan_fetch(d, L.sel, st_c, lu_c, 10 ** 6, L.fetch_slot, L.fetch_block,
-                                             L.n_fetch, stream=s),
+        "plan_fetch": lambda: lsk.plan_fetch(d, L.sel, st_c, lu_c, 10 ** 6, fs_c, fb_c, nf_c, stream=s),
         # a1 at admission: summaries of every block from the pinned host KV (rewrites the same values)
         "build_summaries": lambda: lsk.build_summaries(d, L.host_kv, ctx, L.kmin, L.kmax, stream=s),
     }
@@ -748,7 +750,7 @@ def run_longctx(args, device):
                          "h2d_gbs": gbs, "h2d_frac": gbs / h2d["peak_gbs"],
                          "overlap_efficiency": overlap_efficiency(iso, per_ls)["value"],
                          "compute_ms": overlap_efficiency(iso, per_ls)["compute_ms"],
-                         "isolated_ms": {k: iso[k] for k in ("sparse_attn", "score_select", "plan_fetch", "prefetch")}})
+                         "isolated_ms": {k: iso[k] for k in ("sparse_attn", "score_select_plan", "prefetch")}})
             del pipe
         del layers
         torch.cuda.empty_cache()
@@ -855,7 +857,7 @@ def run_reasoning(args, device):
             "overlap_efficiency": overlap_efficiency(iso, per_ls)["value"],
             "compute_ms": overlap_efficiency(iso, per_ls)["compute_ms"],
             "attention_hbm_gbs": attn_gbs, "host_enqueue_ms_per_step": host_ms / steps,
-            "isolated_ms": {k: iso[k] for k in ("sparse_attn", "score_select", "plan_fetch", "prefetch")}})
+            "isolated_ms": {k: iso[k] for k in ("sparse_attn", "score_select_plan", "prefetch")}})
         del pipe
     line = {
         "metric": "long-output reasoning decode with appends: layer-steps/s, tokens/s, H2D vs PCIe roof, "
@@ -1110,7 +1112,10 @@ def algorithmic_bytes(w, fetched_blocks_per_layer_step):
         # resident KV (every slot is occupied after warm-up) + queries + outputs
         "sparse_attn": units * w.budget_blocks * block + q_bytes + out_bytes,
         # min/max summaries of every valid block + draft queries + scores written and read + selection
-        "score_select": units * nv * 2 * w.head_dim * 2 + q_bytes + 2 * units * nv * 4 + units * w.budget_blocks * 8,
+        # plus the plan's slot table / recency read and written and its fetch lists
+        "score_select_plan": (units * nv * 2 * w.head_dim * 2 + q_bytes + 2 * units * nv * 4
+                              + units * w.budget_blocks * 8 + units * w.budget_blocks * 4 * 4
+                              + units * w.fetch_cap * 8 + units * 4),
         "select_only": units * nv * 4 + units * w.budget_blocks * 8,
         # slot table + last-used read and written, selection read, fetch lists written
         "plan_fetch": units * w.budget_blocks * 4 * 5 + units * w.fetch_cap * 8 + units * 4,
@@ -1126,11 +1131,11 @@ def overlap_efficiency(iso_ms, pipeline_ms_per_layer_step):
     """eta = (T_compute + T_fetch - T_pipeline) / min(T_compute, T_fetch) per
     layer-step: 1 when the gather hides completely behind (or hides) the
     compute, 0 when they run back to back.  T_fetch is the isolated gather;
-    T_compute the compute path of a layer-step as the pipeline runs it, with
-    scores + top-K on their own stream beside the attention:
-    max(attention, scores + top-K) + plan, from isolated times.  T_pipeline
-    is the measured per-layer-step time of the pipeline."""
-    t_c = max(iso_ms["sparse_attn"], iso_ms["score_select"]) + iso_ms["plan_fetch"]
+    T_compute the compute path of a layer-step as the pipeline runs it on
+    one stream: attention + (scores, top-K and plan in one launch), from
+    isolated times.  T_pipeline is the measured per-layer-step time of the
+    pipeline."""
+    t_c = iso_ms["sparse_attn"] + iso_ms["score_select_plan"]
     t_f = iso_ms["prefetch"]
     return {"value": (t_c + t_f - pipeline_ms_per_layer_step) / min(t_c, t_f),
             "compute_ms": t_c, "fetch_ms": t_f, "pipeline_ms": pipeline_ms_per_layer_step}
@@ -1153,9 +1158,9 @@ def token_kv_intensity(w, fetched_blocks_per_layer_step):
 
 
 def launches_per_layer_step(w) -> int:
-    """Kernels of one layer-step: attention and its merge, scores, top-K,
-    plan and gather, plus the residency loss when the workload has one."""
-    return 6 + (1 if w.evict_prob > 0 else 0)
+    """Kernels of one layer-step: attention, scores + top-K + plan (one
+    launch) and gather, plus the residency loss when the workload has one."""
+    return 3 + (1 if w.evict_prob > 0 else 0)
 
 
 def emit_gpu(args, res, world):

@@ -89,9 +89,11 @@ enum {
 #define OASIS_DEVERR_APPEND_FULL 0x4u  /* append position at or beyond N * P */
 #define OASIS_DEVERR_DUPLICATE   0x8u  /* a block resident twice / selected twice */
 
-/* Workspace bytes needed by oasis_score_select and oasis_sparse_attn for
- * these dims (one region each, so the two may run concurrently on different
- * streams with the same workspace).  The workspace is device memory that
+/* Workspace bytes needed by oasis_score_select, oasis_score_select_plan and
+ * oasis_sparse_attn for these dims (the scoring and the attention use
+ * separate regions, so they may run concurrently on different streams with
+ * the same workspace; two attention calls, or two scoring calls, on one
+ * workspace must be stream-ordered).  The workspace is device memory that
  * must be zero-filled once before its first use; the kernels leave it ready
  * for the next call.  One workspace per concurrently running layer. */
 size_t oasis_workspace_bytes(const oasis_dims* d);
@@ -154,6 +156,27 @@ int oasis_score_select(const oasis_dims* d, const void* q, const void* kmin,
 int oasis_score_select_rows(const oasis_dims* d, const void* q, int32_t row_begin,
                             int32_t row_count, const void* kmin, const void* kmax,
                             const int32_t* ctx_len, int32_t* sel, float* sel_score,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* a2 + a3 + a4 in one launch (OasisKV Figure 8: per layer the drafts'
+ * prediction, the selection and the residency diff with the capped plan run
+ * back to back before the transfer can start).  Results are those of
+ * oasis_lookahead_scores, oasis_select_topk and oasis_plan_fetch (scores ==
+ * NULL) or oasis_plan_fetch_scored (scores != NULL) called in turn, bit for
+ * bit.  scores: NULL keeps the block scores in the workspace; else device fp32
+ * [B][Hkv][N] that receives them and orders the victims by score.  step_dev:
+ * NULL uses `step`, else the step number is read from device memory at run
+ * time (graph capture).  sel_score may be NULL.  Every buffer is device
+ * memory; ws: a workspace of oasis_workspace_bytes(d) bytes.  The plan reads
+ * and rewrites slot_table / last_used, so it must run after any attention
+ * that reads this layer's slot table.  EINVAL also when the fused kernel's
+ * shared memory cannot hold one unit's N keys and plan (4*N + 8*K + 36*K
+ * bytes above 226 KiB, i.e. only near N = 32768 with a large K). */
+int oasis_score_select_plan(const oasis_dims* d, const void* q, const void* kmin,
+                            const void* kmax, const int32_t* ctx_len, int32_t* sel,
+                            float* sel_score, float* scores, int32_t* slot_table,
+                            int32_t* last_used, int32_t step, const int32_t* step_dev,
+                            int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
                             void* ws, size_t ws_bytes, void* stream);
 
 /* Prediction quality (OasisKV Figure 4: top-K accuracy of the previous token
@@ -270,34 +293,28 @@ typedef struct oasis_layer {
 } oasis_layer;
 
 /* Streams (cudaStream_t; NULL is the default stream) and this layer's events
- * (cudaEvent_t, created by the caller) of a layer-step.  score may equal main
- * (no overlap).  With in_graph
- * set (inside a capture of a whole step) the main stream does not wait for
- * fetch_done and the score stream forks from main through `fork` instead of
- * waiting for plan_ready.  timing: optional begin / end events recorded
- * around attention (main), score+select (score), plan (main) and gather (copy),
- * in that order; NULL entries are skipped. */
+ * (cudaEvent_t, created by the caller) of a layer-step.  With in_graph set
+ * (inside a capture of a whole step) the main stream does not wait for
+ * fetch_done.  timing: optional begin / end events recorded around the
+ * attention (main), the fused scores + top-K + plan (main) and the gather
+ * (copy), in that order; NULL entries are skipped. */
 typedef struct oasis_step_sync {
     void* main;
-    void* score;
     void* copy;
     void* fetch_done;       /* recorded on copy after the gather */
     void* plan_ready;       /* recorded on main after the plan */
-    void* sel_ready;        /* recorded on score after the selection */
-    void* fork;             /* in_graph only */
     int32_t in_graph;
-    void* timing[8];
+    void* timing[6];
 } oasis_step_sync;
 
 /* Decode step `step` of one layer, in the order above: [wait fetch_done] ->
  * attention(q, scale) -> [residency loss: evict_mask, may be NULL] -> scores +
- * top-K -> plan (step number `step`, or *step_dev when step_dev != NULL) ->
- * gather.  Same buffers, workspace and results as the individual calls; the
- * first error returns before anything after it is enqueued.  q is read on
- * main (attention) and on score (scores + top-K); outside a graph the score
- * stream follows earlier main-stream work only through plan_ready, so a
- * caller that writes q on main must also order score after that write (an
- * event recorded on main and waited on by score). */
+ * top-K + plan in one launch (oasis_score_select_plan; step number `step`, or
+ * *step_dev when step_dev != NULL) -> gather on copy.  Same buffers,
+ * workspace and results as the individual calls; the first error returns
+ * before anything after it is enqueued.  Everything but the gather runs on
+ * main, so queries written on main before the call are ordered before both
+ * readers. */
 int oasis_decode_layer_step(const oasis_dims* d, const oasis_layer* layer, const void* q,
                             const int32_t* ctx_len, const uint8_t* evict_mask, int32_t step,
                             const int32_t* step_dev, float scale, void* ws, size_t ws_bytes,
@@ -319,8 +336,11 @@ int oasis_prefetch(const oasis_dims* d, const void* host_kv, const int32_t* fetc
  * every occupied slot of (b, h),
  *   out = sum softmax(scale * q.k) v,   lse = log sum exp(scale * q.k);
  * no occupied slot / no valid token gives out = 0, lse = -inf.  bf16 inputs,
- * fp32 accumulation.  scale must be positive and finite (OASIS_EINVAL
- * otherwise).  q, pool, slot_table, ctx_len, out, lse, ws: device. */
+ * fp32 accumulation (the softmax weights enter the P.V product as a bf16
+ * head plus a bf16 remainder).  scale must be positive and finite
+ * (OASIS_EINVAL otherwise).  q, pool, slot_table, ctx_len, out, lse, ws:
+ * device.  Value rows past the context in a partly filled block are never
+ * multiplied in (non-finite stale bytes there do not reach out). */
 int oasis_sparse_attn(const oasis_dims* d, const void* q, const void* pool,
                       const int32_t* slot_table, const int32_t* ctx_len, float scale,
                       float* out, float* lse, void* ws, size_t ws_bytes, void* stream);

@@ -74,10 +74,10 @@ class Layer(ctypes.Structure):
 
 
 class StepSync(ctypes.Structure):
-    """oasis_step_sync: streams, this layer's events, graph flag, timing events."""
-    _fields_ = [("main", ctypes.c_void_p), ("score", ctypes.c_void_p), ("copy", ctypes.c_void_p),
-                ("fetch_done", ctypes.c_void_p), ("plan_ready", ctypes.c_void_p), ("sel_ready", ctypes.c_void_p),
-                ("fork", ctypes.c_void_p), ("in_graph", ctypes.c_int32), ("timing", ctypes.c_void_p * 8)]
+    """oasis_step_sync: streams, this layer's events, graph flag, timing events
+    (begin / end of the attention, the fused scores + top-K + plan, the gather)."""
+    _fields_ = [("main", ctypes.c_void_p), ("copy", ctypes.c_void_p), ("fetch_done", ctypes.c_void_p),
+                ("plan_ready", ctypes.c_void_p), ("in_graph", ctypes.c_int32), ("timing", ctypes.c_void_p * 6)]
 
 
 _LIB = None
@@ -94,6 +94,8 @@ _SIGS = {
     "oasis_score_select_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V]),
     "oasis_score_select_rows": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _I32, _I32, _V, _V, _V, _V, _V, _V,
                                                ctypes.c_size_t, _V]),
+    "oasis_score_select_plan": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _V, _V, _V, _V, _V, _I32, _V,
+                                               _V, _V, _V, _V, ctypes.c_size_t, _V]),
     "oasis_block_overlap": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V]),
     "oasis_plan_fetch": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _I32, _V, _V, _V, _V]),
     "oasis_plan_fetch_scored": (ctypes.c_int, [ctypes.POINTER(Dims), _V, _V, _V, _V, _I32, _V, _V, _V, _V]),
@@ -287,6 +289,29 @@ def score_select_rows(d, q, row_begin, row_count, kmin, kmax, ctx_len, sel, sel_
                                          _stream(stream)), w)
 
 
+def score_select_plan(d, q, kmin, kmax, ctx_len, sel, sel_score, scores, slot_table, last_used, step, step_dev,
+                      fetch_slot, fetch_block, n_fetch, ws, stream=None):
+    """Scores, top-K and the capped plan in one launch.  scores: None keeps the
+    block scores in the workspace (LRU victims), else fp32 [B][Hkv][N] that
+    receives them (score-ordered victims); step_dev: None uses ``step``, else an
+    int32 device tensor whose first element is read on the device."""
+    w = "oasis_score_select_plan"
+    z = _Sizes(d, w)
+    _check(lib().oasis_score_select_plan(ctypes.byref(d), _arg(q, w, "q", _BF16, z.q),
+                                         _arg(kmin, w, "kmin", _BF16, z.summary),
+                                         _arg(kmax, w, "kmax", _BF16, z.summary),
+                                         _arg(ctx_len, w, "ctx_len", _I32_T, z.b), _arg(sel, w, "sel", _I32_T, z.k),
+                                         _arg(sel_score, w, "sel_score", _F32, z.k, nullable=True),
+                                         _arg(scores, w, "scores", _F32, z.scores, nullable=True),
+                                         _arg(slot_table, w, "slot_table", _I32_T, z.k),
+                                         _arg(last_used, w, "last_used", _I32_T, z.k), int(step),
+                                         _arg(step_dev, w, "step_dev", _I32_T, 1, nullable=True),
+                                         z.fetch_list(fetch_slot, "fetch_slot"),
+                                         z.fetch_list(fetch_block, "fetch_block"),
+                                         _arg(n_fetch, w, "n_fetch", _I32_T, z.units), *_ws(ws, w),
+                                         _stream(stream)), w)
+
+
 def block_overlap(d, a, b, count, stream=None):
     """count[b][h] = distinct ids of list b also in list a (int32 [B][Hkv][K] each)."""
     w = "oasis_block_overlap"
@@ -369,7 +394,7 @@ def make_layer(d, host_kv, kmin, kmax, pool, slot_table, last_used, sel, sel_sco
 
 
 def decode_layer_step(d, layer: Layer, q, ctx_len, evict_mask, step, step_dev, scale, ws, sync: StepSync):
-    """One layer's decode step (attention, [loss], scores + top-K, plan, gather) in one call;
+    """One layer's decode step (attention, [loss], scores + top-K + plan in one launch, gather) in one call;
     `layer` comes from make_layer, which checked its buffers."""
     w = "oasis_decode_layer_step"
     z = _Sizes(d, w)

@@ -1,4 +1,5 @@
-// attn.cuh - sparse GQA decode attention over the resident pool slots.
+// attn.cuh - sparse GQA decode attention over the resident pool slots, on
+// the 5th-generation tensor cores.
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
 // Prefetching, Figure 7 (right): the verification query and the drafts are
@@ -6,47 +7,72 @@
 // per-head slot table says which block each pool slot holds.
 //
 // Work split (stream-K): the T = B*Hkv*K pool slots, in (sequence, KV head,
-// slot) order, are cut into NS contiguous ranges, one per "stream".  A
-// stream is QG warps that share a 3-stage ring of 8 KiB shared-memory
-// buffers; its first warp's lane 0 fills the ring with TMA (two 64-column
-// boxes per slot, 128-byte swizzle, L2 evict-first), skipping free slots and
-// blocks beyond the context.  Streams are independent - there is no CTA-wide
-// barrier anywhere in the kernel - so an SM keeps up to 8 streams x 24 KiB
-// of KV in flight.  A stream writes one normalised partial (output and
-// log-sum-exp) for every (sequence, KV head) unit its range touches; a second
-// kernel, launched as a programmatic dependent, merges the partials of each
-// unit in stream order (one warp per query row, every load in flight).
+// slot) order, are cut into NS contiguous ranges, one per CTA (one CTA per
+// SM).  A CTA walks its range one (sequence, KV head) "unit" piece at a
+// time.  Per piece the producer warp lists the occupied slots (free slots and
+// blocks past the context skipped), TMA-loads the unit's query rows, and
+// streams the listed slots through a 4-stage ring in tiles of 4 slots (64
+// tokens): four 2 KiB boxes per slot (K and V, each as two 64-column halves,
+// 128-byte swizzle) so that a tile lands as K[64 tokens][128] and
+// V[64 tokens][128] in the layouts the tensor core reads.
 //
-// Math per slot (16 tokens), per warp, on the warp-level tensor-core path
-// (mma.sync m16n8k16, bf16 in, fp32 accumulate), tokens as the M dimension
-// and the Qn*G query rows of the KV head as N (8 per n-tile):
-//   S^T[16 x 8] = K[16 x 128] . Q^T           (8 k-steps per n-tile)
-//   online softmax per query column (max over tokens by xor-shuffles)
-//   P^T fragments -> PV B operand by movmatrix.trans (no smem round trip);
-//   P enters as a bf16 head plus a bf16 remainder (two MMAs), so the weights
-//   keep ~16 significant bits
-//   O^T[128 x 8] += V^T[128 x 16] . P^T       (8 m-tiles per n-tile)
-// With more than 4 n-tiles (Qn*G > 32) a stream is two warps, each owning
-// half of the query n-tiles.
+// Math per tile, with the unit's Qn*G query rows as the MMA M dimension
+// (padded to 64; M = 64 puts row r in TMEM lane 32*(r/16) + r%16):
+//   S[64 x 64]   = Q[64 x 128] . K^T          8 tcgen05.mma, K-major A and B
+//   softmax      4 warps, one per TMEM lane quadrant, each thread owning two
+//                query rows of 16 tokens (a quad of threads shares a row):
+//                running max (moved only when a tile exceeds it by 2^8, so
+//                the accumulator is rarely rescaled), exponentials, row sums
+//   P            written to shared memory as a bf16 head plus a bf16
+//                remainder (~16 significant bits), 128-byte swizzled
+//   O[64 x 128] += P_head . V + P_rest . V    V read MN-major, 4 x 2 MMAs
+// S is double-buffered in TMEM (S of tile i+1 runs while tile i's softmax
+// does), P double-buffered in shared memory; O stays in TMEM for the whole
+// piece.  One thread issues every MMA; mbarriers carry every hand-off, with
+// bounded waits.
+//
+// A unit covered by one CTA is normalised and written directly.  A unit
+// split over CTAs: each writes a normalised partial (output, log2-sum-exp),
+// then takes a ticket with an atomic counter; the last CTA to arrive merges
+// all partials of the unit (they are in L2), writes the output and resets the
+// counter for the next call.  No CTA ever waits for another.
 #pragma once
 
 #include "common.cuh"
 
 namespace oasis {
 
-constexpr int kAttnStreamsPerCta = 4;
-constexpr int kAttnStages = 3;
-constexpr int kAttnWindow = 256;                          // slots listed per pass
-constexpr int kAttnStreamSmem = kAttnStages * kBlockBytes + kAttnWindow * 8 + 64;
+constexpr int kAttnTileSlots = 4;                                 // slots per tile
+constexpr int kAttnStages = 4;                                    // K/V ring depth
+constexpr int kAttnRegion = 64 * 128;                             // 64 rows x 128 B = 8 KiB
+constexpr int kAttnStageBytes = 4 * kAttnRegion;                  // K lo, K hi, V lo, V hi
+constexpr int kAttnRows = 64;                                     // MMA M
+constexpr int kAttnMaxList = 1024;                                // slots of one unit (K <= 1024)
+constexpr int kAttnThreads = 192;                                 // producer, MMA, 4 softmax warps
+constexpr int kAttnTmemCols = 256;                                // S x 2 (64 columns each) + O (128)
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int NTW, int QG>
-struct AttnCfg {
-    static constexpr int kWarps = kAttnStreamsPerCta * QG;
-    static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kStreamStride = (kAttnStreamSmem + 1023) / 1024 * 1024;
-    static constexpr int kSmem = kAttnStreamsPerCta * kStreamStride + 1024;
-};
+constexpr int kAttnOffQ = kAttnStages * kAttnStageBytes;          // 2 buffers x (lo, hi)
+constexpr int kAttnOffP = kAttnOffQ + 4 * kAttnRegion;            // 2 buffers x (head, rest)
+constexpr int kAttnOffList = kAttnOffP + 4 * kAttnRegion;         // 2 x kAttnMaxList ints
+constexpr int kAttnOffBar = kAttnOffList + 2 * kAttnMaxList * 4;
+constexpr int kAttnNumBars = 26;
+constexpr int kAttnOffMisc = kAttnOffBar + kAttnNumBars * 8;
+constexpr int kAttnSmem = kAttnOffMisc + 64 + 1024;              // + alignment slack
+
+// mbarrier indices
+constexpr int kBarFull = 0;     // [4]  tile landed (producer expect_tx)
+constexpr int kBarEmpty = 4;    // [4]  tile's K and V consumed (MMA commit)
+constexpr int kBarSFull = 8;    // [2]  S computed (MMA commit)
+constexpr int kBarSFree = 10;   // [2]  S read by the 4 softmax warps
+constexpr int kBarPFull = 12;   // [2]  P written by the 4 softmax warps
+constexpr int kBarPFree = 14;   // [2]  P consumed (MMA commit after PV)
+constexpr int kBarQFull = 16;   // [2]  unit's query rows landed
+constexpr int kBarQFree = 18;   // [2]  query rows no longer read (MMA commit)
+constexpr int kBarLFull = 20;   // [2]  piece's slot list written (producer)
+constexpr int kBarLFree = 22;   // [2]  slot list no longer read (MMA thread + softmax leader)
+constexpr int kBarODone = 24;   // the piece's last PV has completed
+constexpr int kBarFinal = 25;   // teardown: every MMA issued has completed
 
 // Streams whose ranges touch unit u: [first, last].  Slot s belongs to
 // stream floor(s * NS / T), so every stream in between touches u.
@@ -56,420 +82,480 @@ __host__ __device__ __forceinline__ void attn_unit_streams(long long u, long lon
     *last = ((u + 1) * K - 1) * NS / T;
 }
 
-// floor(x / t) for x < 2^53, t < 2^31 without the 64-bit integer division
-// routine: a double quotient, then an exact integer correction.
-__device__ __forceinline__ long long floor_div_small(long long x, long long t) {
-    long long q = static_cast<long long>(static_cast<double>(x) / static_cast<double>(t));
-    if (q * t > x) --q;
-    else if ((q + 1) * t <= x) ++q;
-    return q;
+// Waits unless the CTA has given up; a wait that runs out flags the CTA and
+// the device error word.  Returns whether the awaited phase completed.
+__device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *abort_flag = 1;
+    raise_dev_error(OASIS_DEVERR_TIMEOUT);
+    return false;
 }
 
-// Merges the stream partials of each (unit, query row) in stream order:
-// lse = log sum_p exp(lse_p), out = sum_p exp(lse_p - lse) * o_p.  One warp
-// per (unit, row); lane j holds partial j's lse, lane c owns channels
-// 4c..4c+3.  Up to 12 partials (the usual case: 8 streams per SM give about
-// 10 per unit on the 32K Llama layer) are read in one round trip: every lse
-// and output load is issued before any of them is used.  Small CTAs, and at
-// most 80 registers so that 12 CTAs fit an SM and the grid runs in one wave.
-constexpr int kMergeWarps = 2;
-constexpr int kMergeFast = 12;
-
-__global__ void __launch_bounds__(32 * kMergeWarps, 12) attn_merge_kernel(Dims d, int n_streams,
-                                                                      const float* __restrict__ ws_o,
-                                                                      const float* __restrict__ ws_lse,
-                                                                      float* __restrict__ out,
-                                                                      float* __restrict__ lse_out) {
-    const float kNegInf = -__int_as_float(0x7f800000);
-    const int lane = threadIdx.x & 31;
-    const int G = d.G();
-    const int rows = d.Qn * G;
-    const int units = d.B * d.Hkv;
-    const int gw = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);   // < units * rows <= 2^22
-    // partials are produced by the attention grid this kernel depends on
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (gw >= units * rows) return;
-    const int u = gw / rows;
-    const int r = gw - u * rows;
-    // streams whose ranges touch unit u (attn_unit_streams): slot s is in stream floor(s*NS/T)
-    const long long T = static_cast<long long>(units) * d.K;
-    const long long first = floor_div_small(static_cast<long long>(u) * d.K * n_streams, T);
-    const long long last = floor_div_small((static_cast<long long>(u + 1) * d.K - 1) * n_streams, T);
-    const int np = static_cast<int>(last - first + 1);
-    const long long p0 = first + u;
-    const float4* src = reinterpret_cast<const float4*>(ws_o + (p0 * rows + r) * kHeadDim) + lane;
-    const long long pstride = static_cast<long long>(rows) * (kHeadDim / 4);
-    float M = kNegInf, L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (np <= kMergeFast) {
-        const float lj = lane < np ? ws_lse[(p0 + lane) * rows + r] : kNegInf;
-        float4 v[kMergeFast];
-#pragma unroll
-        for (int k = 0; k < kMergeFast; ++k) v[k] = k < np ? src[k * pstride] : make_float4(0.f, 0.f, 0.f, 0.f);
-        M = lj;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
-        const float wj = (lj == kNegInf) ? 0.f : __expf(lj - M);
-        L = wj;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
-#pragma unroll
-        for (int k = 0; k < kMergeFast; ++k) {
-            const float w = __shfl_sync(0xFFFFFFFFu, wj, k);
-            if (w > 0.f) {                      // empty partials may hold stale outputs
-                acc.x += w * v[k].x;
-                acc.y += w * v[k].y;
-                acc.z += w * v[k].z;
-                acc.w += w * v[k].w;
-            }
-        }
-    } else {
-        for (int j0 = 0; j0 < np; j0 += 32) {
-            const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;
-            M = fmaxf(M, lj);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
-        if (M != kNegInf) {
-            for (int j0 = 0; j0 < np; j0 += 32) {
-                const float lj = j0 + lane < np ? ws_lse[(p0 + j0 + lane) * rows + r] : kNegInf;
-                const float wj = lj == kNegInf ? 0.f : __expf(lj - M);
-                float ws = wj;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xFFFFFFFFu, ws, o);
-                L += ws;
-                const int nj = min(32, np - j0);
-                for (int k0 = 0; k0 < nj; k0 += 8) {
-                    float4 v[8];
-                    float wk[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        wk[k] = __shfl_sync(0xFFFFFFFFu, wj, (k0 + k) & 31);
-                        v[k] = (k0 + k < nj && wk[k] > 0.f) ? src[(j0 + k0 + k) * pstride]
-                                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float w = k0 + k < nj ? wk[k] : 0.f;
-                        acc.x += w * v[k].x;
-                        acc.y += w * v[k].y;
-                        acc.z += w * v[k].z;
-                        acc.w += w * v[k].w;
-                    }
-                }
-            }
-        }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    acc.x *= inv;
-    acc.y *= inv;
-    acc.z *= inv;
-    acc.w *= inv;
-    const int b = u / d.Hkv, h = u - b * d.Hkv;
-    const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
-    reinterpret_cast<float4*>(out + orow * kHeadDim)[lane] = acc;
-    if (lane == 0) lse_out[orow] = L > 0.f ? M + logf(L) : kNegInf;
-}
-
-template <int NTW, int QG>
-__global__ void __launch_bounds__(AttnCfg<NTW, QG>::kThreads)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_pool, Dims d, const uint16_t* __restrict__ q,
-                       const int32_t* __restrict__ slot_table, const int32_t* __restrict__ ctx_len,
-                       float scale_log2, int n_streams, float* __restrict__ ws_o, float* __restrict__ ws_lse) {
-    using Cfg = AttnCfg<NTW, QG>;
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_pool, const __grid_constant__ CUtensorMap tm_q, Dims d,
+                       const int32_t* __restrict__ slot_table, const int32_t* __restrict__ ctx_len, float scale_log2,
+                       int n_streams, float* __restrict__ out, float* __restrict__ lse_out, float* ws_o,
+                       float* ws_lse, int* ws_ticket) {
     const float kNegInf = -__int_as_float(0x7f800000);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ring = smem;
+    uint8_t* sQ = smem + kAttnOffQ;
+    uint8_t* sP = smem + kAttnOffP;
+    int* s_list = reinterpret_cast<int*>(smem + kAttnOffList);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kAttnOffBar);
+    int* misc = reinterpret_cast<int*>(smem + kAttnOffMisc);
+    int* s_nlist = misc;                                  // [2]
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc + 2);
+    volatile int* s_abort = misc + 3;
+    volatile int* s_last = misc + 4;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ls = warp / QG, qg = warp % QG;             // local stream, query group
-    const long long gs = static_cast<long long>(blockIdx.x) * kAttnStreamsPerCta + ls;
-
-    uint8_t* ring = smem + ls * Cfg::kStreamStride;
-    int* l_slot = reinterpret_cast<int*>(ring + kAttnStages * kBlockBytes);
-    int* l_nv = l_slot + kAttnWindow;
-    uint64_t* full = reinterpret_cast<uint64_t*>(l_nv + kAttnWindow);   // [stages]
-    uint64_t* empty = full + kAttnStages;                                // [stages]
-
-    const int g = lane >> 2, t = lane & 3;
-    const int G = d.G();
-    const int rows = d.Qn * G;
     const long long K = d.K;
     const long long T = static_cast<long long>(d.B) * d.Hkv * K;
-    const long long s_begin = gs < n_streams ? (gs * T + n_streams - 1) / n_streams : 0;
-    const long long s_end = gs < n_streams ? ((gs + 1) * T + n_streams - 1) / n_streams : 0;
+    const long long gs = blockIdx.x;
+    const long long s_begin = (gs * T + n_streams - 1) / n_streams;
+    const long long s_end = ((gs + 1) * T + n_streams - 1) / n_streams;
+    if (s_begin >= s_end) return;                         // whole CTA: empty range
     const long long u_first = s_begin / K, u_last = (s_end - 1) / K;
-    if (s_begin < s_end) {
+    const int G = d.G();
+    const int rows = d.Qn * G;
 
-    if (qg == 0) {
-        if (lane < kAttnStages) {
-            mbar_init(&full[lane], 1);
-            mbar_init(&empty[lane], QG);
-        }
+    // ---------------------------------------------------------- set-up
+    if (tid == 0) {
+        const int counts[kAttnNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 4, 4, 4, 1, 1,
+                                          1, 1, 1, 1, 1, 1, 2, 2, 1, 1};
+        for (int i = 0; i < kAttnNumBars; ++i) mbar_init(&bar[i], counts[i]);
         fence_mbar_init();
+        *s_abort = 0;
+        *s_last = 0;
     }
-    if (QG > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + ls), "r"(32 * QG) : "memory");
-    __syncwarp();
+    if (warp == 1) {
+        tmem_alloc(s_tmem, kAttnTmemCols);
+        tmem_relinquish();
+    }
+    // zero Q and P: rows past the real query rows stay zero for the whole call
+    for (int i = tid; i < 8 * kAttnRegion / 16; i += kAttnThreads)
+        reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tmem_o = tmem + 128;
 
-    const uint64_t pol = l2_policy_evict_first();
-    const uint32_t ring_addr = smem_addr(ring);
-    auto issue = [&](int idx, long long pos) {
-        const int stage = static_cast<int>(pos % kAttnStages);
-        uint64_t* bar = &full[stage];
-        const int y = l_slot[idx] * (2 * kBlockTokens);
-        mbar_arrive_expect_tx(bar, kBlockBytes);
-        tma_load_2d(ring + stage * kBlockBytes, &tm_pool, bar, 0, y, pol);
-        tma_load_2d(ring + stage * kBlockBytes + kBlockBytes / 2, &tm_pool, bar, 64, y, pol);
-    };
-
-    float o[8][NTW][4];
-    float m_run[NTW][2], l_run[NTW][2];
-    uint32_t qf[NTW][8][2];
-
-    auto load_unit = [&](long long u) {
-        const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
-#pragma unroll
-        for (int nt = 0; nt < NTW; ++nt) {
-            const int r = 8 * (qg * NTW + nt) + g;
-            const bool valid = r < rows;
-            const uint16_t* qrow = q + ((static_cast<long long>(b) * d.Qn + (valid ? r / G : 0)) * d.Hq + h * G +
-                                        (valid ? r % G : 0)) *
-                                           kHeadDim;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                qf[nt][ks][0] = valid ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * t)) : 0u;
-                qf[nt][ks][1] = valid ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * t + 8)) : 0u;
-            }
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                m_run[nt][c] = kNegInf;
-                l_run[nt][c] = 0.f;
-            }
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+    if (warp == 0) {
+        // ===================================================== producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_pool);
+            prefetch_tensormap(&tm_q);
         }
-    };
-
-    // Normalised partial of unit u into entry p = gs + u of the workspace
-    // (unique: a later stream starts at or after this stream's last unit).
-    auto finalize = [&](long long u, bool any) {
-        const long long p = gs + u;
+        const uint64_t pol_kv = l2_policy_evict_first();
+        const uint64_t pol_q = l2_policy_evict_last();
+        long long pos = 0;
+        long long last_pos[kAttnStages] = {-1, -1, -1, -1};
+        int p = 0;
+        for (long long u = u_first; u <= u_last; ++u, ++p) {
+            const int pb = p & 1;
+            const long long lo = max(s_begin, u * K), hi = min(s_end, (u + 1) * K);
+            const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
+            if (lane == 0 && p >= 2) attn_wait(&bar[kBarLFree + pb], ((p >> 1) - 1) & 1, s_abort);
+            __syncwarp();
+            // the occupied slots of the piece, in slot order: (slot in unit) << 5 | valid tokens
+            int* list = s_list + pb * kAttnMaxList;
+            const int ctx = ctx_len[b];
+            int n = 0;
+            for (long long base = lo; base < hi; base += 32) {
+                const long long s = base + lane;
+                int nv = 0;
+                if (s < hi) {
+                    int blk = slot_table[s];
+                    if (blk < -1 || blk >= d.N) {
+                        raise_dev_error(OASIS_DEVERR_ID_RANGE);
+                        blk = -1;
+                    }
+                    if (blk >= 0) nv = min(kBlockTokens, max(0, ctx - blk * kBlockTokens));
+                }
+                const unsigned m = __ballot_sync(0xFFFFFFFFu, nv > 0);
+                if (nv > 0) list[n + __popc(m & ((1u << lane) - 1u))] = (static_cast<int>(s - u * K) << 5) | nv;
+                n += __popc(m);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                s_nlist[pb] = n;
+                __threadfence_block();
+                mbar_arrive(&bar[kBarLFull + pb]);
+                // the unit's query rows: box {64 columns, G heads, Qn rows} per 64-column half
+                if (p >= 2) attn_wait(&bar[kBarQFree + pb], ((p >> 1) - 1) & 1, s_abort);
+                mbar_arrive_expect_tx(&bar[kBarQFull + pb], static_cast<uint32_t>(rows) * kRowBytes);
+                if (!*s_abort) {
+                    uint8_t* q_dst = sQ + pb * 2 * kAttnRegion;
+                    tma_load_3d(q_dst, &tm_q, &bar[kBarQFull + pb], 0, h * G, b * d.Qn, pol_q);
+                    tma_load_3d(q_dst + kAttnRegion, &tm_q, &bar[kBarQFull + pb], 64, h * G, b * d.Qn, pol_q);
+                }
+                const int ntiles = (n + kAttnTileSlots - 1) / kAttnTileSlots;
+                for (int i = 0; i < ntiles; ++i, ++pos) {
+                    const int stage = static_cast<int>(pos % kAttnStages);
+                    if (pos >= kAttnStages)
+                        attn_wait(&bar[kBarEmpty + stage], static_cast<uint32_t>((pos / kAttnStages - 1) & 1),
+                                  s_abort);
+                    const int ns = min(kAttnTileSlots, n - i * kAttnTileSlots);
+                    mbar_arrive_expect_tx(&bar[kBarFull + stage], static_cast<uint32_t>(ns) * kBlockBytes);
+                    last_pos[stage] = pos;
+                    if (*s_abort) continue;
+                    uint8_t* st = ring + stage * kAttnStageBytes;
+                    for (int j = 0; j < ns; ++j) {
+                        const int slot = list[i * kAttnTileSlots + j] >> 5;
+                        const int y = static_cast<int>((u * K + slot) * (2 * kBlockTokens));
+                        const int off = j * (kBlockTokens * 128);
+                        tma_load_2d(st + 0 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 0, y, pol_kv);
+                        tma_load_2d(st + 1 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 64, y, pol_kv);
+                        tma_load_2d(st + 2 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 0,
+                                    y + kBlockTokens, pol_kv);
+                        tma_load_2d(st + 3 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 64,
+                                    y + kBlockTokens, pol_kv);
+                    }
+                }
+            }
+            __syncwarp();
+            n = __shfl_sync(0xFFFFFFFFu, n, 0);
+            pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+        }
+        // no copy may still be writing this CTA's shared memory when it exits
+        if (lane == 0)
+            for (int s = 0; s < kAttnStages; ++s)
+                if (last_pos[s] >= 0) mbar_wait(&bar[kBarFull + s], static_cast<uint32_t>((last_pos[s] / kAttnStages) & 1));
+    } else if (warp == 1) {
+        // =================================================== MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16_f32(kAttnRows, kAttnTileSlots * kBlockTokens);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16_f32_bmn(kAttnRows, kHeadDim);
+            long long pos = 0;
+            int p = 0;
+            bool have_prev = false, prev_first = false, prev_last = false;
+            long long prev_pos = 0;
+            int prev_ns = 0;
+            auto issue_pv = [&](long long ppos, int pns, bool pfirst, bool plast) {
+                const int sb = static_cast<int>(ppos & 1);
+                const int stage = static_cast<int>(ppos % kAttnStages);
+                const bool ok = attn_wait(&bar[kBarPFull + sb], static_cast<uint32_t>((ppos >> 1) & 1), s_abort);
+                tc_fence_after_sync();
+                if (ok) {
+                    const uint32_t pa = smem_addr(sP + sb * 2 * kAttnRegion);
+                    const uint32_t va = smem_addr(ring + stage * kAttnStageBytes + 2 * kAttnRegion);
+                    for (int kk = 0; kk < pns; ++kk) {
+                        const uint64_t bd = umma_desc_sw128_lbo_sbo(va + kk * (kBlockTokens * 128), kAttnRegion, 1024);
+                        umma_bf16(tmem_o, umma_desc_sw128_lbo_sbo(pa + kk * 32, 16, 1024), bd, idesc_pv,
+                                  (pfirst && kk == 0) ? 0u : 1u);
+                        umma_bf16(tmem_o, umma_desc_sw128_lbo_sbo(pa + kAttnRegion + kk * 32, 16, 1024), bd,
+                                  idesc_pv, 1u);
+                    }
+                }
+                umma_commit(&bar[kBarEmpty + stage]);
+                umma_commit(&bar[kBarPFree + sb]);
+                if (plast) umma_commit(&bar[kBarODone]);
+            };
+            for (long long u = u_first; u <= u_last; ++u, ++p) {
+                const int pb = p & 1;
+                attn_wait(&bar[kBarLFull + pb], static_cast<uint32_t>((p >> 1) & 1), s_abort);
+                const int n = s_nlist[pb];
+                const int ntiles = (n + kAttnTileSlots - 1) / kAttnTileSlots;
+                attn_wait(&bar[kBarQFull + pb], static_cast<uint32_t>((p >> 1) & 1), s_abort);
+                const uint32_t qa = smem_addr(sQ + pb * 2 * kAttnRegion);
+                for (int i = 0; i < ntiles; ++i, ++pos) {
+                    const int stage = static_cast<int>(pos % kAttnStages);
+                    const int sb = static_cast<int>(pos & 1);
+                    bool ok = attn_wait(&bar[kBarFull + stage], static_cast<uint32_t>((pos / kAttnStages) & 1),
+                                        s_abort);
+                    if (pos >= 2) ok = attn_wait(&bar[kBarSFree + sb], static_cast<uint32_t>(((pos >> 1) - 1) & 1),
+                                                 s_abort) && ok;
+                    tc_fence_after_sync();
+                    if (ok) {
+                        const uint32_t ka = smem_addr(ring + stage * kAttnStageBytes);
 #pragma unroll
-        for (int nt = 0; nt < NTW; ++nt) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float l = l_run[nt][c];
-                l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
-                l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
-                l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
-                const int col = 8 * (qg * NTW + nt) + 2 * t + c;
-                const bool live = any && l > 0.f;
-                const float inv = live ? 1.f / l : 0.f;
-                if (col < rows) {
-                    if (g == 0) ws_lse[p * rows + col] = live ? (m_run[nt][c] + log2f(l)) * kLn2 : kNegInf;
-                    if (live) {
-                        float* dst = ws_o + (p * rows + col) * kHeadDim;
-#pragma unroll
-                        for (int mt = 0; mt < 8; ++mt) {
-                            dst[16 * mt + g] = o[mt][nt][c] * inv;
-                            dst[16 * mt + g + 8] = o[mt][nt][2 + c] * inv;
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t off = (ks >> 2) * kAttnRegion + (ks & 3) * 32;
+                            umma_bf16(tmem + sb * 64, umma_desc_sw128_lbo_sbo(qa + off, 16, 1024),
+                                      umma_desc_sw128_lbo_sbo(ka + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                         }
                     }
+                    umma_commit(&bar[kBarSFull + sb]);
+                    if (have_prev) issue_pv(prev_pos, prev_ns, prev_first, prev_last);
+                    have_prev = true;
+                    prev_pos = pos;
+                    prev_ns = min(kAttnTileSlots, n - i * kAttnTileSlots);
+                    prev_first = i == 0;
+                    prev_last = i == ntiles - 1;
                 }
+                umma_commit(&bar[kBarQFree + pb]);            // after the piece's last S
+                mbar_arrive(&bar[kBarLFree + pb]);
             }
+            if (have_prev) issue_pv(prev_pos, prev_ns, prev_first, prev_last);
+            umma_commit(&bar[kBarFinal]);
+            mbar_wait(&bar[kBarFinal], 0);
         }
-    };
-    auto write_empty = [&](long long u) {
-        const long long p = gs + u;
-        const int c1 = min(rows, 8 * (qg + 1) * NTW);
-        for (int col = 8 * qg * NTW + lane; col < c1; col += 32) ws_lse[p * rows + col] = kNegInf;
-    };
-
-    const int rowK = lane & 15, hiK = lane >> 4;
-    const int tokV = (lane & 7) + ((lane >> 4) << 3), hiV = (lane >> 3) & 1;
-    long long rp = 0;            // ring position of the next slot consumed
-    long long u_cur = -1;
-    long long u_end = 0;         // first slot past the current unit
-    bool any = false;            // the current unit has seen a slot
-    bool failed = false;
-
-    // A failed (timed-out) wait does not leave the loops early: every warp of
-    // a stream must reach the same named barriers, so the remaining slots are
-    // walked without waiting or computing.
-    for (long long w0 = s_begin; w0 < s_end; w0 += kAttnWindow) {
-        const long long w1 = min(s_end, w0 + kAttnWindow);
-        // ---- the occupied slots of this window, in slot order
-        int n_list = 0;
-        for (long long base = w0; base < w1; base += 32) {
-            const long long s = base + lane;
-            int nv = 0;
-            if (s < w1) {
-                int blk = slot_table[s];
-                if (blk < -1 || blk >= d.N) {
-                    if (qg == 0) raise_dev_error(OASIS_DEVERR_ID_RANGE);
-                    blk = -1;
-                }
-                // slot indices stay below 2^26 (host check): 32-bit division
-                const unsigned unit = static_cast<unsigned>(s) / static_cast<unsigned>(K);
-                if (blk >= 0) nv = min(kBlockTokens, ctx_len[unit / static_cast<unsigned>(d.Hkv)] - blk * kBlockTokens);
-            }
-            const unsigned m = __ballot_sync(0xFFFFFFFFu, nv > 0);
-            if (nv > 0 && qg == 0) {
-                const int pos = n_list + __popc(m & ((1u << lane) - 1u));
-                l_slot[pos] = static_cast<int>(s);
-                l_nv[pos] = nv;
-            }
-            n_list += __popc(m);
-        }
-        if (QG > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + ls), "r"(32 * QG) : "memory");
         __syncwarp();
-        if (qg == 0 && lane == 0 && !failed)
-            for (int i = 0; i < kAttnStages && i < n_list; ++i) issue(i, rp + i);
-
-        for (int i = 0; i < n_list; ++i, ++rp) {
-            if (l_slot[i] >= u_end) {
-                // slots are listed in order: divide only when the unit changes
-                const long long u = l_slot[i] / K;
-                if (u_cur >= 0) finalize(u_cur, any);
-                for (long long uu = (u_cur < 0 ? u_first : u_cur + 1); uu < u; ++uu) write_empty(uu);
-                u_cur = u;
-                u_end = (u + 1) * K;
-                any = false;
-                load_unit(u);
-            }
-            if (failed) continue;
-            const int stage = static_cast<int>(rp % kAttnStages);
-            const uint32_t parity = static_cast<uint32_t>((rp / kAttnStages) & 1);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[stage], parity))) {
-                if (lane == 0) raise_dev_error(OASIS_DEVERR_TIMEOUT);
-                failed = true;
-                continue;
-            }
-            any = true;
-            const int nv = l_nv[i];
-            const uint32_t sbase = ring_addr + stage * kBlockBytes;
-
-            // S^T = K . Q^T
-            float sacc[NTW][4];
+    } else {
+        // ============================================ softmax / epilogue
+        const int qd = warp & 3;                              // TMEM lane quadrant
+        const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        const int rA = 16 * qd + (lane >> 2), rB = rA + 8;   // this thread's query rows
+        const bool realA = rA < rows, realB = rB < rows;
+        const int cp = 2 * (lane & 3);                        // column pair within each 8-column chunk
+        long long pos = 0;
+        int nonempty = 0;
+        int p = 0;
+        for (long long u = u_first; u <= u_last; ++u, ++p) {
+            const int pb = p & 1;
+            attn_wait(&bar[kBarLFull + pb], static_cast<uint32_t>((p >> 1) & 1), s_abort);
+            const int n = s_nlist[pb];
+            const int* list = s_list + pb * kAttnMaxList;
+            const int ntiles = (n + kAttnTileSlots - 1) / kAttnTileSlots;
+            float mA = kNegInf, mB = kNegInf, lA = 0.f, lB = 0.f;
+            for (int i = 0; i < ntiles; ++i, ++pos) {
+                const int sb = static_cast<int>(pos & 1);
+                const int stage = static_cast<int>(pos % kAttnStages);
+                const int ns = min(kAttnTileSlots, n - i * kAttnTileSlots);
+                int nvj[kAttnTileSlots];
 #pragma unroll
-            for (int nt = 0; nt < NTW; ++nt)
+                for (int j = 0; j < kAttnTileSlots; ++j) nvj[j] = j < ns ? (list[i * kAttnTileSlots + j] & 31) : 0;
+                attn_wait(&bar[kBarSFull + sb], static_cast<uint32_t>((pos >> 1) & 1), s_abort);
+                tc_fence_after_sync();
+                uint32_t v[32];
+                tmem_ld_16x256b_x8(tmem + lane_base + sb * 64, v);
+                tmem_ld_wait();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kBarSFree + sb]);
+                float s[32];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+                for (int c = 0; c < 8; ++c) {
+                    const int j = c >> 1;                      // slot of this chunk
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const int c16 = ((ks & 3) << 1) | hiK;
-                const uint32_t addr = sbase + (ks >> 2) * (kBlockBytes / 2) + rowK * 128 + ((c16 ^ (rowK & 7)) << 4);
-                uint32_t a[4];
-                ldsm_x4(addr, a);
-#pragma unroll
-                for (int nt = 0; nt < NTW; ++nt) mma_bf16_m16n8k16(sacc[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
-            }
-            if (nv < kBlockTokens) {
-#pragma unroll
-                for (int nt = 0; nt < NTW; ++nt) {
-                    if (g >= nv) sacc[nt][0] = sacc[nt][1] = kNegInf;
-                    if (g + 8 >= nv) sacc[nt][2] = sacc[nt][3] = kNegInf;
-                }
-            }
-            // online softmax over tokens, per query column (log2 domain).  The
-            // reference max only moves when a tile's max exceeds it by more
-            // than 8 (weights stay <= 2^8), so O and l are rarely rescaled;
-            // lse = m + log2(l) is exact for any reference.  scale > 0.
-            float alpha[NTW][2];
-            bool rescale = false;
-#pragma unroll
-            for (int nt = 0; nt < NTW; ++nt) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float mx = fmaxf(sacc[nt][c], sacc[nt][2 + c]);
-                    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-                    const float mx_s = mx * scale_log2;
-                    alpha[nt][c] = 1.f;
-                    if (mx_s > m_run[nt][c] + 8.f) {
-                        alpha[nt][c] = exp2f(m_run[nt][c] - mx_s);
-                        m_run[nt][c] = mx_s;
-                        rescale = true;
+                    for (int e = 0; e < 2; ++e) {
+                        const int tt = (c & 1) * 8 + cp + e;   // token within the slot
+                        const bool ok = tt < nvj[j];
+                        s[4 * c + e] = ok ? __uint_as_float(v[4 * c + e]) : kNegInf;
+                        s[4 * c + 2 + e] = ok ? __uint_as_float(v[4 * c + 2 + e]) : kNegInf;
                     }
-                    sacc[nt][c] = exp2f(fmaf(sacc[nt][c], scale_log2, -m_run[nt][c]));
-                    sacc[nt][2 + c] = exp2f(fmaf(sacc[nt][2 + c], scale_log2, -m_run[nt][c]));
                 }
-            }
-            if (__any_sync(0xFFFFFFFFu, rescale)) {
+                float mxA = kNegInf, mxB = kNegInf;
 #pragma unroll
-                for (int nt = 0; nt < NTW; ++nt) {
-#pragma unroll
-                    for (int mt = 0; mt < 8; ++mt) {
-                        o[mt][nt][0] *= alpha[nt][0];
-                        o[mt][nt][1] *= alpha[nt][1];
-                        o[mt][nt][2] *= alpha[nt][0];
-                        o[mt][nt][3] *= alpha[nt][1];
+                for (int c = 0; c < 8; ++c) {
+                    mxA = fmaxf(mxA, fmaxf(s[4 * c], s[4 * c + 1]));
+                    mxB = fmaxf(mxB, fmaxf(s[4 * c + 2], s[4 * c + 3]));
+                }
+                mxA = fmaxf(mxA, __shfl_xor_sync(0xFFFFFFFFu, mxA, 1));
+                mxA = fmaxf(mxA, __shfl_xor_sync(0xFFFFFFFFu, mxA, 2));
+                mxB = fmaxf(mxB, __shfl_xor_sync(0xFFFFFFFFu, mxB, 1));
+                mxB = fmaxf(mxB, __shfl_xor_sync(0xFFFFFFFFu, mxB, 2));
+                mxA *= scale_log2;
+                mxB *= scale_log2;
+                // P buffer sb is free once PV of tile pos-2 has completed
+                if (pos >= 2) attn_wait(&bar[kBarPFree + sb], static_cast<uint32_t>(((pos >> 1) - 1) & 1), s_abort);
+                // running max: moved only by more than 2^8 (exact lse for any reference)
+                float alA = 1.f, alB = 1.f;
+                bool resc = false;
+                if (mxA > mA + 8.f) {
+                    if (i > 0) {
+                        alA = exp2f(mA - mxA);
+                        resc = true;
                     }
-                    l_run[nt][0] *= alpha[nt][0];
-                    l_run[nt][1] *= alpha[nt][1];
+                    mA = mxA;
                 }
-            }
-            // P^T -> B fragments of O^T += V^T . P^T (head + remainder)
-            uint32_t pb[NTW][2], pr[NTW][2];
-#pragma unroll
-            for (int nt = 0; nt < NTW; ++nt) {
-                const uint32_t h0 = pack_bf16x2(sacc[nt][0], sacc[nt][1]);   // token g
-                const uint32_t h1 = pack_bf16x2(sacc[nt][2], sacc[nt][3]);   // token g + 8
-                const uint32_t r0 = pack_bf16x2(sacc[nt][0] - bf16_lo(h0), sacc[nt][1] - bf16_hi(h0));
-                const uint32_t r1 = pack_bf16x2(sacc[nt][2] - bf16_lo(h1), sacc[nt][3] - bf16_hi(h1));
-                l_run[nt][0] += sacc[nt][0] + sacc[nt][2];
-                l_run[nt][1] += sacc[nt][1] + sacc[nt][3];
-                pb[nt][0] = movmatrix_trans(h0);
-                pb[nt][1] = movmatrix_trans(h1);
-                pr[nt][0] = movmatrix_trans(r0);
-                pr[nt][1] = movmatrix_trans(r1);
-            }
-            uint32_t vmask_lo = 0xFFFFFFFFu, vmask_hi = 0xFFFFFFFFu;
-            if (nv < kBlockTokens) {
-                vmask_lo = (2 * t < nv ? 0xFFFFu : 0u) | (2 * t + 1 < nv ? 0xFFFF0000u : 0u);
-                vmask_hi = (2 * t + 8 < nv ? 0xFFFFu : 0u) | (2 * t + 9 < nv ? 0xFFFF0000u : 0u);
-            }
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                const int row = kBlockTokens + tokV;
-                const int c16 = ((mt & 3) << 1) | hiV;
-                const uint32_t addr = sbase + (mt >> 2) * (kBlockBytes / 2) + row * 128 + ((c16 ^ (row & 7)) << 4);
-                uint32_t a[4];
-                ldsm_x4_trans(addr, a);
-                a[0] &= vmask_lo;
-                a[1] &= vmask_lo;
-                a[2] &= vmask_hi;
-                a[3] &= vmask_hi;
-#pragma unroll
-                for (int nt = 0; nt < NTW; ++nt) {
-                    mma_bf16_m16n8k16(o[mt][nt], a, pb[nt][0], pb[nt][1]);
-                    mma_bf16_m16n8k16(o[mt][nt], a, pr[nt][0], pr[nt][1]);
+                if (mxB > mB + 8.f) {
+                    if (i > 0) {
+                        alB = exp2f(mB - mxB);
+                        resc = true;
+                    }
+                    mB = mxB;
                 }
+                lA *= alA;
+                lB *= alB;
+                if (__any_sync(0xFFFFFFFFu, resc)) {
+                    // PV of tile pos-1 must have landed in O before it is rescaled
+                    attn_wait(&bar[kBarPFree + (sb ^ 1)], static_cast<uint32_t>(((pos - 1) >> 1) & 1), s_abort);
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t o[32];
+                        tmem_ld_16x256b_x8(tmem_o + lane_base + half * 64, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            o[4 * c + 0] = __float_as_uint(__uint_as_float(o[4 * c + 0]) * alA);
+                            o[4 * c + 1] = __float_as_uint(__uint_as_float(o[4 * c + 1]) * alA);
+                            o[4 * c + 2] = __float_as_uint(__uint_as_float(o[4 * c + 2]) * alB);
+                            o[4 * c + 3] = __float_as_uint(__uint_as_float(o[4 * c + 3]) * alB);
+                        }
+                        tmem_st_16x256b_x8(tmem_o + lane_base + half * 64, o);
+                    }
+                    tmem_st_wait();
+                }
+                // probabilities: head + remainder in bf16, written 128-byte swizzled
+                uint8_t* p_head = sP + sb * 2 * kAttnRegion;
+                uint8_t* p_rest = p_head + kAttnRegion;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float a0 = exp2f(fmaf(s[4 * c + 0], scale_log2, -mA));
+                    const float a1 = exp2f(fmaf(s[4 * c + 1], scale_log2, -mA));
+                    const float b0 = exp2f(fmaf(s[4 * c + 2], scale_log2, -mB));
+                    const float b1 = exp2f(fmaf(s[4 * c + 3], scale_log2, -mB));
+                    lA += a0 + a1;
+                    lB += b0 + b1;
+                    if (realA) {
+                        const uint32_t hd = pack_bf16x2(a0, a1);
+                        const uint32_t rs = pack_bf16x2(a0 - bf16_lo(hd), a1 - bf16_hi(hd));
+                        const int off = rA * 128 + ((c ^ (rA & 7)) << 4) + cp * 2;
+                        *reinterpret_cast<uint32_t*>(p_head + off) = hd;
+                        *reinterpret_cast<uint32_t*>(p_rest + off) = rs;
+                    }
+                    if (realB) {
+                        const uint32_t hd = pack_bf16x2(b0, b1);
+                        const uint32_t rs = pack_bf16x2(b0 - bf16_lo(hd), b1 - bf16_hi(hd));
+                        const int off = rB * 128 + ((c ^ (rB & 7)) << 4) + cp * 2;
+                        *reinterpret_cast<uint32_t*>(p_head + off) = hd;
+                        *reinterpret_cast<uint32_t*>(p_rest + off) = rs;
+                    }
+                }
+                // value rows past the context of a partly filled block read as zero
+                // (their weights are zero, and zero times a non-finite stale value is not)
+                if (qd < ns && nvj[qd] < kBlockTokens) {
+                    // the tile's copy is complete (already awaited by the MMA thread; this
+                    // wait returns at once and orders the copy before these writes)
+                    attn_wait(&bar[kBarFull + stage], static_cast<uint32_t>((pos / kAttnStages) & 1), s_abort);
+                    uint8_t* vbase = ring + stage * kAttnStageBytes + 2 * kAttnRegion + qd * (kBlockTokens * 128);
+                    const int first_row = nvj[qd];
+                    for (int k = lane; k < (kBlockTokens - first_row) * 16; k += 32) {
+                        const int row = first_row + (k >> 4), chunk = k & 15;
+                        *reinterpret_cast<uint4*>(vbase + (chunk >> 3) * kAttnRegion + row * 128 + (chunk & 7) * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kBarPFull + sb]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-            if (qg == 0 && lane == 0 && i + kAttnStages < n_list) {
-                if (mbar_wait(&empty[stage], parity)) {
-                    fence_proxy_async_smem();
-                    issue(i + kAttnStages, rp + kAttnStages);
+
+            // ------------------------------------------------- epilogue
+            if (ntiles > 0) {
+                attn_wait(&bar[kBarODone], static_cast<uint32_t>(nonempty & 1), s_abort);
+                ++nonempty;
+                tc_fence_after_sync();
+            }
+            lA += __shfl_xor_sync(0xFFFFFFFFu, lA, 1);
+            lA += __shfl_xor_sync(0xFFFFFFFFu, lA, 2);
+            lB += __shfl_xor_sync(0xFFFFFFFFu, lB, 1);
+            lB += __shfl_xor_sync(0xFFFFFFFFu, lB, 2);
+            const float invA = lA > 0.f ? 1.f / lA : 0.f, invB = lB > 0.f ? 1.f / lB : 0.f;
+            const bool direct = u * K >= s_begin && (u + 1) * K <= s_end;
+            const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
+            const long long pidx = gs + u;                    // this CTA's partial of unit u
+            const long long orowA = (static_cast<long long>(b) * d.Qn + rA / G) * d.Hq + h * G + rA % G;
+            const long long orowB = (static_cast<long long>(b) * d.Qn + rB / G) * d.Hq + h * G + rB % G;
+            float* dstA = direct ? out + orowA * kHeadDim : ws_o + (pidx * rows + rA) * kHeadDim;
+            float* dstB = direct ? out + orowB * kHeadDim : ws_o + (pidx * rows + rB) * kHeadDim;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t o[32];
+                if (ntiles > 0) {
+                    tmem_ld_16x256b_x8(tmem_o + lane_base + half * 64, o);
+                    tmem_ld_wait();
                 } else {
-                    raise_dev_error(OASIS_DEVERR_TIMEOUT);
-                    failed = true;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = 0u;
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int col = half * 64 + 8 * c + cp;
+                    if (realA)
+                        *reinterpret_cast<float2*>(dstA + col) =
+                            make_float2(__uint_as_float(o[4 * c]) * invA, __uint_as_float(o[4 * c + 1]) * invA);
+                    if (realB)
+                        *reinterpret_cast<float2*>(dstB + col) = make_float2(__uint_as_float(o[4 * c + 2]) * invB,
+                                                                             __uint_as_float(o[4 * c + 3]) * invB);
                 }
             }
-            __syncwarp();
+            tc_fence_before_sync();
+            if ((lane & 3) == 0) {
+                const float l2A = lA > 0.f ? mA + log2f(lA) : kNegInf;
+                const float l2B = lB > 0.f ? mB + log2f(lB) : kNegInf;
+                if (direct) {
+                    if (realA) lse_out[orowA] = lA > 0.f ? l2A * kLn2 : kNegInf;
+                    if (realB) lse_out[orowB] = lB > 0.f ? l2B * kLn2 : kNegInf;
+                } else {
+                    if (realA) ws_lse[pidx * rows + rA] = l2A;
+                    if (realB) ws_lse[pidx * rows + rB] = l2B;
+                }
+            }
+            if (!direct) {
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (warp == 2 && lane == 0) {
+                    long long first, last;
+                    attn_unit_streams(u, K, n_streams, T, &first, &last);
+                    const int old = atomicAdd(ws_ticket + u, 1);
+                    *s_last = old == static_cast<int>(last - first) ? 1 : 0;
+                }
+                named_bar_sync(1, 128);
+                if (*s_last) {
+                    __threadfence();
+                    long long first, last;
+                    attn_unit_streams(u, K, n_streams, T, &first, &last);
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int r = rr == 0 ? rA : rB;
+                        if (r >= rows) continue;
+                        const long long orow = rr == 0 ? orowA : orowB;
+                        float M = kNegInf;
+                        for (long long sp = first; sp <= last; ++sp) M = fmaxf(M, __ldcg(ws_lse + (sp + u) * rows + r));
+                        float L = 0.f;
+                        float2 acc[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) acc[k] = make_float2(0.f, 0.f);
+                        if (M != kNegInf) {
+                            for (long long sp = first; sp <= last; ++sp) {
+                                const float lj = __ldcg(ws_lse + (sp + u) * rows + r);
+                                if (lj == kNegInf) continue;             // empty partial: its output is not read
+                                const float w = exp2f(lj - M);
+                                L += w;
+                                const float* src = ws_o + ((sp + u) * rows + r) * kHeadDim;
+#pragma unroll
+                                for (int k = 0; k < 16; ++k) {
+                                    const int col = (k >> 3) * 64 + 8 * (k & 7) + cp;
+                                    const float2 x = __ldcg(reinterpret_cast<const float2*>(src + col));
+                                    acc[k].x += w * x.x;
+                                    acc[k].y += w * x.y;
+                                }
+                            }
+                        }
+                        const float inv = L > 0.f ? 1.f / L : 0.f;
+                        float* dst = out + orow * kHeadDim;
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int col = (k >> 3) * 64 + 8 * (k & 7) + cp;
+                            *reinterpret_cast<float2*>(dst + col) = make_float2(acc[k].x * inv, acc[k].y * inv);
+                        }
+                        if ((lane & 3) == 0) lse_out[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : kNegInf;
+                    }
+                    if (warp == 2 && lane == 0) ws_ticket[u] = 0;         // ready for the next call
+                }
+            }
+            named_bar_sync(1, 128);                                         // every warp is done with the list
+            if (warp == 2 && lane == 0) {
+                *s_last = 0;
+                mbar_arrive(&bar[kBarLFree + pb]);
+            }
         }
-        // every warp of the stream is done with this window's list
-        if (QG > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + ls), "r"(32 * QG) : "memory");
     }
-    if (u_cur >= 0) finalize(u_cur, any);
-    for (long long uu = (u_cur < 0 ? u_first : u_cur + 1); uu <= u_last; ++uu) write_empty(uu);
-    }   // s_begin < s_end
-    // let the merge kernel (launched as a programmatic dependent) start early
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // ---------------------------------------------------------- teardown
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc(tmem, kAttnTmemCols);
 }
 
 }  // namespace oasis

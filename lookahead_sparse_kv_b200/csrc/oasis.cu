@@ -19,6 +19,7 @@
 
 #include "attn.cuh"
 #include "common.cuh"
+#include "fused.cuh"
 #include "overlap.cuh"
 #include "plan.cuh"
 #include "prefetch.cuh"
@@ -140,6 +141,26 @@ int make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned
     return OASIS_OK;
 }
 
+// The query rows of every (sequence, KV head): bf16 q [B][Qn][Hq][128] seen
+// as a 3-D tensor (128 columns, Hq heads, B*Qn query positions), boxes of
+// 64 columns x G heads x Qn positions, so one box per 64-column half brings
+// the unit's Qn*G rows in (j, g) order, 128-byte swizzled.
+int make_map_q(CUtensorMap* m, const void* q, const Dims& d) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(oasis::kHeadDim), static_cast<cuuint64_t>(d.Hq),
+                                static_cast<cuuint64_t>(d.B) * d.Qn};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(oasis::kRowBytes),
+                                   static_cast<cuuint64_t>(oasis::kRowBytes) * d.Hq};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(d.G()), static_cast<cuuint32_t>(d.Qn)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled(q) failed: %d", static_cast<int>(r));
+    return OASIS_OK;
+}
+
 template <typename K>
 int set_smem(K kernel, int bytes, const char* what) {
     const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -157,8 +178,13 @@ long long attn_max_streams(const Dims& d) {
     return std::max<long long>(1, std::min(T, std::max(cap, (T + 255) / 256)));
 }
 
+// Workspace: block scores [B*Hkv*N] fp32, then the attention partials of
+// units split over CTAs (log2-sum-exp [P][rows] and normalised outputs
+// [P][rows][128], P = streams + units), then one ticket counter per unit for
+// the attention merge and one for the fused score / select / plan (all zero
+// between calls).
 struct WsLayout {
-    size_t scores, lse, o, total;
+    size_t scores, lse, o, ticket, sticket, total;
     long long partials;
 };
 
@@ -170,7 +196,9 @@ WsLayout ws_layout(const Dims& d) {
     w.scores = 0;
     w.lse = align256(units * d.N * sizeof(float));
     w.o = align256(w.lse + static_cast<size_t>(w.partials) * rows * sizeof(float));
-    w.total = align256(w.o + static_cast<size_t>(w.partials) * rows * oasis::kHeadDim * sizeof(float));
+    w.ticket = align256(w.o + static_cast<size_t>(w.partials) * rows * oasis::kHeadDim * sizeof(float));
+    w.sticket = align256(w.ticket + units * sizeof(int));
+    w.total = align256(w.sticket + units * sizeof(int));
     return w;
 }
 
@@ -187,45 +215,12 @@ int sm_count() {
     return n;
 }
 
-// Streams for this launch: 8 per SM (4 with two-warp streams), at least 4
-// slots each, never more than the workspace holds.
-long long attn_streams(const Dims& d, int qg) {
+// CTAs (streams) of an attention launch: one per SM, each range at least 16
+// slots (four tiles), never more than the workspace holds.
+long long attn_streams(const Dims& d) {
     const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
-    long long ns = static_cast<long long>(sm_count()) * (qg == 1 ? 8 : 4);
-    ns = std::max(ns, (T + 255) / 256);
-    ns = std::min(ns, std::max(1ll, T / 4));
+    long long ns = std::min<long long>(sm_count(), std::max(1ll, T / 16));
     return std::min(ns, attn_max_streams(d));
-}
-
-template <int NTW, int QG>
-int launch_attn(const CUtensorMap& tm, const Dims& d, const uint16_t* q, const int32_t* st, const int32_t* ctx,
-                float scale_log2, float* out, float* lse, float* ws_o, float* ws_lse, cudaStream_t s) {
-    using Cfg = oasis::AttnCfg<NTW, QG>;
-    auto k = oasis::sparse_attn_kernel<NTW, QG>;
-    if (int rc = set_smem(k, Cfg::kSmem, "sparse_attn smem")) return rc;
-    const long long ns = attn_streams(d, QG);
-    const long long ctas = (ns + oasis::kAttnStreamsPerCta - 1) / oasis::kAttnStreamsPerCta;
-    k<<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmem, s>>>(tm, d, q, st, ctx, scale_log2,
-                                                                      static_cast<int>(ns), ws_o, ws_lse);
-    if (int rc = check_launch("sparse_attn launch")) return rc;
-    // merge, as a programmatic dependent launch: its launch overlaps the
-    // attention tail and griddepcontrol.wait orders its reads after it
-    const long long warps = static_cast<long long>(d.B) * d.Hkv * d.Qn * d.G();
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((warps + oasis::kMergeWarps - 1) / oasis::kMergeWarps));
-    cfg.blockDim = dim3(32 * oasis::kMergeWarps);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, oasis::attn_merge_kernel, d, static_cast<int>(ns),
-                                             static_cast<const float*>(ws_o), static_cast<const float*>(ws_lse),
-                                             out, lse);
-    if (e != cudaSuccess) return cuda_fail(e, "attn_merge launch");
-    return check_launch("attn_merge launch");
 }
 
 template <int NPAD>
@@ -237,6 +232,38 @@ int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d
     dim3 grid((d.N + oasis::kScoreTile - 1) / oasis::kScoreTile, d.B * d.Hkv);
     k<<<grid, 128, S::kBytes, s>>>(tmax, tmin, d, q, ctx, scores, row0, rows);
     return check_launch("lookahead_score launch");
+}
+
+template <int NPAD, bool kScored>
+int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
+                 const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int32_t* sel, float* sel_score,
+                 int32_t* st, int32_t* lu, int32_t step, const int32_t* step_dev, int32_t* fs, int32_t* fb,
+                 int32_t* nf, cudaStream_t s) {
+    auto k = oasis::score_select_plan_kernel<NPAD, kScored>;
+    const int smem = std::max(oasis::ScoreSmem<NPAD>::kBytes, oasis::fused_tail_bytes(d.N, d.K) + 1024);
+    if (int rc = set_smem(k, smem, "score_select_plan smem")) return rc;
+    dim3 grid((d.N + oasis::kScoreTile - 1) / oasis::kScoreTile, d.B * d.Hkv);
+    k<<<grid, 128, smem, s>>>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu, step,
+                              step_dev, fs, fb, nf);
+    return check_launch("score_select_plan launch");
+}
+
+template <bool kScored>
+int launch_fused_rows(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
+                      const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int32_t* sel,
+                      float* sel_score, int32_t* st, int32_t* lu, int32_t step, const int32_t* step_dev, int32_t* fs,
+                      int32_t* fb, int32_t* nf, cudaStream_t s) {
+    if (rows <= 16)
+        return launch_fused<16, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu,
+                                         step, step_dev, fs, fb, nf, s);
+    if (rows <= 32)
+        return launch_fused<32, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu,
+                                         step, step_dev, fs, fb, nf, s);
+    if (rows <= 48)
+        return launch_fused<48, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu,
+                                         step, step_dev, fs, fb, nf, s);
+    return launch_fused<64, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu, step,
+                                     step_dev, fs, fb, nf, s);
 }
 
 }  // namespace
@@ -311,14 +338,13 @@ int plan(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t*
         if (int rc = check_ptr(fetch_slot, "fetch_slot")) return rc;
         if (int rc = check_ptr(fetch_block, "fetch_block")) return rc;
     }
-    const int threads = (d.K + 31) / 32 * 32;
-    const int smem = 7 * d.K * static_cast<int>(sizeof(int32_t));
+    const int smem = oasis::plan_smem_ints(d.K) * static_cast<int>(sizeof(int32_t));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (scores != nullptr)
-        oasis::plan_fetch_kernel<true><<<d.B * d.Hkv, threads, smem, s>>>(
+        oasis::plan_fetch_kernel<true><<<d.B * d.Hkv, oasis::kPlanThreads, smem, s>>>(
             d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
     else
-        oasis::plan_fetch_kernel<false><<<d.B * d.Hkv, threads, smem, s>>>(
+        oasis::plan_fetch_kernel<false><<<d.B * d.Hkv, oasis::kPlanThreads, smem, s>>>(
             d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
     return check_launch("plan_fetch launch");
 }
@@ -437,6 +463,51 @@ int oasis_score_select_rows(const oasis_dims* dp, const void* q, int32_t row_beg
     return oasis_select_topk(dp, scores, ctx_len, sel, sel_score, stream);
 }
 
+int oasis_score_select_plan(const oasis_dims* dp, const void* q, const void* kmin, const void* kmax,
+                            const int32_t* ctx_len, int32_t* sel, float* sel_score, float* scores,
+                            int32_t* slot_table, int32_t* last_used, int32_t step, const int32_t* step_dev,
+                            int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch, void* ws, size_t ws_bytes,
+                            void* stream) {
+    Dims d;
+    if (int rc = validate(dp, &d)) return rc;
+    if (int rc = check_ptr(q, "q")) return rc;
+    if (int rc = check_ptr(kmin, "kmin")) return rc;
+    if (int rc = check_ptr(kmax, "kmax")) return rc;
+    if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
+    if (int rc = check_ptr(sel, "sel")) return rc;
+    if (int rc = check_ptr(sel_score, "sel_score", true)) return rc;
+    if (int rc = check_ptr(scores, "scores", true)) return rc;
+    if (int rc = check_ptr(slot_table, "slot_table")) return rc;
+    if (int rc = check_ptr(last_used, "last_used")) return rc;
+    if (int rc = check_ptr(step_dev, "step_dev", true)) return rc;
+    if (int rc = check_ptr(n_fetch, "n_fetch")) return rc;
+    if (d.C > 0) {
+        if (int rc = check_ptr(fetch_slot, "fetch_slot")) return rc;
+        if (int rc = check_ptr(fetch_block, "fetch_block")) return rc;
+    }
+    if (int rc = check_ptr(ws, "ws")) return rc;
+    const WsLayout w = ws_layout(d);
+    if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
+    if (oasis::fused_tail_bytes(d.N, d.K) + 1024 > 227 * 1024)
+        return fail(OASIS_EINVAL, "max_blocks %d with budget %d exceeds the fused kernel's shared memory", d.N, d.K);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* sc = scores != nullptr ? scores : reinterpret_cast<float*>(base + w.scores);
+    int* ticket = reinterpret_cast<int*>(base + w.sticket);
+    const int row0 = d.Qn > 1 ? 1 : 0;
+    const int rows = (d.Qn > 1 ? d.Qn - 1 : 1) * d.G();
+    const unsigned long long total_rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.N;
+    CUtensorMap tmax, tmin;
+    if (int rc = make_map(&tmax, kmax, total_rows, oasis::kScoreTile, "kmax")) return rc;
+    if (int rc = make_map(&tmin, kmin, total_rows, oasis::kScoreTile, "kmin")) return rc;
+    const auto* qq = static_cast<const uint16_t*>(q);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (scores != nullptr)
+        return launch_fused_rows<true>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sel, sel_score,
+                                       slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch, s);
+    return launch_fused_rows<false>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sel, sel_score, slot_table,
+                                    last_used, step, step_dev, fetch_slot, fetch_block, n_fetch, s);
+}
+
 int oasis_block_overlap(const oasis_dims* dp, const int32_t* a, const int32_t* b, int32_t* count, void* stream) {
     Dims d;
     if (int rc = validate(dp, &d)) return rc;
@@ -499,10 +570,8 @@ int oasis_decode_layer_step(const oasis_dims* dp, const oasis_layer* L, const vo
                             const uint8_t* evict_mask, int32_t step, const int32_t* step_dev, float scale, void* ws,
                             size_t ws_bytes, const oasis_step_sync* S) {
     if (L == nullptr || S == nullptr) return fail(OASIS_EINVAL, "layer and sync must not be NULL");
-    if (S->fetch_done == nullptr || S->plan_ready == nullptr || S->sel_ready == nullptr)
-        return fail(OASIS_EINVAL, "fetch_done, plan_ready and sel_ready events must be given");
-    if (S->in_graph && S->fork == nullptr) return fail(OASIS_EINVAL, "in_graph needs the fork event");
-    const bool overlap = S->score != S->main;
+    if (S->fetch_done == nullptr || S->plan_ready == nullptr)
+        return fail(OASIS_EINVAL, "fetch_done and plan_ready events must be given");
     int rc;
     if (!S->in_graph && (rc = ev_wait(S->main, S->fetch_done, "wait fetch_done"))) return rc;
     // attention over the working set staged by the previous step
@@ -512,48 +581,21 @@ int oasis_decode_layer_step(const oasis_dims* dp, const oasis_layer* L, const vo
         return rc;
     if ((rc = ev_record(S->timing[1], S->main, "timing"))) return rc;
     if (evict_mask != nullptr && (rc = oasis_evict_slots(dp, evict_mask, L->slot_table, S->main))) return rc;
-    // lookahead scores + top-K, concurrent with the attention
-    if (overlap) {
-        if (S->in_graph) {
-            if ((rc = ev_record(S->fork, S->main, "record fork")) || (rc = ev_wait(S->score, S->fork, "wait fork")))
-                return rc;
-        } else if ((rc = ev_wait(S->score, S->plan_ready, "wait plan_ready"))) {   // previous plan read sel
-            return rc;
-        }
-    }
-    if ((rc = ev_record(S->timing[2], S->score, "timing"))) return rc;
-    if (L->scores != nullptr) {
-        if ((rc = oasis_lookahead_scores(dp, q, L->kmin, L->kmax, ctx_len, L->scores, S->score)) ||
-            (rc = oasis_select_topk(dp, L->scores, ctx_len, L->sel, L->sel_score, S->score)))
-            return rc;
-    } else if ((rc = oasis_score_select(dp, q, L->kmin, L->kmax, ctx_len, L->sel, L->sel_score, ws, ws_bytes,
-                                        S->score))) {
+    // lookahead scores + top-K + residency diff and capped plan, one launch,
+    // after the attention that read this layer's slot table
+    if ((rc = ev_record(S->timing[2], S->main, "timing"))) return rc;
+    if ((rc = oasis_score_select_plan(dp, q, L->kmin, L->kmax, ctx_len, L->sel, L->sel_score, L->scores,
+                                      L->slot_table, L->last_used, step, step_dev, L->fetch_slot, L->fetch_block,
+                                      L->n_fetch, ws, ws_bytes, S->main)))
         return rc;
-    }
-    if ((rc = ev_record(S->timing[3], S->score, "timing"))) return rc;
-    if (overlap && ((rc = ev_record(S->sel_ready, S->score, "record sel_ready")) ||
-                    (rc = ev_wait(S->main, S->sel_ready, "wait sel_ready"))))
-        return rc;
-    // residency diff + capped plan
-    if ((rc = ev_record(S->timing[4], S->main, "timing"))) return rc;
-    if (step_dev != nullptr)
-        rc = oasis_plan_fetch_at(dp, L->sel, L->scores, L->slot_table, L->last_used, step_dev, L->fetch_slot,
-                                 L->fetch_block, L->n_fetch, S->main);
-    else if (L->scores != nullptr)
-        rc = oasis_plan_fetch_scored(dp, L->sel, L->scores, L->slot_table, L->last_used, step, L->fetch_slot,
-                                     L->fetch_block, L->n_fetch, S->main);
-    else
-        rc = oasis_plan_fetch(dp, L->sel, L->slot_table, L->last_used, step, L->fetch_slot, L->fetch_block,
-                              L->n_fetch, S->main);
-    if (rc) return rc;
-    if ((rc = ev_record(S->timing[5], S->main, "timing"))) return rc;
+    if ((rc = ev_record(S->timing[3], S->main, "timing"))) return rc;
     if ((rc = ev_record(S->plan_ready, S->main, "record plan_ready")) ||
         (rc = ev_wait(S->copy, S->plan_ready, "wait plan_ready")))
         return rc;
     // the gather of the missing blocks, on the copy stream
-    if ((rc = ev_record(S->timing[6], S->copy, "timing"))) return rc;
+    if ((rc = ev_record(S->timing[4], S->copy, "timing"))) return rc;
     if ((rc = oasis_prefetch(dp, L->host_kv, L->fetch_slot, L->fetch_block, L->n_fetch, L->pool, S->copy))) return rc;
-    if ((rc = ev_record(S->timing[7], S->copy, "timing"))) return rc;
+    if ((rc = ev_record(S->timing[5], S->copy, "timing"))) return rc;
     return ev_record(S->fetch_done, S->copy, "record fetch_done");
 }
 
@@ -597,25 +639,21 @@ int oasis_sparse_attn(const oasis_dims* dp, const void* q, const void* pool, con
     if (!(scale > 0.f) || !(scale < 3.0e38f)) return fail(OASIS_EINVAL, "scale must be a positive finite float");
     const WsLayout w = ws_layout(d);
     if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
-    CUtensorMap tm;
+    CUtensorMap tm, tq;
     const unsigned long long rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.K * 2 * oasis::kBlockTokens;
-    if (int rc = make_map(&tm, pool, rows, 2 * oasis::kBlockTokens, "pool")) return rc;
+    if (int rc = make_map(&tm, pool, rows, oasis::kBlockTokens, "pool")) return rc;
+    if (int rc = make_map_q(&tq, q, d)) return rc;
     uint8_t* base = static_cast<uint8_t*>(ws);
     float* ws_lse = reinterpret_cast<float*>(base + w.lse);
     float* ws_o = reinterpret_cast<float*>(base + w.o);
+    int* ws_ticket = reinterpret_cast<int*>(base + w.ticket);
     const float scale_log2 = scale * 1.4426950408889634f;
-    const auto* qq = static_cast<const uint16_t*>(q);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int nt = (d.Qn * d.G() + 7) / 8;
-    switch (nt) {
-        case 1: return launch_attn<1, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
-        case 2: return launch_attn<2, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
-        case 3: return launch_attn<3, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
-        case 4: return launch_attn<4, 1>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
-        case 5:
-        case 6: return launch_attn<3, 2>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
-        default: return launch_attn<4, 2>(tm, d, qq, slot_table, ctx_len, scale_log2, out, lse, ws_o, ws_lse, s);
-    }
+    if (int rc = set_smem(oasis::sparse_attn_kernel, oasis::kAttnSmem, "sparse_attn smem")) return rc;
+    const long long ns = attn_streams(d);
+    oasis::sparse_attn_kernel<<<static_cast<unsigned>(ns), oasis::kAttnThreads, oasis::kAttnSmem, s>>>(
+        tm, tq, d, slot_table, ctx_len, scale_log2, static_cast<int>(ns), out, lse, ws_o, ws_lse, ws_ticket);
+    return check_launch("sparse_attn launch");
 }
 
 int oasis_read_device_error(uint32_t* out, int clear, void* stream) {

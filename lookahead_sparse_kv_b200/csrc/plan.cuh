@@ -58,21 +58,18 @@ __device__ __forceinline__ unsigned long long victim_key(int slot, int blk, uint
            static_cast<unsigned long long>(static_cast<uint32_t>(blk));
 }
 
-// blockDim.x = K rounded up to a multiple of 32; dynamic smem 7*K ints.
-// kScored: victims by the block's score (scores fp32 [B][Hkv][N]), else LRU.
-// step_dev (nullable): the step number is read from device memory instead of
-// `step`, so a captured graph can replay the plan at every step.
-template <bool kScored>
-__global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t* __restrict__ sel,
-                                                          const float* __restrict__ scores,
-                                                          int32_t* __restrict__ slot_table,
-                                                          int32_t* __restrict__ last_used, int step,
-                                                          const int32_t* __restrict__ step_dev,
-                                                          int32_t* __restrict__ fetch_slot,
-                                                          int32_t* __restrict__ fetch_block,
-                                                          int32_t* __restrict__ n_fetch) {
-    extern __shared__ int32_t sp[];
-    const int K = d.K, C = d.C, N = d.N;
+constexpr int kPlanThreads = 256;
+
+// Shared-memory ints plan_unit needs for budget K.
+__host__ __device__ constexpr int plan_smem_ints(int K) { return 9 * K; }
+
+// Plan of one (b, h) with NT threads (each loops over slots / ranks):
+// sel, st, lu point at the unit's K entries, fs/fb at its C fetch entries,
+// nf at its fetch count; scores_u (kScored) at its N block scores.  sp:
+// plan_smem_ints(K) ints of shared memory; tmp: 32 ints.
+template <int NT, bool kScored>
+__device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* scores_u, int32_t* st, int32_t* lu,
+                          int step, int32_t* fs, int32_t* fb, int32_t* nf, int32_t* sp, int* tmp) {
     int32_t* s_st = sp;
     int32_t* s_lu = sp + K;
     int32_t* s_prot = sp + 2 * K;
@@ -80,49 +77,56 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
     int32_t* s_nst = sp + 4 * K;
     int32_t* s_nlu = sp + 5 * K;
     uint32_t* s_ord = reinterpret_cast<uint32_t*>(sp + 6 * K);
-    __shared__ int tmp[32];
-
-    const int i = threadIdx.x;
-    const long long base = static_cast<long long>(blockIdx.x) * K;
-    if (step_dev != nullptr) step = *step_dev;
-    int sv = -1;
-    if (i < K) {
-        int st = slot_table[base + i];
-        if (st < -1 || st >= N) {
+    int32_t* s_sel = sp + 7 * K;
+    int32_t* s_mpos = sp + 8 * K;          // miss flag, then the miss's position in rank order (-1: no miss)
+    const int tid = threadIdx.x;
+    for (int i = tid; i < K; i += NT) {
+        int x = st[i];
+        if (x < -1 || x >= N) {
             raise_dev_error(OASIS_DEVERR_ID_RANGE);
-            st = -1;
+            x = -1;
         }
-        s_st[i] = st;
-        s_lu[i] = last_used[base + i];
+        s_st[i] = x;
+        s_lu[i] = lu[i];
         s_prot[i] = 0;
         if constexpr (kScored)
-            s_ord[i] = st >= 0 ? ordered_key(scores[static_cast<long long>(blockIdx.x) * N + st]) : 0u;
+            s_ord[i] = x >= 0 ? ordered_key(__ldcg(scores_u + x)) : 0u;
         else
             s_ord[i] = static_cast<uint32_t>(s_lu[i]) ^ 0x80000000u;   // signed order
-        sv = sel[base + i];
+        int sv = sel[i];
         if (sv < -1 || sv >= N) {
             raise_dev_error(OASIS_DEVERR_ID_RANGE);
             sv = -1;
         }
+        s_sel[i] = sv;
     }
     __syncthreads();
-
-    int hit = -1;
-    if (i < K) {
-        const int own = s_st[i];
+    // 1. residency lookup of every selected block; hits are protected
+    for (int i = tid; i < K; i += NT) {
+        const int sv = s_sel[i], own = s_st[i];
+        int hit = -1;
         for (int j = 0; j < K; ++j) {
             const int x = s_st[j];
             if (sv >= 0 && hit < 0 && x == sv) hit = j;
             if (own >= 0 && j < i && x == own) raise_dev_error(OASIS_DEVERR_DUPLICATE);
         }
         if (hit >= 0) s_prot[hit] = 1;
+        s_mpos[i] = (sv >= 0 && hit < 0) ? 1 : 0;
     }
-    const int miss = (i < K && sv >= 0 && hit < 0) ? 1 : 0;
-    int total_miss;
-    const int mpos = block_excl_sum_any(miss, tmp, &total_miss);   // syncs: s_prot visible after
-    const int nF = min(C, total_miss);
-
-    if (i < K) {
+    __syncthreads();
+    // 2. misses numbered in rank order
+    int running = 0;
+    for (int base = 0; base < K; base += NT) {
+        const int i = base + tid;
+        const int m = i < K ? s_mpos[i] : 0;
+        int total;
+        const int excl = block_excl_sum_any(m, tmp, &total);     // syncs
+        if (i < K) s_mpos[i] = m ? running + excl : -1;
+        running += total;
+    }
+    const int nF = min(C, running);
+    // 3. victims: rank of every unprotected slot among the candidates
+    for (int i = tid; i < K; i += NT) {
         const bool prot = s_prot[i] != 0;
         s_nst[i] = s_st[i];
         s_nlu[i] = prot ? step : s_lu[i];
@@ -135,23 +139,50 @@ __global__ void __launch_bounds__(1024) plan_fetch_kernel(Dims d, const int32_t*
         }
     }
     __syncthreads();
-    if (miss && mpos < nF) {
-        const int v = s_vict[mpos];
-        s_nst[v] = sv;
-        s_nlu[v] = step;
-        fetch_slot[static_cast<long long>(blockIdx.x) * C + mpos] = v;
-        fetch_block[static_cast<long long>(blockIdx.x) * C + mpos] = sv;
+    // 4. the first nF misses replace the victims in order
+    for (int i = tid; i < K; i += NT) {
+        const int mp = s_mpos[i];
+        if (mp >= 0 && mp < nF) {
+            const int v = s_vict[mp];
+            s_nst[v] = s_sel[i];
+            s_nlu[v] = step;
+            fs[mp] = v;
+            fb[mp] = s_sel[i];
+        }
     }
     __syncthreads();
-    if (i < K) {
-        slot_table[base + i] = s_nst[i];
-        last_used[base + i] = s_nlu[i];
+    for (int i = tid; i < K; i += NT) {
+        st[i] = s_nst[i];
+        lu[i] = s_nlu[i];
     }
-    for (int f = nF + i; f < C; f += blockDim.x) {
-        fetch_slot[static_cast<long long>(blockIdx.x) * C + f] = -1;
-        fetch_block[static_cast<long long>(blockIdx.x) * C + f] = -1;
+    for (int f = nF + tid; f < C; f += NT) {
+        fs[f] = -1;
+        fb[f] = -1;
     }
-    if (i == 0) n_fetch[blockIdx.x] = nF;
+    if (tid == 0) *nf = nF;
+}
+
+// One CTA of kPlanThreads per (b, h); dynamic smem plan_smem_ints(K) ints.
+// kScored: victims by the block's score (scores fp32 [B][Hkv][N]), else LRU.
+// step_dev (nullable): the step number is read from device memory instead of
+// `step`, so a captured graph can replay the plan at every step.
+template <bool kScored>
+__global__ void __launch_bounds__(kPlanThreads) plan_fetch_kernel(Dims d, const int32_t* __restrict__ sel,
+                                                                  const float* __restrict__ scores,
+                                                                  int32_t* __restrict__ slot_table,
+                                                                  int32_t* __restrict__ last_used, int step,
+                                                                  const int32_t* __restrict__ step_dev,
+                                                                  int32_t* __restrict__ fetch_slot,
+                                                                  int32_t* __restrict__ fetch_block,
+                                                                  int32_t* __restrict__ n_fetch) {
+    extern __shared__ int32_t sp[];
+    __shared__ int tmp[32];
+    const long long bh = blockIdx.x;
+    const long long base = bh * d.K;
+    if (step_dev != nullptr) step = *step_dev;
+    plan_unit<kPlanThreads, kScored>(d.K, d.C, d.N, sel + base, kScored ? scores + bh * d.N : nullptr,
+                                     slot_table + base, last_used + base, step, fetch_slot + bh * d.C,
+                                     fetch_block + bh * d.C, n_fetch + bh, sp, tmp);
 }
 
 // Residency loss: frees every slot whose mask byte is set (n = B*Hkv*K).

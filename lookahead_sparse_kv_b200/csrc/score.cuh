@@ -34,28 +34,24 @@ struct ScoreSmem {
     static constexpr int kTmemCols = NPAD <= 32 ? 32 : (NPAD <= 64 ? 64 : (NPAD <= 128 ? 128 : 256));
 };
 
-// rows = real query vectors (scored query rows x G), the scored rows being
-// row0, row0+1, ...; NPAD = rows rounded up to 16.
+// Scores of the 128-block tile starting at n0 of unit bh (b, h) into
+// scores[bh][n0, nv): called by all 128 threads of the CTA with `smem`
+// (1024-aligned, ScoreSmem<NPAD>::kBytes - 1024 bytes).  rows = real query
+// vectors (scored query rows x G), the scored rows being row0, row0+1, ...;
+// NPAD = rows rounded up to 16.  The shared memory may be reused when it
+// returns (its barriers are invalidated).
 template <int NPAD>
-__global__ void __launch_bounds__(128) lookahead_score_kernel(const __grid_constant__ CUtensorMap tm_kmax,
-                                                              const __grid_constant__ CUtensorMap tm_kmin,
-                                                              Dims d, const uint16_t* __restrict__ q,
-                                                              const int32_t* __restrict__ ctx_len,
-                                                              float* __restrict__ scores, int row0, int rows) {
+__device__ __forceinline__ void score_tile(const CUtensorMap* tm_kmax, const CUtensorMap* tm_kmin, const Dims& d,
+                                           const uint16_t* __restrict__ q, int b, int h, int n0, int nv,
+                                           float* __restrict__ scores, int row0, int rows, uint8_t* smem) {
     using S = ScoreSmem<NPAD>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* a_tile = smem;
     uint8_t* b_tile = smem + kScoreABytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(b_tile + 4 * S::kBRegion);   // [0] tma full, [1] mma done
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
     int* flag = reinterpret_cast<int*>(bars + 3);
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.y, b = bh / d.Hkv, h = bh % d.Hkv;
-    const int nv = n_valid_blocks(ctx_len[b], d.N);
-    const int n0 = blockIdx.x * kScoreTile;
-    if (n0 >= nv) return;   // whole CTA: tile beyond the sequence's context
+    const int bh = b * d.Hkv + h;
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
@@ -68,10 +64,10 @@ __global__ void __launch_bounds__(128) lookahead_score_kernel(const __grid_const
         const uint64_t pol = l2_policy_evict_first();
         const int y = bh * d.N + n0;
         mbar_arrive_expect_tx(&bars[0], kScoreABytes);
-        tma_load_2d(a_tile + 0 * kScoreRegionBytes, &tm_kmax, &bars[0], 0, y, pol);
-        tma_load_2d(a_tile + 1 * kScoreRegionBytes, &tm_kmax, &bars[0], 64, y, pol);
-        tma_load_2d(a_tile + 2 * kScoreRegionBytes, &tm_kmin, &bars[0], 0, y, pol);
-        tma_load_2d(a_tile + 3 * kScoreRegionBytes, &tm_kmin, &bars[0], 64, y, pol);
+        tma_load_2d(a_tile + 0 * kScoreRegionBytes, tm_kmax, &bars[0], 0, y, pol);
+        tma_load_2d(a_tile + 1 * kScoreRegionBytes, tm_kmax, &bars[0], 64, y, pol);
+        tma_load_2d(a_tile + 2 * kScoreRegionBytes, tm_kmin, &bars[0], 0, y, pol);
+        tma_load_2d(a_tile + 3 * kScoreRegionBytes, tm_kmin, &bars[0], 64, y, pol);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, S::kTmemCols);
@@ -110,8 +106,10 @@ __global__ void __launch_bounds__(128) lookahead_score_kernel(const __grid_const
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
+    bool tma_done = false;
     if (tid == 0) {
         if (mbar_wait(&bars[0], 0)) {
+            tma_done = true;
             constexpr uint32_t idesc = umma_idesc_bf16_f32(kScoreTile, NPAD);
             const uint32_t a0 = smem_addr(a_tile), b0 = smem_addr(b_tile);
 #pragma unroll
@@ -153,6 +151,28 @@ __global__ void __launch_bounds__(128) lookahead_score_kernel(const __grid_const
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, S::kTmemCols);
+    if (tid == 0) {
+        // a copy that never completed must not land in memory reused below
+        if (!tma_done && !mbar_wait(&bars[0], 0)) raise_dev_error(OASIS_DEVERR_TIMEOUT);
+        mbar_inval(&bars[0]);
+        mbar_inval(&bars[1]);
+    }
+    __syncthreads();
+}
+
+template <int NPAD>
+__global__ void __launch_bounds__(128) lookahead_score_kernel(const __grid_constant__ CUtensorMap tm_kmax,
+                                                              const __grid_constant__ CUtensorMap tm_kmin,
+                                                              Dims d, const uint16_t* __restrict__ q,
+                                                              const int32_t* __restrict__ ctx_len,
+                                                              float* __restrict__ scores, int row0, int rows) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int bh = blockIdx.y, b = bh / d.Hkv, h = bh % d.Hkv;
+    const int nv = n_valid_blocks(ctx_len[b], d.N);
+    const int n0 = blockIdx.x * kScoreTile;
+    if (n0 >= nv) return;   // whole CTA: tile beyond the sequence's context
+    score_tile<NPAD>(&tm_kmax, &tm_kmin, d, q, b, h, n0, nv, scores, row0, rows, smem);
 }
 
 }  // namespace oasis

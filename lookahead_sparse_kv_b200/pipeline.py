@@ -10,12 +10,16 @@ step t-1.
 
 Streams (all work is in liboasis kernels; this module only orders them):
 
-* main  - [append] -> sparse attention -> plan        (per layer, in order)
-* score - lookahead scores + top-K, concurrent with the attention of the same
-          layer (they read disjoint buffers); waits for the layer's previous
-          plan before overwriting its selection
+* main  - [append] -> sparse attention -> [residency loss] -> scores + top-K +
+          plan in one launch                            (per layer, in order)
 * copy  - host-to-HBM gather, high priority, after the layer's plan; the next
           step's append/attention of that layer waits for it
+
+Scoring follows the attention of its layer on the main stream: the plan
+rewrites the slot table the attention reads, and the attention kernel holds
+all of every SM's shared memory while it runs, so scoring beside it would
+only queue behind it.  The gathers of the layers overlap the compute of the
+other layers (Figure 8).
 
 Exact-set mode (OasisKV Figures 4 and 6; prediction misses need corrective
 fetches): before a layer's attention at step t the main stream ranks the
@@ -26,38 +30,35 @@ the missing blocks of E_t with no cap, in stream order before the attention.
 
 Victim order: LRU (OasisKV Table 2) or, with ``victims="score"``, the stale
 block with the lowest current lookahead score first; the scores of each
-layer then go to a buffer of its own so the plan on the main stream can
-read them while the score stream moves on to the next layer.
+layer then go to a buffer of its own.
 
 Native steps: unless the exact-set stage is on, a layer's decode step is one
 call into the library (``oasis_decode_layer_step``), which enqueues the
 kernels and does the stream / event order above in C, so the host cost per
-layer-step is one call instead of a dozen.
+layer-step is one call instead of several.
 
 Graph mode (``device_step=True``): the step number lives in device memory
 (advanced by a kernel at the start of each step, read by the planner), so a
 whole multi-layer decode step can be captured once as a CUDA graph
 (``capture``) and replayed (``replay``) with one launch per step.  Inside
-the graph the score stream forks from the main stream at each layer and all
-gathers join the main stream at the end, so a replay is self-contained; the
-price is that the last layers' gathers no longer overlap the next step's
-first layers, which matters little for deep stacks.  Appends and the
+the graph all gathers join the main stream at the end, so a replay is
+self-contained; the price is that the last layers' gathers no longer overlap
+the next step's first layers, which matters little for deep stacks.  Appends and the
 exact-set stage take per-step host values and are not captured.
 
 Memory: the full KV of every layer lives in pinned host memory; HBM holds per
 layer the per-block summaries (N x 512 B per KV head), the fixed pool of K
 slots (8 KiB each) and a few small int tables.  One workspace serves all
-layers because each stream runs its layers in order and the two workspace
-regions (scores, attention partials) are disjoint.
+layers because the main stream runs the layers' kernels in order.
 """
 
 from __future__ import annotations
 
 import torch
 
-from . import (StepSync, append_kv, block_overlap, build_summaries, decode_layer_step, evict_slots,
-               lookahead_scores, make_dims, make_layer, plan_fetch, plan_fetch_at, plan_fetch_scored, prefetch,
-               score_select, score_select_rows, select_topk, sparse_attn, step_advance, workspace_bytes)
+from . import (StepSync, append_kv, block_overlap, build_summaries, decode_layer_step, evict_slots, make_dims,
+               make_layer, plan_fetch, plan_fetch_at, prefetch, score_select_plan, score_select_rows, sparse_attn,
+               step_advance, workspace_bytes)
 
 HEAD_DIM, BLOCK_TOKENS = 128, 16
 
@@ -101,7 +102,6 @@ class LayerState:
         self.cfetch_block = torch.full((B, H, K), -1, dtype=torch.int32, device=device)
         # each [B, Hkv] slice padded to 16 bytes (the library's pointer alignment)
         self.hist = torch.zeros((4, steps_cap, (B * H + 3) // 4 * 4), dtype=torch.int32, device=device)
-        self.sel_read = torch.cuda.Event()
 
     def hist_slot(self, k: int, slot: int) -> torch.Tensor:
         d = self.d
@@ -117,7 +117,7 @@ class DecodePipeline:
     """Drives priming and decode steps over a list of layers."""
 
     def __init__(self, d, layers, ctx_len: torch.Tensor, scale: float, device="cuda",
-                 overlap_score: bool = True, exact: str | None = None, steps_cap: int = 256,
+                 single_stream: bool = False, exact: str | None = None, steps_cap: int = 256,
                  victims: str = "lru", device_step: bool = False):
         assert exact in (None, "measure", "correct") and victims in ("lru", "score")
         assert not (device_step and exact is not None), "the exact-set stage is not graph-capturable"
@@ -134,8 +134,7 @@ class DecodePipeline:
                                            device=device)
         self.steps_cap = steps_cap
         if exact is not None:
-            # uncapped plan / gather for the corrective fetch; a workspace of its own
-            # because the score stream may be scoring the previous layer meanwhile
+            # uncapped plan / gather for the corrective fetch, with a workspace of its own
             self.d_full = make_dims(d.batch, d.n_q_heads, d.n_kv_heads, d.max_blocks, d.budget_blocks,
                                     d.n_queries, d.budget_blocks, d.head_dim, d.block_tokens)
             self.ws_exact = torch.zeros(workspace_bytes(d), dtype=torch.uint8, device=device)
@@ -148,16 +147,14 @@ class DecodePipeline:
         self.main = torch.cuda.Stream(device) if device_step else torch.cuda.current_stream(device)
         if device_step:
             self.main.wait_stream(torch.cuda.current_stream(device))
-        self.score_stream = torch.cuda.Stream(device) if overlap_score else self.main
         lo, hi = torch.cuda.Stream.priority_range()
-        self.copy_stream = torch.cuda.Stream(device, priority=hi)
-        self.step_start = torch.cuda.Event()
-        self.sel_ready = [torch.cuda.Event() for _ in layers]
-        self.fork = [torch.cuda.Event() for _ in layers]
+        # single_stream: the gathers too run on the main stream (the order a
+        # one-stream caller would get; the tests compare the two)
+        self.copy_stream = self.main if single_stream else torch.cuda.Stream(device, priority=hi)
         # the native step takes raw event handles: create every event now (torch creates them
         # on first record; recording on an idle stream completes at once)
-        for i, L in enumerate(layers):
-            for ev in (L.plan_ready, L.fetch_done, self.sel_ready[i], self.fork[i]):
+        for L in layers:
+            for ev in (L.plan_ready, L.fetch_done):
                 ev.record(self.main)
         self._native = [None] * len(layers)
         self.timer = None        # optional: begin(name, stream) / end(name, stream) around each call
@@ -178,37 +175,16 @@ class DecodePipeline:
         if self.step_dev is not None:
             plan_fetch_at(d, sel, scores, L.slot_table, L.last_used, self.step_dev, fetch_slot, fetch_block,
                           n_fetch, stream=self.main)
-        elif scores is not None:
-            plan_fetch_scored(d, sel, scores, L.slot_table, L.last_used, step, fetch_slot, fetch_block, n_fetch,
-                              stream=self.main)
         else:
             plan_fetch(d, sel, L.slot_table, L.last_used, step, fetch_slot, fetch_block, n_fetch, stream=self.main)
 
-    def _select_plan_fetch(self, i, L, q, step, ctx, in_graph=False):
+    def _select_plan_fetch(self, i, L, q, step, ctx):
         d, main = self.d, self.main
-        if self.score_stream is not main:
-            if in_graph:
-                # fork from this replay's main stream; the previous plan ran in the previous replay
-                self.fork[i].record(main)
-                self.score_stream.wait_event(self.fork[i])
-            else:
-                self.score_stream.wait_event(L.plan_ready)     # previous plan has read L.sel
-            if self.exact is not None and step > 0:
-                self.score_stream.wait_event(L.sel_read)   # so has the agreement count
-        self._t("begin", "score_select", self.score_stream)
-        if self.victims == "score":
-            lookahead_scores(d, q, L.kmin, L.kmax, ctx, L.scores, stream=self.score_stream)
-            select_topk(d, L.scores, ctx, L.sel, L.sel_score, stream=self.score_stream)
-        else:
-            score_select(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, self.ws, stream=self.score_stream)
-        self._t("end", "score_select", self.score_stream)
-        if self.score_stream is not main:
-            self.sel_ready[i].record(self.score_stream)
-            main.wait_event(self.sel_ready[i])
-        self._t("begin", "plan_fetch", main)
-        self._plan(d, L.sel, L.scores if self.victims == "score" else None, L, step, L.fetch_slot, L.fetch_block,
-                   L.n_fetch)
-        self._t("end", "plan_fetch", main)
+        self._t("begin", "score_select_plan", main)
+        score_select_plan(d, q, L.kmin, L.kmax, ctx, L.sel, L.sel_score, L.scores if self.victims == "score" else None,
+                          L.slot_table, L.last_used, 0 if step is None else step, self.step_dev, L.fetch_slot,
+                          L.fetch_block, L.n_fetch, self.ws, stream=main)
+        self._t("end", "score_select_plan", main)
         L.plan_ready.record(main)
         self.copy_stream.wait_event(L.plan_ready)
         self._t("begin", "prefetch", self.copy_stream)
@@ -224,9 +200,8 @@ class DecodePipeline:
         return self._native[i]
 
     def _native_sync(self, i, L, in_graph):
-        sync = StepSync(self.main.cuda_stream, self.score_stream.cuda_stream, self.copy_stream.cuda_stream,
-                        L.fetch_done.cuda_event, L.plan_ready.cuda_event, self.sel_ready[i].cuda_event,
-                        self.fork[i].cuda_event, 1 if in_graph else 0)
+        sync = StepSync(self.main.cuda_stream, self.copy_stream.cuda_stream, L.fetch_done.cuda_event,
+                        L.plan_ready.cuda_event, 1 if in_graph else 0)
         if self.timer is not None and hasattr(self.timer, "native_handles"):
             for k, h in enumerate(self.timer.native_handles()):
                 sync.timing[k] = h
@@ -243,7 +218,6 @@ class DecodePipeline:
         if t > 1:
             block_overlap(d, prev, cur, h[1], stream=main)
         block_overlap(d, L.slot_table, cur, h[2], stream=main)
-        L.sel_read.record(main)
         self._t("end", "exact_set", main)
         if self.exact == "correct":
             self._t("begin", "corrective", main)
@@ -262,24 +236,22 @@ class DecodePipeline:
     def prime(self, q_per_layer):
         """Step 0: select, plan and fetch from the drafts before decoding starts."""
         for i, (L, q) in enumerate(zip(self.layers, q_per_layer)):
-            L.plan_ready.record(self.main)
-            self._select_plan_fetch(i, L, q, 0, self.ctx_len)
+            self._select_plan_fetch(i, L, q, None if self.step_dev is not None else 0, self.ctx_len)
 
     def step(self, t, q_per_layer, appended=None, evict=None, inputs_ready=None, layer_done=None):
         """Decode step t >= 1: per layer [append] -> attention -> [loss] -> select/plan/fetch.
 
-        Each layer's queries are read on the main stream (attention) and on the
-        score stream (scores); the score stream starts the step after all work
-        enqueued on the main stream before this call, so queries written there
-        (a non-blocking copy, say) are seen by both.
+        Each layer's queries are read on the main stream (attention, then
+        scores), so queries written there before this call (a non-blocking copy,
+        say) are seen by both.
         appended: optional list of (k_new, v_new) per layer, bf16 [B, Hkv, D],
         the token accepted at the previous step; it is written at position
         ctx_len[b] and the context is one token longer from this step on.
         evict: optional list of uint8 masks [B, Hkv, K] per layer; the marked
         slots are freed after the layer's attention (residency loss).
         inputs_ready: optional list of CUDA events, one per layer; layer i's
-        work on both streams waits for event i first, so a caller can bring
-        each layer's queries in on a stream of its own.
+        work waits for event i first, so a caller can bring each layer's
+        queries in on a stream of its own.
         layer_done: optional list of CUDA events, one per layer; event i is
         recorded on the main stream once layer i's attention and plan are
         enqueued (its out and lse are final from there on).
@@ -299,25 +271,15 @@ class DecodePipeline:
             ctx_in = ctx = self.ctx_len
         else:
             ctx_in, ctx = self.ctx[self.cur], self.ctx[1 - self.cur]
-        if not in_graph and self.score_stream is not main:
-            # the queries may have been written on main just before this step
-            self.step_start.record(main)
-            self.score_stream.wait_event(self.step_start)
         for i, (L, q) in enumerate(zip(self.layers, q_per_layer)):
             if inputs_ready is not None and inputs_ready[i] is not None:
                 main.wait_event(inputs_ready[i])
-                if self.score_stream is not main:
-                    self.score_stream.wait_event(inputs_ready[i])
             if not in_graph and (self.exact is not None or appended is not None):
                 main.wait_event(L.fetch_done)          # (the native step waits for it itself)
             if appended is not None:
                 k_new, v_new = appended[i]
                 append_kv(d, k_new, v_new, ctx_in, ctx if i == 0 else None, L.host_kv, L.kmin, L.kmax,
                           L.slot_table, L.pool, stream=main)
-                if self.score_stream is not main:
-                    ev = torch.cuda.Event()
-                    ev.record(main)
-                    self.score_stream.wait_event(ev)       # grown summaries and context
             if self.exact is None:
                 decode_layer_step(d, self._native_layer(i, L), q, ctx, None if evict is None else evict[i],
                                   0 if t is None else t, self.step_dev, self.scale, self.ws,
@@ -329,7 +291,7 @@ class DecodePipeline:
                 self._t("end", "sparse_attn", main)
                 if evict is not None:
                     evict_slots(d, evict[i], L.slot_table, stream=main)
-                self._select_plan_fetch(i, L, q, t, ctx, in_graph)
+                self._select_plan_fetch(i, L, q, t, ctx)
             if layer_done is not None and layer_done[i] is not None:
                 layer_done[i].record(main)
         if appended is not None:

@@ -31,8 +31,8 @@ def test_kernel_hash_ignores_comment_edits_only(tmp_path, monkeypatch):
 
 
 def test_overlap_efficiency_bounds():
-    iso = {"sparse_attn": 0.04, "score_select": 0.05, "plan_fetch": 0.01, "prefetch": 0.25}
-    t_c, t_f = 0.06, 0.25                 # max(attention, scores + top-K) + plan
+    iso = {"sparse_attn": 0.03, "score_select_plan": 0.035, "prefetch": 0.25}
+    t_c, t_f = 0.065, 0.25                # attention + (scores, top-K and plan)
     full = bench.overlap_efficiency(iso, max(t_c, t_f))          # perfect overlap
     none = bench.overlap_efficiency(iso, t_c + t_f)              # back to back
     assert math.isclose(full["value"], 1.0) and math.isclose(none["value"], 0.0, abs_tol=1e-12)
@@ -73,12 +73,12 @@ def test_gpu_line_keeps_the_contract(capsys):
     import torch
     w = W.WORKLOADS[bench.WORKLOAD]
     nl, steps = 8, 10
-    ms_pipe = {"sparse_attn": 0.16, "score_select": 0.16, "plan_fetch": 0.01, "prefetch": 0.277}
+    ms_pipe = {"sparse_attn": 0.03, "score_select_plan": 0.04, "prefetch": 0.277}
     res = {
         "w": w, "timer": _FakeTimer(ms_pipe), "layers": [None] * nl,
         "fetch_hist": torch.full((steps * nl,), 1583.0),
         "h2d": {"memcpy_gbs": 55.6, "zero_copy_gbs": 51.1, "peak_gbs": 55.6},
-        "iso": {"sparse_attn": 0.043, "score_select": 0.046, "plan_fetch": 0.012, "prefetch": 0.26,
+        "iso": {"sparse_attn": 0.03, "score_select_plan": 0.04, "plan_fetch": 0.012, "prefetch": 0.26,
                 "select_only": 0.016, "build_summaries": 20.9, "_prefetch_blocks": 1572},
         "ms": 2.25 * steps, "e2e_steps": steps, "e2e_ms": 2.4 * steps, "layer": _FakeLayer(w),
         "reuse": [0.9, 0.89], "host_ms": 2.1 * steps, "host_cost_ms": 0.19,

@@ -90,6 +90,11 @@ def test_no_call_writes_outside_its_buffers():
     lsk.score_select(d, qs[0], t["kmin"], t["kmax"], t["ctx"], t["sel"], t["sel_score"], t["ws"])
     lsk.plan_fetch(d, t["sel"], t["slot_table"], t["last_used"], 0, t["fetch_slot"], t["fetch_block"], t["n_fetch"])
     lsk.prefetch(d, t["host_kv"], t["fetch_slot"], t["fetch_block"], t["n_fetch"], t["pool"])
+    # scores + top-K + plan in one launch, LRU (scores in the workspace) and score-ordered victims
+    lsk.score_select_plan(d, qs[0], t["kmin"], t["kmax"], t["ctx"], t["sel"], t["sel_score"], None, t["slot_table"],
+                          t["last_used"], 0, None, t["fetch_slot"], t["fetch_block"], t["n_fetch"], t["ws"])
+    lsk.score_select_plan(d, qs[0], t["kmin"], t["kmax"], t["ctx"], t["sel"], None, t["scores"], t["slot_table"],
+                          t["last_used"], 0, t["step"], t["fetch_slot"], t["fetch_block"], t["n_fetch"], t["ws"])
     for step in range(1, 4):
         q = qs[step]
         lsk.sparse_attn(d, q, t["pool"], t["slot_table"], t["ctx"], scale, t["out"], t["lse"], t["ws"])
@@ -114,8 +119,7 @@ def test_no_call_writes_outside_its_buffers():
     layer = lsk.make_layer(d, t["host_kv"], t["kmin"], t["kmax"], t["pool"], t["slot_table"], t["last_used"],
                            t["sel"], t["sel_score"], None, t["fetch_slot"], t["fetch_block"], t["n_fetch"], t["out"],
                            t["lse"])
-    sync = lsk.StepSync(s.cuda_stream, s.cuda_stream, s.cuda_stream, evs[0].cuda_event, evs[1].cuda_event,
-                        evs[2].cuda_event, None, 0)
+    sync = lsk.StepSync(s.cuda_stream, s.cuda_stream, evs[0].cuda_event, evs[1].cuda_event, 0)
     t["step"].fill_(4)
     for step in range(4, 7):
         lsk.step_advance(t["step"])

@@ -84,13 +84,13 @@ def test_tiny_decode_stage_by_stage():
     assert (np_i32(L.slot_table) >= 0).all()
 
 
-def _run(w, overlap, steps):
+def _run(w, single_stream, steps):
     """Runs priming + steps with the stream pipeline; returns per-step outputs."""
     d = lsk.dims_for(w)
     host = W.make_host_kv(w).pin_memory()
     L = LayerState(d, host, DEV)
     pipe = DecodePipeline(d, [L], W.initial_ctx_len(w).to(DEV), 1 / math.sqrt(128), DEV,
-                          overlap_score=overlap)
+                          single_stream=single_stream)
     pipe.build_summaries()
     qs = W.QueryStream(w)
     pipe.prime([qs.next().to(DEV)])
@@ -106,8 +106,8 @@ def _run(w, overlap, steps):
 def test_pipeline_streams_match_sequential_order():
     w = W.WORKLOADS["llama8b_32k"].with_(batch=2, n_q_heads=8, n_kv_heads=2, context=8192,
                                           max_blocks=512, budget_blocks=64, fetch_cap=8)
-    a = _run(w, overlap=True, steps=5)
-    b = _run(w, overlap=False, steps=5)
+    a = _run(w, single_stream=False, steps=5)
+    b = _run(w, single_stream=True, steps=5)
     for x, y in zip(a, b):
         for u, v in zip(x, y):
             assert torch.equal(u, v)
@@ -122,7 +122,7 @@ def _run_fed(w, mode, steps):
     w = w.with_(layers=2)
     d = lsk.dims_for(w)
     layers = [LayerState(d, W.make_host_kv(w, l).pin_memory(), DEV) for l in range(2)]
-    pipe = DecodePipeline(d, layers, W.initial_ctx_len(w).to(DEV), 1 / math.sqrt(128), DEV, overlap_score=True)
+    pipe = DecodePipeline(d, layers, W.initial_ctx_len(w).to(DEV), 1 / math.sqrt(128), DEV)
     pipe.build_summaries()
     streams = [W.QueryStream(w, l) for l in range(2)]
     pipe.prime([s.next().to(DEV) for s in streams])
@@ -190,7 +190,7 @@ def test_multilayer_append_decode():
     hosts = [W.make_host_kv(w, l).pin_memory() for l in range(w.layers)]
     layers = [LayerState(d, h, DEV) for h in hosts]
     ctx = W.initial_ctx_len(w)
-    pipe = DecodePipeline(d, layers, ctx.to(DEV), scale, DEV, overlap_score=True)
+    pipe = DecodePipeline(d, layers, ctx.to(DEV), scale, DEV)
     pipe.build_summaries()
     streams = [W.QueryStream(w, l) for l in range(w.layers)]
     # oracle state per layer (float64 keys / values mirror the host KV)

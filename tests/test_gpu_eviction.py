@@ -71,7 +71,7 @@ def test_pipeline_with_score_victims_step_by_step():
     ctx = W.initial_ctx_len(w)
     cnp = ctx.numpy()
     L = LayerState(d, host, DEV)
-    pipe = DecodePipeline(d, [L], ctx.to(DEV), 1 / math.sqrt(128), DEV, overlap_score=True, victims="score")
+    pipe = DecodePipeline(d, [L], ctx.to(DEV), 1 / math.sqrt(128), DEV, victims="score")
     pipe.build_summaries()
     kmin, kmax = O.block_summaries(keys, cnp)
     qs = W.QueryStream(w)

@@ -245,6 +245,92 @@ def test_plan_fetch_bit_exact_random(K, C, N):
         st, lu = plan["slot_table"], plan["last_used"]
 
 
+# ------------------------------------------- scores + top-K + plan, fused
+@pytest.mark.parametrize("Hq,Hkv,Qn,N,K,C,victims", [(8, 2, 5, 300, 32, 6, "lru"), (32, 8, 5, 1000, 128, 16, "lru"),
+                                                     (64, 8, 8, 700, 128, 16, "score"), (12, 4, 3, 257, 64, 64, "score"),
+                                                     (8, 8, 1, 129, 16, 0, "lru"), (16, 2, 4, 4096, 1024, 40, "lru")])
+def test_score_select_plan_matches_separate_kernels_and_oracle(Hq, Hkv, Qn, N, K, C, victims):
+    """The one-launch scores + top-K + plan against the three separate
+    kernels (bit for bit: selection, selected scores, slot table, recency,
+    fetch lists) and against the oracle (selection under the tie rule, plan
+    bit-exact on the GPU's selection), over several steps of a random decode
+    state, with the step number given by value and read from device memory
+    on alternate steps.  Sequences cover a context that fits the budget, one
+    with no context at all, and ragged last tiles."""
+    B = 3
+    d = _dims(B, Hq, Hkv, N, K, Qn, C)
+    g = _gen(500 + N + K)
+    kv = random_kv(B, Hkv, N, g)
+    ctx = torch.tensor([N * 16 - 7, min(N, K) * 16 - 20, 0], dtype=torch.int32)
+    ctx_d = ctx.to(DEV)
+    kmin = torch.zeros((B, Hkv, N, 128), dtype=torch.bfloat16, device=DEV)
+    kmax = kmin.clone()
+    lsk.build_summaries(d, kv.to(DEV), ctx_d, kmin, kmax)
+    ws = torch.zeros(lsk.workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    ws2 = torch.zeros_like(ws)
+    okmin, okmax = f64(kmin), f64(kmax)
+    c = max(C, 1)
+    # fused (F) and separate (S) states, both starting from the same random residency
+    rng = np.random.default_rng(N + K)
+    st0 = np.full((B, Hkv, K), -1, dtype=np.int32)
+    for b in range(B):
+        nvb = int(O.n_valid_blocks(ctx.numpy(), 16)[b])
+        for h in range(Hkv):
+            ids = rng.permutation(max(nvb, 1))[: rng.integers(0, min(K, nvb) + 1)] if nvb else []
+            st0[b, h, :len(ids)] = ids
+            st0[b, h] = rng.permutation(st0[b, h])
+    lu0 = np.where(st0 >= 0, rng.integers(-1, 5, size=st0.shape), -1).astype(np.int32)
+    F = {k: torch.from_numpy(v.copy()).to(DEV) for k, v in (("st", st0), ("lu", lu0))}
+    S = {k: torch.from_numpy(v.copy()).to(DEV) for k, v in (("st", st0), ("lu", lu0))}
+    for X in (F, S):
+        X.update(sel=torch.empty((B, Hkv, K), dtype=torch.int32, device=DEV),
+                 sel_score=torch.empty((B, Hkv, K), device=DEV),
+                 fs=torch.full((B, Hkv, c), -9, dtype=torch.int32, device=DEV),
+                 fb=torch.full((B, Hkv, c), -9, dtype=torch.int32, device=DEV),
+                 nf=torch.full((B, Hkv), -9, dtype=torch.int32, device=DEV),
+                 scores=torch.zeros((B, Hkv, N), device=DEV))
+    step_dev = torch.zeros(4, dtype=torch.int32, device=DEV)
+    st, lu = st0, lu0
+    for step in range(5, 10):
+        q = (torch.randn(B, Qn, Hq, 128, generator=g) * 1.3).to(torch.bfloat16)
+        qd = q.to(DEV)
+        scored = victims == "score"
+        step_dev.fill_(step)
+        lsk.score_select_plan(d, qd, kmin, kmax, ctx_d, F["sel"], F["sel_score"], F["scores"] if scored else None,
+                              F["st"], F["lu"], -1 if step % 2 else step, step_dev if step % 2 else None, F["fs"],
+                              F["fb"], F["nf"], ws)
+        if scored:
+            lsk.lookahead_scores(d, qd, kmin, kmax, ctx_d, S["scores"])
+            lsk.select_topk(d, S["scores"], ctx_d, S["sel"], S["sel_score"])
+            lsk.plan_fetch_scored(d, S["sel"], S["scores"], S["st"], S["lu"], step, S["fs"], S["fb"], S["nf"])
+        else:
+            lsk.score_select(d, qd, kmin, kmax, ctx_d, S["sel"], S["sel_score"], ws2)
+            lsk.plan_fetch(d, S["sel"], S["st"], S["lu"], step, S["fs"], S["fb"], S["nf"])
+        torch.cuda.synchronize()
+        nf_np = np_i32(F["nf"])
+        for key in ("sel", "sel_score", "st", "lu", "nf"):
+            assert torch.equal(F[key], S[key]), f"{key} differs from the separate kernels at step {step}"
+        if C:
+            for b in range(B):
+                for h in range(Hkv):
+                    n = nf_np[b, h]
+                    assert torch.equal(F["fs"][b, h, :C], S["fs"][b, h, :C]) and n <= C
+                    assert torch.equal(F["fb"][b, h, :C], S["fb"][b, h, :C])
+        sc = O.lookahead_scores(f64(q), okmin, okmax, ctx.numpy(), 16)
+        ref_sel, _ = O.select_topk(sc, ctx.numpy(), K, 16)
+        sel = np_i32(F["sel"])
+        assert_selection_matches(sel, ref_sel, sc, ctx.numpy(), K)
+        assert (sel[2] == -1).all()                                         # no context: nothing selected
+        plan = O.plan_fetch(sel, st, lu, step, C, scores=F["scores"].cpu().numpy() if scored else None)
+        np.testing.assert_array_equal(np_i32(F["st"]), plan["slot_table"])
+        np.testing.assert_array_equal(np_i32(F["lu"]), plan["last_used"])
+        np.testing.assert_array_equal(nf_np, plan["n_fetch"])
+        if C:
+            np.testing.assert_array_equal(np_i32(F["fs"])[..., :C], plan["fetch_slot"])
+            np.testing.assert_array_equal(np_i32(F["fb"])[..., :C], plan["fetch_block"])
+        st, lu = plan["slot_table"], plan["last_used"]
+
+
 # --------------------------------------------------------------- prefetch
 def test_prefetch_bytes_exact():
     B, H, N, K, C = 2, 3, 50, 16, 6

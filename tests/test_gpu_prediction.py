@@ -121,7 +121,7 @@ def test_exact_set_pipeline_step_by_step(mode):
     cnp = ctx.numpy()
     L = LayerState(d, host, DEV)
     scale = 1 / math.sqrt(128)
-    pipe = DecodePipeline(d, [L], ctx.to(DEV), scale, DEV, overlap_score=True, exact=mode, steps_cap=8)
+    pipe = DecodePipeline(d, [L], ctx.to(DEV), scale, DEV, exact=mode, steps_cap=8)
     pipe.build_summaries()
     kmin, kmax = O.block_summaries(keys, cnp)
     qs = W.QueryStream(w)
