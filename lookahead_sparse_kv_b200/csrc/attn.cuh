@@ -6,547 +6,737 @@
 // attended in one pass over the resident sparse working set; Figure 9: the
 // per-head slot table says which block each pool slot holds.
 //
-// Work split (stream-K): the T = B*Hkv*K pool slots, in (sequence, KV head,
-// slot) order, are cut into NS contiguous ranges, one per CTA (one CTA per
-// SM).  A CTA walks its range one (sequence, KV head) "unit" piece at a
-// time.  Per piece the producer warp lists the occupied slots (free slots and
-// blocks past the context skipped), TMA-loads the unit's query rows, and
-// streams the listed slots through a 4-stage ring in tiles of 4 slots (64
-// tokens): four 2 KiB boxes per slot (K and V, each as two 64-column halves,
-// 128-byte swizzle) so that a tile lands as K[64 tokens][128] and
-// V[64 tokens][128] in the layouts the tensor core reads.
+// Shapes.  A (sequence, KV head) "unit" has rows = Qn*G query rows (at most
+// 64) and K pool slots of 16 tokens.  Decode has few query rows and many
+// tokens, so the tokens are the MMA's M dimension:
+//   S^T [128 tokens x NR]   = K_tile [128 x 128] . Q^T        8 MMAs, both K-major
+//   O^T [128 dims x NR]    += V_tile^T . P^T [128 tokens x NR]
+//                             two MMAs per occupied slot (16 tokens), both
+//                             operands MN-major: V is read in place, P^T is
+//                             written one 128-B row per token as a bf16 head
+//                             and a bf16 remainder (~16 significant bits); with
+//                             32 rows head and remainder share the row (the
+//                             remainder's MMA starts 64 B in) and P^T is
+//                             double-buffered, with 64 they take a row each
+// NR = 32 or 64 is the row count padded to the MMA's N.  A tile is 8 pool
+// slots (128 tokens).  In TMEM, lane i of S^T is token i of the tile (a
+// softmax thread owns a token and reads its NR scores), lane i of O^T is
+// head-dimension channel i (an epilogue thread owns a channel and writes it
+// for every row), so only real rows are ever exponentiated and every TMEM
+// access is a plain 32x32b row per thread.
 //
-// Math per tile, with the unit's Qn*G query rows as the MMA M dimension
-// (padded to 64; M = 64 puts row r in TMEM lane 32*(r/16) + r%16):
-//   S[64 x 64]   = Q[64 x 128] . K^T          8 tcgen05.mma, K-major A and B
-//   softmax      4 warps, one per TMEM lane quadrant, each thread owning two
-//                query rows of 16 tokens (a quad of threads shares a row):
-//                running max (moved only when a tile exceeds it by 2^8, so
-//                the accumulator is rarely rescaled), exponentials, row sums
-//   P            written to shared memory as a bf16 head plus a bf16
-//                remainder (~16 significant bits), 128-byte swizzled
-//   O[64 x 128] += P_head . V + P_rest . V    V read MN-major, 4 x 2 MMAs
-// S is double-buffered in TMEM (S of tile i+1 runs while tile i's softmax
-// does), P double-buffered in shared memory; O stays in TMEM for the whole
-// piece.  One thread issues every MMA; mbarriers carry every hand-off, with
-// bounded waits.
+// Work split.  A unit's slots are cut into chunks of `ct` tiles (`cpu`
+// chunks per unit, `nc` in all).  Persistent CTAs (at most one per SM) take
+// chunks from an atomic counter in the workspace, so a CTA that runs slowly
+// (beside a gather on its SM, say) simply takes fewer.  A chunk that is a
+// whole unit is normalised and written directly; otherwise it writes a
+// normalised partial (output, log2-sum-exp) and takes a ticket, and the last
+// chunk of the unit to finish merges the unit's partials (still in L2) and
+// resets the ticket.  The last CTA to exit resets the chunk counter, so the
+// workspace is ready for the next call.
 //
-// A unit covered by one CTA is normalised and written directly.  A unit
-// split over CTAs: each writes a normalised partial (output, log2-sum-exp),
-// then takes a ticket with an atomic counter; the last CTA to arrive merges
-// all partials of the unit (they are in L2), writes the output and resets the
-// counter for the next call.  No CTA ever waits for another.
+// Roles (12 warps, mbarriers for every hand-off, every wait bounded):
+//   warp 11    lister: takes chunks (the next one is requested while the
+//              current one is listed), lists a chunk's tiles that hold a
+//              valid token (valid-token count of each slot) and loads the
+//              unit's query rows;
+//   warp 8     loader: streams the listed tiles' K and V through two 2-stage
+//              TMA rings (per tile and tensor two 16-KiB boxes of 8 slots x
+//              16 rows x 64 columns, 128-byte swizzle).
+//   warp 9     issues S^T (and holds the TMEM allocation).
+//   warp 10    issues O^T; a free slot's product is not issued.
+//   warps 0-3  softmax, one token per thread.  The running max of a row
+//              moves only when a tile exceeds it by more than 2^8 (found
+//              with one barrier-wide vote per tile); then the tile's row
+//              maxima are reduced across the four warps and O^T and the row
+//              sums are rescaled.  Value rows past the context in a partly
+//              filled slot are zeroed so stale bytes never meet a zero
+//              weight.
+//   warps 4-7  epilogue, one channel per thread, double-buffered against
+//              the next chunk (two O^T accumulators in TMEM).
 #pragma once
 
 #include "common.cuh"
 
 namespace oasis {
 
-constexpr int kAttnTileSlots = 4;                                 // slots per tile
-constexpr int kAttnStages = 4;                                    // K/V ring depth
-constexpr int kAttnRegion = 64 * 128;                             // 64 rows x 128 B = 8 KiB
-constexpr int kAttnStageBytes = 4 * kAttnRegion;                  // K lo, K hi, V lo, V hi
-constexpr int kAttnRows = 64;                                     // MMA M
-constexpr int kAttnMaxList = 1024;                                // slots of one unit (K <= 1024)
-constexpr int kAttnThreads = 192;                                 // producer, MMA, 4 softmax warps
-constexpr int kAttnTmemCols = 256;                                // S x 2 (64 columns each) + O (128)
+constexpr int kAttnTileSlots = 8;                                  // slots per tile
+constexpr int kAttnTileTokens = kAttnTileSlots * kBlockTokens;     // 128: the MMA's M
+constexpr int kAttnHalf = kAttnTileTokens * 128;                   // one 64-column half of a tile: 16 KiB
+constexpr int kAttnStageBytes = 2 * kAttnHalf;                     // K (or V) of one tile
+constexpr int kAttnQHalf = 64 * 128;                               // 64 query rows x 128 B
+constexpr int kAttnMaxChunkTiles = 16;
+constexpr int kAttnInfoInts = 8 + 4 * kAttnMaxChunkTiles;          // chunk header + 4 ints per tile
+constexpr int kAttnLoaderWarp = 8, kAttnSWarp = 9, kAttnOWarp = 10, kAttnListerWarp = 11;
+constexpr int kAttnThreads = 32 * 12;
+constexpr int kAttnTmemCols = 256;                                 // S^T x 2, O^T x 2 (64 columns each)
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int kAttnOffQ = kAttnStages * kAttnStageBytes;          // 2 buffers x (lo, hi)
-constexpr int kAttnOffP = kAttnOffQ + 4 * kAttnRegion;            // 2 buffers x (head, rest)
-constexpr int kAttnOffList = kAttnOffP + 4 * kAttnRegion;         // 2 x kAttnMaxList ints
-constexpr int kAttnOffBar = kAttnOffList + 2 * kAttnMaxList * 4;
-constexpr int kAttnNumBars = 26;
-constexpr int kAttnOffMisc = kAttnOffBar + kAttnNumBars * 8;
-constexpr int kAttnSmem = kAttnOffMisc + 64 + 1024;              // + alignment slack
+// shared memory, from the 1024-B aligned base
+constexpr int kAttnOffK = 0;                                       // K ring, 2 stages
+constexpr int kAttnOffV = kAttnOffK + 2 * kAttnStageBytes;         // V ring, 2 stages
+constexpr int kAttnOffQ = kAttnOffV + 2 * kAttnStageBytes;         // 2 buffers x 2 halves
+constexpr int kAttnOffP = kAttnOffQ + 4 * kAttnQHalf;              // P^T: two [128 tokens][128 B] regions
+constexpr int kAttnOffInfo = kAttnOffP + 2 * kAttnHalf;            // 2 chunk descriptions
+constexpr int kAttnOffBar = kAttnOffInfo + 2 * kAttnInfoInts * 4;
+constexpr int kAttnNumBars = 32;
+constexpr int kAttnOffMisc = kAttnOffBar + kAttnNumBars * 8;       // 8 ints
+constexpr int kAttnOffM = kAttnOffMisc + 32;                       // [2][64] running max (log2 units)
+constexpr int kAttnOffAlpha = kAttnOffM + 2 * 64 * 4;              // [64] rescale factors of a tile
+constexpr int kAttnOffWmax = kAttnOffAlpha + 64 * 4;               // [4][64] per-warp tile maxima
+constexpr int kAttnOffLw = kAttnOffWmax + 4 * 64 * 4;              // [2][4][64] per-warp row sums
+constexpr int kAttnOffFin = kAttnOffLw + 2 * 4 * 64 * 4;           // [2][64] 1/sum, [2][64] log2-sum-exp
+constexpr int kAttnMaxChunks = 8;                                  // chunks per unit (merge weights)
+constexpr int kAttnOffMw = kAttnOffFin + 4 * 64 * 4;               // [64][8] merge weights
+constexpr int kAttnSmem = kAttnOffMw + 64 * kAttnMaxChunks * 4 + 1024;   // + alignment slack
 
-// mbarrier indices
-constexpr int kBarFull = 0;     // [4]  tile landed (producer expect_tx)
-constexpr int kBarEmpty = 4;    // [4]  tile's K and V consumed (MMA commit)
-constexpr int kBarSFull = 8;    // [2]  S computed (MMA commit)
-constexpr int kBarSFree = 10;   // [2]  S read by the 4 softmax warps
-constexpr int kBarPFull = 12;   // [2]  P written by the 4 softmax warps
-constexpr int kBarPFree = 14;   // [2]  P consumed (MMA commit after PV)
-constexpr int kBarQFull = 16;   // [2]  unit's query rows landed
-constexpr int kBarQFree = 18;   // [2]  query rows no longer read (MMA commit)
-constexpr int kBarLFull = 20;   // [2]  piece's slot list written (producer)
-constexpr int kBarLFree = 22;   // [2]  slot list no longer read (MMA thread + softmax leader)
-constexpr int kBarODone = 24;   // the piece's last PV has completed
-constexpr int kBarFinal = 25;   // teardown: every MMA issued has completed
+// mbarriers ([2] = one per ring stage / buffer)
+constexpr int kBarKFull = 0;     // K tile landed (producer expect_tx)
+constexpr int kBarKEmpty = 2;    // K tile read by S^T (commit)
+constexpr int kBarVFull = 4;     // V tile landed
+constexpr int kBarVEmpty = 6;    // V tile read by O^T (commit)
+constexpr int kBarSFull = 8;     // S^T computed (commit)
+constexpr int kBarSFree = 10;    // S^T read by the 4 softmax warps
+constexpr int kBarPFull = 12;    // P^T written by the 4 softmax warps (per P^T buffer)
+constexpr int kBarPFree = 14;    // P^T read by O^T (commit)
+constexpr int kBarQFull = 16;    // chunk's query rows landed
+constexpr int kBarQFree = 18;    // query rows no longer read (commit after the chunk's last S^T)
+constexpr int kBarLFull = 20;    // chunk description written (producer)
+constexpr int kBarLFree = 22;    // description read by all 11 consumer warps
+constexpr int kBarODone = 24;    // chunk's last O^T product completed (commit)
+constexpr int kBarOFree = 26;    // O^T accumulator, running max and row sums read by the epilogue
+constexpr int kBarSMDone = 28;   // chunk's row sums written by the 4 softmax warps
+constexpr int kBarFinalS = 30;   // teardown: every S^T issued has completed
+constexpr int kBarFinalO = 31;   // teardown: every O^T issued has completed
+constexpr int kAttnLFreeCount = 11;
 
-// Streams whose ranges touch unit u: [first, last].  Slot s belongs to
-// stream floor(s * NS / T), so every stream in between touches u.
-__host__ __device__ __forceinline__ void attn_unit_streams(long long u, long long K, long long NS, long long T,
-                                                           long long* first, long long* last) {
-    *first = (u * K) * NS / T;
-    *last = ((u + 1) * K - 1) * NS / T;
+// named barriers (0 is __syncthreads)
+constexpr uint32_t kNbSoftmax = 1, kNbSoftmaxVote = 2, kNbEpi = 3, kNbEpiVote = 4;
+
+// Chunking of the attention work (host and device agree through these).
+struct AttnChunks {
+    int ct;    // tiles per chunk
+    int cpu;   // chunks per unit
+    int nc;    // chunks in all
+};
+
+// 2^x on the multi-function unit (approximate, |rel err| about 2^-22; -inf -> +0).
+__device__ __forceinline__ float attn_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-// Waits unless the CTA has given up; a wait that runs out flags the CTA and
-// the device error word.  Returns whether the awaited phase completed.
-__device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    if (*abort_flag) return false;
-    if (mbar_wait(bar, parity)) return true;
-    *abort_flag = 1;
-    raise_dev_error(OASIS_DEVERR_TIMEOUT);
-    return false;
+// Butterfly reduce-scatter over the warp: v[0..31] in every lane; on return
+// lane t holds the max (or the sum) over all lanes of v[t].  v is clobbered.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool up = (lane & w) != 0;
+#pragma unroll
+        for (int k = 0; k < w; ++k) {
+            const float send = up ? v[k] : v[k + w];
+            const float keep = up ? v[k + w] : v[k];
+            const float got = __shfl_xor_sync(0xFFFFFFFFu, send, w);
+            v[k] = kMax ? fmaxf(keep, got) : keep + got;
+        }
+    }
+    return v[0];
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_pool, const __grid_constant__ CUtensorMap tm_q, Dims d,
-                       const int32_t* __restrict__ slot_table, const int32_t* __restrict__ ctx_len, float scale_log2,
-                       int n_streams, float* __restrict__ out, float* __restrict__ lse_out, float* ws_o,
-                       float* ws_lse, int* ws_ticket) {
+template <int NR>
+// 152 registers a thread: 384 x 152 leaves room for a gather CTA (128 x 48) on
+// the same SM.
+__global__ void __maxnreg__(152)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_q, Dims d, const int32_t* __restrict__ slot_table,
+                       const int32_t* __restrict__ ctx_len, float scale_log2, AttnChunks ch,
+                       float* __restrict__ out, float* __restrict__ lse_out, float* ws_o, float* ws_lse,
+                       int* ws_ticket, int* ws_sched) {
+    static_assert(NR == 32 || NR == 64, "rows are padded to 32 or 64");
+    // P^T buffers: with 32 rows one 128-B row per token holds the head (bytes
+    // 0-63 of the row before swizzling) and the remainder (64-127), two
+    // buffers; with 64 rows head and remainder fill one region each, one buffer.
+    constexpr int kPBufs = NR == 32 ? 2 : 1;
+    constexpr uint32_t kRestOff = NR == 32 ? 64u : static_cast<uint32_t>(kAttnHalf);
     const float kNegInf = -__int_as_float(0x7f800000);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* ring = smem;
+    uint8_t* sK = smem + kAttnOffK;
+    uint8_t* sV = smem + kAttnOffV;
     uint8_t* sQ = smem + kAttnOffQ;
     uint8_t* sP = smem + kAttnOffP;
-    int* s_list = reinterpret_cast<int*>(smem + kAttnOffList);
+    int* s_info = reinterpret_cast<int*>(smem + kAttnOffInfo);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kAttnOffBar);
     int* misc = reinterpret_cast<int*>(smem + kAttnOffMisc);
-    int* s_nlist = misc;                                  // [2]
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc + 2);
-    volatile int* s_abort = misc + 3;
-    volatile int* s_last = misc + 4;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc);
+    volatile int* s_abort = misc + 1;
+    volatile int* s_last = misc + 2;
+    float* s_m = reinterpret_cast<float*>(smem + kAttnOffM);
+    float* s_alpha = reinterpret_cast<float*>(smem + kAttnOffAlpha);
+    float* s_wmax = reinterpret_cast<float*>(smem + kAttnOffWmax);
+    float* s_lw = reinterpret_cast<float*>(smem + kAttnOffLw);
+    float* s_fin = reinterpret_cast<float*>(smem + kAttnOffFin);
+    float* s_mw = reinterpret_cast<float*>(smem + kAttnOffMw);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long K = d.K;
-    const long long T = static_cast<long long>(d.B) * d.Hkv * K;
-    const long long gs = blockIdx.x;
-    const long long s_begin = (gs * T + n_streams - 1) / n_streams;
-    const long long s_end = ((gs + 1) * T + n_streams - 1) / n_streams;
-    if (s_begin >= s_end) return;                         // whole CTA: empty range
-    const long long u_first = s_begin / K, u_last = (s_end - 1) / K;
+    const int K = d.K;
     const int G = d.G();
     const int rows = d.Qn * G;
 
     // ---------------------------------------------------------- set-up
     if (tid == 0) {
-        const int counts[kAttnNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 4, 4, 4, 1, 1,
-                                          1, 1, 1, 1, 1, 1, 2, 2, 1, 1};
-        for (int i = 0; i < kAttnNumBars; ++i) mbar_init(&bar[i], counts[i]);
+        for (int i = 0; i < kAttnNumBars; ++i) {
+            int cnt = 1;
+            if (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1 || i == kBarSMDone ||
+                i == kBarSMDone + 1)
+                cnt = 4;
+            if (i == kBarLFree || i == kBarLFree + 1) cnt = kAttnLFreeCount;
+            mbar_init(&bar[i], cnt);
+        }
         fence_mbar_init();
         *s_abort = 0;
         *s_last = 0;
     }
-    if (warp == 1) {
+    if (warp == kAttnSWarp) {
         tmem_alloc(s_tmem, kAttnTmemCols);
         tmem_relinquish();
     }
-    // zero Q and P: rows past the real query rows stay zero for the whole call
-    for (int i = tid; i < 8 * kAttnRegion / 16; i += kAttnThreads)
-        reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tmem_o = tmem + 128;
 
-    if (warp == 0) {
-        // ===================================================== producer
-        if (lane == 0) {
-            prefetch_tensormap(&tm_pool);
-            prefetch_tensormap(&tm_q);
-        }
-        const uint64_t pol_kv = l2_policy_evict_first();
+    if (warp == kAttnListerWarp) {
+        // ======================================================= lister
+        if (lane == 0) prefetch_tensormap(&tm_q);
         const uint64_t pol_q = l2_policy_evict_last();
-        long long pos = 0;
-        long long last_pos[kAttnStages] = {-1, -1, -1, -1};
-        int p = 0;
-        for (long long u = u_first; u <= u_last; ++u, ++p) {
+        int c_next = 0;
+        if (lane == 0) c_next = atomicAdd(ws_sched, 1);
+        for (int p = 0;; ++p) {
             const int pb = p & 1;
-            const long long lo = max(s_begin, u * K), hi = min(s_end, (u + 1) * K);
-            const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
-            if (lane == 0 && p >= 2) attn_wait(&bar[kBarLFree + pb], ((p >> 1) - 1) & 1, s_abort);
-            __syncwarp();
-            // the occupied slots of the piece, in slot order: (slot in unit) << 5 | valid tokens
-            int* list = s_list + pb * kAttnMaxList;
-            const int ctx = ctx_len[b];
-            int n = 0;
-            for (long long base = lo; base < hi; base += 32) {
-                const long long s = base + lane;
-                int nv = 0;
-                if (s < hi) {
-                    int blk = slot_table[s];
-                    if (blk < -1 || blk >= d.N) {
-                        raise_dev_error(OASIS_DEVERR_ID_RANGE);
-                        blk = -1;
-                    }
-                    if (blk >= 0) nv = min(kBlockTokens, max(0, ctx - blk * kBlockTokens));
+            int* info = s_info + pb * kAttnInfoInts;
+            if (lane == 0 && p >= 2) cta_wait(&bar[kBarLFree + pb], ((p >> 1) - 1) & 1, s_abort);
+            int c = c_next;
+            if (lane == 0 && *s_abort) c = ch.nc;
+            c = __shfl_sync(0xFFFFFFFFu, c, 0);
+            if (c >= ch.nc) {
+                if (lane == 0) {
+                    info[0] = -1;
+                    mbar_arrive(&bar[kBarLFull + pb]);
                 }
-                const unsigned m = __ballot_sync(0xFFFFFFFFu, nv > 0);
-                if (nv > 0) list[n + __popc(m & ((1u << lane) - 1u))] = (static_cast<int>(s - u * K) << 5) | nv;
-                n += __popc(m);
+                break;
+            }
+            if (lane == 0) c_next = atomicAdd(ws_sched, 1);    // lands while this chunk is listed
+            const int u = c / ch.cpu, j = c - u * ch.cpu;
+            const int lo = j * ch.ct * kAttnTileSlots, hi = min(lo + ch.ct * kAttnTileSlots, K);
+            const int b = u / d.Hkv, h = u - b * d.Hkv;
+            const int ctx = ctx_len[b];
+            const int ntiles = (hi - lo + kAttnTileSlots - 1) / kAttnTileSlots;   // <= 16
+            // lane i lists tile i: valid-token count of each of its 8 slots, a byte each
+            uint32_t nvlo = 0u, nvhi = 0u;
+            bool any = false;
+            if (lane < ntiles) {
+                const int s0 = lo + kAttnTileSlots * lane;
+                int blk[kAttnTileSlots];
+#pragma unroll
+                for (int jj = 0; jj < kAttnTileSlots; ++jj)
+                    blk[jj] = s0 + jj < hi ? slot_table[static_cast<long long>(u) * K + s0 + jj] : -1;
+#pragma unroll
+                for (int jj = 0; jj < kAttnTileSlots; ++jj) {
+                    int bk = blk[jj];
+                    if (bk < -1 || bk >= d.N) {
+                        raise_dev_error(OASIS_DEVERR_ID_RANGE);
+                        bk = -1;
+                    }
+                    const int nv = bk >= 0 ? min(kBlockTokens, max(0, ctx - bk * kBlockTokens)) : 0;
+                    if (jj < 4)
+                        nvlo |= static_cast<uint32_t>(nv) << (8 * jj);
+                    else
+                        nvhi |= static_cast<uint32_t>(nv) << (8 * (jj - 4));
+                    any |= nv > 0;
+                }
+            }
+            const unsigned m = __ballot_sync(0xFFFFFFFFu, any);
+            const int n = __popc(m);
+            if (any) {
+                int* e = info + 8 + 4 * __popc(m & ((1u << lane) - 1u));
+                e[0] = lo + kAttnTileSlots * lane;
+                e[1] = static_cast<int>(nvlo);
+                e[2] = static_cast<int>(nvhi);
             }
             __syncwarp();
             if (lane == 0) {
-                s_nlist[pb] = n;
-                __threadfence_block();
+                info[0] = n;
+                info[1] = c;
+                info[2] = u;
+                info[3] = ch.cpu;
                 mbar_arrive(&bar[kBarLFull + pb]);
                 // the unit's query rows: box {64 columns, G heads, Qn rows} per 64-column half
-                if (p >= 2) attn_wait(&bar[kBarQFree + pb], ((p >> 1) - 1) & 1, s_abort);
+                if (p >= 2) cta_wait(&bar[kBarQFree + pb], ((p >> 1) - 1) & 1, s_abort);
                 mbar_arrive_expect_tx(&bar[kBarQFull + pb], static_cast<uint32_t>(rows) * kRowBytes);
                 if (!*s_abort) {
-                    uint8_t* q_dst = sQ + pb * 2 * kAttnRegion;
+                    uint8_t* q_dst = sQ + pb * 2 * kAttnQHalf;
                     tma_load_3d(q_dst, &tm_q, &bar[kBarQFull + pb], 0, h * G, b * d.Qn, pol_q);
-                    tma_load_3d(q_dst + kAttnRegion, &tm_q, &bar[kBarQFull + pb], 64, h * G, b * d.Qn, pol_q);
-                }
-                const int ntiles = (n + kAttnTileSlots - 1) / kAttnTileSlots;
-                for (int i = 0; i < ntiles; ++i, ++pos) {
-                    const int stage = static_cast<int>(pos % kAttnStages);
-                    if (pos >= kAttnStages)
-                        attn_wait(&bar[kBarEmpty + stage], static_cast<uint32_t>((pos / kAttnStages - 1) & 1),
-                                  s_abort);
-                    const int ns = min(kAttnTileSlots, n - i * kAttnTileSlots);
-                    mbar_arrive_expect_tx(&bar[kBarFull + stage], static_cast<uint32_t>(ns) * kBlockBytes);
-                    last_pos[stage] = pos;
-                    if (*s_abort) continue;
-                    uint8_t* st = ring + stage * kAttnStageBytes;
-                    for (int j = 0; j < ns; ++j) {
-                        const int slot = list[i * kAttnTileSlots + j] >> 5;
-                        const int y = static_cast<int>((u * K + slot) * (2 * kBlockTokens));
-                        const int off = j * (kBlockTokens * 128);
-                        tma_load_2d(st + 0 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 0, y, pol_kv);
-                        tma_load_2d(st + 1 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 64, y, pol_kv);
-                        tma_load_2d(st + 2 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 0,
-                                    y + kBlockTokens, pol_kv);
-                        tma_load_2d(st + 3 * kAttnRegion + off, &tm_pool, &bar[kBarFull + stage], 64,
-                                    y + kBlockTokens, pol_kv);
-                    }
+                    tma_load_3d(q_dst + kAttnQHalf, &tm_q, &bar[kBarQFull + pb], 64, h * G, b * d.Qn, pol_q);
                 }
             }
             __syncwarp();
-            n = __shfl_sync(0xFFFFFFFFu, n, 0);
-            pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
         }
-        // no copy may still be writing this CTA's shared memory when it exits
-        if (lane == 0)
-            for (int s = 0; s < kAttnStages; ++s)
-                if (last_pos[s] >= 0) mbar_wait(&bar[kBarFull + s], static_cast<uint32_t>((last_pos[s] / kAttnStages) & 1));
-    } else if (warp == 1) {
-        // =================================================== MMA issuer
+    } else if (warp == kAttnLoaderWarp) {
+        // ======================================================= loader
         if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16_f32(kAttnRows, kAttnTileSlots * kBlockTokens);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16_f32_bmn(kAttnRows, kHeadDim);
-            long long pos = 0;
-            int p = 0;
-            bool have_prev = false, prev_first = false, prev_last = false;
-            long long prev_pos = 0;
-            int prev_ns = 0;
-            auto issue_pv = [&](long long ppos, int pns, bool pfirst, bool plast) {
-                const int sb = static_cast<int>(ppos & 1);
-                const int stage = static_cast<int>(ppos % kAttnStages);
-                const bool ok = attn_wait(&bar[kBarPFull + sb], static_cast<uint32_t>((ppos >> 1) & 1), s_abort);
-                tc_fence_after_sync();
-                if (ok) {
-                    const uint32_t pa = smem_addr(sP + sb * 2 * kAttnRegion);
-                    const uint32_t va = smem_addr(ring + stage * kAttnStageBytes + 2 * kAttnRegion);
-                    for (int kk = 0; kk < pns; ++kk) {
-                        const uint64_t bd = umma_desc_sw128_lbo_sbo(va + kk * (kBlockTokens * 128), kAttnRegion, 1024);
-                        umma_bf16(tmem_o, umma_desc_sw128_lbo_sbo(pa + kk * 32, 16, 1024), bd, idesc_pv,
-                                  (pfirst && kk == 0) ? 0u : 1u);
-                        umma_bf16(tmem_o, umma_desc_sw128_lbo_sbo(pa + kAttnRegion + kk * 32, 16, 1024), bd,
-                                  idesc_pv, 1u);
-                    }
-                }
-                umma_commit(&bar[kBarEmpty + stage]);
-                umma_commit(&bar[kBarPFree + sb]);
-                if (plast) umma_commit(&bar[kBarODone]);
-            };
-            for (long long u = u_first; u <= u_last; ++u, ++p) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            const uint64_t pol_kv = l2_policy_evict_first();
+            int pos = 0;
+            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+            for (int p = 0;; ++p) {
                 const int pb = p & 1;
-                attn_wait(&bar[kBarLFull + pb], static_cast<uint32_t>((p >> 1) & 1), s_abort);
-                const int n = s_nlist[pb];
-                const int ntiles = (n + kAttnTileSlots - 1) / kAttnTileSlots;
-                attn_wait(&bar[kBarQFull + pb], static_cast<uint32_t>((p >> 1) & 1), s_abort);
-                const uint32_t qa = smem_addr(sQ + pb * 2 * kAttnRegion);
-                for (int i = 0; i < ntiles; ++i, ++pos) {
-                    const int stage = static_cast<int>(pos % kAttnStages);
-                    const int sb = static_cast<int>(pos & 1);
-                    bool ok = attn_wait(&bar[kBarFull + stage], static_cast<uint32_t>((pos / kAttnStages) & 1),
-                                        s_abort);
-                    if (pos >= 2) ok = attn_wait(&bar[kBarSFree + sb], static_cast<uint32_t>(((pos >> 1) - 1) & 1),
-                                                 s_abort) && ok;
-                    tc_fence_after_sync();
-                    if (ok) {
-                        const uint32_t ka = smem_addr(ring + stage * kAttnStageBytes);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t off = (ks >> 2) * kAttnRegion + (ks & 3) * 32;
-                            umma_bf16(tmem + sb * 64, umma_desc_sw128_lbo_sbo(qa + off, 16, 1024),
-                                      umma_desc_sw128_lbo_sbo(ka + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
-                        }
+                if (!cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort)) break;
+                const int* info = s_info + pb * kAttnInfoInts;
+                const int n = info[0];
+                if (n < 0) break;
+                const int zu = info[2] * K;
+                for (int i = 0; i < n; ++i, ++pos) {
+                    const int st = pos & 1;
+                    const int z = zu + info[8 + 4 * i];              // first pool slot of the tile
+                    if (pos >= 2) cta_wait(&bar[kBarKEmpty + st], ((pos >> 1) - 1) & 1, s_abort);
+                    mbar_arrive_expect_tx(&bar[kBarKFull + st], kAttnStageBytes);
+                    if (!*s_abort) {
+                        last_k[st] = pos;
+                        uint8_t* dk = sK + st * kAttnStageBytes;
+                        tma_load_3d(dk, &tm_k, &bar[kBarKFull + st], 0, 0, z, pol_kv);
+                        tma_load_3d(dk + kAttnHalf, &tm_k, &bar[kBarKFull + st], 64, 0, z, pol_kv);
                     }
-                    umma_commit(&bar[kBarSFull + sb]);
-                    if (have_prev) issue_pv(prev_pos, prev_ns, prev_first, prev_last);
-                    have_prev = true;
-                    prev_pos = pos;
-                    prev_ns = min(kAttnTileSlots, n - i * kAttnTileSlots);
-                    prev_first = i == 0;
-                    prev_last = i == ntiles - 1;
+                    if (pos >= 2) cta_wait(&bar[kBarVEmpty + st], ((pos >> 1) - 1) & 1, s_abort);
+                    mbar_arrive_expect_tx(&bar[kBarVFull + st], kAttnStageBytes);
+                    if (!*s_abort) {
+                        last_v[st] = pos;
+                        uint8_t* dv = sV + st * kAttnStageBytes;
+                        tma_load_3d(dv, &tm_v, &bar[kBarVFull + st], 0, 0, z, pol_kv);
+                        tma_load_3d(dv + kAttnHalf, &tm_v, &bar[kBarVFull + st], 64, 0, z, pol_kv);
+                    }
                 }
-                umma_commit(&bar[kBarQFree + pb]);            // after the piece's last S
                 mbar_arrive(&bar[kBarLFree + pb]);
             }
-            if (have_prev) issue_pv(prev_pos, prev_ns, prev_first, prev_last);
-            umma_commit(&bar[kBarFinal]);
-            mbar_wait(&bar[kBarFinal], 0);
+            // no copy may still be writing this CTA's shared memory when it exits
+            for (int st = 0; st < 2; ++st) {
+                if (last_k[st] >= 0) mbar_wait(&bar[kBarKFull + st], static_cast<uint32_t>((last_k[st] >> 1) & 1));
+                if (last_v[st] >= 0) mbar_wait(&bar[kBarVFull + st], static_cast<uint32_t>((last_v[st] >> 1) & 1));
+            }
         }
         __syncwarp();
-    } else {
-        // ============================================ softmax / epilogue
-        const int qd = warp & 3;                              // TMEM lane quadrant
-        const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-        const int rA = 16 * qd + (lane >> 2), rB = rA + 8;   // this thread's query rows
-        const bool realA = rA < rows, realB = rB < rows;
-        const int cp = 2 * (lane & 3);                        // column pair within each 8-column chunk
-        long long pos = 0;
-        int nonempty = 0;
-        int p = 0;
-        for (long long u = u_first; u <= u_last; ++u, ++p) {
-            const int pb = p & 1;
-            attn_wait(&bar[kBarLFull + pb], static_cast<uint32_t>((p >> 1) & 1), s_abort);
-            const int n = s_nlist[pb];
-            const int* list = s_list + pb * kAttnMaxList;
-            const int ntiles = (n + kAttnTileSlots - 1) / kAttnTileSlots;
-            float mA = kNegInf, mB = kNegInf, lA = 0.f, lB = 0.f;
-            for (int i = 0; i < ntiles; ++i, ++pos) {
-                const int sb = static_cast<int>(pos & 1);
-                const int stage = static_cast<int>(pos % kAttnStages);
-                const int ns = min(kAttnTileSlots, n - i * kAttnTileSlots);
-                int nvj[kAttnTileSlots];
-#pragma unroll
-                for (int j = 0; j < kAttnTileSlots; ++j) nvj[j] = j < ns ? (list[i * kAttnTileSlots + j] & 31) : 0;
-                attn_wait(&bar[kBarSFull + sb], static_cast<uint32_t>((pos >> 1) & 1), s_abort);
-                tc_fence_after_sync();
-                uint32_t v[32];
-                tmem_ld_16x256b_x8(tmem + lane_base + sb * 64, v);
-                tmem_ld_wait();
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kBarSFree + sb]);
-                float s[32];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int j = c >> 1;                      // slot of this chunk
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int tt = (c & 1) * 8 + cp + e;   // token within the slot
-                        const bool ok = tt < nvj[j];
-                        s[4 * c + e] = ok ? __uint_as_float(v[4 * c + e]) : kNegInf;
-                        s[4 * c + 2 + e] = ok ? __uint_as_float(v[4 * c + 2 + e]) : kNegInf;
-                    }
-                }
-                float mxA = kNegInf, mxB = kNegInf;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    mxA = fmaxf(mxA, fmaxf(s[4 * c], s[4 * c + 1]));
-                    mxB = fmaxf(mxB, fmaxf(s[4 * c + 2], s[4 * c + 3]));
-                }
-                mxA = fmaxf(mxA, __shfl_xor_sync(0xFFFFFFFFu, mxA, 1));
-                mxA = fmaxf(mxA, __shfl_xor_sync(0xFFFFFFFFu, mxA, 2));
-                mxB = fmaxf(mxB, __shfl_xor_sync(0xFFFFFFFFu, mxB, 1));
-                mxB = fmaxf(mxB, __shfl_xor_sync(0xFFFFFFFFu, mxB, 2));
-                mxA *= scale_log2;
-                mxB *= scale_log2;
-                // P buffer sb is free once PV of tile pos-2 has completed
-                if (pos >= 2) attn_wait(&bar[kBarPFree + sb], static_cast<uint32_t>(((pos >> 1) - 1) & 1), s_abort);
-                // running max: moved only by more than 2^8 (exact lse for any reference)
-                float alA = 1.f, alB = 1.f;
-                bool resc = false;
-                if (mxA > mA + 8.f) {
-                    if (i > 0) {
-                        alA = exp2f(mA - mxA);
-                        resc = true;
-                    }
-                    mA = mxA;
-                }
-                if (mxB > mB + 8.f) {
-                    if (i > 0) {
-                        alB = exp2f(mB - mxB);
-                        resc = true;
-                    }
-                    mB = mxB;
-                }
-                lA *= alA;
-                lB *= alB;
-                if (__any_sync(0xFFFFFFFFu, resc)) {
-                    // PV of tile pos-1 must have landed in O before it is rescaled
-                    attn_wait(&bar[kBarPFree + (sb ^ 1)], static_cast<uint32_t>(((pos - 1) >> 1) & 1), s_abort);
+    } else if (warp == kAttnSWarp) {
+        // =========================================== S^T = K . Q^T issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16_f32(kAttnTileTokens, NR);
+            int sp = 0;
+            for (int p = 0;; ++p) {
+                const int pb = p & 1;
+                if (!cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort)) break;
+                const int n = s_info[pb * kAttnInfoInts];
+                if (n < 0) break;
+                cta_wait(&bar[kBarQFull + pb], (p >> 1) & 1, s_abort);
+                const uint32_t qa = smem_addr(sQ + pb * 2 * kAttnQHalf);
+                for (int i = 0; i < n; ++i, ++sp) {
+                    const int st = sp & 1;
+                    bool ok = cta_wait(&bar[kBarKFull + st], (sp >> 1) & 1, s_abort);
+                    if (sp >= 2) ok = cta_wait(&bar[kBarSFree + st], ((sp >> 1) - 1) & 1, s_abort) && ok;
                     tc_fence_after_sync();
+                    if (ok) {
+                        const uint32_t ka = smem_addr(sK + st * kAttnStageBytes);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t o[32];
-                        tmem_ld_16x256b_x8(tmem_o + lane_base + half * 64, o);
+                        for (int ks = 0; ks < 8; ++ks)
+                            umma_bf16(tmem + st * 64,
+                                      umma_desc_sw128_lbo_sbo(ka + (ks >> 2) * kAttnHalf + (ks & 3) * 32, 16, 1024),
+                                      umma_desc_sw128_lbo_sbo(qa + (ks >> 2) * kAttnQHalf + (ks & 3) * 32, 16, 1024),
+                                      idesc, ks > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&bar[kBarKEmpty + st]);
+                    umma_commit(&bar[kBarSFull + st]);
+                }
+                umma_commit(&bar[kBarQFree + pb]);                // after the chunk's last S^T
+                mbar_arrive(&bar[kBarLFree + pb]);
+            }
+            umma_commit(&bar[kBarFinalS]);
+            mbar_wait(&bar[kBarFinalS], 0);
+        }
+        __syncwarp();
+    } else if (warp == kAttnOWarp) {
+        // ======================================== O^T += V^T . P^T issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16_f32_amn_bmn(kHeadDim, NR);
+            int pv = 0;
+            for (int p = 0;; ++p) {
+                const int pb = p & 1;
+                if (!cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort)) break;
+                const int* info = s_info + pb * kAttnInfoInts;
+                const int n = info[0];
+                if (n < 0) break;
+                if (p >= 2) cta_wait(&bar[kBarOFree + pb], ((p >> 1) - 1) & 1, s_abort);
+                const uint32_t d_o = tmem + 128 + pb * 64;
+                bool fresh = true;                                // the chunk's first product overwrites O^T
+                for (int i = 0; i < n; ++i, ++pv) {
+                    const int st = pv & 1;
+                    const int pbuf = pv % kPBufs;
+                    bool ok = cta_wait(&bar[kBarPFull + pbuf], (pv / kPBufs) & 1, s_abort);
+                    ok = cta_wait(&bar[kBarVFull + st], (pv >> 1) & 1, s_abort) && ok;
+                    tc_fence_after_sync();
+                    if (ok) {
+                        const uint32_t nvlo = static_cast<uint32_t>(info[8 + 4 * i + 1]);
+                        const uint32_t nvhi = static_cast<uint32_t>(info[8 + 4 * i + 2]);
+                        const uint32_t va = smem_addr(sV + st * kAttnStageBytes);
+                        const uint32_t pa = smem_addr(sP + pbuf * kAttnHalf);
+#pragma unroll
+                        for (int kk = 0; kk < kAttnTileSlots; ++kk) {
+                            const uint32_t nv = ((kk < 4 ? nvlo : nvhi) >> (8 * (kk & 3))) & 0xFFu;
+                            if (nv == 0) continue;                // free slot: no product
+                            const uint32_t off = kk * kBlockTokens * 128;
+                            const uint64_t ad = umma_desc_sw128_lbo_sbo(va + off, kAttnHalf, 1024);
+                            umma_bf16(d_o, ad, umma_desc_sw128_lbo_sbo(pa + off, kAttnHalf, 1024), idesc,
+                                      fresh ? 0u : 1u);
+                            umma_bf16(d_o, ad, umma_desc_sw128_lbo_sbo(pa + kRestOff + off, kAttnHalf, 1024), idesc,
+                                      1u);
+                            fresh = false;
+                        }
+                    }
+                    umma_commit(&bar[kBarVEmpty + st]);
+                    umma_commit(&bar[kBarPFree + pbuf]);
+                }
+                umma_commit(&bar[kBarODone + pb]);
+                mbar_arrive(&bar[kBarLFree + pb]);
+            }
+            umma_commit(&bar[kBarFinalO]);
+            mbar_wait(&bar[kBarFinalO], 0);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ============================================ softmax (token / thread)
+        const int q = warp;                                   // TMEM lane quadrant
+        const int tok = 32 * q + lane;                        // token of the tile this thread owns
+        const int myslot = tok >> 4, mytok = tok & 15;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        int pos = 0;
+        for (int p = 0;; ++p) {
+            const int pb = p & 1;
+            cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort);
+            const int* info = s_info + pb * kAttnInfoInts;
+            const int n = info[0];
+            if (named_bar_or(kNbSoftmaxVote, 128, n < 0 || *s_abort)) break;
+            // the epilogue of chunk p-2 has read this buffer's running max and sums
+            if (p >= 2) cta_wait(&bar[kBarOFree + pb], ((p >> 1) - 1) & 1, s_abort);
+            float* mr = s_m + pb * 64;
+            if (q == 0) {                                     // rows past the real ones stay at 0
+                mr[lane] = lane < rows ? kNegInf : 0.f;
+                mr[lane + 32] = lane + 32 < rows ? kNegInf : 0.f;
+            }
+            named_bar_sync(kNbSoftmax, 128);
+            // row sums: with 32 rows each thread keeps its token's sums (reduced over the
+            // warp at the chunk's end); with 64, to save registers, every tile's sums are
+            // reduced over the warp at once and lane t keeps rows t and t + 32
+            constexpr int kL = NR == 32 ? 32 : 1;
+            float l[kL];
+#pragma unroll
+            for (int r = 0; r < kL; ++r) l[r] = 0.f;
+            float lsc0 = 0.f, lsc1 = 0.f;
+            for (int i = 0; i < n; ++i, ++pos) {
+                const int st = pos & 1;
+                const int* e = info + 8 + 4 * i;
+                const int nvj = (static_cast<uint32_t>(myslot < 4 ? e[1] : e[2]) >> (8 * (myslot & 3))) & 0xFF;
+                const bool valid = mytok < nvj;
+                cta_wait(&bar[kBarSFull + st], (pos >> 1) & 1, s_abort);
+                tc_fence_after_sync();
+                float x[NR];
+                {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + st * 64, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int r = 0; r < 32; ++r)
+                        x[r] = (valid && r < rows) ? __uint_as_float(v[r]) * scale_log2 : kNegInf;
+                    if constexpr (NR == 64) {
+                        tmem_ld_32x32b_x32(tmem + lane_base + st * 64 + 32, v);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            o[4 * c + 0] = __float_as_uint(__uint_as_float(o[4 * c + 0]) * alA);
-                            o[4 * c + 1] = __float_as_uint(__uint_as_float(o[4 * c + 1]) * alA);
-                            o[4 * c + 2] = __float_as_uint(__uint_as_float(o[4 * c + 2]) * alB);
-                            o[4 * c + 3] = __float_as_uint(__uint_as_float(o[4 * c + 3]) * alB);
-                        }
-                        tmem_st_16x256b_x8(tmem_o + lane_base + half * 64, o);
+                        for (int r = 0; r < 32; ++r)
+                            x[32 + r] = (valid && 32 + r < rows) ? __uint_as_float(v[r]) * scale_log2 : kNegInf;
                     }
-                    tmem_st_wait();
                 }
-                // probabilities: head + remainder in bf16, written 128-byte swizzled
-                uint8_t* p_head = sP + sb * 2 * kAttnRegion;
-                uint8_t* p_rest = p_head + kAttnRegion;
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kBarSFree + st]);
+                // does any row's running max move (by more than 2^8)?
+                bool up = false;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float a0 = exp2f(fmaf(s[4 * c + 0], scale_log2, -mA));
-                    const float a1 = exp2f(fmaf(s[4 * c + 1], scale_log2, -mA));
-                    const float b0 = exp2f(fmaf(s[4 * c + 2], scale_log2, -mB));
-                    const float b1 = exp2f(fmaf(s[4 * c + 3], scale_log2, -mB));
-                    lA += a0 + a1;
-                    lB += b0 + b1;
-                    if (realA) {
-                        const uint32_t hd = pack_bf16x2(a0, a1);
-                        const uint32_t rs = pack_bf16x2(a0 - bf16_lo(hd), a1 - bf16_hi(hd));
-                        const int off = rA * 128 + ((c ^ (rA & 7)) << 4) + cp * 2;
-                        *reinterpret_cast<uint32_t*>(p_head + off) = hd;
-                        *reinterpret_cast<uint32_t*>(p_rest + off) = rs;
+                for (int r = 0; r < NR; r += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4*>(mr + r);
+                    up |= (x[r] > m4.x + 8.f) | (x[r + 1] > m4.y + 8.f) | (x[r + 2] > m4.z + 8.f) |
+                          (x[r + 3] > m4.w + 8.f);
+                }
+                if (named_bar_or(kNbSoftmaxVote, 128, up)) {
+                    // tile maxima: lane t of each warp gets rows t and t + 32 over its tokens
+#pragma unroll
+                    for (int hh = 0; hh < NR / 32; ++hh) {
+                        float t[32];
+#pragma unroll
+                        for (int r = 0; r < 32; ++r) t[r] = x[32 * hh + r];
+                        s_wmax[q * 64 + 32 * hh + lane] = warp_reduce_scatter32<true>(t, lane);
                     }
-                    if (realB) {
-                        const uint32_t hd = pack_bf16x2(b0, b1);
-                        const uint32_t rs = pack_bf16x2(b0 - bf16_lo(hd), b1 - bf16_hi(hd));
-                        const int off = rB * 128 + ((c ^ (rB & 7)) << 4) + cp * 2;
-                        *reinterpret_cast<uint32_t*>(p_head + off) = hd;
-                        *reinterpret_cast<uint32_t*>(p_rest + off) = rs;
+                    named_bar_sync(kNbSoftmax, 128);
+                    if (q == 0) {
+#pragma unroll
+                        for (int hh = 0; hh < NR / 32; ++hh) {
+                            const int r = 32 * hh + lane;
+                            const float tmx = fmaxf(fmaxf(s_wmax[r], s_wmax[64 + r]), fmaxf(s_wmax[128 + r], s_wmax[192 + r]));
+                            const float mo = mr[r];
+                            float a = 1.f;
+                            if (tmx > mo + 8.f) {
+                                a = attn_exp2(mo - tmx);              // 0 on the chunk's first tile
+                                mr[r] = tmx;
+                            }
+                            s_alpha[r] = a;
+                        }
+                    }
+                    named_bar_sync(kNbSoftmax, 128);
+                    if constexpr (NR == 32) {
+#pragma unroll
+                        for (int r = 0; r < 32; ++r) l[r] *= s_alpha[r];
+                    } else {
+                        lsc0 *= s_alpha[lane];
+                        lsc1 *= s_alpha[32 + lane];
+                    }
+                    if (i > 0) {
+                        // the previous tile's product must have landed in O^T before it is rescaled
+                        cta_wait(&bar[kBarPFree + (pos - 1) % kPBufs], ((pos - 1) / kPBufs) & 1, s_abort);
+                        tc_fence_after_sync();
+#pragma unroll
+                        for (int hh = 0; hh < NR / 32; ++hh) {
+                            const uint32_t oaddr = tmem + lane_base + 128 + pb * 64 + 32 * hh;
+                            uint32_t o[32];
+                            tmem_ld_32x32b_x32(oaddr, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int r = 0; r < 32; ++r)
+                                o[r] = __float_as_uint(__uint_as_float(o[r]) * s_alpha[32 * hh + r]);
+                            tmem_st_32x32b_x32(oaddr, o);
+                        }
+                        tmem_st_wait();
                     }
                 }
-                // value rows past the context of a partly filled block read as zero
-                // (their weights are zero, and zero times a non-finite stale value is not)
-                if (qd < ns && nvj[qd] < kBlockTokens) {
-                    // the tile's copy is complete (already awaited by the MMA thread; this
-                    // wait returns at once and orders the copy before these writes)
-                    attn_wait(&bar[kBarFull + stage], static_cast<uint32_t>((pos / kAttnStages) & 1), s_abort);
-                    uint8_t* vbase = ring + stage * kAttnStageBytes + 2 * kAttnRegion + qd * (kBlockTokens * 128);
-                    const int first_row = nvj[qd];
-                    for (int k = lane; k < (kBlockTokens - first_row) * 16; k += 32) {
-                        const int row = first_row + (k >> 4), chunk = k & 15;
-                        *reinterpret_cast<uint4*>(vbase + (chunk >> 3) * kAttnRegion + row * 128 + (chunk & 7) * 16) =
-                            make_uint4(0u, 0u, 0u, 0u);
+                // this token's probabilities for every row, head and remainder (bf16 each),
+                // once the product that last read this P^T buffer is done
+                const int pbuf = pos % kPBufs;
+                if (pos >= kPBufs) cta_wait(&bar[kBarPFree + pbuf], ((pos / kPBufs) - 1) & 1, s_abort);
+                uint8_t* prow = sP + pbuf * kAttnHalf + tok * 128;
+#pragma unroll
+                for (int c8 = 0; c8 < NR / 8; ++c8) {
+                    const float4 ma = *reinterpret_cast<const float4*>(mr + 8 * c8);
+                    const float4 mb = *reinterpret_cast<const float4*>(mr + 8 * c8 + 4);
+                    const int r = 8 * c8;
+                    const float p0 = attn_exp2(x[r + 0] - ma.x), p1 = attn_exp2(x[r + 1] - ma.y);
+                    const float p2 = attn_exp2(x[r + 2] - ma.z), p3 = attn_exp2(x[r + 3] - ma.w);
+                    const float p4 = attn_exp2(x[r + 4] - mb.x), p5 = attn_exp2(x[r + 5] - mb.y);
+                    const float p6 = attn_exp2(x[r + 6] - mb.z), p7 = attn_exp2(x[r + 7] - mb.w);
+                    if constexpr (NR == 32) {
+                        l[r + 0] += p0;
+                        l[r + 1] += p1;
+                        l[r + 2] += p2;
+                        l[r + 3] += p3;
+                        l[r + 4] += p4;
+                        l[r + 5] += p5;
+                        l[r + 6] += p6;
+                        l[r + 7] += p7;
+                    } else {
+                        x[r + 0] = p0;
+                        x[r + 1] = p1;
+                        x[r + 2] = p2;
+                        x[r + 3] = p3;
+                        x[r + 4] = p4;
+                        x[r + 5] = p5;
+                        x[r + 6] = p6;
+                        x[r + 7] = p7;
+                    }
+                    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+                    const uint32_t h45 = pack_bf16x2(p4, p5), h67 = pack_bf16x2(p6, p7);
+                    const int off = (c8 ^ (tok & 7)) << 4;
+                    const int roff = NR == 32 ? (((c8 + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
+                    *reinterpret_cast<uint4*>(prow + off) = make_uint4(h01, h23, h45, h67);
+                    *reinterpret_cast<uint4*>(prow + roff) =
+                        make_uint4(pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01)),
+                                   pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23)),
+                                   pack_bf16x2(p4 - bf16_lo(h45), p5 - bf16_hi(h45)),
+                                   pack_bf16x2(p6 - bf16_lo(h67), p7 - bf16_hi(h67)));
+                }
+                // a value row past the context in an occupied slot reads as zero (its weight is
+                // zero, and zero times a non-finite stale value is not)
+                if (!valid && nvj > 0) {
+                    cta_wait(&bar[kBarVFull + st], (pos >> 1) & 1, s_abort);   // orders the copy first
+                    uint8_t* vrow = sV + st * kAttnStageBytes + tok * 128;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        *reinterpret_cast<uint4*>(vrow + 16 * k) = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(vrow + kAttnHalf + 16 * k) = make_uint4(0u, 0u, 0u, 0u);
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kBarPFull + sb]);
+                if (lane == 0) mbar_arrive(&bar[kBarPFull + pbuf]);
+                if constexpr (NR == 64) {                     // x now holds the probabilities
+                    lsc0 += warp_reduce_scatter32<false>(*reinterpret_cast<float(*)[32]>(x), lane);
+                    lsc1 += warp_reduce_scatter32<false>(*reinterpret_cast<float(*)[32]>(x + 32), lane);
+                }
             }
-
-            // ------------------------------------------------- epilogue
-            if (ntiles > 0) {
-                attn_wait(&bar[kBarODone], static_cast<uint32_t>(nonempty & 1), s_abort);
-                ++nonempty;
-                tc_fence_after_sync();
+            // the chunk's row sums over this warp's tokens: lane t gets rows t and t + 32
+            float* lw = s_lw + (pb * 4 + q) * 64;
+            if constexpr (NR == 32) {
+                lw[lane] = warp_reduce_scatter32<false>(l, lane);
+                lw[32 + lane] = 0.f;
+            } else {
+                lw[lane] = lsc0;
+                lw[32 + lane] = lsc1;
             }
-            lA += __shfl_xor_sync(0xFFFFFFFFu, lA, 1);
-            lA += __shfl_xor_sync(0xFFFFFFFFu, lA, 2);
-            lB += __shfl_xor_sync(0xFFFFFFFFu, lB, 1);
-            lB += __shfl_xor_sync(0xFFFFFFFFu, lB, 2);
-            const float invA = lA > 0.f ? 1.f / lA : 0.f, invB = lB > 0.f ? 1.f / lB : 0.f;
-            const bool direct = u * K >= s_begin && (u + 1) * K <= s_end;
-            const int b = static_cast<int>(u / d.Hkv), h = static_cast<int>(u % d.Hkv);
-            const long long pidx = gs + u;                    // this CTA's partial of unit u
-            const long long orowA = (static_cast<long long>(b) * d.Qn + rA / G) * d.Hq + h * G + rA % G;
-            const long long orowB = (static_cast<long long>(b) * d.Qn + rB / G) * d.Hq + h * G + rB % G;
-            float* dstA = direct ? out + orowA * kHeadDim : ws_o + (pidx * rows + rA) * kHeadDim;
-            float* dstB = direct ? out + orowB * kHeadDim : ws_o + (pidx * rows + rB) * kHeadDim;
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar[kBarSMDone + pb]);
+                mbar_arrive(&bar[kBarLFree + pb]);
+            }
+        }
+    } else {
+        // ============================================ epilogue (channel / thread)
+        const int q = warp & 3;                               // TMEM lane quadrant
+        const int chn = 32 * q + lane;                        // head-dimension channel
+        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        const bool leader = warp == 4 && lane == 0;
+        for (int p = 0;; ++p) {
+            const int pb = p & 1;
+            cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort);
+            const int* info = s_info + pb * kAttnInfoInts;
+            const int n = info[0], c = info[1], u = info[2], ncu = info[3];
+            const bool stop = named_bar_or(kNbEpiVote, 128, n < 0 || *s_abort);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kBarLFree + pb]);
+            if (stop) break;
+            cta_wait(&bar[kBarSMDone + pb], (p >> 1) & 1, s_abort);
+            cta_wait(&bar[kBarODone + pb], (p >> 1) & 1, s_abort);
+            tc_fence_after_sync();
+            float* f_inv = s_fin + pb * 64;
+            float* f_lse = s_fin + 128 + pb * 64;
+            if (q < 2) {
+                const int r = 32 * q + lane;
+                const float* lw = s_lw + pb * 4 * 64;
+                const float L = (lw[r] + lw[64 + r]) + (lw[128 + r] + lw[192 + r]);
+                f_inv[r] = L > 0.f ? 1.f / L : 0.f;
+                f_lse[r] = L > 0.f ? s_m[pb * 64 + r] + log2f(L) : kNegInf;
+            }
+            float o[NR];
+            if (n > 0) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t o[32];
-                if (ntiles > 0) {
-                    tmem_ld_16x256b_x8(tmem_o + lane_base + half * 64, o);
+                for (int hh = 0; hh < NR / 32; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + 128 + pb * 64 + 32 * hh, v);
                     tmem_ld_wait();
-                } else {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = 0u;
+                    for (int r = 0; r < 32; ++r) o[32 * hh + r] = __uint_as_float(v[r]);
                 }
+            } else {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int col = half * 64 + 8 * c + cp;
-                    if (realA)
-                        *reinterpret_cast<float2*>(dstA + col) =
-                            make_float2(__uint_as_float(o[4 * c]) * invA, __uint_as_float(o[4 * c + 1]) * invA);
-                    if (realB)
-                        *reinterpret_cast<float2*>(dstB + col) = make_float2(__uint_as_float(o[4 * c + 2]) * invB,
-                                                                             __uint_as_float(o[4 * c + 3]) * invB);
-                }
+                for (int r = 0; r < NR; ++r) o[r] = 0.f;
             }
             tc_fence_before_sync();
-            if ((lane & 3) == 0) {
-                const float l2A = lA > 0.f ? mA + log2f(lA) : kNegInf;
-                const float l2B = lB > 0.f ? mB + log2f(lB) : kNegInf;
-                if (direct) {
-                    if (realA) lse_out[orowA] = lA > 0.f ? l2A * kLn2 : kNegInf;
-                    if (realB) lse_out[orowB] = lB > 0.f ? l2B * kLn2 : kNegInf;
-                } else {
-                    if (realA) ws_lse[pidx * rows + rA] = l2A;
-                    if (realB) ws_lse[pidx * rows + rB] = l2B;
+            named_bar_sync(kNbEpi, 128);       // O^T, running max and sums read; 1/sum and lse ready
+            if (leader) mbar_arrive(&bar[kBarOFree + pb]);
+            const int b = u / d.Hkv, h = u - b * d.Hkv;
+            if (ncu == 1) {
+                // the chunk is the whole unit: final output
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    if (r >= rows) break;
+                    const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
+                    out[orow * kHeadDim + chn] = o[r] * f_inv[r];
                 }
-            }
-            if (!direct) {
+                if (q < 2 && 32 * q + lane < rows) {
+                    const int r = 32 * q + lane;
+                    const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
+                    lse_out[orow] = f_lse[r] * kLn2;
+                }
+            } else {
+                float* dst = ws_o + static_cast<long long>(c) * rows * kHeadDim;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    if (r >= rows) break;
+                    dst[r * kHeadDim + chn] = o[r] * f_inv[r];
+                }
+                if (q < 2 && 32 * q + lane < rows) ws_lse[static_cast<long long>(c) * rows + 32 * q + lane] = f_lse[32 * q + lane];
                 __threadfence();
-                named_bar_sync(1, 128);
-                if (warp == 2 && lane == 0) {
-                    long long first, last;
-                    attn_unit_streams(u, K, n_streams, T, &first, &last);
-                    const int old = atomicAdd(ws_ticket + u, 1);
-                    *s_last = old == static_cast<int>(last - first) ? 1 : 0;
-                }
-                named_bar_sync(1, 128);
+                named_bar_sync(kNbEpi, 128);
+                if (leader) *s_last = atomicAdd(ws_ticket + u, 1) == ncu - 1 ? 1 : 0;
+                named_bar_sync(kNbEpi, 128);
                 if (*s_last) {
+                    // merge the unit's partials: out = sum_j 2^(lse_j - M) o_j / sum_j 2^(lse_j - M).
+                    // Thread r < rows turns row r's log2-sum-exps into weights, then every
+                    // thread (one channel) sums the weighted partials, loads in flight together.
                     __threadfence();
-                    long long first, last;
-                    attn_unit_streams(u, K, n_streams, T, &first, &last);
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int r = rr == 0 ? rA : rB;
-                        if (r >= rows) continue;
-                        const long long orow = rr == 0 ? orowA : orowB;
+                    const long long c0 = static_cast<long long>(u) * ncu;
+                    const int t = 32 * q + lane;
+                    if (t < rows) {
+                        float lj[kAttnMaxChunks];
                         float M = kNegInf;
-                        for (long long sp = first; sp <= last; ++sp) M = fmaxf(M, __ldcg(ws_lse + (sp + u) * rows + r));
+#pragma unroll
+                        for (int jj = 0; jj < kAttnMaxChunks; ++jj) {
+                            lj[jj] = jj < ncu ? __ldcg(ws_lse + (c0 + jj) * rows + t) : kNegInf;
+                            M = fmaxf(M, lj[jj]);
+                        }
                         float L = 0.f;
-                        float2 acc[16];
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) acc[k] = make_float2(0.f, 0.f);
-                        if (M != kNegInf) {
-                            for (long long sp = first; sp <= last; ++sp) {
-                                const float lj = __ldcg(ws_lse + (sp + u) * rows + r);
-                                if (lj == kNegInf) continue;             // empty partial: its output is not read
-                                const float w = exp2f(lj - M);
-                                L += w;
-                                const float* src = ws_o + ((sp + u) * rows + r) * kHeadDim;
-#pragma unroll
-                                for (int k = 0; k < 16; ++k) {
-                                    const int col = (k >> 3) * 64 + 8 * (k & 7) + cp;
-                                    const float2 x = __ldcg(reinterpret_cast<const float2*>(src + col));
-                                    acc[k].x += w * x.x;
-                                    acc[k].y += w * x.y;
-                                }
-                            }
+                        for (int jj = 0; jj < kAttnMaxChunks; ++jj) {
+                            lj[jj] = (M != kNegInf && lj[jj] != kNegInf) ? exp2f(lj[jj] - M) : 0.f;   // empty partial: 0
+                            L += lj[jj];
                         }
                         const float inv = L > 0.f ? 1.f / L : 0.f;
-                        float* dst = out + orow * kHeadDim;
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const int col = (k >> 3) * 64 + 8 * (k & 7) + cp;
-                            *reinterpret_cast<float2*>(dst + col) = make_float2(acc[k].x * inv, acc[k].y * inv);
-                        }
-                        if ((lane & 3) == 0) lse_out[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : kNegInf;
+                        for (int jj = 0; jj < kAttnMaxChunks; ++jj) s_mw[t * kAttnMaxChunks + jj] = lj[jj] * inv;
+                        const long long orow = (static_cast<long long>(b) * d.Qn + t / G) * d.Hq + h * G + t % G;
+                        lse_out[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : kNegInf;
                     }
-                    if (warp == 2 && lane == 0) ws_ticket[u] = 0;         // ready for the next call
+                    named_bar_sync(kNbEpi, 128);
+                    // 32 threads per row (4 channels each), 4 rows per row-set, two row-sets per
+                    // pass: up to 16 float4 loads in flight per thread
+                    const int et = 32 * q + lane;
+                    const int rsub = et >> 5, c4 = (et & 31) * 4;
+                    for (int r0 = 0; r0 < rows; r0 += 8) {
+                        float4 xv[2][kAttnMaxChunks];
+#pragma unroll
+                        for (int s2 = 0; s2 < 2; ++s2) {
+                            const int r = r0 + 4 * s2 + rsub;
+#pragma unroll
+                            for (int jj = 0; jj < kAttnMaxChunks; ++jj)
+                                xv[s2][jj] = (r < rows && jj < ncu)
+                                                 ? __ldcg(reinterpret_cast<const float4*>(
+                                                       ws_o + ((c0 + jj) * rows + r) * kHeadDim + c4))
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+#pragma unroll
+                        for (int s2 = 0; s2 < 2; ++s2) {
+                            const int r = r0 + 4 * s2 + rsub;
+                            if (r >= rows) continue;
+                            const float* w = s_mw + r * kAttnMaxChunks;
+                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int jj = 0; jj < kAttnMaxChunks; ++jj) {
+                                acc.x += w[jj] * xv[s2][jj].x;
+                                acc.y += w[jj] * xv[s2][jj].y;
+                                acc.z += w[jj] * xv[s2][jj].z;
+                                acc.w += w[jj] * xv[s2][jj].w;
+                            }
+                            const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
+                            *reinterpret_cast<float4*>(out + orow * kHeadDim + c4) = acc;
+                        }
+                    }
+                    if (leader) ws_ticket[u] = 0;             // ready for the next call
                 }
-            }
-            named_bar_sync(1, 128);                                         // every warp is done with the list
-            if (warp == 2 && lane == 0) {
-                *s_last = 0;
-                mbar_arrive(&bar[kBarLFree + pb]);
             }
         }
     }
@@ -555,7 +745,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (warp == 1) tmem_dealloc(tmem, kAttnTmemCols);
+    if (warp == kAttnSWarp) tmem_dealloc(tmem, kAttnTmemCols);
+    if (tid == 0) {
+        // the last CTA out resets the chunk counter for the next call
+        __threadfence();
+        if (atomicAdd(ws_sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+            atomicExch(ws_sched, 0);
+            atomicExch(ws_sched + 1, 0);
+        }
+    }
 }
 
 }  // namespace oasis

@@ -1,22 +1,36 @@
 // fused.cuh - lookahead scores, top-K selection and the capped fetch plan in
-// one launch.
+// one persistent launch.
 //
 // OasisKV: Scaling In-Decode KV Cache Beyond HBM with Lookahead Sparse
 // Prefetching, Figure 8: per layer the drafts drive the top-K prediction,
 // the prediction is diffed against the resident blocks, and only then can
 // the transfer start, so the three steps sit back to back on the path to the
-// copy; method sketch item 4.
+// copy; method sketch item 4.  The per-block bound is Quest's (Quest:
+// Query-Aware Sparsity for Efficient Long-Context LLM Inference), computed on
+// the tensor cores as in score.cuh: for 128 blocks and the R = draft rows x G
+// query vectors of a (sequence, KV head) unit,
+//     S[128 x R] = [kmax | kmin][128 x 256] . [q+ | q-]^T[256 x R].
 //
-// The grid is the scorer's: one CTA per 128-block tile of each (b, h) unit
-// (lookahead_score_kernel's tile, on the tensor cores).  After writing its
-// scores a CTA takes a ticket on the unit's counter; the CTA that completes
-// the unit (the last of its ceil(valid blocks / 128) tiles to finish) reads
-// all of the unit's scores back from L2 and runs the top-K selection and the
-// plan of the unit in its tail, then resets the counter.  No CTA waits for
-// another: the selection and the plan of a unit overlap the scoring of the
-// others, and the two separate launches (and their serial latency) are gone.
-// The results are those of the three separate kernels bit for bit: the same
-// scores, select_unit and plan_unit.
+// Work split: a unit's ceil(N / 128) block tiles are cut into chunks of `cts`
+// tiles; CTAs (at most one per SM) take chunks from an atomic counter in
+// unit-major order, skipping chunks past the unit's context, so units finish
+// one after another through the launch and a CTA slowed down by a neighbour
+// on its SM simply takes fewer chunks.  Warps are specialised:
+//   warp 0    producer: takes a chunk, streams its 64 KiB summary tiles
+//             through a 2-stage TMA ring and builds the unit's [q+ | q-]
+//             operand (double buffered when it fits);
+//   warp 1    one thread issues the 16 tcgen05.mma of each tile into one of
+//             two TMEM accumulators;
+//   warps 2-5 read the accumulators back (one TMEM lane quadrant each: 32
+//             blocks per warp), take the max over the real columns and store
+//             the fp32 scores; after a chunk they take a ticket on the unit's
+//             counter, and the chunk that completes the unit hands it to
+//   warps 6-9 which read the unit's scores back from L2 into shared memory
+//             and run the top-K selection (select_unit) and the plan
+//             (plan_unit) while the other warps score on.
+// Results are those of the separate lookahead_score / select_topk / plan
+// kernels bit for bit (the same MMA, the same select_unit and plan_unit).
+// The last CTA to exit resets the chunk counter for the next call.
 #pragma once
 
 #include "common.cuh"
@@ -26,62 +40,374 @@
 
 namespace oasis {
 
-// Shared memory of the fused tail: keys [N] u32, candidates
-// [next_pow2(min(K, N))] u64, plan scratch.
-__host__ __device__ inline int fused_tail_bytes(int N, int K) {
-    int kp = 1;
-    while (kp < (K < N ? K : N)) kp <<= 1;
-    return ((N * 4 + 7) / 8) * 8 + kp * 8 + plan_smem_ints(K) * 4;
-}
+constexpr int kSspThreads = 320;                           // 10 warps
+constexpr int kSspStages = 2;                              // summary-tile ring
+constexpr int kSspTileBytes = kScoreABytes;                // 64 KiB: kmax lo/hi, kmin lo/hi
+constexpr int kSspInfoInts = 8;                            // per chunk: end, u, nv, t0, ts, vt
+using SspTailGroup = WarpGroup<128, 2, 192>;               // warps 6-9
+using SspEpiGroup = WarpGroup<128, 1, 64>;                 // warps 2-5
 
-// slot_table == NULL: scores and selection only (no plan).  kScored: victims
-// by the block's score (read from `scores`), else LRU.  step_dev (nullable):
-// the step number is read from device memory.
+// barrier indices
+constexpr int kSspFull = 0;       // [2] tile landed
+constexpr int kSspEmpty = 2;      // [2] tile consumed by its MMAs
+constexpr int kSspAccFull = 4;    // [2] accumulator written
+constexpr int kSspAccFree = 6;    // [2] accumulator read (4 epilogue warps)
+constexpr int kSspBFull = 8;      // [2] unit operand built
+constexpr int kSspBFree = 10;     // [2] unit operand no longer read
+constexpr int kSspDecFull = 12;   // [2] chunk decided (epilogue leader): tail or not
+constexpr int kSspDecFree = 14;   // [2] decision consumed (tail leader)
+constexpr int kSspCFull = 16;     // [2] chunk description written (producer)
+constexpr int kSspCFree = 18;     // [2] description read (MMA issuer, epilogue leader)
+constexpr int kSspFinal = 20;
+constexpr int kSspNumBars = 21;
+constexpr uint32_t kSspNbEpiVote = 3;                      // named barrier of the epilogue's stop vote
+
+// Chunking of the scoring work (host and device agree through these).
+struct SspChunks {
+    int cts;   // tiles per chunk
+    int cpu;   // chunks per unit (ceil(ceil(N / 128) / cts))
+    int nc;    // chunks in all
+};
+
+template <int NPAD>
+struct SspSmem {
+    static constexpr int kBBytes = 4 * NPAD * 128;                     // q+ lo/hi, q- lo/hi
+    static constexpr int kOffB = kSspStages * kSspTileBytes;
+    static constexpr int kOffBar(int nbuf) { return kOffB + nbuf * kBBytes; }
+    static constexpr int kOffMisc(int nbuf) { return kOffBar(nbuf) + kSspNumBars * 8; }   // 64 ints
+    static constexpr int kOffCand(int nbuf) { return kOffMisc(nbuf) + 256; }
+    static constexpr int kAccStride = NPAD <= 16 ? 16 : (NPAD <= 32 ? 32 : 64);   // TMEM columns per accumulator
+    static constexpr int kTmemCols = 2 * kAccStride < 32 ? 32 : 2 * kAccStride;
+    // total dynamic bytes for nbuf operand buffers, budget K and N blocks
+    // (candidates, plan scratch, the unit's keys; +1024 alignment slack)
+    static constexpr int bytes(int nbuf, int K, int N) {
+        int kp = 1;
+        while (kp < K) kp <<= 1;
+        return kOffCand(nbuf) + kp * 8 + plan_smem_ints(K) * 4 + N * 4 + 1024;
+    }
+};
+
 template <int NPAD, bool kScored>
-__global__ void __launch_bounds__(128) score_select_plan_kernel(
+__global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
     const __grid_constant__ CUtensorMap tm_kmax, const __grid_constant__ CUtensorMap tm_kmin, Dims d,
     const uint16_t* __restrict__ q, const int32_t* __restrict__ ctx_len, float* scores, int row0, int rows,
-    int* ticket, int32_t* sel, float* sel_score, int32_t* slot_table, int32_t* last_used, int step,
-    const int32_t* __restrict__ step_dev, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch) {
+    int* ticket, int* sched, int32_t* sel, float* sel_score, int32_t* slot_table, int32_t* last_used, int step,
+    const int32_t* __restrict__ step_dev, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
+    SspChunks ch, int nbuf) {
+    using S = SspSmem<NPAD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ SelScratch sc;
     __shared__ int tmp[32];
-    __shared__ int s_last;
-    const int tid = threadIdx.x;
-    const int bh = blockIdx.y, b = bh / d.Hkv, h = bh % d.Hkv;
-    const int nv = n_valid_blocks(ctx_len[b], d.N);
-    const int parts = max(1, (nv + kScoreTile - 1) / kScoreTile);   // CTAs that take a ticket
-    if (static_cast<int>(blockIdx.x) >= parts) return;
-    const int n0 = blockIdx.x * kScoreTile;
-    if (n0 < nv) score_tile<NPAD>(&tm_kmax, &tm_kmin, d, q, b, h, n0, nv, scores, row0, rows, smem);
-
-    // the CTA that finishes the unit selects and plans it
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(ticket + bh, 1) == parts - 1 ? 1 : 0;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (tid == 0) ticket[bh] = 0;                                     // ready for the next call
-    const int N = d.N, K = d.K;
-    const float* su = scores + static_cast<long long>(bh) * N;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
-    unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + ((N * 4 + 7) / 8) * 8);
+    uint8_t* ring = smem;
+    uint8_t* bbuf = smem + S::kOffB;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + S::kOffBar(nbuf));
+    int* misc = reinterpret_cast<int*>(smem + S::kOffMisc(nbuf));
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc);
+    volatile int* s_abort = misc + 1;
+    int* s_info = misc + 8;                               // [2][kSspInfoInts] chunk descriptions
+    volatile int* s_dec = misc + 24;                      // [2][4] decisions (mine, unit, nv, end) + a copy
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + S::kOffCand(nbuf));
     int kp = 1;
-    while (kp < min(K, N)) kp <<= 1;
+    while (kp < d.K) kp <<= 1;
     int32_t* sp = reinterpret_cast<int32_t*>(cand + kp);
-    for (int i = tid; i < nv; i += 128) keys[i] = ordered_key(__ldcg(su + i));
+    uint32_t* keys = reinterpret_cast<uint32_t*>(sp + plan_smem_ints(d.K));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long N = d.N;
+
+    if (tid == 0) {
+        for (int i = 0; i < kSspNumBars; ++i)
+            mbar_init(&bar[i], (i == kSspAccFree || i == kSspAccFree + 1) ? 4
+                               : (i == kSspCFree || i == kSspCFree + 1) ? 2
+                                                                         : 1);
+        fence_mbar_init();
+        *s_abort = 0;
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem, S::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
     __syncthreads();
-    int32_t* sel_u = sel + static_cast<long long>(bh) * K;
-    select_unit<128>(keys, nv, K, cand, &sc, su, sel_u, sel_score ? sel_score + static_cast<long long>(bh) * K : nullptr);
-    if (slot_table == nullptr) return;
-    __syncthreads();                                                  // the selection is in memory
-    if (step_dev != nullptr) step = *step_dev;
-    plan_unit<128, kScored>(K, d.C, N, sel_u, kScored ? su : nullptr, slot_table + static_cast<long long>(bh) * K,
-                            last_used + static_cast<long long>(bh) * K, step,
-                            fetch_slot + static_cast<long long>(bh) * d.C, fetch_block + static_cast<long long>(bh) * d.C,
-                            n_fetch + bh, sp, tmp);
+    tc_fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+    const int G = d.G();
+
+    if (warp == 0) {
+        // ========================================================= producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_kmax);
+            prefetch_tensormap(&tm_kmin);
+        }
+        const uint64_t pol = l2_policy_evict_first();
+        int pos = 0, nb = 0;
+        int last_pos[kSspStages] = {-1, -1};
+        // tile t of unit u into the ring (lane 0)
+        auto load_tile = [&](int u, int t) {
+            const int stage = pos % kSspStages;
+            if (pos >= kSspStages) cta_wait(&bar[kSspEmpty + stage], ((pos / kSspStages) - 1) & 1, s_abort);
+            mbar_arrive_expect_tx(&bar[kSspFull + stage], kSspTileBytes);
+            if (!*s_abort) {
+                last_pos[stage] = pos;
+                uint8_t* st = ring + stage * kSspTileBytes;
+                const int y = static_cast<int>(u * N + t * kScoreTile);
+                tma_load_2d(st + 0 * kScoreRegionBytes, &tm_kmax, &bar[kSspFull + stage], 0, y, pol);
+                tma_load_2d(st + 1 * kScoreRegionBytes, &tm_kmax, &bar[kSspFull + stage], 64, y, pol);
+                tma_load_2d(st + 2 * kScoreRegionBytes, &tm_kmin, &bar[kSspFull + stage], 0, y, pol);
+                tma_load_2d(st + 3 * kScoreRegionBytes, &tm_kmin, &bar[kSspFull + stage], 64, y, pol);
+            }
+            ++pos;
+        };
+        for (int p = 0;; ++p) {
+            const int pb = p & 1;
+            int* info = s_info + pb * kSspInfoInts;
+            if (lane == 0 && p >= 2) cta_wait(&bar[kSspCFree + pb], ((p >> 1) - 1) & 1, s_abort);
+            // the next chunk that holds valid blocks (every unit has one: its chunk 0)
+            int u = 0, nv = 0, t0 = 0, vt = 0, c = 0;
+            while (true) {
+                if (lane == 0) c = *s_abort ? ch.nc : atomicAdd(sched, 1);
+                c = __shfl_sync(0xFFFFFFFFu, c, 0);
+                if (c >= ch.nc) break;
+                u = c / ch.cpu;
+                t0 = (c - u * ch.cpu) * ch.cts;
+                nv = n_valid_blocks(ctx_len[u / d.Hkv], d.N);
+                vt = max(1, (nv + kScoreTile - 1) / kScoreTile);
+                if (t0 < vt) break;
+            }
+            if (c >= ch.nc) {
+                if (lane == 0) {
+                    info[0] = 1;
+                    mbar_arrive(&bar[kSspCFull + pb]);
+                }
+                break;
+            }
+            const int ts = min(t0 + ch.cts, (nv + kScoreTile - 1) / kScoreTile);   // scored tiles [t0, ts)
+            // as many tiles as the ring holds go out first: they wait only on earlier
+            // chunks' products; the rest wait on this chunk's, so the operand comes first
+            const int t_pre = min(ts, t0 + kSspStages);
+            if (lane == 0) {
+                info[0] = 0;
+                info[1] = u;
+                info[2] = nv;
+                info[3] = t0;
+                info[4] = ts;
+                info[5] = vt;
+                mbar_arrive(&bar[kSspCFull + pb]);
+                for (int t = t0; t < t_pre; ++t) load_tile(u, t);
+            }
+            __syncwarp();
+            if (ts > t0) {
+                // [q+ | q-] of the unit's scored rows, four 64-column regions, 128-byte swizzled
+                const int b = u / d.Hkv, h = u - b * d.Hkv;
+                const int bb = nb % nbuf;
+                if (lane == 0 && nb >= nbuf) cta_wait(&bar[kSspBFree + bb], ((nb / nbuf) - 1) & 1, s_abort);
+                __syncwarp();
+                uint8_t* bt = bbuf + bb * S::kBBytes;
+                // NPAD*16 16-B pieces, 32 lanes: loads go out in batches of 8 per lane
+                constexpr int kPer = NPAD / 2, kBatch = kPer < 8 ? kPer : 8;
+#pragma unroll
+                for (int i0 = 0; i0 < kPer; i0 += kBatch) {
+                  uint4 vb[kBatch];
+#pragma unroll
+                  for (int k = 0; k < kBatch; ++k) {
+                    const int it = lane + 32 * (i0 + k);
+                    const int r = it >> 4, cc16 = it & 15;
+                    vb[k] = make_uint4(0, 0, 0, 0);
+                    if (r < rows) {
+                        const int j = row0 + r / G, g = r % G;
+                        vb[k] = *reinterpret_cast<const uint4*>(
+                            q + ((static_cast<long long>(b) * d.Qn + j) * d.Hq + h * G + g) * kHeadDim + cc16 * 8);
+                    }
+                  }
+#pragma unroll
+                  for (int k = 0; k < kBatch; ++k) {
+                    const int it = lane + 32 * (i0 + k);
+                    const int r = it >> 4, cc16 = it & 15;
+                    const uint4 v = vb[k];
+                    uint32_t w[4] = {v.x, v.y, v.z, v.w}, pos4[4], neg4[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t neg_mask = ((w[i] & 0x80008000u) >> 15) * 0xFFFFu;
+                        neg4[i] = w[i] & neg_mask;
+                        pos4[i] = w[i] & ~neg_mask;
+                    }
+                    const int region = cc16 >> 3, cc = cc16 & 7;
+                    const int off = (r >> 3) * 1024 + (r & 7) * 128 + ((cc ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4*>(bt + region * NPAD * 128 + off) =
+                        make_uint4(pos4[0], pos4[1], pos4[2], pos4[3]);
+                    *reinterpret_cast<uint4*>(bt + (2 + region) * NPAD * 128 + off) =
+                        make_uint4(neg4[0], neg4[1], neg4[2], neg4[3]);
+                  }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bar[kSspBFull + bb]);
+                    for (int t = t_pre; t < ts; ++t) load_tile(u, t);
+                }
+                ++nb;
+            }
+            __syncwarp();
+            pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+        }
+        if (lane == 0)                                     // no copy may land after the CTA exits
+            for (int s = 0; s < kSspStages; ++s)
+                if (last_pos[s] >= 0) mbar_wait(&bar[kSspFull + s], static_cast<uint32_t>((last_pos[s] / kSspStages) & 1));
+    } else if (warp == 1) {
+        // ======================================================= MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16_f32(kScoreTile, NPAD);
+            int pos = 0, nb = 0;
+            for (int p = 0;; ++p) {
+                const int pb = p & 1;
+                if (!cta_wait(&bar[kSspCFull + pb], (p >> 1) & 1, s_abort)) break;
+                const int* info = s_info + pb * kSspInfoInts;
+                if (info[0]) break;
+                const int t0 = info[3], ts = info[4];
+                if (ts > t0) {
+                    const int bb = nb % nbuf;
+                    cta_wait(&bar[kSspBFull + bb], (nb / nbuf) & 1, s_abort);
+                    const uint32_t b0 = smem_addr(bbuf + bb * S::kBBytes);
+                    for (int t = t0; t < ts; ++t, ++pos) {
+                        const int stage = pos % kSspStages;
+                        const int ab = pos & 1;
+                        bool ok = cta_wait(&bar[kSspFull + stage], (pos / kSspStages) & 1, s_abort);
+                        if (pos >= 2) ok = cta_wait(&bar[kSspAccFree + ab], ((pos >> 1) - 1) & 1, s_abort) && ok;
+                        tc_fence_after_sync();
+                        if (ok) {
+                            const uint32_t a0 = smem_addr(ring + stage * kSspTileBytes);
+#pragma unroll
+                            for (int reg = 0; reg < 4; ++reg)
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    umma_bf16(tmem + ab * S::kAccStride,
+                                              umma_desc_sw128(a0 + reg * kScoreRegionBytes + ks * 32),
+                                              umma_desc_sw128(b0 + reg * NPAD * 128 + ks * 32), idesc,
+                                              (reg | ks) != 0);
+                        }
+                        umma_commit(&bar[kSspAccFull + ab]);
+                        umma_commit(&bar[kSspEmpty + stage]);
+                    }
+                    umma_commit(&bar[kSspBFree + bb]);         // after the chunk's last MMA
+                    ++nb;
+                }
+                mbar_arrive(&bar[kSspCFree + pb]);
+            }
+            umma_commit(&bar[kSspFinal]);
+            mbar_wait(&bar[kSspFinal], 0);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ========================================== score epilogue (2..5)
+        const int qd = warp & 3;                               // TMEM lane quadrant = 32 blocks of the tile
+        const bool leader = warp == 2 && lane == 0;
+        int pos = 0;
+        for (int p = 0;; ++p) {
+            const int pb = p & 1, db = p & 1;
+            cta_wait(&bar[kSspCFull + pb], (p >> 1) & 1, s_abort);
+            const int* info = s_info + pb * kSspInfoInts;
+            const int end = info[0], u = info[1], nv = info[2], t0 = info[3], ts = info[4], vt = info[5];
+            if (named_bar_or(kSspNbEpiVote, 128, end != 0 || *s_abort)) {
+                if (leader) {                                  // the tail group finishes too
+                    if (p >= 2) cta_wait(&bar[kSspDecFree + db], ((p >> 1) - 1) & 1, s_abort);
+                    s_dec[db * 4 + 3] = 1;
+                    mbar_arrive(&bar[kSspDecFull + db]);
+                }
+                break;
+            }
+            for (int t = t0; t < ts; ++t, ++pos) {
+                const int ab = pos & 1;
+                const bool ok = cta_wait(&bar[kSspAccFull + ab], (pos >> 1) & 1, s_abort);
+                tc_fence_after_sync();
+                float best = -__int_as_float(0x7f800000);
+                if (ok) {
+#pragma unroll
+                    for (int c0 = 0; c0 < NPAD; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld_x16(tmem + (static_cast<uint32_t>(qd * 32) << 16) + ab * S::kAccStride + c0, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < rows) best = fmaxf(best, __uint_as_float(v[i]));
+                    }
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kSspAccFree + ab]);
+                const int n = t * kScoreTile + qd * 32 + lane;
+                if (ok && n < nv) scores[u * N + n] = best;
+            }
+            // the chunk's scores are out: take the unit's ticket; the chunk that
+            // completes the unit hands it to the tail warps
+            __threadfence();
+            SspEpiGroup::sync();
+            if (leader) {
+                const int chunks = (vt + ch.cts - 1) / ch.cts;     // the unit's chunks that hold valid blocks
+                const int old = atomicAdd(ticket + u, 1);
+                mbar_arrive(&bar[kSspCFree + pb]);
+                if (p >= 2) cta_wait(&bar[kSspDecFree + db], ((p >> 1) - 1) & 1, s_abort);
+                s_dec[db * 4 + 0] = old == chunks - 1 ? 1 : 0;
+                s_dec[db * 4 + 1] = u;
+                s_dec[db * 4 + 2] = nv;
+                s_dec[db * 4 + 3] = 0;
+                mbar_arrive(&bar[kSspDecFull + db]);            // release: the decision and the scores
+            }
+        }
+    } else {
+        // ====================================== top-K + plan tail (6..9)
+        const int ttid = SspTailGroup::tid();
+        for (int p = 0;; ++p) {
+            const int db = p & 1;
+            cta_wait(&bar[kSspDecFull + db], (p >> 1) & 1, s_abort);
+            // one thread copies the decision and the group reads the copy after the
+            // barrier, so every thread sees the same values (they then meet the same
+            // barriers below)
+            if (ttid == 0) {
+                const int end = (s_dec[db * 4 + 3] != 0 || *s_abort) ? 1 : 0;
+                s_dec[8] = end ? 0 : s_dec[db * 4 + 0];
+                s_dec[9] = s_dec[db * 4 + 1];
+                s_dec[10] = s_dec[db * 4 + 2];
+                s_dec[11] = end;
+            }
+            SspTailGroup::sync();
+            const int mine = s_dec[8], u = s_dec[9], nv = s_dec[10], end = s_dec[11];
+            SspTailGroup::sync();
+            if (ttid == 0) mbar_arrive(&bar[kSspDecFree + db]);
+            if (end) break;
+            if (!mine) continue;
+            __threadfence();                                   // every CTA's scores of the unit are visible
+            if (ttid == 0) ticket[u] = 0;                      // ready for the next call
+            const float* su = scores + u * N;
+            for (int i = ttid; i < nv; i += SspTailGroup::kThreads) keys[i] = ordered_key(__ldcg(su + i));
+            SspTailGroup::sync();
+            int32_t* sel_u = sel + static_cast<long long>(u) * d.K;
+            select_unit<SspTailGroup>(SmemKeys{keys}, nv, d.K, cand, &sc, su, sel_u,
+                                      sel_score ? sel_score + static_cast<long long>(u) * d.K : nullptr);
+            if (slot_table == nullptr) continue;
+            SspTailGroup::sync();                              // the selection is in memory
+            const int stp = step_dev != nullptr ? *step_dev : step;
+            const long long uk = static_cast<long long>(u) * d.K, uc = static_cast<long long>(u) * d.C;
+            plan_unit<SspTailGroup, kScored>(d.K, d.C, d.N, sel_u, kScored ? su : nullptr, slot_table + uk,
+                                             last_used + uk, stp, fetch_slot + uc, fetch_block + uc, n_fetch + u, sp,
+                                             tmp);
+            SspTailGroup::sync();                              // scratch free for the next unit
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc(tmem, S::kTmemCols);
+    if (tid == 0) {
+        // the last CTA out resets the chunk counter for the next call
+        __threadfence();
+        if (atomicAdd(sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+            atomicExch(sched, 0);
+            atomicExch(sched + 1, 0);
+        }
+    }
 }
 
 }  // namespace oasis

@@ -141,6 +141,26 @@ int make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned
     return OASIS_OK;
 }
 
+// Keys (or values, from base + 4 KiB) of the pool: bf16 [B*Hkv*K slots][32
+// rows][128] seen as a 3-D tensor (128 columns, 16 rows of one slot's K or V,
+// slots 8 KiB apart), boxes of 64 columns x 16 rows x 4 consecutive slots.
+int make_map_pool(CUtensorMap* m, const void* base, unsigned long long slots, const char* name) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(oasis::kHeadDim), static_cast<cuuint64_t>(oasis::kBlockTokens),
+                                static_cast<cuuint64_t>(slots)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(oasis::kRowBytes),
+                                   static_cast<cuuint64_t>(oasis::kBlockBytes)};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(oasis::kBlockTokens),
+                               static_cast<cuuint32_t>(oasis::kAttnTileSlots)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled(%s) failed: %d", name, static_cast<int>(r));
+    return OASIS_OK;
+}
+
 // The query rows of every (sequence, KV head): bf16 q [B][Qn][Hq][128] seen
 // as a 3-D tensor (128 columns, Hq heads, B*Qn query positions), boxes of
 // 64 columns x G heads x Qn positions, so one box per 64-column half brings
@@ -161,30 +181,61 @@ int make_map_q(CUtensorMap* m, const void* q, const Dims& d) {
     return OASIS_OK;
 }
 
+// Every kernel asks for the largest shared-memory carve-out.  An SM's split
+// between L1 and shared memory is set when a CTA lands on an idle SM, and an
+// SM split for a kernel that needs little shared memory (the gather, the
+// plan) cannot take a 200-KB attention or scoring CTA until it drains: the
+// attention launched beside a running gather then ran in two waves.
 template <typename K>
-int set_smem(K kernel, int bytes, const char* what) {
-    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+int carveout(K kernel, const char* what) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_fail(e, what);
     return OASIS_OK;
 }
 
+template <typename K>
+int set_smem(K kernel, int bytes, const char* what) {
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return carveout(kernel, what);
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Upper bound of attention streams the workspace is sized for: 148 SMs x 8
-// streams (two CTAs of four per SM), or more when ranges would exceed 256 slots.
-long long attn_max_streams(const Dims& d) {
-    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
-    const long long cap = 148ll * 8;
-    return std::max<long long>(1, std::min(T, std::max(cap, (T + 255) / 256)));
+// Attention chunks: a unit's ceil(K / 8) tiles cut into chunks of `ct`
+// tiles.  Chunks are at least 2 tiles (4 with more than 32 query rows) so the
+// partials a split unit writes stay under ~1/8 of the bytes it reads, at
+// most 8 per unit (the merge's limit), and otherwise sized for about six per
+// CTA so that CTAs taking chunks from the counter finish together.
+int attn_min_chunk_tiles(const Dims& d) {
+    const int tpu = (d.K + oasis::kAttnTileSlots - 1) / oasis::kAttnTileSlots;
+    return std::min(tpu, d.Qn * d.G() <= 32 ? 2 : 4);
+}
+
+oasis::AttnChunks attn_chunks(const Dims& d, int ctas) {
+    const int tpu = (d.K + oasis::kAttnTileSlots - 1) / oasis::kAttnTileSlots;
+    const long long units = static_cast<long long>(d.B) * d.Hkv;
+    const long long per = units * tpu / (6ll * std::max(1, ctas));
+    int ct = static_cast<int>(std::min<long long>(std::max<long long>(per, attn_min_chunk_tiles(d)),
+                                                  oasis::kAttnMaxChunkTiles));
+    ct = std::max(ct, (tpu + oasis::kAttnMaxChunks - 1) / oasis::kAttnMaxChunks);   // the merge takes <= 8
+    ct = std::min(ct, tpu);
+    oasis::AttnChunks c;
+    c.ct = ct;
+    c.cpu = (tpu + ct - 1) / ct;
+    c.nc = static_cast<int>(units * c.cpu);
+    return c;
 }
 
 // Workspace: block scores [B*Hkv*N] fp32, then the attention partials of
-// units split over CTAs (log2-sum-exp [P][rows] and normalised outputs
-// [P][rows][128], P = streams + units), then one ticket counter per unit for
-// the attention merge and one for the fused score / select / plan (all zero
-// between calls).
+// split units (log2-sum-exp [P][rows] and normalised outputs [P][rows][128],
+// P = the most chunks any launch makes), then one ticket counter per unit
+// for the attention merge, one per unit for the fused score / select / plan,
+// and the chunk and exit counters of the attention and of the fused scoring
+// (all zero between calls).
 struct WsLayout {
-    size_t scores, lse, o, ticket, sticket, total;
+    size_t scores, lse, o, ticket, sticket, sched, ssched, total;
     long long partials;
 };
 
@@ -192,13 +243,17 @@ WsLayout ws_layout(const Dims& d) {
     WsLayout w;
     const size_t units = static_cast<size_t>(d.B) * d.Hkv;
     const size_t rows = static_cast<size_t>(d.Qn) * d.G();
-    w.partials = attn_max_streams(d) + static_cast<long long>(units);
+    const long long tpu = (d.K + oasis::kAttnTileSlots - 1) / oasis::kAttnTileSlots;
+    const long long mct = attn_min_chunk_tiles(d);
+    w.partials = static_cast<long long>(units) * ((tpu + mct - 1) / mct);
     w.scores = 0;
     w.lse = align256(units * d.N * sizeof(float));
     w.o = align256(w.lse + static_cast<size_t>(w.partials) * rows * sizeof(float));
     w.ticket = align256(w.o + static_cast<size_t>(w.partials) * rows * oasis::kHeadDim * sizeof(float));
     w.sticket = align256(w.ticket + units * sizeof(int));
-    w.total = align256(w.sticket + units * sizeof(int));
+    w.sched = align256(w.sticket + units * sizeof(int));
+    w.ssched = align256(w.sched + 2 * sizeof(int));
+    w.total = align256(w.ssched + 2 * sizeof(int));
     return w;
 }
 
@@ -215,14 +270,6 @@ int sm_count() {
     return n;
 }
 
-// CTAs (streams) of an attention launch: one per SM, each range at least 16
-// slots (four tiles), never more than the workspace holds.
-long long attn_streams(const Dims& d) {
-    const long long T = static_cast<long long>(d.B) * d.Hkv * d.K;
-    long long ns = std::min<long long>(sm_count(), std::max(1ll, T / 16));
-    return std::min(ns, attn_max_streams(d));
-}
-
 template <int NPAD>
 int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
                  const int32_t* ctx, float* scores, int row0, int rows, cudaStream_t s) {
@@ -234,35 +281,47 @@ int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d
     return check_launch("lookahead_score launch");
 }
 
+// Scoring chunks: 2 tiles of 128 blocks each (128 KiB of summaries), one per
+// unit when a unit has fewer.
 template <int NPAD, bool kScored>
 int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
-                 const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int32_t* sel, float* sel_score,
-                 int32_t* st, int32_t* lu, int32_t step, const int32_t* step_dev, int32_t* fs, int32_t* fb,
-                 int32_t* nf, cudaStream_t s) {
+                 const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int* sched, int32_t* sel,
+                 float* sel_score, int32_t* st, int32_t* lu, int32_t step, const int32_t* step_dev, int32_t* fs,
+                 int32_t* fb, int32_t* nf, cudaStream_t s) {
+    using S = oasis::SspSmem<NPAD>;
     auto k = oasis::score_select_plan_kernel<NPAD, kScored>;
-    const int smem = std::max(oasis::ScoreSmem<NPAD>::kBytes, oasis::fused_tail_bytes(d.N, d.K) + 1024);
+    // two unit operands when they fit beside the ring and the tail scratch, else one
+    const int nbuf = S::bytes(2, d.K, d.N) <= 227 * 1024 ? 2 : 1;
+    const int smem = S::bytes(nbuf, d.K, d.N);
+    if (smem > 227 * 1024)
+        return fail(OASIS_EINVAL, "budget_blocks %d / max_blocks %d need more shared memory than a CTA has", d.K, d.N);
     if (int rc = set_smem(k, smem, "score_select_plan smem")) return rc;
-    dim3 grid((d.N + oasis::kScoreTile - 1) / oasis::kScoreTile, d.B * d.Hkv);
-    k<<<grid, 128, smem, s>>>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu, step,
-                              step_dev, fs, fb, nf);
+    const int tpu = (d.N + oasis::kScoreTile - 1) / oasis::kScoreTile;
+    oasis::SspChunks ch;
+    ch.cts = std::min(2, tpu);
+    ch.cpu = (tpu + ch.cts - 1) / ch.cts;
+    ch.nc = d.B * d.Hkv * ch.cpu;
+    const int ctas = std::min(sm_count(), ch.nc);
+    k<<<ctas, oasis::kSspThreads, smem, s>>>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score,
+                                             st, lu, step, step_dev, fs, fb, nf, ch, nbuf);
     return check_launch("score_select_plan launch");
 }
 
 template <bool kScored>
 int launch_fused_rows(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
-                      const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int32_t* sel,
+                      const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int* sched, int32_t* sel,
                       float* sel_score, int32_t* st, int32_t* lu, int32_t step, const int32_t* step_dev, int32_t* fs,
                       int32_t* fb, int32_t* nf, cudaStream_t s) {
     if (rows <= 16)
-        return launch_fused<16, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu,
+        return launch_fused<16, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
                                          step, step_dev, fs, fb, nf, s);
     if (rows <= 32)
-        return launch_fused<32, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu,
+        return launch_fused<32, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
                                          step, step_dev, fs, fb, nf, s);
     if (rows <= 48)
-        return launch_fused<48, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu,
+        return launch_fused<48, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
                                          step, step_dev, fs, fb, nf, s);
-    return launch_fused<64, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sel, sel_score, st, lu, step,
+    return launch_fused<64, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu, step,
                                      step_dev, fs, fb, nf, s);
 }
 
@@ -340,12 +399,15 @@ int plan(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t*
     }
     const int smem = oasis::plan_smem_ints(d.K) * static_cast<int>(sizeof(int32_t));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (scores != nullptr)
+    if (scores != nullptr) {
+        if (int rc = carveout(oasis::plan_fetch_kernel<true>, "plan carve-out")) return rc;
         oasis::plan_fetch_kernel<true><<<d.B * d.Hkv, oasis::kPlanThreads, smem, s>>>(
             d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
-    else
+    } else {
+        if (int rc = carveout(oasis::plan_fetch_kernel<false>, "plan carve-out")) return rc;
         oasis::plan_fetch_kernel<false><<<d.B * d.Hkv, oasis::kPlanThreads, smem, s>>>(
             d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
+    }
     return check_launch("plan_fetch launch");
 }
 
@@ -381,6 +443,7 @@ int oasis_build_summaries(const oasis_dims* dp, const void* kv, const int32_t* c
     const long long items = static_cast<long long>(d.B) * d.Hkv * n_blocks;
     const long long grid = (items + oasis::kSumGroups - 1) / oasis::kSumGroups;
     if (grid > 0x7FFFFFFFll) return fail(OASIS_EINVAL, "too many blocks");
+    if (int rc = carveout(oasis::build_summaries_kernel, "summaries carve-out")) return rc;
     oasis::build_summaries_kernel<<<static_cast<unsigned>(grid), oasis::kSumThreads, 0,
                                     static_cast<cudaStream_t>(stream)>>>(
         d, static_cast<const uint4*>(src), ctx_len, first_block, n_blocks, static_cast<uint4*>(kmin),
@@ -408,6 +471,7 @@ int oasis_append_kv(const oasis_dims* dp, const void* k_new, const void* v_new, 
     const void* hv = nullptr;
     if (host_kv != nullptr)
         if (int rc = device_view(host_kv, "host_kv", false, &hv)) return rc;
+    if (int rc = carveout(oasis::append_kv_kernel, "append carve-out")) return rc;
     oasis::append_kv_kernel<<<d.B * d.Hkv, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         d, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), ctx_len, ctx_len_out,
         static_cast<uint4*>(const_cast<void*>(hv)), static_cast<uint4*>(kmin), static_cast<uint4*>(kmax), slot_table,
@@ -488,11 +552,10 @@ int oasis_score_select_plan(const oasis_dims* dp, const void* q, const void* kmi
     if (int rc = check_ptr(ws, "ws")) return rc;
     const WsLayout w = ws_layout(d);
     if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
-    if (oasis::fused_tail_bytes(d.N, d.K) + 1024 > 227 * 1024)
-        return fail(OASIS_EINVAL, "max_blocks %d with budget %d exceeds the fused kernel's shared memory", d.N, d.K);
     uint8_t* base = static_cast<uint8_t*>(ws);
     float* sc = scores != nullptr ? scores : reinterpret_cast<float*>(base + w.scores);
     int* ticket = reinterpret_cast<int*>(base + w.sticket);
+    int* sched = reinterpret_cast<int*>(base + w.ssched);
     const int row0 = d.Qn > 1 ? 1 : 0;
     const int rows = (d.Qn > 1 ? d.Qn - 1 : 1) * d.G();
     const unsigned long long total_rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.N;
@@ -502,9 +565,9 @@ int oasis_score_select_plan(const oasis_dims* dp, const void* q, const void* kmi
     const auto* qq = static_cast<const uint16_t*>(q);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (scores != nullptr)
-        return launch_fused_rows<true>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sel, sel_score,
+        return launch_fused_rows<true>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sched, sel, sel_score,
                                        slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch, s);
-    return launch_fused_rows<false>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sel, sel_score, slot_table,
+    return launch_fused_rows<false>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sched, sel, sel_score, slot_table,
                                     last_used, step, step_dev, fetch_slot, fetch_block, n_fetch, s);
 }
 
@@ -515,6 +578,7 @@ int oasis_block_overlap(const oasis_dims* dp, const int32_t* a, const int32_t* b
     if (int rc = check_ptr(b, "b")) return rc;
     if (int rc = check_ptr(count, "count")) return rc;
     const int smem = 2 * ((d.N + 31) / 32) * static_cast<int>(sizeof(uint32_t));
+    if (int rc = carveout(oasis::block_overlap_kernel, "overlap carve-out")) return rc;
     oasis::block_overlap_kernel<<<d.B * d.Hkv, oasis::kOverlapThreads, smem, static_cast<cudaStream_t>(stream)>>>(
         d, a, b, count);
     return check_launch("block_overlap launch");
@@ -547,6 +611,7 @@ int oasis_evict_slots(const oasis_dims* dp, const uint8_t* mask, int32_t* slot_t
     if (int rc = check_ptr(slot_table, "slot_table")) return rc;
     const long long n = static_cast<long long>(d.B) * d.Hkv * d.K;
     const unsigned grid = static_cast<unsigned>(std::min<long long>((n + 255) / 256, 4 * 148));
+    if (int rc = carveout(oasis::evict_slots_kernel, "evict carve-out")) return rc;
     oasis::evict_slots_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(n, mask, slot_table);
     return check_launch("evict_slots launch");
 }
@@ -601,6 +666,7 @@ int oasis_decode_layer_step(const oasis_dims* dp, const oasis_layer* L, const vo
 
 int oasis_step_advance(int32_t* step, void* stream) {
     if (int rc = check_ptr(step, "step")) return rc;
+    if (int rc = carveout(oasis::step_advance_kernel, "step carve-out")) return rc;
     oasis::step_advance_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(step);
     return check_launch("step_advance launch");
 }
@@ -619,6 +685,7 @@ int oasis_prefetch(const oasis_dims* dp, const void* host_kv, const int32_t* fet
     if (int rc = device_view(host_kv, "host_kv", false, &hv)) return rc;
     const long long entries = static_cast<long long>(d.B) * d.Hkv * d.C;
     const unsigned grid = static_cast<unsigned>(std::min<long long>(oasis::kPrefetchCtas, (entries + 1) / 2));
+    if (int rc = carveout(oasis::prefetch_kernel, "prefetch carve-out")) return rc;
     oasis::prefetch_kernel<<<grid, oasis::kPrefetchThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         d, static_cast<const uint4*>(hv), fetch_slot, fetch_block, n_fetch, static_cast<uint4*>(pool));
     return check_launch("prefetch launch");
@@ -639,20 +706,25 @@ int oasis_sparse_attn(const oasis_dims* dp, const void* q, const void* pool, con
     if (!(scale > 0.f) || !(scale < 3.0e38f)) return fail(OASIS_EINVAL, "scale must be a positive finite float");
     const WsLayout w = ws_layout(d);
     if (ws_bytes < w.total) return fail(OASIS_EINVAL, "workspace too small: %zu < %zu", ws_bytes, w.total);
-    CUtensorMap tm, tq;
-    const unsigned long long rows = static_cast<unsigned long long>(d.B) * d.Hkv * d.K * 2 * oasis::kBlockTokens;
-    if (int rc = make_map(&tm, pool, rows, oasis::kBlockTokens, "pool")) return rc;
+    CUtensorMap tk, tv, tq;
+    const unsigned long long slots = static_cast<unsigned long long>(d.B) * d.Hkv * d.K;
+    if (int rc = make_map_pool(&tk, pool, slots, "pool keys")) return rc;
+    if (int rc = make_map_pool(&tv, static_cast<const uint8_t*>(pool) + oasis::kBlockBytes / 2, slots, "pool values"))
+        return rc;
     if (int rc = make_map_q(&tq, q, d)) return rc;
     uint8_t* base = static_cast<uint8_t*>(ws);
     float* ws_lse = reinterpret_cast<float*>(base + w.lse);
     float* ws_o = reinterpret_cast<float*>(base + w.o);
     int* ws_ticket = reinterpret_cast<int*>(base + w.ticket);
+    int* ws_sched = reinterpret_cast<int*>(base + w.sched);
     const float scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (int rc = set_smem(oasis::sparse_attn_kernel, oasis::kAttnSmem, "sparse_attn smem")) return rc;
-    const long long ns = attn_streams(d);
-    oasis::sparse_attn_kernel<<<static_cast<unsigned>(ns), oasis::kAttnThreads, oasis::kAttnSmem, s>>>(
-        tm, tq, d, slot_table, ctx_len, scale_log2, static_cast<int>(ns), out, lse, ws_o, ws_lse, ws_ticket);
+    const oasis::AttnChunks chunks = attn_chunks(d, sm_count());
+    const unsigned ctas = static_cast<unsigned>(std::min(sm_count(), chunks.nc));
+    auto kern = d.Qn * d.G() <= 32 ? oasis::sparse_attn_kernel<32> : oasis::sparse_attn_kernel<64>;
+    if (int rc = set_smem(kern, oasis::kAttnSmem, "sparse_attn smem")) return rc;
+    kern<<<ctas, oasis::kAttnThreads, oasis::kAttnSmem, s>>>(tk, tv, tq, d, slot_table, ctx_len, scale_log2, chunks,
+                                                             out, lse, ws_o, ws_lse, ws_ticket, ws_sched);
     return check_launch("sparse_attn launch");
 }
 

@@ -25,32 +25,6 @@
 
 namespace oasis {
 
-__device__ __forceinline__ int block_excl_sum_any(int v, int* tmp, int* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, x, o);
-        if (lane >= o) x += n;
-    }
-    if (lane == 31) tmp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nw ? tmp[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xFFFFFFFFu, w, o);
-            if (lane >= o) w += n;
-        }
-        tmp[lane] = w;
-    }
-    __syncthreads();
-    const int incl = x + (warp > 0 ? tmp[warp - 1] : 0);
-    *total = tmp[nw - 1];
-    __syncthreads();
-    return incl - v;
-}
-
 // order: an unsigned key, smaller = evicted earlier (blk < 15 bits, N <= 32768)
 __device__ __forceinline__ unsigned long long victim_key(int slot, int blk, uint32_t order) {
     if (blk < 0) return static_cast<unsigned long long>(slot);
@@ -63,13 +37,14 @@ constexpr int kPlanThreads = 256;
 // Shared-memory ints plan_unit needs for budget K.
 __host__ __device__ constexpr int plan_smem_ints(int K) { return 9 * K; }
 
-// Plan of one (b, h) with NT threads (each loops over slots / ranks):
-// sel, st, lu point at the unit's K entries, fs/fb at its C fetch entries,
-// nf at its fetch count; scores_u (kScored) at its N block scores.  sp:
-// plan_smem_ints(K) ints of shared memory; tmp: 32 ints.
-template <int NT, bool kScored>
+// Plan of one (b, h) by a group of threads (each loops over slots /
+// ranks): sel, st, lu point at the unit's K entries, fs/fb at its C fetch
+// entries, nf at its fetch count; scores_u (kScored) at its N block scores.
+// sp: plan_smem_ints(K) ints of shared memory; tmp: 32 ints.
+template <class Grp, bool kScored>
 __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* scores_u, int32_t* st, int32_t* lu,
                           int step, int32_t* fs, int32_t* fb, int32_t* nf, int32_t* sp, int* tmp) {
+    constexpr int NT = Grp::kThreads;
     int32_t* s_st = sp;
     int32_t* s_lu = sp + K;
     int32_t* s_prot = sp + 2 * K;
@@ -79,7 +54,7 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
     uint32_t* s_ord = reinterpret_cast<uint32_t*>(sp + 6 * K);
     int32_t* s_sel = sp + 7 * K;
     int32_t* s_mpos = sp + 8 * K;          // miss flag, then the miss's position in rank order (-1: no miss)
-    const int tid = threadIdx.x;
+    const int tid = Grp::tid();
     for (int i = tid; i < K; i += NT) {
         int x = st[i];
         if (x < -1 || x >= N) {
@@ -100,7 +75,7 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
         }
         s_sel[i] = sv;
     }
-    __syncthreads();
+    Grp::sync();
     // 1. residency lookup of every selected block; hits are protected
     for (int i = tid; i < K; i += NT) {
         const int sv = s_sel[i], own = s_st[i];
@@ -113,14 +88,14 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
         if (hit >= 0) s_prot[hit] = 1;
         s_mpos[i] = (sv >= 0 && hit < 0) ? 1 : 0;
     }
-    __syncthreads();
+    Grp::sync();
     // 2. misses numbered in rank order
     int running = 0;
     for (int base = 0; base < K; base += NT) {
         const int i = base + tid;
         const int m = i < K ? s_mpos[i] : 0;
         int total;
-        const int excl = block_excl_sum_any(m, tmp, &total);     // syncs
+        const int excl = group_excl_sum<Grp>(m, tmp, &total);     // syncs
         if (i < K) s_mpos[i] = m ? running + excl : -1;
         running += total;
     }
@@ -138,7 +113,7 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
             if (rank < nF) s_vict[rank] = i;
         }
     }
-    __syncthreads();
+    Grp::sync();
     // 4. the first nF misses replace the victims in order
     for (int i = tid; i < K; i += NT) {
         const int mp = s_mpos[i];
@@ -150,7 +125,7 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
             fb[mp] = s_sel[i];
         }
     }
-    __syncthreads();
+    Grp::sync();
     for (int i = tid; i < K; i += NT) {
         st[i] = s_nst[i];
         lu[i] = s_nlu[i];
@@ -180,7 +155,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fetch_kernel(Dims d, const 
     const long long bh = blockIdx.x;
     const long long base = bh * d.K;
     if (step_dev != nullptr) step = *step_dev;
-    plan_unit<kPlanThreads, kScored>(d.K, d.C, d.N, sel + base, kScored ? scores + bh * d.N : nullptr,
+    plan_unit<CtaGroup<kPlanThreads>, kScored>(d.K, d.C, d.N, sel + base, kScored ? scores + bh * d.N : nullptr,
                                      slot_table + base, last_used + base, step, fetch_slot + bh * d.C,
                                      fetch_block + bh * d.C, n_fetch + bh, sp, tmp);
 }

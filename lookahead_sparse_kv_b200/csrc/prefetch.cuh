@@ -8,11 +8,14 @@
 // The kernel reads the pinned host KV directly over PCIe (zero-copy) and
 // writes each 8 KiB block into its pool slot, so the gather stays ordered on
 // the stream after the planner with no host round trip.  It is persistent
-// and small on purpose: a few dozen CTAs, each thread keeping eight 16-B
-// loads in flight (two blocks per CTA at a time), which covers the link's
-// bandwidth-delay product (~55 GB/s x a few microseconds) while leaving the
-// SMs and their register files to the attention and scoring kernels that run
-// beside it.  Only real fetches are visited: a CTA takes the prefix sum of
+// and small on purpose: 16 CTAs, each thread keeping eight 16-B loads in
+// flight (two blocks per CTA at a time), which covers the link's
+// bandwidth-delay product (~55 GB/s x a few microseconds).  Measured on B200:
+// 16, 32 and 64 CTAs all gather at 51 GB/s, 8 at 45 GB/s; and an attention or
+// scoring CTA that shares an SM with a gather CTA runs 1.4-2.5x slower, so
+// the fewer SMs the gather occupies the better.  Its 48 registers a thread
+// (launch bound of 10 CTAs per SM) leave room beside an attention CTA
+// (384 threads x 152 registers) in the 64K-register file.  Only real fetches are visited: a CTA takes the prefix sum of
 // the units' fetch counts (1,024 units per pass, in shared memory), numbers
 // the fetches of all units consecutively, and takes every gridDim-th pair;
 // a binary search over the prefix maps a fetch number back to (unit, entry).
@@ -25,7 +28,7 @@
 namespace oasis {
 
 constexpr int kPrefetchThreads = 128;
-constexpr int kPrefetchCtas = 32;
+constexpr int kPrefetchCtas = 16;
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     uint4 v;
@@ -50,7 +53,7 @@ __device__ __forceinline__ int prefetch_unit_of(const int* s_pre, int nu, int r)
     return lo;
 }
 
-__global__ void __launch_bounds__(kPrefetchThreads) prefetch_kernel(Dims d, const uint4* __restrict__ host_kv,
+__global__ void __launch_bounds__(kPrefetchThreads, 10) prefetch_kernel(Dims d, const uint4* __restrict__ host_kv,
                                                                     const int32_t* __restrict__ fetch_slot,
                                                                     const int32_t* __restrict__ fetch_block,
                                                                     const int32_t* __restrict__ n_fetch,

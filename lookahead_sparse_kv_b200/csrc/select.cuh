@@ -19,31 +19,6 @@ namespace oasis {
 constexpr int kSelThreads = 512;
 constexpr int kSelMaxK = 1024;
 
-// Inclusive block-wide sum over kSelThreads threads; `tmp` holds 32 ints.
-__device__ __forceinline__ int block_inclusive_sum(int v, int* tmp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, v, o);
-        if (lane >= o) v += n;
-    }
-    if (lane == 31) tmp[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < (blockDim.x >> 5) ? tmp[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xFFFFFFFFu, w, o);
-            if (lane >= o) w += n;
-        }
-        tmp[lane] = w;
-    }
-    __syncthreads();
-    const int r = v + (warp > 0 ? tmp[warp - 1] : 0);
-    __syncthreads();
-    return r;
-}
-
 // Scratch of select_unit in shared memory.
 struct SelScratch {
     int hist[256];
@@ -51,20 +26,32 @@ struct SelScratch {
     int chosen, remaining, gt, pad;
 };
 
-// Top-K of one (b, h) with NT threads: keys[0, nv) are the monotone keys of
-// the valid blocks (in shared memory, written and synced by the caller);
-// cand holds next_pow2(min(K, nv)) entries.  Writes out[0, K) (rank order,
-// -1 padded) and, if out_s is not NULL, the scores s[id] of the winners.
-template <int NT>
-__device__ void select_unit(const uint32_t* keys, int nv, int K, unsigned long long* cand, SelScratch* sc,
-                            const float* s, int32_t* out, float* out_s) {
+// Monotone keys of a unit's scores: from shared memory, or computed from the
+// fp32 scores in global memory (read through L2) when they do not fit there.
+struct SmemKeys {
+    const uint32_t* k;
+    __device__ __forceinline__ uint32_t operator()(int i) const { return k[i]; }
+};
+struct GlobalKeys {
+    const float* s;
+    __device__ __forceinline__ uint32_t operator()(int i) const { return ordered_key(__ldcg(s + i)); }
+};
+
+// Top-K of one (b, h) by a group of threads: key(i), i < nv, is the monotone
+// key of valid block i (keys in shared memory written and synced by the
+// caller); cand holds next_pow2(min(K, nv)) entries.  Writes out[0, K)
+// (rank order, -1 padded) and, if out_s is not NULL, the scores s[id] of the
+// winners.
+template <class Grp, class Key>
+__device__ void select_unit(Key key, int nv, int K, unsigned long long* cand, SelScratch* sc, const float* s,
+                            int32_t* out, float* out_s) {
+    constexpr int NT = Grp::kThreads;
     constexpr int kBpt = NT >= 256 ? 1 : 256 / NT;     // histogram bins per thread
-    const int tid = threadIdx.x;
+    const int tid = Grp::tid();
     const int take = min(K, nv);
     int kp = 1;
     while (kp < take) kp <<= 1;
-    if (tid == 0) sc->gt = 0;
-    __syncthreads();
+    Grp::sync();
 
     uint32_t T = 0;
     int need_eq = 0;
@@ -73,12 +60,20 @@ __device__ void select_unit(const uint32_t* keys, int nv, int K, unsigned long l
         int remaining = K;
         for (int shift = 24; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += NT) sc->hist[i] = 0;
-            __syncthreads();
-            for (int i = tid; i < nv; i += NT) {
-                const uint32_t u = keys[i];
-                if ((u & mask) == prefix) atomicAdd(&sc->hist[(u >> shift) & 0xFF], 1);
+            Grp::sync();
+            // scores of one unit cluster in a few bins: lanes of a warp that share a
+            // bin add to it once (one shared-memory atomic per distinct bin per warp)
+            for (int base = 0; base < nv; base += NT) {
+                const int i = base + tid;
+                int bin = -1;
+                if (i < nv) {
+                    const uint32_t u = key(i);
+                    if ((u & mask) == prefix) bin = static_cast<int>((u >> shift) & 0xFF);
+                }
+                const unsigned same = __match_any_sync(0xFFFFFFFFu, bin);
+                if (bin >= 0 && __ffs(same) - 1 == (tid & 31)) atomicAdd(&sc->hist[bin], __popc(same));
             }
-            __syncthreads();
+            Grp::sync();
             // suffix sums over bins (bin 255 first): thread t holds bins 255-t*kBpt-k
             int c[kBpt];
             int cnt = 0;
@@ -88,8 +83,8 @@ __device__ void select_unit(const uint32_t* keys, int nv, int K, unsigned long l
                 c[k] = idx < 256 ? sc->hist[255 - idx] : 0;
                 cnt += c[k];
             }
-            const int incl = block_inclusive_sum(cnt, sc->tmp);
-            int above = incl - cnt;                     // keys in bins above this thread's first bin
+            int total;
+            int above = group_excl_sum<Grp>(cnt, sc->tmp, &total);   // keys in bins above this thread's first bin
 #pragma unroll
             for (int k = 0; k < kBpt; ++k) {
                 const int idx = tid * kBpt + k;
@@ -99,37 +94,43 @@ __device__ void select_unit(const uint32_t* keys, int nv, int K, unsigned long l
                 }
                 above += c[k];
             }
-            __syncthreads();
+            Grp::sync();
             prefix |= static_cast<uint32_t>(sc->chosen) << shift;
             mask |= 0xFFu << shift;
             remaining = sc->remaining;
-            __syncthreads();
+            Grp::sync();
         }
         T = prefix;
         need_eq = remaining;
     }
 
     // Gather the winners.  Keys > T in any order (sorted below); keys == T in
-    // block-id order, the first need_eq of them.
+    // block-id order, the first need_eq of them.  Each thread takes a
+    // contiguous chunk; block scans place the chunks' winners.
     const int per = (nv + NT - 1) / NT;
     const int i0 = tid * per, i1 = min(nv, i0 + per);
-    int eq_local = 0;
+    int gt_local = 0, eq_local = 0;
     for (int i = i0; i < i1; ++i) {
-        const uint32_t u = keys[i];
-        const bool win = nv <= K || u > T;
-        if (win) {
-            const int p = atomicAdd(&sc->gt, 1);
-            cand[p] = (static_cast<unsigned long long>(~u) << 32) | static_cast<uint32_t>(i);
-        } else if (u == T) {
-            ++eq_local;
+        const uint32_t u = key(i);
+        if (nv <= K || u > T) ++gt_local;
+        else if (u == T) ++eq_local;
+    }
+    int total;
+    int p = group_excl_sum<Grp>(gt_local, sc->tmp, &total);
+    if (tid == 0) sc->gt = total;
+    for (int i = i0; i < i1 && gt_local > 0; ++i) {
+        const uint32_t u = key(i);
+        if (nv <= K || u > T) {
+            cand[p++] = (static_cast<unsigned long long>(~u) << 32) | static_cast<uint32_t>(i);
+            --gt_local;
         }
     }
-    const int eq_before = block_inclusive_sum(eq_local, sc->tmp) - eq_local;
+    const int eq_before = group_excl_sum<Grp>(eq_local, sc->tmp, &total);   // (syncs: sc->gt visible)
     const int n_gt = sc->gt;   // == take - need_eq
     if (nv > K) {
         int e = eq_before;
         for (int i = i0; i < i1 && e < need_eq; ++i) {
-            const uint32_t u = keys[i];
+            const uint32_t u = key(i);
             if (u == T) {
                 cand[n_gt + e] = (static_cast<unsigned long long>(~u) << 32) | static_cast<uint32_t>(i);
                 ++e;
@@ -137,7 +138,7 @@ __device__ void select_unit(const uint32_t* keys, int nv, int K, unsigned long l
         }
     }
     for (int i = take + tid; i < kp; i += NT) cand[i] = ~0ull;
-    __syncthreads();
+    Grp::sync();
 
     // Bitonic sort of kp entries, ascending (~key, id) = score desc, id asc.
     for (int k = 2; k <= kp; k <<= 1) {
@@ -153,7 +154,7 @@ __device__ void select_unit(const uint32_t* keys, int nv, int K, unsigned long l
                     }
                 }
             }
-            __syncthreads();
+            Grp::sync();
         }
     }
 
@@ -166,6 +167,93 @@ __device__ void select_unit(const uint32_t* keys, int nv, int K, unsigned long l
             out[i] = -1;
             if (out_s) out_s[i] = -__int_as_float(0x7f800000);
         }
+    }
+}
+
+// Fast path of select_unit for nv <= 2048 blocks and K <= 128, by a group of
+// 4 warps.  Warp w bitonic-sorts the composites (~key << 32 | id) of blocks
+// [512w, 512w + 512) in registers (16 per lane, element e = 16*lane + j;
+// strides below 16 stay in a lane, larger ones exchange with lane ^
+// (stride / 16)); ascending composites are descending scores with ties to the
+// lower id, the order select_unit produces.  Each warp's first 128 entries go
+// to cand[128w ..]; a candidate's rank among the four heads is its position
+// plus, in each other head, the number of smaller entries (binary search), and
+// the first K ranks are written in rank order.  key(i) gives block i's
+// monotone key; cand holds 512 entries.
+constexpr int kSelFastMaxN = 2048, kSelFastMaxK = 128;
+
+template <class Grp, class Key>
+__device__ void select_unit_fast(Key key, int nv, int K, unsigned long long* cand, const float* s, int32_t* out,
+                                 float* out_s) {
+    static_assert(Grp::kThreads == 128, "four warps");
+    const int t = Grp::tid(), lane = t & 31, w = t >> 5;
+    unsigned long long v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int i = 512 * w + 16 * lane + j;
+        v[j] = i < nv ? (static_cast<unsigned long long>(~key(i)) << 32) | static_cast<uint32_t>(i) : ~0ull;
+    }
+#pragma unroll
+    for (int k = 2; k <= 512; k <<= 1) {
+#pragma unroll
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+            if (jj < 16) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int pj = j ^ jj;
+                    if (pj > j) {
+                        const bool asc = ((16 * lane + j) & k) == 0;
+                        const unsigned long long a = v[j], b = v[pj];
+                        const bool sw = (a > b) == asc;
+                        v[j] = sw ? b : a;
+                        v[pj] = sw ? a : b;
+                    }
+                }
+            } else {
+                const int lm = jj >> 4;
+                const bool lower = (lane & lm) == 0;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const bool asc = ((16 * lane + j) & k) == 0;
+                    const unsigned long long o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
+                    const bool keep_min = lower == asc;
+                    v[j] = keep_min ? (v[j] < o ? v[j] : o) : (v[j] < o ? o : v[j]);
+                }
+            }
+        }
+    }
+    if (lane < 8) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cand[128 * w + 16 * lane + j] = v[j];
+    }
+    Grp::sync();
+    const int take = min(K, nv);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        const int idx = t + 128 * c4, lst = idx >> 7, p = idx & 127;
+        const unsigned long long c = cand[idx];
+        if (c == ~0ull) continue;                      // past the unit's blocks
+        int rank = p;
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+            if (o == lst) continue;
+            const unsigned long long* L = cand + 128 * o;
+            int lo = 0, hi = 128;                      // entries of L below c
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (L[mid] < c) lo = mid + 1; else hi = mid;
+            }
+            rank += lo;
+        }
+        if (rank < take) {
+            const int id = static_cast<int>(c & 0xFFFFFFFFu);
+            out[rank] = id;
+            if (out_s) out_s[rank] = __ldcg(s + id);
+        }
+    }
+    for (int i = take + t; i < K; i += 128) {
+        out[i] = -1;
+        if (out_s) out_s[i] = -__int_as_float(0x7f800000);
     }
 }
 
@@ -182,8 +270,8 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(Dims d, const 
     const float* s = scores + static_cast<long long>(bh) * d.N;
     for (int i = tid; i < nv; i += kSelThreads) keys[i] = ordered_key(s[i]);
     __syncthreads();
-    select_unit<kSelThreads>(keys, nv, d.K, cand, &sc, s, sel + static_cast<long long>(bh) * d.K,
-                             sel_score ? sel_score + static_cast<long long>(bh) * d.K : nullptr);
+    select_unit<CtaGroup<kSelThreads>>(SmemKeys{keys}, nv, d.K, cand, &sc, s, sel + static_cast<long long>(bh) * d.K,
+                                       sel_score ? sel_score + static_cast<long long>(bh) * d.K : nullptr);
 }
 
 }  // namespace oasis
