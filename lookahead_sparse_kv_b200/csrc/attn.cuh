@@ -10,14 +10,15 @@
 // 64) and K pool slots of 16 tokens.  Decode has few query rows and many
 // tokens, so the tokens are the MMA's M dimension:
 //   S^T [128 tokens x NR]   = K_tile [128 x 128] . Q^T        8 MMAs, both K-major
-//   O^T [128 dims x NR]    += V_tile^T . P^T [128 tokens x NR]
-//                             two MMAs per occupied slot (16 tokens), both
+//   O^T [128 dims x 2 NR]  += V_tile^T . [P_head | P_rest]^T [128 tokens x 2 NR]
+//                             one MMA per occupied slot (16 tokens), both
 //                             operands MN-major: V is read in place, P^T is
-//                             written one 128-B row per token as a bf16 head
-//                             and a bf16 remainder (~16 significant bits); with
-//                             32 rows head and remainder share the row (the
-//                             remainder's MMA starts 64 B in) and P^T is
-//                             double-buffered, with 64 they take a row each
+//                             written one row per token as a bf16 head and a
+//                             bf16 remainder (~16 significant bits), side by
+//                             side along N, so head and remainder products land
+//                             in two column ranges that the epilogue adds; with
+//                             32 rows the two share a 128-B row and P^T is
+//                             double-buffered, with 64 they take a region each
 // NR = 32 or 64 is the row count padded to the MMA's N.  A tile is 8 pool
 // slots (128 tokens).  In TMEM, lane i of S^T is token i of the tile (a
 // softmax thread owns a token and reads its NR scores), lane i of O^T is
@@ -69,7 +70,7 @@ constexpr int kAttnMaxChunkTiles = 16;
 constexpr int kAttnInfoInts = 8 + 4 * kAttnMaxChunkTiles;          // chunk header + 4 ints per tile
 constexpr int kAttnLoaderWarp = 8, kAttnSWarp = 9, kAttnOWarp = 10, kAttnListerWarp = 11;
 constexpr int kAttnThreads = 32 * 12;
-constexpr int kAttnTmemCols = 256;                                 // S^T x 2, O^T x 2 (64 columns each)
+constexpr int kAttnTmemCols = 512;                                 // S^T x 2 (64 columns each), O^T x 2 (2 NR each), row sums
 constexpr float kLn2 = 0.6931471805599453f;
 
 // shared memory, from the 1024-B aligned base
@@ -88,7 +89,8 @@ constexpr int kAttnOffLw = kAttnOffWmax + 4 * 64 * 4;              // [2][4][64]
 constexpr int kAttnOffFin = kAttnOffLw + 2 * 4 * 64 * 4;           // [2][64] 1/sum, [2][64] log2-sum-exp
 constexpr int kAttnMaxChunks = 8;                                  // chunks per unit (merge weights)
 constexpr int kAttnOffMw = kAttnOffFin + 4 * 64 * 4;               // [64][8] merge weights
-constexpr int kAttnSmem = kAttnOffMw + 64 * kAttnMaxChunks * 4 + 1024;   // + alignment slack
+constexpr int kAttnOffThr = kAttnOffMw + 64 * kAttnMaxChunks * 4;  // [2][64] raw-score thresholds
+constexpr int kAttnSmem = kAttnOffThr + 2 * 64 * 4 + 1024;         // + alignment slack
 
 // mbarriers ([2] = one per ring stage / buffer)
 constexpr int kBarKFull = 0;     // K tile landed (producer expect_tx)
@@ -159,7 +161,9 @@ __global__ void __maxnreg__(152)
     // 0-63 of the row before swizzling) and the remainder (64-127), two
     // buffers; with 64 rows head and remainder fill one region each, one buffer.
     constexpr int kPBufs = NR == 32 ? 2 : 1;
-    constexpr uint32_t kRestOff = NR == 32 ? 64u : static_cast<uint32_t>(kAttnHalf);
+    // TMEM columns: S^T buffers at 0 and 64, O^T buffers (head and remainder
+    // products side by side) at 128 and 128 + 2 NR, 64-row sums after them
+    constexpr uint32_t kOCol = 128, kOStride = 2 * NR, kLCol = 128 + 2 * 2 * NR;
     const float kNegInf = -__int_as_float(0x7f800000);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -179,6 +183,7 @@ __global__ void __maxnreg__(152)
     float* s_lw = reinterpret_cast<float*>(smem + kAttnOffLw);
     float* s_fin = reinterpret_cast<float*>(smem + kAttnOffFin);
     float* s_mw = reinterpret_cast<float*>(smem + kAttnOffMw);
+    float* s_thr = reinterpret_cast<float*>(smem + kAttnOffThr);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int K = d.K;
@@ -367,7 +372,7 @@ __global__ void __maxnreg__(152)
     } else if (warp == kAttnOWarp) {
         // ======================================== O^T += V^T . P^T issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_bf16_f32_amn_bmn(kHeadDim, NR);
+            constexpr uint32_t idesc = umma_idesc_bf16_f32_amn_bmn(kHeadDim, 2 * NR);
             int pv = 0;
             for (int p = 0;; ++p) {
                 const int pb = p & 1;
@@ -376,7 +381,7 @@ __global__ void __maxnreg__(152)
                 const int n = info[0];
                 if (n < 0) break;
                 if (p >= 2) cta_wait(&bar[kBarOFree + pb], ((p >> 1) - 1) & 1, s_abort);
-                const uint32_t d_o = tmem + 128 + pb * 64;
+                const uint32_t d_o = tmem + kOCol + pb * kOStride;
                 bool fresh = true;                                // the chunk's first product overwrites O^T
                 for (int i = 0; i < n; ++i, ++pv) {
                     const int st = pv & 1;
@@ -394,11 +399,8 @@ __global__ void __maxnreg__(152)
                             const uint32_t nv = ((kk < 4 ? nvlo : nvhi) >> (8 * (kk & 3))) & 0xFFu;
                             if (nv == 0) continue;                // free slot: no product
                             const uint32_t off = kk * kBlockTokens * 128;
-                            const uint64_t ad = umma_desc_sw128_lbo_sbo(va + off, kAttnHalf, 1024);
-                            umma_bf16(d_o, ad, umma_desc_sw128_lbo_sbo(pa + off, kAttnHalf, 1024), idesc,
-                                      fresh ? 0u : 1u);
-                            umma_bf16(d_o, ad, umma_desc_sw128_lbo_sbo(pa + kRestOff + off, kAttnHalf, 1024), idesc,
-                                      1u);
+                            umma_bf16(d_o, umma_desc_sw128_lbo_sbo(va + off, kAttnHalf, 1024),
+                                      umma_desc_sw128_lbo_sbo(pa + off, kAttnHalf, 1024), idesc, fresh ? 0u : 1u);
                             fresh = false;
                         }
                     }
@@ -427,20 +429,34 @@ __global__ void __maxnreg__(152)
             if (named_bar_or(kNbSoftmaxVote, 128, n < 0 || *s_abort)) break;
             // the epilogue of chunk p-2 has read this buffer's running max and sums
             if (p >= 2) cta_wait(&bar[kBarOFree + pb], ((p >> 1) - 1) & 1, s_abort);
+            // running max m (log2 units) and the raw-score threshold (m + 8) / scale of
+            // every row; rows past the real ones have both at +inf, so their scores never
+            // vote and their probabilities are 0 (the padded columns are never read)
             float* mr = s_m + pb * 64;
-            if (q == 0) {                                     // rows past the real ones stay at 0
-                mr[lane] = lane < rows ? kNegInf : 0.f;
-                mr[lane + 32] = lane + 32 < rows ? kNegInf : 0.f;
+            float* thr = s_thr + pb * 64;
+            if (q == 0) {
+                const float kPosInf = __int_as_float(0x7f800000);
+                mr[lane] = lane < rows ? kNegInf : kPosInf;
+                mr[lane + 32] = lane + 32 < rows ? kNegInf : kPosInf;
+                thr[lane] = mr[lane];
+                thr[lane + 32] = mr[lane + 32];
             }
             named_bar_sync(kNbSoftmax, 128);
-            // row sums: with 32 rows each thread keeps its token's sums (reduced over the
-            // warp at the chunk's end); with 64, to save registers, every tile's sums are
-            // reduced over the warp at once and lane t keeps rows t and t + 32
-            constexpr int kL = NR == 32 ? 32 : 1;
-            float l[kL];
+            // this token's share of the row sums: registers with 32 rows, TMEM columns
+            // of the token's lane with 64 (registers are short there)
+            constexpr bool kLT = NR == 64;
+            const uint32_t l_addr = tmem + lane_base + kLCol;
+            float l[kLT ? 1 : NR];
 #pragma unroll
-            for (int r = 0; r < kL; ++r) l[r] = 0.f;
-            float lsc0 = 0.f, lsc1 = 0.f;
+            for (int r = 0; r < (kLT ? 1 : NR); ++r) l[r] = 0.f;
+            if constexpr (kLT) {
+                uint32_t z[32];
+#pragma unroll
+                for (int r = 0; r < 32; ++r) z[r] = 0u;
+                tmem_st_32x32b_x32(l_addr, z);
+                tmem_st_32x32b_x32(l_addr + 32, z);
+                tmem_st_wait();
+            }
             for (int i = 0; i < n; ++i, ++pos) {
                 const int st = pos & 1;
                 const int* e = info + 8 + 4 * i;
@@ -448,20 +464,18 @@ __global__ void __maxnreg__(152)
                 const bool valid = mytok < nvj;
                 cta_wait(&bar[kBarSFull + st], (pos >> 1) & 1, s_abort);
                 tc_fence_after_sync();
-                float x[NR];
+                float x[NR];                                  // raw scores q.k of this token
                 {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tmem + lane_base + st * 64, v);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int r = 0; r < 32; ++r)
-                        x[r] = (valid && r < rows) ? __uint_as_float(v[r]) * scale_log2 : kNegInf;
+                    for (int r = 0; r < 32; ++r) x[r] = __uint_as_float(v[r]);
                     if constexpr (NR == 64) {
                         tmem_ld_32x32b_x32(tmem + lane_base + st * 64 + 32, v);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int r = 0; r < 32; ++r)
-                            x[32 + r] = (valid && 32 + r < rows) ? __uint_as_float(v[r]) * scale_log2 : kNegInf;
+                        for (int r = 0; r < 32; ++r) x[32 + r] = __uint_as_float(v[r]);
                     }
                 }
                 tc_fence_before_sync();
@@ -469,19 +483,21 @@ __global__ void __maxnreg__(152)
                 if (lane == 0) mbar_arrive(&bar[kBarSFree + st]);
                 // does any row's running max move (by more than 2^8)?
                 bool up = false;
+                if (valid) {
 #pragma unroll
-                for (int r = 0; r < NR; r += 4) {
-                    const float4 m4 = *reinterpret_cast<const float4*>(mr + r);
-                    up |= (x[r] > m4.x + 8.f) | (x[r + 1] > m4.y + 8.f) | (x[r + 2] > m4.z + 8.f) |
-                          (x[r + 3] > m4.w + 8.f);
+                    for (int r = 0; r < NR; r += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(thr + r);
+                        up |= (x[r] > t4.x) | (x[r + 1] > t4.y) | (x[r + 2] > t4.z) | (x[r + 3] > t4.w);
+                    }
                 }
                 if (named_bar_or(kNbSoftmaxVote, 128, up)) {
-                    // tile maxima: lane t of each warp gets rows t and t + 32 over its tokens
+                    // tile maxima (log2 units): lane t of each warp gets rows t and t + 32
 #pragma unroll
                     for (int hh = 0; hh < NR / 32; ++hh) {
                         float t[32];
 #pragma unroll
-                        for (int r = 0; r < 32; ++r) t[r] = x[32 * hh + r];
+                        for (int r = 0; r < 32; ++r)
+                            t[r] = (valid && 32 * hh + r < rows) ? x[32 * hh + r] * scale_log2 : kNegInf;
                         s_wmax[q * 64 + 32 * hh + lane] = warp_reduce_scatter32<true>(t, lane);
                     }
                     named_bar_sync(kNbSoftmax, 128);
@@ -492,34 +508,45 @@ __global__ void __maxnreg__(152)
                             const float tmx = fmaxf(fmaxf(s_wmax[r], s_wmax[64 + r]), fmaxf(s_wmax[128 + r], s_wmax[192 + r]));
                             const float mo = mr[r];
                             float a = 1.f;
-                            if (tmx > mo + 8.f) {
+                            if (r < rows && tmx > mo + 8.f) {
                                 a = attn_exp2(mo - tmx);              // 0 on the chunk's first tile
                                 mr[r] = tmx;
+                                thr[r] = (tmx + 8.f) / scale_log2;
                             }
                             s_alpha[r] = a;
                         }
                     }
                     named_bar_sync(kNbSoftmax, 128);
-                    if constexpr (NR == 32) {
+                    if constexpr (kLT) {
 #pragma unroll
-                        for (int r = 0; r < 32; ++r) l[r] *= s_alpha[r];
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t lv[32];
+                            tmem_ld_32x32b_x32(l_addr + 32 * hh, lv);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int r = 0; r < 32; ++r)
+                                lv[r] = __float_as_uint(__uint_as_float(lv[r]) * s_alpha[32 * hh + r]);
+                            tmem_st_32x32b_x32(l_addr + 32 * hh, lv);
+                        }
+                        tmem_st_wait();
                     } else {
-                        lsc0 *= s_alpha[lane];
-                        lsc1 *= s_alpha[32 + lane];
+#pragma unroll
+                        for (int r = 0; r < NR; ++r) l[r] *= s_alpha[r];
                     }
                     if (i > 0) {
                         // the previous tile's product must have landed in O^T before it is rescaled
                         cta_wait(&bar[kBarPFree + (pos - 1) % kPBufs], ((pos - 1) / kPBufs) & 1, s_abort);
                         tc_fence_after_sync();
 #pragma unroll
-                        for (int hh = 0; hh < NR / 32; ++hh) {
-                            const uint32_t oaddr = tmem + lane_base + 128 + pb * 64 + 32 * hh;
+                        for (int hh = 0; hh < 2 * NR / 32; ++hh) {            // head and remainder columns
+                            const uint32_t oaddr = tmem + lane_base + kOCol + pb * kOStride + 32 * hh;
+                            const int r0 = (32 * hh) % NR;
                             uint32_t o[32];
                             tmem_ld_32x32b_x32(oaddr, o);
                             tmem_ld_wait();
 #pragma unroll
                             for (int r = 0; r < 32; ++r)
-                                o[r] = __float_as_uint(__uint_as_float(o[r]) * s_alpha[32 * hh + r]);
+                                o[r] = __float_as_uint(__uint_as_float(o[r]) * s_alpha[r0 + r]);
                             tmem_st_32x32b_x32(oaddr, o);
                         }
                         tmem_st_wait();
@@ -530,73 +557,105 @@ __global__ void __maxnreg__(152)
                 const int pbuf = pos % kPBufs;
                 if (pos >= kPBufs) cta_wait(&bar[kBarPFree + pbuf], ((pos / kPBufs) - 1) & 1, s_abort);
                 uint8_t* prow = sP + pbuf * kAttnHalf + tok * 128;
+                if (valid) {
 #pragma unroll
-                for (int c8 = 0; c8 < NR / 8; ++c8) {
-                    const float4 ma = *reinterpret_cast<const float4*>(mr + 8 * c8);
-                    const float4 mb = *reinterpret_cast<const float4*>(mr + 8 * c8 + 4);
-                    const int r = 8 * c8;
-                    const float p0 = attn_exp2(x[r + 0] - ma.x), p1 = attn_exp2(x[r + 1] - ma.y);
-                    const float p2 = attn_exp2(x[r + 2] - ma.z), p3 = attn_exp2(x[r + 3] - ma.w);
-                    const float p4 = attn_exp2(x[r + 4] - mb.x), p5 = attn_exp2(x[r + 5] - mb.y);
-                    const float p6 = attn_exp2(x[r + 6] - mb.z), p7 = attn_exp2(x[r + 7] - mb.w);
-                    if constexpr (NR == 32) {
-                        l[r + 0] += p0;
-                        l[r + 1] += p1;
-                        l[r + 2] += p2;
-                        l[r + 3] += p3;
-                        l[r + 4] += p4;
-                        l[r + 5] += p5;
-                        l[r + 6] += p6;
-                        l[r + 7] += p7;
-                    } else {
-                        x[r + 0] = p0;
-                        x[r + 1] = p1;
-                        x[r + 2] = p2;
-                        x[r + 3] = p3;
-                        x[r + 4] = p4;
-                        x[r + 5] = p5;
-                        x[r + 6] = p6;
-                        x[r + 7] = p7;
+                    for (int c8 = 0; c8 < NR / 8; ++c8) {
+                        const float4 ma = *reinterpret_cast<const float4*>(mr + 8 * c8);
+                        const float4 mb = *reinterpret_cast<const float4*>(mr + 8 * c8 + 4);
+                        const int r = 8 * c8;
+                        const float p0 = attn_exp2(fmaf(x[r + 0], scale_log2, -ma.x));
+                        const float p1 = attn_exp2(fmaf(x[r + 1], scale_log2, -ma.y));
+                        const float p2 = attn_exp2(fmaf(x[r + 2], scale_log2, -ma.z));
+                        const float p3 = attn_exp2(fmaf(x[r + 3], scale_log2, -ma.w));
+                        const float p4 = attn_exp2(fmaf(x[r + 4], scale_log2, -mb.x));
+                        const float p5 = attn_exp2(fmaf(x[r + 5], scale_log2, -mb.y));
+                        const float p6 = attn_exp2(fmaf(x[r + 6], scale_log2, -mb.z));
+                        const float p7 = attn_exp2(fmaf(x[r + 7], scale_log2, -mb.w));
+                        if constexpr (kLT) {
+                            x[r + 0] = p0;
+                            x[r + 1] = p1;
+                            x[r + 2] = p2;
+                            x[r + 3] = p3;
+                            x[r + 4] = p4;
+                            x[r + 5] = p5;
+                            x[r + 6] = p6;
+                            x[r + 7] = p7;
+                        } else {
+                            l[r + 0] += p0;
+                            l[r + 1] += p1;
+                            l[r + 2] += p2;
+                            l[r + 3] += p3;
+                            l[r + 4] += p4;
+                            l[r + 5] += p5;
+                            l[r + 6] += p6;
+                            l[r + 7] += p7;
+                        }
+                        const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+                        const uint32_t h45 = pack_bf16x2(p4, p5), h67 = pack_bf16x2(p6, p7);
+                        const int off = (c8 ^ (tok & 7)) << 4;
+                        const int roff = NR == 32 ? (((c8 + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
+                        *reinterpret_cast<uint4*>(prow + off) = make_uint4(h01, h23, h45, h67);
+                        *reinterpret_cast<uint4*>(prow + roff) =
+                            make_uint4(pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01)),
+                                       pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23)),
+                                       pack_bf16x2(p4 - bf16_lo(h45), p5 - bf16_hi(h45)),
+                                       pack_bf16x2(p6 - bf16_lo(h67), p7 - bf16_hi(h67)));
                     }
-                    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
-                    const uint32_t h45 = pack_bf16x2(p4, p5), h67 = pack_bf16x2(p6, p7);
-                    const int off = (c8 ^ (tok & 7)) << 4;
-                    const int roff = NR == 32 ? (((c8 + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
-                    *reinterpret_cast<uint4*>(prow + off) = make_uint4(h01, h23, h45, h67);
-                    *reinterpret_cast<uint4*>(prow + roff) =
-                        make_uint4(pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01)),
-                                   pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23)),
-                                   pack_bf16x2(p4 - bf16_lo(h45), p5 - bf16_hi(h45)),
-                                   pack_bf16x2(p6 - bf16_lo(h67), p7 - bf16_hi(h67)));
-                }
-                // a value row past the context in an occupied slot reads as zero (its weight is
-                // zero, and zero times a non-finite stale value is not)
-                if (!valid && nvj > 0) {
-                    cta_wait(&bar[kBarVFull + st], (pos >> 1) & 1, s_abort);   // orders the copy first
-                    uint8_t* vrow = sV + st * kAttnStageBytes + tok * 128;
+                } else {
+                    // a token past the context or in a free slot: zero weights; in an occupied
+                    // slot its value row reads as zero too (zero times a stale non-finite
+                    // value is not zero)
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        *reinterpret_cast<uint4*>(vrow + 16 * k) = make_uint4(0u, 0u, 0u, 0u);
-                        *reinterpret_cast<uint4*>(vrow + kAttnHalf + 16 * k) = make_uint4(0u, 0u, 0u, 0u);
+                    for (int c8 = 0; c8 < NR / 8; ++c8) {
+                        const int off = (c8 ^ (tok & 7)) << 4;
+                        const int roff = NR == 32 ? (((c8 + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
+                        *reinterpret_cast<uint4*>(prow + off) = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(prow + roff) = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    if (nvj > 0) {
+                        cta_wait(&bar[kBarVFull + st], (pos >> 1) & 1, s_abort);   // orders the copy first
+                        uint8_t* vrow = sV + st * kAttnStageBytes + tok * 128;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            *reinterpret_cast<uint4*>(vrow + 16 * k) = make_uint4(0u, 0u, 0u, 0u);
+                            *reinterpret_cast<uint4*>(vrow + kAttnHalf + 16 * k) = make_uint4(0u, 0u, 0u, 0u);
+                        }
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[kBarPFull + pbuf]);
-                if constexpr (NR == 64) {                     // x now holds the probabilities
-                    lsc0 += warp_reduce_scatter32<false>(*reinterpret_cast<float(*)[32]>(x), lane);
-                    lsc1 += warp_reduce_scatter32<false>(*reinterpret_cast<float(*)[32]>(x + 32), lane);
+                if constexpr (kLT) {                          // x holds the probabilities now
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t lv[32];
+                        tmem_ld_32x32b_x32(l_addr + 32 * hh, lv);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int r = 0; r < 32; ++r)
+                            lv[r] = __float_as_uint(__uint_as_float(lv[r]) + (valid ? x[32 * hh + r] : 0.f));
+                        tmem_st_32x32b_x32(l_addr + 32 * hh, lv);
+                    }
+                    tmem_st_wait();
                 }
             }
             // the chunk's row sums over this warp's tokens: lane t gets rows t and t + 32
             float* lw = s_lw + (pb * 4 + q) * 64;
-            if constexpr (NR == 32) {
-                lw[lane] = warp_reduce_scatter32<false>(l, lane);
-                lw[32 + lane] = 0.f;
+            if constexpr (kLT) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t lv[32];
+                    tmem_ld_32x32b_x32(l_addr + 32 * hh, lv);
+                    tmem_ld_wait();
+                    float t[32];
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) t[r] = __uint_as_float(lv[r]);
+                    lw[32 * hh + lane] = warp_reduce_scatter32<false>(t, lane);
+                }
             } else {
-                lw[lane] = lsc0;
-                lw[32 + lane] = lsc1;
+                lw[lane] = warp_reduce_scatter32<false>(*reinterpret_cast<float(*)[32]>(l), lane);
+                lw[32 + lane] = 0.f;
             }
             __syncwarp();
             if (lane == 0) {
@@ -634,12 +693,13 @@ __global__ void __maxnreg__(152)
             float o[NR];
             if (n > 0) {
 #pragma unroll
-                for (int hh = 0; hh < NR / 32; ++hh) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem + lane_base + 128 + pb * 64 + 32 * hh, v);
+                for (int hh = 0; hh < NR / 32; ++hh) {                 // head + remainder products
+                    uint32_t v[32], w[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + kOCol + pb * kOStride + 32 * hh, v);
+                    tmem_ld_32x32b_x32(tmem + lane_base + kOCol + pb * kOStride + NR + 32 * hh, w);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int r = 0; r < 32; ++r) o[32 * hh + r] = __uint_as_float(v[r]);
+                    for (int r = 0; r < 32; ++r) o[32 * hh + r] = __uint_as_float(v[r]) + __uint_as_float(w[r]);
                 }
             } else {
 #pragma unroll

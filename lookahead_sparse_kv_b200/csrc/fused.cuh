@@ -17,20 +17,24 @@
 // one after another through the launch and a CTA slowed down by a neighbour
 // on its SM simply takes fewer chunks.  Warps are specialised:
 //   warp 0    producer: takes a chunk, streams its 64 KiB summary tiles
-//             through a 2-stage TMA ring and builds the unit's [q+ | q-]
-//             operand (double buffered when it fits);
+//             through a 2-stage TMA ring, and TMA-loads the unit's query
+//             rows into the operand buffer (double buffered when it fits),
+//             where it splits them into [q+ | q-] in place;
 //   warp 1    one thread issues the 16 tcgen05.mma of each tile into one of
 //             two TMEM accumulators;
 //   warps 2-5 read the accumulators back (one TMEM lane quadrant each: 32
 //             blocks per warp), take the max over the real columns and store
-//             the fp32 scores; after a chunk they take a ticket on the unit's
-//             counter, and the chunk that completes the unit hands it to
-//   warps 6-9 which read the unit's scores back from L2 into shared memory
-//             and run the top-K selection (select_unit) and the plan
-//             (plan_unit) while the other warps score on.
+//             the fp32 scores; after a chunk they add one to the unit's
+//             ticket;
+//   warps 6-9 claim units in order from a second counter (so every CTA
+//             selects and plans about B*Hkv / CTAs units, whichever CTAs
+//             scored them), wait until the unit's ticket shows all its chunks
+//             scored, read its scores back from L2 into shared memory and run
+//             the top-K selection (select_unit) and the plan (plan_unit),
+//             while the other warps score on.
 // Results are those of the separate lookahead_score / select_topk / plan
 // kernels bit for bit (the same MMA, the same select_unit and plan_unit).
-// The last CTA to exit resets the chunk counter for the next call.
+// The last CTA to exit resets the counters for the next call.
 #pragma once
 
 #include "common.cuh"
@@ -54,12 +58,11 @@ constexpr int kSspAccFull = 4;    // [2] accumulator written
 constexpr int kSspAccFree = 6;    // [2] accumulator read (4 epilogue warps)
 constexpr int kSspBFull = 8;      // [2] unit operand built
 constexpr int kSspBFree = 10;     // [2] unit operand no longer read
-constexpr int kSspDecFull = 12;   // [2] chunk decided (epilogue leader): tail or not
-constexpr int kSspDecFree = 14;   // [2] decision consumed (tail leader)
-constexpr int kSspCFull = 16;     // [2] chunk description written (producer)
-constexpr int kSspCFree = 18;     // [2] description read (MMA issuer, epilogue leader)
-constexpr int kSspFinal = 20;
-constexpr int kSspNumBars = 21;
+constexpr int kSspQFull = 12;     // [2] unit's query rows landed in the operand buffer
+constexpr int kSspCFull = 14;     // [2] chunk description written (producer)
+constexpr int kSspCFree = 16;     // [2] description read (MMA issuer, epilogue leader)
+constexpr int kSspFinal = 18;
+constexpr int kSspNumBars = 19;
 constexpr uint32_t kSspNbEpiVote = 3;                      // named barrier of the epilogue's stop vote
 
 // Chunking of the scoring work (host and device agree through these).
@@ -75,13 +78,13 @@ struct SspSmem {
     static constexpr int kOffB = kSspStages * kSspTileBytes;
     static constexpr int kOffBar(int nbuf) { return kOffB + nbuf * kBBytes; }
     static constexpr int kOffMisc(int nbuf) { return kOffBar(nbuf) + kSspNumBars * 8; }   // 64 ints
-    static constexpr int kOffCand(int nbuf) { return kOffMisc(nbuf) + 256; }
+    static constexpr int kOffCand(int nbuf) { return (kOffMisc(nbuf) + 256 + 15) / 16 * 16; }
     static constexpr int kAccStride = NPAD <= 16 ? 16 : (NPAD <= 32 ? 32 : 64);   // TMEM columns per accumulator
     static constexpr int kTmemCols = 2 * kAccStride < 32 ? 32 : 2 * kAccStride;
     // total dynamic bytes for nbuf operand buffers, budget K and N blocks
     // (candidates, plan scratch, the unit's keys; +1024 alignment slack)
     static constexpr int bytes(int nbuf, int K, int N) {
-        int kp = 1;
+        int kp = 2;                                  // >= 2 keeps the plan scratch 16-B aligned
         while (kp < K) kp <<= 1;
         return kOffCand(nbuf) + kp * 8 + plan_smem_ints(K) * 4 + N * 4 + 1024;
     }
@@ -89,7 +92,8 @@ struct SspSmem {
 
 template <int NPAD, bool kScored>
 __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
-    const __grid_constant__ CUtensorMap tm_kmax, const __grid_constant__ CUtensorMap tm_kmin, Dims d,
+    const __grid_constant__ CUtensorMap tm_kmax, const __grid_constant__ CUtensorMap tm_kmin,
+    const __grid_constant__ CUtensorMap tm_q, Dims d,
     const uint16_t* __restrict__ q, const int32_t* __restrict__ ctx_len, float* scores, int row0, int rows,
     int* ticket, int* sched, int32_t* sel, float* sel_score, int32_t* slot_table, int32_t* last_used, int step,
     const int32_t* __restrict__ step_dev, int32_t* fetch_slot, int32_t* fetch_block, int32_t* n_fetch,
@@ -106,11 +110,11 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc);
     volatile int* s_abort = misc + 1;
     int* s_info = misc + 8;                               // [2][kSspInfoInts] chunk descriptions
-    volatile int* s_dec = misc + 24;                      // [2][4] decisions (mine, unit, nv, end) + a copy
+    volatile int* s_claim = misc + 24;                    // the tail group's claimed unit
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + S::kOffCand(nbuf));
-    int kp = 1;
+    int kp = 2;
     while (kp < d.K) kp <<= 1;
-    int32_t* sp = reinterpret_cast<int32_t*>(cand + kp);
+    int32_t* sp = reinterpret_cast<int32_t*>(cand + kp);   // 16-B aligned
     uint32_t* keys = reinterpret_cast<uint32_t*>(sp + plan_smem_ints(d.K));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -139,8 +143,10 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
         if (lane == 0) {
             prefetch_tensormap(&tm_kmax);
             prefetch_tensormap(&tm_kmin);
+            prefetch_tensormap(&tm_q);
         }
         const uint64_t pol = l2_policy_evict_first();
+        const uint64_t pol_q = l2_policy_evict_last();
         int pos = 0, nb = 0;
         int last_pos[kSspStages] = {-1, -1};
         // tile t of unit u into the ring (lane 0)
@@ -159,6 +165,8 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             }
             ++pos;
         };
+        int c_next = 0;                                    // requested one chunk ahead
+        if (lane == 0) c_next = atomicAdd(sched, 1);
         for (int p = 0;; ++p) {
             const int pb = p & 1;
             int* info = s_info + pb * kSspInfoInts;
@@ -166,7 +174,10 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             // the next chunk that holds valid blocks (every unit has one: its chunk 0)
             int u = 0, nv = 0, t0 = 0, vt = 0, c = 0;
             while (true) {
-                if (lane == 0) c = *s_abort ? ch.nc : atomicAdd(sched, 1);
+                if (lane == 0) {
+                    c = *s_abort ? ch.nc : c_next;
+                    if (c < ch.nc) c_next = atomicAdd(sched, 1);
+                }
                 c = __shfl_sync(0xFFFFFFFFu, c, 0);
                 if (c >= ch.nc) break;
                 u = c / ch.cpu;
@@ -198,33 +209,27 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             }
             __syncwarp();
             if (ts > t0) {
-                // [q+ | q-] of the unit's scored rows, four 64-column regions, 128-byte swizzled
+                // [q+ | q-] of the unit's scored rows in four 64-column regions (128-byte
+                // swizzle): the rows land in the q+ regions by TMA, and each 16-B piece is
+                // split there, its negative lanes going to the same place in the q- regions
                 const int b = u / d.Hkv, h = u - b * d.Hkv;
                 const int bb = nb % nbuf;
-                if (lane == 0 && nb >= nbuf) cta_wait(&bar[kSspBFree + bb], ((nb / nbuf) - 1) & 1, s_abort);
-                __syncwarp();
                 uint8_t* bt = bbuf + bb * S::kBBytes;
-                // NPAD*16 16-B pieces, 32 lanes: loads go out in batches of 8 per lane
-                constexpr int kPer = NPAD / 2, kBatch = kPer < 8 ? kPer : 8;
-#pragma unroll
-                for (int i0 = 0; i0 < kPer; i0 += kBatch) {
-                  uint4 vb[kBatch];
-#pragma unroll
-                  for (int k = 0; k < kBatch; ++k) {
-                    const int it = lane + 32 * (i0 + k);
-                    const int r = it >> 4, cc16 = it & 15;
-                    vb[k] = make_uint4(0, 0, 0, 0);
-                    if (r < rows) {
-                        const int j = row0 + r / G, g = r % G;
-                        vb[k] = *reinterpret_cast<const uint4*>(
-                            q + ((static_cast<long long>(b) * d.Qn + j) * d.Hq + h * G + g) * kHeadDim + cc16 * 8);
+                if (lane == 0) {
+                    if (nb >= nbuf) cta_wait(&bar[kSspBFree + bb], ((nb / nbuf) - 1) & 1, s_abort);
+                    mbar_arrive_expect_tx(&bar[kSspQFull + bb], static_cast<uint32_t>(rows) * kRowBytes);
+                    if (!*s_abort) {
+                        tma_load_3d(bt, &tm_q, &bar[kSspQFull + bb], 0, h * G, b * d.Qn + row0, pol_q);
+                        tma_load_3d(bt + NPAD * 128, &tm_q, &bar[kSspQFull + bb], 64, h * G, b * d.Qn + row0, pol_q);
                     }
-                  }
-#pragma unroll
-                  for (int k = 0; k < kBatch; ++k) {
-                    const int it = lane + 32 * (i0 + k);
+                }
+                __syncwarp();
+                cta_wait(&bar[kSspQFull + bb], (nb / nbuf) & 1, s_abort);
+                for (int it = lane; it < rows * 16; it += 32) {
                     const int r = it >> 4, cc16 = it & 15;
-                    const uint4 v = vb[k];
+                    const int region = cc16 >> 3, cc = cc16 & 7;
+                    const int off = region * NPAD * 128 + (r >> 3) * 1024 + (r & 7) * 128 + ((cc ^ (r & 7)) << 4);
+                    const uint4 v = *reinterpret_cast<const uint4*>(bt + off);
                     uint32_t w[4] = {v.x, v.y, v.z, v.w}, pos4[4], neg4[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -232,13 +237,8 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
                         neg4[i] = w[i] & neg_mask;
                         pos4[i] = w[i] & ~neg_mask;
                     }
-                    const int region = cc16 >> 3, cc = cc16 & 7;
-                    const int off = (r >> 3) * 1024 + (r & 7) * 128 + ((cc ^ (r & 7)) << 4);
-                    *reinterpret_cast<uint4*>(bt + region * NPAD * 128 + off) =
-                        make_uint4(pos4[0], pos4[1], pos4[2], pos4[3]);
-                    *reinterpret_cast<uint4*>(bt + (2 + region) * NPAD * 128 + off) =
-                        make_uint4(neg4[0], neg4[1], neg4[2], neg4[3]);
-                  }
+                    *reinterpret_cast<uint4*>(bt + off) = make_uint4(pos4[0], pos4[1], pos4[2], pos4[3]);
+                    *reinterpret_cast<uint4*>(bt + 2 * NPAD * 128 + off) = make_uint4(neg4[0], neg4[1], neg4[2], neg4[3]);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -304,18 +304,11 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
         const bool leader = warp == 2 && lane == 0;
         int pos = 0;
         for (int p = 0;; ++p) {
-            const int pb = p & 1, db = p & 1;
+            const int pb = p & 1;
             cta_wait(&bar[kSspCFull + pb], (p >> 1) & 1, s_abort);
             const int* info = s_info + pb * kSspInfoInts;
-            const int end = info[0], u = info[1], nv = info[2], t0 = info[3], ts = info[4], vt = info[5];
-            if (named_bar_or(kSspNbEpiVote, 128, end != 0 || *s_abort)) {
-                if (leader) {                                  // the tail group finishes too
-                    if (p >= 2) cta_wait(&bar[kSspDecFree + db], ((p >> 1) - 1) & 1, s_abort);
-                    s_dec[db * 4 + 3] = 1;
-                    mbar_arrive(&bar[kSspDecFull + db]);
-                }
-                break;
-            }
+            const int end = info[0], u = info[1], nv = info[2], t0 = info[3], ts = info[4];
+            if (named_bar_or(kSspNbEpiVote, 128, end != 0 || *s_abort)) break;
             for (int t = t0; t < ts; ++t, ++pos) {
                 const int ab = pos & 1;
                 const bool ok = cta_wait(&bar[kSspAccFull + ab], (pos >> 1) & 1, s_abort);
@@ -338,46 +331,45 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
                 const int n = t * kScoreTile + qd * 32 + lane;
                 if (ok && n < nv) scores[u * N + n] = best;
             }
-            // the chunk's scores are out: take the unit's ticket; the chunk that
-            // completes the unit hands it to the tail warps
+            // the chunk's scores are out: one more chunk of the unit done
             __threadfence();
             SspEpiGroup::sync();
             if (leader) {
-                const int chunks = (vt + ch.cts - 1) / ch.cts;     // the unit's chunks that hold valid blocks
-                const int old = atomicAdd(ticket + u, 1);
+                atomicAdd(ticket + u, 1);
                 mbar_arrive(&bar[kSspCFree + pb]);
-                if (p >= 2) cta_wait(&bar[kSspDecFree + db], ((p >> 1) - 1) & 1, s_abort);
-                s_dec[db * 4 + 0] = old == chunks - 1 ? 1 : 0;
-                s_dec[db * 4 + 1] = u;
-                s_dec[db * 4 + 2] = nv;
-                s_dec[db * 4 + 3] = 0;
-                mbar_arrive(&bar[kSspDecFull + db]);            // release: the decision and the scores
             }
         }
     } else {
         // ====================================== top-K + plan tail (6..9)
         const int ttid = SspTailGroup::tid();
-        for (int p = 0;; ++p) {
-            const int db = p & 1;
-            cta_wait(&bar[kSspDecFull + db], (p >> 1) & 1, s_abort);
-            // one thread copies the decision and the group reads the copy after the
-            // barrier, so every thread sees the same values (they then meet the same
-            // barriers below)
+        const int units = d.B * d.Hkv;
+        while (true) {
+            // claim the next unit; wait until every chunk of it holding valid blocks is scored
             if (ttid == 0) {
-                const int end = (s_dec[db * 4 + 3] != 0 || *s_abort) ? 1 : 0;
-                s_dec[8] = end ? 0 : s_dec[db * 4 + 0];
-                s_dec[9] = s_dec[db * 4 + 1];
-                s_dec[10] = s_dec[db * 4 + 2];
-                s_dec[11] = end;
+                int u = *s_abort ? units : atomicAdd(sched + 2, 1);
+                if (u < units) {
+                    const int nvu = n_valid_blocks(ctx_len[u / d.Hkv], d.N);
+                    const int vt = max(1, (nvu + kScoreTile - 1) / kScoreTile);
+                    const int chunks = (vt + ch.cts - 1) / ch.cts;
+                    const uint64_t t0 = global_timer_ns();
+                    while (ld_acquire_gpu(ticket + u) < chunks) {
+                        if (global_timer_ns() - t0 > kWaitLimitNs) {   // bounded: give up, flag it
+                            *s_abort = 1;
+                            raise_dev_error(OASIS_DEVERR_TIMEOUT);
+                            u = units;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+                *s_claim = u;
             }
             SspTailGroup::sync();
-            const int mine = s_dec[8], u = s_dec[9], nv = s_dec[10], end = s_dec[11];
+            const int u = *s_claim;
             SspTailGroup::sync();
-            if (ttid == 0) mbar_arrive(&bar[kSspDecFree + db]);
-            if (end) break;
-            if (!mine) continue;
-            __threadfence();                                   // every CTA's scores of the unit are visible
+            if (u >= units) break;
             if (ttid == 0) ticket[u] = 0;                      // ready for the next call
+            const int nv = n_valid_blocks(ctx_len[u / d.Hkv], d.N);
             const float* su = scores + u * N;
             for (int i = ttid; i < nv; i += SspTailGroup::kThreads) keys[i] = ordered_key(__ldcg(su + i));
             SspTailGroup::sync();
@@ -405,6 +397,7 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
         __threadfence();
         if (atomicAdd(sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
             atomicExch(sched, 0);
+            atomicExch(sched + 2, 0);
             atomicExch(sched + 1, 0);
         }
     }

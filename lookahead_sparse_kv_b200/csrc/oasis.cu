@@ -163,16 +163,16 @@ int make_map_pool(CUtensorMap* m, const void* base, unsigned long long slots, co
 
 // The query rows of every (sequence, KV head): bf16 q [B][Qn][Hq][128] seen
 // as a 3-D tensor (128 columns, Hq heads, B*Qn query positions), boxes of
-// 64 columns x G heads x Qn positions, so one box per 64-column half brings
-// the unit's Qn*G rows in (j, g) order, 128-byte swizzled.
-int make_map_q(CUtensorMap* m, const void* q, const Dims& d) {
+// 64 columns x G heads x nq positions, so one box per 64-column half brings
+// nq of the unit's query positions in (j, g) order, 128-byte swizzled.
+int make_map_q(CUtensorMap* m, const void* q, const Dims& d, int nq) {
     auto fn = encode_fn();
     if (fn == nullptr) return fail(OASIS_ECUDA, "cuTensorMapEncodeTiled unavailable");
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(oasis::kHeadDim), static_cast<cuuint64_t>(d.Hq),
                                 static_cast<cuuint64_t>(d.B) * d.Qn};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(oasis::kRowBytes),
                                    static_cast<cuuint64_t>(oasis::kRowBytes) * d.Hq};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(d.G()), static_cast<cuuint32_t>(d.Qn)};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(d.G()), static_cast<cuuint32_t>(nq)};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -232,8 +232,8 @@ oasis::AttnChunks attn_chunks(const Dims& d, int ctas) {
 // split units (log2-sum-exp [P][rows] and normalised outputs [P][rows][128],
 // P = the most chunks any launch makes), then one ticket counter per unit
 // for the attention merge, one per unit for the fused score / select / plan,
-// and the chunk and exit counters of the attention and of the fused scoring
-// (all zero between calls).
+// the attention's chunk and exit counters and the fused scoring's chunk,
+// exit and tail-claim counters (all zero between calls).
 struct WsLayout {
     size_t scores, lse, o, ticket, sticket, sched, ssched, total;
     long long partials;
@@ -253,7 +253,7 @@ WsLayout ws_layout(const Dims& d) {
     w.sticket = align256(w.ticket + units * sizeof(int));
     w.sched = align256(w.sticket + units * sizeof(int));
     w.ssched = align256(w.sched + 2 * sizeof(int));
-    w.total = align256(w.ssched + 2 * sizeof(int));
+    w.total = align256(w.ssched + 4 * sizeof(int));
     return w;
 }
 
@@ -284,7 +284,8 @@ int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d
 // Scoring chunks: 2 tiles of 128 blocks each (128 KiB of summaries), one per
 // unit when a unit has fewer.
 template <int NPAD, bool kScored>
-int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
+int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const CUtensorMap& tq, const Dims& d,
+                 const uint16_t* q,
                  const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int* sched, int32_t* sel,
                  float* sel_score, int32_t* st, int32_t* lu, int32_t step, const int32_t* step_dev, int32_t* fs,
                  int32_t* fb, int32_t* nf, cudaStream_t s) {
@@ -302,26 +303,27 @@ int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d
     ch.cpu = (tpu + ch.cts - 1) / ch.cts;
     ch.nc = d.B * d.Hkv * ch.cpu;
     const int ctas = std::min(sm_count(), ch.nc);
-    k<<<ctas, oasis::kSspThreads, smem, s>>>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score,
+    k<<<ctas, oasis::kSspThreads, smem, s>>>(tmax, tmin, tq, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score,
                                              st, lu, step, step_dev, fs, fb, nf, ch, nbuf);
     return check_launch("score_select_plan launch");
 }
 
 template <bool kScored>
-int launch_fused_rows(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d, const uint16_t* q,
+int launch_fused_rows(const CUtensorMap& tmax, const CUtensorMap& tmin, const CUtensorMap& tq, const Dims& d,
+                      const uint16_t* q,
                       const int32_t* ctx, float* scores, int row0, int rows, int* ticket, int* sched, int32_t* sel,
                       float* sel_score, int32_t* st, int32_t* lu, int32_t step, const int32_t* step_dev, int32_t* fs,
                       int32_t* fb, int32_t* nf, cudaStream_t s) {
     if (rows <= 16)
-        return launch_fused<16, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
+        return launch_fused<16, kScored>(tmax, tmin, tq, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
                                          step, step_dev, fs, fb, nf, s);
     if (rows <= 32)
-        return launch_fused<32, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
+        return launch_fused<32, kScored>(tmax, tmin, tq, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
                                          step, step_dev, fs, fb, nf, s);
     if (rows <= 48)
-        return launch_fused<48, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
+        return launch_fused<48, kScored>(tmax, tmin, tq, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu,
                                          step, step_dev, fs, fb, nf, s);
-    return launch_fused<64, kScored>(tmax, tmin, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu, step,
+    return launch_fused<64, kScored>(tmax, tmin, tq, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score, st, lu, step,
                                      step_dev, fs, fb, nf, s);
 }
 
@@ -562,12 +564,14 @@ int oasis_score_select_plan(const oasis_dims* dp, const void* q, const void* kmi
     CUtensorMap tmax, tmin;
     if (int rc = make_map(&tmax, kmax, total_rows, oasis::kScoreTile, "kmax")) return rc;
     if (int rc = make_map(&tmin, kmin, total_rows, oasis::kScoreTile, "kmin")) return rc;
+    CUtensorMap tq;
+    if (int rc = make_map_q(&tq, q, d, rows / d.G())) return rc;
     const auto* qq = static_cast<const uint16_t*>(q);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (scores != nullptr)
-        return launch_fused_rows<true>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sched, sel, sel_score,
+        return launch_fused_rows<true>(tmax, tmin, tq, d, qq, ctx_len, sc, row0, rows, ticket, sched, sel, sel_score,
                                        slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch, s);
-    return launch_fused_rows<false>(tmax, tmin, d, qq, ctx_len, sc, row0, rows, ticket, sched, sel, sel_score, slot_table,
+    return launch_fused_rows<false>(tmax, tmin, tq, d, qq, ctx_len, sc, row0, rows, ticket, sched, sel, sel_score, slot_table,
                                     last_used, step, step_dev, fetch_slot, fetch_block, n_fetch, s);
 }
 
@@ -711,7 +715,7 @@ int oasis_sparse_attn(const oasis_dims* dp, const void* q, const void* pool, con
     if (int rc = make_map_pool(&tk, pool, slots, "pool keys")) return rc;
     if (int rc = make_map_pool(&tv, static_cast<const uint8_t*>(pool) + oasis::kBlockBytes / 2, slots, "pool values"))
         return rc;
-    if (int rc = make_map_q(&tq, q, d)) return rc;
+    if (int rc = make_map_q(&tq, q, d, d.Qn)) return rc;
     uint8_t* base = static_cast<uint8_t*>(ws);
     float* ws_lse = reinterpret_cast<float*>(base + w.lse);
     float* ws_o = reinterpret_cast<float*>(base + w.o);

@@ -34,8 +34,10 @@ __device__ __forceinline__ unsigned long long victim_key(int slot, int blk, uint
 
 constexpr int kPlanThreads = 256;
 
-// Shared-memory ints plan_unit needs for budget K.
-__host__ __device__ constexpr int plan_smem_ints(int K) { return 9 * K; }
+// Shared-memory ints plan_unit needs for budget K (nine arrays of K rounded
+// up to a multiple of 4, so the scans over slots read 16 B at a time).
+__host__ __device__ constexpr int plan_k4(int K) { return (K + 3) & ~3; }
+__host__ __device__ constexpr int plan_smem_ints(int K) { return 9 * plan_k4(K); }
 
 // Plan of one (b, h) by a group of threads (each loops over slots /
 // ranks): sel, st, lu point at the unit's K entries, fs/fb at its C fetch
@@ -45,16 +47,22 @@ template <class Grp, bool kScored>
 __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* scores_u, int32_t* st, int32_t* lu,
                           int step, int32_t* fs, int32_t* fb, int32_t* nf, int32_t* sp, int* tmp) {
     constexpr int NT = Grp::kThreads;
+    const int K4 = plan_k4(K);
     int32_t* s_st = sp;
-    int32_t* s_lu = sp + K;
-    int32_t* s_prot = sp + 2 * K;
-    int32_t* s_vict = sp + 3 * K;
-    int32_t* s_nst = sp + 4 * K;
-    int32_t* s_nlu = sp + 5 * K;
-    uint32_t* s_ord = reinterpret_cast<uint32_t*>(sp + 6 * K);
-    int32_t* s_sel = sp + 7 * K;
-    int32_t* s_mpos = sp + 8 * K;          // miss flag, then the miss's position in rank order (-1: no miss)
+    int32_t* s_lu = sp + K4;
+    int32_t* s_prot = sp + 2 * K4;
+    int32_t* s_vict = sp + 3 * K4;
+    int32_t* s_nst = sp + 4 * K4;
+    int32_t* s_nlu = sp + 5 * K4;
+    uint32_t* s_ord = reinterpret_cast<uint32_t*>(sp + 6 * K4);
+    int32_t* s_sel = sp + 7 * K4;
+    int32_t* s_mpos = sp + 8 * K4;         // miss flag, then the miss's position in rank order (-1: no miss)
     const int tid = Grp::tid();
+    for (int i = K + tid; i < K4; i += NT) {   // padding: never matches, never a victim
+        s_st[i] = -2;
+        s_prot[i] = 1;
+        s_ord[i] = 0u;
+    }
     for (int i = tid; i < K; i += NT) {
         int x = st[i];
         if (x < -1 || x >= N) {
@@ -76,17 +84,28 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
         s_sel[i] = sv;
     }
     Grp::sync();
-    // 1. residency lookup of every selected block; hits are protected
+    // 1. residency lookup of every selected block (hits are protected), and a
+    //    check that no block is resident twice; 4 slots per shared-memory read
+    const int4* st4 = reinterpret_cast<const int4*>(s_st);
     for (int i = tid; i < K; i += NT) {
         const int sv = s_sel[i], own = s_st[i];
-        int hit = -1;
-        for (int j = 0; j < K; ++j) {
-            const int x = s_st[j];
-            if (sv >= 0 && hit < 0 && x == sv) hit = j;
-            if (own >= 0 && j < i && x == own) raise_dev_error(OASIS_DEVERR_DUPLICATE);
+        int hit = 0x7FFFFFFF;
+        bool dup = false;
+#pragma unroll 4
+        for (int j4 = 0; j4 < K4 / 4; ++j4) {
+            const int4 x = st4[j4];
+            const int j = 4 * j4;
+            if (x.w == sv) hit = min(hit, j + 3);
+            if (x.z == sv) hit = min(hit, j + 2);
+            if (x.y == sv) hit = min(hit, j + 1);
+            if (x.x == sv) hit = min(hit, j);
+            dup |= (x.x == own && j < i) | (x.y == own && j + 1 < i) | (x.z == own && j + 2 < i) |
+                   (x.w == own && j + 3 < i);
         }
-        if (hit >= 0) s_prot[hit] = 1;
-        s_mpos[i] = (sv >= 0 && hit < 0) ? 1 : 0;
+        if (sv < 0) hit = 0x7FFFFFFF;
+        if (own >= 0 && dup) raise_dev_error(OASIS_DEVERR_DUPLICATE);
+        if (hit != 0x7FFFFFFF) s_prot[hit] = 1;
+        s_mpos[i] = (sv >= 0 && hit == 0x7FFFFFFF) ? 1 : 0;
     }
     Grp::sync();
     // 2. misses numbered in rank order
@@ -105,11 +124,19 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
         const bool prot = s_prot[i] != 0;
         s_nst[i] = s_st[i];
         s_nlu[i] = prot ? step : s_lu[i];
-        if (!prot) {
+        if (!prot && nF > 0) {
             const unsigned long long mine = victim_key(i, s_st[i], s_ord[i]);
+            const int4* pr4 = reinterpret_cast<const int4*>(s_prot);
+            const uint4* or4 = reinterpret_cast<const uint4*>(s_ord);
             int rank = 0;
-            for (int j = 0; j < K; ++j)
-                if (!s_prot[j] && victim_key(j, s_st[j], s_ord[j]) < mine) ++rank;
+#pragma unroll 2
+            for (int j4 = 0; j4 < K4 / 4; ++j4) {
+                const int4 pr = pr4[j4], x = st4[j4];
+                const uint4 od = or4[j4];
+                const int j = 4 * j4;
+                rank += (!pr.x && victim_key(j, x.x, od.x) < mine) + (!pr.y && victim_key(j + 1, x.y, od.y) < mine) +
+                        (!pr.z && victim_key(j + 2, x.z, od.z) < mine) + (!pr.w && victim_key(j + 3, x.w, od.w) < mine);
+            }
             if (rank < nF) s_vict[rank] = i;
         }
     }

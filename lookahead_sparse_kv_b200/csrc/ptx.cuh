@@ -83,6 +83,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// Load with acquire semantics at GPU scope (pairs with a release by a
+// __threadfence() + atomic in another CTA).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // Makes this thread's generic-proxy shared-memory writes visible to the async
 // proxy (TMA, tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -55,23 +55,60 @@ __device__ void select_unit(Key key, int nv, int K, unsigned long long* cand, Se
 
     uint32_t T = 0;
     int need_eq = 0;
-    if (nv > K) {
+    if (nv > K && NT <= 128 && nv <= 32 * NT) {
+        // small groups: the K-th largest key by bisection on the key value (each
+        // thread holds its, at most 32, keys in registers; one barrier per step;
+        // padding keys are 0, below every score's key); large groups take the radix
+        // passes below
+        const int per = (nv + NT - 1) / NT;
+        const int i0 = tid * per;
+        uint32_t kk[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) kk[j] = (j < per && i0 + j < nv) ? key(i0 + j) : 0u;
+        uint32_t lo = 0u, hi = 0xFFFFFFFFu;          // count(>= lo) >= K > count(>= hi + 1)
+        for (int it = 0; lo < hi; ++it) {
+            const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
+            int c = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) c += kk[j] >= mid ? 1 : 0;
+            c = __reduce_add_sync(0xFFFFFFFFu, c);
+            if ((tid & 31) == 0) sc->hist[(it & 1) * 32 + (tid >> 5)] = c;
+            Grp::sync();
+            int tot = 0;
+#pragma unroll
+            for (int w = 0; w < NT / 32; ++w) tot += sc->hist[(it & 1) * 32 + w];
+            if (tot >= K) lo = mid; else hi = mid - 1u;
+        }
+        T = lo;
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) c += kk[j] > T ? 1 : 0;
+        int gt_all;
+        group_excl_sum<Grp>(c, sc->tmp, &gt_all);
+        need_eq = K - gt_all;
+    } else if (nv > K) {
         uint32_t prefix = 0, mask = 0;
         int remaining = K;
         for (int shift = 24; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += NT) sc->hist[i] = 0;
             Grp::sync();
             // scores of one unit cluster in a few bins: lanes of a warp that share a
-            // bin add to it once (one shared-memory atomic per distinct bin per warp)
-            for (int base = 0; base < nv; base += NT) {
-                const int i = base + tid;
-                int bin = -1;
-                if (i < nv) {
-                    const uint32_t u = key(i);
-                    if ((u & mask) == prefix) bin = static_cast<int>((u >> shift) & 0xFF);
+            // bin add to it once (one shared-memory atomic per distinct bin per warp);
+            // four keys per thread are read before any is binned
+            for (int base = 0; base < nv; base += 4 * NT) {
+                uint32_t uk[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = base + k * NT + tid;
+                    uk[k] = i < nv ? key(i) : 0u;
                 }
-                const unsigned same = __match_any_sync(0xFFFFFFFFu, bin);
-                if (bin >= 0 && __ffs(same) - 1 == (tid & 31)) atomicAdd(&sc->hist[bin], __popc(same));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = base + k * NT + tid;
+                    const int bin = (i < nv && (uk[k] & mask) == prefix) ? static_cast<int>((uk[k] >> shift) & 0xFF) : -1;
+                    const unsigned same = __match_any_sync(0xFFFFFFFFu, bin);
+                    if (bin >= 0 && __ffs(same) - 1 == (tid & 31)) atomicAdd(&sc->hist[bin], __popc(same));
+                }
             }
             Grp::sync();
             // suffix sums over bins (bin 255 first): thread t holds bins 255-t*kBpt-k
@@ -140,7 +177,33 @@ __device__ void select_unit(Key key, int nv, int K, unsigned long long* cand, Se
     for (int i = take + tid; i < kp; i += NT) cand[i] = ~0ull;
     Grp::sync();
 
-    // Bitonic sort of kp entries, ascending (~key, id) = score desc, id asc.
+    // Rank order (~key, id) ascending = score desc, id asc.  Up to two winners
+    // a thread: each winner's rank is the number of smaller entries (they are
+    // distinct); more: bitonic sort of kp entries.
+    if (take <= 2 * NT) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int i = tid + h * NT;
+            if (i >= take) continue;
+            const unsigned long long c = cand[i];
+            int rank = 0;
+            int j = 0;
+#pragma unroll 4
+            for (; j + 1 < take; j += 2) {
+                const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(cand + j);
+                rank += (x.x < c) + (x.y < c);
+            }
+            if (j < take) rank += cand[j] < c;
+            const int id = static_cast<int>(c & 0xFFFFFFFFu);
+            out[rank] = id;
+            if (out_s) out_s[rank] = __ldcg(s + id);
+        }
+        for (int i = take + tid; i < K; i += NT) {
+            out[i] = -1;
+            if (out_s) out_s[i] = -__int_as_float(0x7f800000);
+        }
+        return;
+    }
     for (int k = 2; k <= kp; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
             for (int i = tid; i < kp; i += NT) {
@@ -170,99 +233,12 @@ __device__ void select_unit(Key key, int nv, int K, unsigned long long* cand, Se
     }
 }
 
-// Fast path of select_unit for nv <= 2048 blocks and K <= 128, by a group of
-// 4 warps.  Warp w bitonic-sorts the composites (~key << 32 | id) of blocks
-// [512w, 512w + 512) in registers (16 per lane, element e = 16*lane + j;
-// strides below 16 stay in a lane, larger ones exchange with lane ^
-// (stride / 16)); ascending composites are descending scores with ties to the
-// lower id, the order select_unit produces.  Each warp's first 128 entries go
-// to cand[128w ..]; a candidate's rank among the four heads is its position
-// plus, in each other head, the number of smaller entries (binary search), and
-// the first K ranks are written in rank order.  key(i) gives block i's
-// monotone key; cand holds 512 entries.
-constexpr int kSelFastMaxN = 2048, kSelFastMaxK = 128;
-
-template <class Grp, class Key>
-__device__ void select_unit_fast(Key key, int nv, int K, unsigned long long* cand, const float* s, int32_t* out,
-                                 float* out_s) {
-    static_assert(Grp::kThreads == 128, "four warps");
-    const int t = Grp::tid(), lane = t & 31, w = t >> 5;
-    unsigned long long v[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const int i = 512 * w + 16 * lane + j;
-        v[j] = i < nv ? (static_cast<unsigned long long>(~key(i)) << 32) | static_cast<uint32_t>(i) : ~0ull;
-    }
-#pragma unroll
-    for (int k = 2; k <= 512; k <<= 1) {
-#pragma unroll
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            if (jj < 16) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int pj = j ^ jj;
-                    if (pj > j) {
-                        const bool asc = ((16 * lane + j) & k) == 0;
-                        const unsigned long long a = v[j], b = v[pj];
-                        const bool sw = (a > b) == asc;
-                        v[j] = sw ? b : a;
-                        v[pj] = sw ? a : b;
-                    }
-                }
-            } else {
-                const int lm = jj >> 4;
-                const bool lower = (lane & lm) == 0;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const bool asc = ((16 * lane + j) & k) == 0;
-                    const unsigned long long o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
-                    const bool keep_min = lower == asc;
-                    v[j] = keep_min ? (v[j] < o ? v[j] : o) : (v[j] < o ? o : v[j]);
-                }
-            }
-        }
-    }
-    if (lane < 8) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) cand[128 * w + 16 * lane + j] = v[j];
-    }
-    Grp::sync();
-    const int take = min(K, nv);
-#pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) {
-        const int idx = t + 128 * c4, lst = idx >> 7, p = idx & 127;
-        const unsigned long long c = cand[idx];
-        if (c == ~0ull) continue;                      // past the unit's blocks
-        int rank = p;
-#pragma unroll
-        for (int o = 0; o < 4; ++o) {
-            if (o == lst) continue;
-            const unsigned long long* L = cand + 128 * o;
-            int lo = 0, hi = 128;                      // entries of L below c
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (L[mid] < c) lo = mid + 1; else hi = mid;
-            }
-            rank += lo;
-        }
-        if (rank < take) {
-            const int id = static_cast<int>(c & 0xFFFFFFFFu);
-            out[rank] = id;
-            if (out_s) out_s[rank] = __ldcg(s + id);
-        }
-    }
-    for (int i = take + t; i < K; i += 128) {
-        out[i] = -1;
-        if (out_s) out_s[i] = -__int_as_float(0x7f800000);
-    }
-}
-
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(Dims d, const float* __restrict__ scores,
                                                                   const int32_t* __restrict__ ctx_len,
                                                                   int32_t* __restrict__ sel,
                                                                   float* __restrict__ sel_score) {
     extern __shared__ uint32_t keys[];                 // [N]
-    __shared__ unsigned long long cand[kSelMaxK];
+    __shared__ __align__(16) unsigned long long cand[kSelMaxK];
     __shared__ SelScratch sc;
     const int tid = threadIdx.x;
     const int bh = blockIdx.x, b = bh / d.Hkv;
