@@ -46,11 +46,13 @@
 //              16 rows x 64 columns, 128-byte swizzle).
 //   warp 9     issues S^T (and holds the TMEM allocation).
 //   warp 10    issues O^T; a free slot's product is not issued.
-//   warps 0-3  softmax, one token per thread.  The running max of a row
-//              moves only when a tile exceeds it by more than 2^8 (found
-//              with one barrier-wide vote per tile); then the tile's row
-//              maxima are reduced across the four warps and O^T and the row
-//              sums are rescaled.  Value rows past the context in a partly
+//   warps 0-3  softmax, one token per thread.  A chunk's running max of a
+//              row starts at the score of the chunk's first valid token and
+//              moves only when a tile exceeds it by more than 2^32 (found with
+//              one barrier-wide vote per tile; probabilities stay below 2^32,
+//              far inside fp32 and bf16 range, and any m gives the exact
+//              log-sum-exp); then the tile's row maxima are reduced across
+//              the four warps and O^T and the row sums are rescaled.  Value rows past the context in a partly
 //              filled slot are zeroed so stale bytes never meet a zero
 //              weight.
 //   warps 4-7  epilogue, one channel per thread, double-buffered against
@@ -72,6 +74,7 @@ constexpr int kAttnLoaderWarp = 8, kAttnSWarp = 9, kAttnOWarp = 10, kAttnListerW
 constexpr int kAttnThreads = 32 * 12;
 constexpr int kAttnTmemCols = 512;                                 // S^T x 2 (64 columns each), O^T x 2 (2 NR each), row sums
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kAttnLazy = 32.f;                                  // rescale when a score passes m + 32 (log2)
 
 // shared memory, from the 1024-B aligned base
 constexpr int kAttnOffK = 0;                                       // K ring, 2 stages
@@ -419,6 +422,7 @@ __global__ void __maxnreg__(152)
         const int q = warp;                                   // TMEM lane quadrant
         const int tok = 32 * q + lane;                        // token of the tile this thread owns
         const int myslot = tok >> 4, mytok = tok & 15;
+        const float inv_scale = 1.f / scale_log2;          // thresholds in raw-score units
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         int pos = 0;
         for (int p = 0;; ++p) {
@@ -429,19 +433,17 @@ __global__ void __maxnreg__(152)
             if (named_bar_or(kNbSoftmaxVote, 128, n < 0 || *s_abort)) break;
             // the epilogue of chunk p-2 has read this buffer's running max and sums
             if (p >= 2) cta_wait(&bar[kBarOFree + pb], ((p >> 1) - 1) & 1, s_abort);
-            // running max m (log2 units) and the raw-score threshold (m + 8) / scale of
-            // every row; rows past the real ones have both at +inf, so their scores never
-            // vote and their probabilities are 0 (the padded columns are never read)
+            // running max m (log2 units) and the raw-score threshold (m + 32) / scale of
+            // every row, set from the chunk's first valid token at its first tile; rows
+            // past the real ones have both at +inf, so their scores never vote and their
+            // probabilities are 0 (the padded columns are never read)
             float* mr = s_m + pb * 64;
             float* thr = s_thr + pb * 64;
             if (q == 0) {
                 const float kPosInf = __int_as_float(0x7f800000);
-                mr[lane] = lane < rows ? kNegInf : kPosInf;
-                mr[lane + 32] = lane + 32 < rows ? kNegInf : kPosInf;
-                thr[lane] = mr[lane];
-                thr[lane + 32] = mr[lane + 32];
+                if (lane >= rows) mr[lane] = thr[lane] = kPosInf;
+                if (lane + 32 >= rows) mr[lane + 32] = thr[lane + 32] = kPosInf;
             }
-            named_bar_sync(kNbSoftmax, 128);
             // this token's share of the row sums: registers with 32 rows, TMEM columns
             // of the token's lane with 64 (registers are short there)
             constexpr bool kLT = NR == 64;
@@ -481,7 +483,22 @@ __global__ void __maxnreg__(152)
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[kBarSFree + st]);
-                // does any row's running max move (by more than 2^8)?
+                if (i == 0) {
+                    // seed the running max: the first token of the tile's first occupied slot
+                    const uint64_t nvs = static_cast<uint32_t>(e[1]) | (static_cast<uint64_t>(static_cast<uint32_t>(e[2])) << 32);
+                    const int j0 = (__ffsll(static_cast<long long>(nvs)) - 1) >> 3;
+                    if (tok == kBlockTokens * j0) {
+#pragma unroll
+                        for (int r = 0; r < NR; ++r)
+                            if (r < rows) {
+                                const float m0 = x[r] * scale_log2;
+                                mr[r] = m0;
+                                thr[r] = (m0 + kAttnLazy) * inv_scale;
+                            }
+                    }
+                    named_bar_sync(kNbSoftmax, 128);
+                }
+                // does any row's running max move (by more than 2^32)?
                 bool up = false;
                 if (valid) {
 #pragma unroll
@@ -508,10 +525,10 @@ __global__ void __maxnreg__(152)
                             const float tmx = fmaxf(fmaxf(s_wmax[r], s_wmax[64 + r]), fmaxf(s_wmax[128 + r], s_wmax[192 + r]));
                             const float mo = mr[r];
                             float a = 1.f;
-                            if (r < rows && tmx > mo + 8.f) {
-                                a = attn_exp2(mo - tmx);              // 0 on the chunk's first tile
+                            if (r < rows && tmx > mo + kAttnLazy) {
+                                a = attn_exp2(mo - tmx);
                                 mr[r] = tmx;
-                                thr[r] = (tmx + 8.f) / scale_log2;
+                                thr[r] = (tmx + kAttnLazy) * inv_scale;
                             }
                             s_alpha[r] = a;
                         }

@@ -204,10 +204,14 @@ int set_smem(K kernel, int bytes, const char* what) {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Attention chunks: a unit's ceil(K / 8) tiles cut into chunks of `ct`
-// tiles.  Chunks are at least 2 tiles (4 with more than 32 query rows) so the
-// partials a split unit writes stay under ~1/8 of the bytes it reads, at
-// most 8 per unit (the merge's limit), and otherwise sized for about six per
-// CTA so that CTAs taking chunks from the counter finish together.
+// tiles.  Every chunk costs a running-max seed, a pipeline refill and, for a
+// split unit, a partial write and its share of the merge; on B200 whole-unit
+// chunks were fastest when there are about as many units as SMs (a 32K layer
+// of 128 units: 38.9 us whole against 43.0 / 51.2 / 65.7 us for 8 / 4 / 2
+// tiles per chunk).  So units are split only when there are fewer of them
+// than CTAs, into about CTAs / units chunks; chunks are at least 2 tiles (4
+// with more than 32 query rows) so a split unit's partials stay under ~1/8 of
+// the bytes it reads, and a unit has at most 8 of them (the merge's limit).
 int attn_min_chunk_tiles(const Dims& d) {
     const int tpu = (d.K + oasis::kAttnTileSlots - 1) / oasis::kAttnTileSlots;
     return std::min(tpu, d.Qn * d.G() <= 32 ? 2 : 4);
@@ -216,9 +220,10 @@ int attn_min_chunk_tiles(const Dims& d) {
 oasis::AttnChunks attn_chunks(const Dims& d, int ctas) {
     const int tpu = (d.K + oasis::kAttnTileSlots - 1) / oasis::kAttnTileSlots;
     const long long units = static_cast<long long>(d.B) * d.Hkv;
-    const long long per = units * tpu / (6ll * std::max(1, ctas));
-    int ct = static_cast<int>(std::min<long long>(std::max<long long>(per, attn_min_chunk_tiles(d)),
-                                                  oasis::kAttnMaxChunkTiles));
+    const int want = static_cast<int>(std::max<long long>(1, ctas / std::max(1ll, units)));   // chunks a unit
+    int ct = (tpu + want - 1) / want;
+    ct = std::max(ct, attn_min_chunk_tiles(d));
+    ct = std::min(ct, oasis::kAttnMaxChunkTiles);
     ct = std::max(ct, (tpu + oasis::kAttnMaxChunks - 1) / oasis::kAttnMaxChunks);   // the merge takes <= 8
     ct = std::min(ct, tpu);
     oasis::AttnChunks c;
@@ -281,8 +286,10 @@ int launch_score(const CUtensorMap& tmax, const CUtensorMap& tmin, const Dims& d
     return check_launch("lookahead_score launch");
 }
 
-// Scoring chunks: 2 tiles of 128 blocks each (128 KiB of summaries), one per
-// unit when a unit has fewer.
+// Scoring chunks: like the attention's, whole units when there are about as
+// many units as SMs (a 32K layer of 128 units: 55.4 us against 59.4 / 61.5 /
+// 64.5 / 71.8 us for chunks of 8 / 4 / 2 / 1 tiles of 128 blocks), else about
+// CTAs / units chunks a unit.
 template <int NPAD, bool kScored>
 int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const CUtensorMap& tq, const Dims& d,
                  const uint16_t* q,
@@ -299,9 +306,11 @@ int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const CUtenso
     if (int rc = set_smem(k, smem, "score_select_plan smem")) return rc;
     const int tpu = (d.N + oasis::kScoreTile - 1) / oasis::kScoreTile;
     oasis::SspChunks ch;
-    ch.cts = std::min(2, tpu);
+    const long long units = static_cast<long long>(d.B) * d.Hkv;
+    const int want = static_cast<int>(std::max<long long>(1, sm_count() / std::max(1ll, units)));
+    ch.cts = (tpu + want - 1) / want;
     ch.cpu = (tpu + ch.cts - 1) / ch.cts;
-    ch.nc = d.B * d.Hkv * ch.cpu;
+    ch.nc = static_cast<int>(units * ch.cpu);
     const int ctas = std::min(sm_count(), ch.nc);
     k<<<ctas, oasis::kSspThreads, smem, s>>>(tmax, tmin, tq, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score,
                                              st, lu, step, step_dev, fs, fb, nf, ch, nbuf);
