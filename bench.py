@@ -106,7 +106,12 @@ def headline_config(w, nl: int, world: int, name: str = WORKLOAD) -> dict:
             "l2": "inputs larger than L2: per layer-step 128 MiB summaries + 128 MiB pool read"}
 QUERY_RING = 256
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic_llama8b_32k.json")
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def traffic_path(workload: str) -> str:
+    """ncu DRAM bytes per launch for one workload (profiles/traffic_<workload>.json)."""
+    return os.path.join(PROFILES, f"traffic_{workload}.json")
 KERNELS = ("sparse_attn", "score_select_plan", "prefetch")
 
 
@@ -442,9 +447,9 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic():
+def load_traffic(workload: str):
     try:
-        with open(TRAFFIC_PATH) as f:
+        with open(traffic_path(workload)) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return {}
@@ -1171,7 +1176,7 @@ def emit_gpu(args, res, world):
     fetched = res["fetch_hist"].sum().item() / layer_steps            # blocks per layer-step (this rank)
     ab = algorithmic_bytes(w, fetched)
     h2d_peak = res["h2d"]["peak_gbs"] if res["h2d"] else None
-    traffic = load_traffic()
+    traffic = load_traffic(w.name)
 
     def roof(k, ms):
         gbs = ab[k] / (ms * 1e-3) / 1e9
