@@ -36,17 +36,18 @@
 // resets the ticket.  The last CTA to exit resets the chunk counter, so the
 // workspace is ready for the next call.
 //
-// Roles (12 warps, mbarriers for every hand-off, every wait bounded):
-//   warp 11    lister: takes chunks (the next one is requested while the
+// Roles (16 warps, mbarriers for every hand-off, every wait bounded):
+//   warp 15    lister: takes chunks (the next one is requested while the
 //              current one is listed), lists a chunk's tiles that hold a
 //              valid token (valid-token count of each slot) and loads the
 //              unit's query rows;
-//   warp 8     loader: streams the listed tiles' K and V through two 2-stage
+//   warp 12    loader: streams the listed tiles' K and V through two 2-stage
 //              TMA rings (per tile and tensor two 16-KiB boxes of 8 slots x
 //              16 rows x 64 columns, 128-byte swizzle).
-//   warp 9     issues S^T (and holds the TMEM allocation).
-//   warp 10    issues O^T; a free slot's product is not issued.
-//   warps 0-3  softmax, one token per thread.  A chunk's running max of a
+//   warp 13    issues S^T (and holds the TMEM allocation).
+//   warp 14    issues O^T; a free slot's product is not issued.
+//   warps 0-7  softmax, one token and half the rows per thread (two warps per
+//              TMEM lane quadrant).  A chunk's running max of a
 //              row starts at the score of the chunk's first valid token and
 //              moves only when a tile exceeds it by more than 2^32 (found with
 //              one barrier-wide vote per tile; probabilities stay below 2^32,
@@ -55,7 +56,7 @@
 //              the four warps and O^T and the row sums are rescaled.  Value rows past the context in a partly
 //              filled slot are zeroed so stale bytes never meet a zero
 //              weight.
-//   warps 4-7  epilogue, one channel per thread, double-buffered against
+//   warps 8-11 epilogue, one channel per thread, double-buffered against
 //              the next chunk (two O^T accumulators in TMEM).
 #pragma once
 
@@ -70,8 +71,10 @@ constexpr int kAttnStageBytes = 2 * kAttnHalf;                     // K (or V) o
 constexpr int kAttnQHalf = 64 * 128;                               // 64 query rows x 128 B
 constexpr int kAttnMaxChunkTiles = 16;
 constexpr int kAttnInfoInts = 8 + 4 * kAttnMaxChunkTiles;          // chunk header + 4 ints per tile
-constexpr int kAttnLoaderWarp = 8, kAttnSWarp = 9, kAttnOWarp = 10, kAttnListerWarp = 11;
-constexpr int kAttnThreads = 32 * 12;
+constexpr int kAttnSoftmaxWarps = 8;                              // warps 0-7 (two per TMEM quadrant)
+constexpr int kAttnEpiWarp = 8;                                    // warps 8-11
+constexpr int kAttnLoaderWarp = 12, kAttnSWarp = 13, kAttnOWarp = 14, kAttnListerWarp = 15;
+constexpr int kAttnThreads = 32 * 16;
 constexpr int kAttnTmemCols = 512;                                 // S^T x 2 (64 columns each), O^T x 2 (2 NR each), row sums
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kAttnLazy = 32.f;                                  // rescale when a score passes m + 32 (log2)
@@ -113,7 +116,7 @@ constexpr int kBarOFree = 26;    // O^T accumulator, running max and row sums re
 constexpr int kBarSMDone = 28;   // chunk's row sums written by the 4 softmax warps
 constexpr int kBarFinalS = 30;   // teardown: every S^T issued has completed
 constexpr int kBarFinalO = 31;   // teardown: every O^T issued has completed
-constexpr int kAttnLFreeCount = 11;
+constexpr int kAttnLFreeCount = 15;
 
 // named barriers (0 is __syncthreads)
 constexpr uint32_t kNbSoftmax = 1, kNbSoftmaxVote = 2, kNbEpi = 3, kNbEpiVote = 4;
@@ -150,10 +153,31 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane)
     return v[0];
 }
 
+// The same over 16 values: the two half-warps are folded first, then lane t
+// (and t + 16) holds the result for v[t & 15].
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter16(float (&v)[16], int lane) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float got = __shfl_xor_sync(0xFFFFFFFFu, v[k], 16);
+        v[k] = kMax ? fmaxf(v[k], got) : v[k] + got;
+    }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {
+        const bool up = (lane & w) != 0;
+#pragma unroll
+        for (int k = 0; k < w; ++k) {
+            const float send = up ? v[k] : v[k + w];
+            const float keep = up ? v[k + w] : v[k];
+            const float got = __shfl_xor_sync(0xFFFFFFFFu, send, w);
+            v[k] = kMax ? fmaxf(keep, got) : keep + got;
+        }
+    }
+    return v[0];
+}
+
 template <int NR>
-// 152 registers a thread: 384 x 152 leaves room for a gather CTA (128 x 48) on
-// the same SM.
-__global__ void __maxnreg__(152)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_q, Dims d, const int32_t* __restrict__ slot_table,
                        const int32_t* __restrict__ ctx_len, float scale_log2, AttnChunks ch,
@@ -166,7 +190,7 @@ __global__ void __maxnreg__(152)
     constexpr int kPBufs = NR == 32 ? 2 : 1;
     // TMEM columns: S^T buffers at 0 and 64, O^T buffers (head and remainder
     // products side by side) at 128 and 128 + 2 NR, 64-row sums after them
-    constexpr uint32_t kOCol = 128, kOStride = 2 * NR, kLCol = 128 + 2 * 2 * NR;
+    constexpr uint32_t kOCol = 128, kOStride = 2 * NR;
     const float kNegInf = -__int_as_float(0x7f800000);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -199,7 +223,7 @@ __global__ void __maxnreg__(152)
             int cnt = 1;
             if (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1 || i == kBarSMDone ||
                 i == kBarSMDone + 1)
-                cnt = 4;
+                cnt = kAttnSoftmaxWarps;
             if (i == kBarLFree || i == kBarLFree + 1) cnt = kAttnLFreeCount;
             mbar_init(&bar[i], cnt);
         }
@@ -417,12 +441,15 @@ __global__ void __maxnreg__(152)
             mbar_wait(&bar[kBarFinalO], 0);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        // ============================================ softmax (token / thread)
-        const int q = warp;                                   // TMEM lane quadrant
+    } else if (warp < kAttnSoftmaxWarps) {
+        // ================================== softmax (token / thread, half the rows / warp)
+        constexpr int kH = NR / 2;                            // rows per thread
+        constexpr int kSm = 32 * kAttnSoftmaxWarps;           // softmax threads
+        const int q = warp & 3;                               // TMEM lane quadrant
+        const int r0 = (warp >> 2) * kH;                      // first row of this warp
         const int tok = 32 * q + lane;                        // token of the tile this thread owns
         const int myslot = tok >> 4, mytok = tok & 15;
-        const float inv_scale = 1.f / scale_log2;          // thresholds in raw-score units
+        const float inv_scale = 1.f / scale_log2;             // thresholds in raw-score units
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         int pos = 0;
         for (int p = 0;; ++p) {
@@ -430,7 +457,7 @@ __global__ void __maxnreg__(152)
             cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort);
             const int* info = s_info + pb * kAttnInfoInts;
             const int n = info[0];
-            if (named_bar_or(kNbSoftmaxVote, 128, n < 0 || *s_abort)) break;
+            if (named_bar_or(kNbSoftmaxVote, kSm, n < 0 || *s_abort)) break;
             // the epilogue of chunk p-2 has read this buffer's running max and sums
             if (p >= 2) cta_wait(&bar[kBarOFree + pb], ((p >> 1) - 1) & 1, s_abort);
             // running max m (log2 units) and the raw-score threshold (m + 32) / scale of
@@ -439,26 +466,14 @@ __global__ void __maxnreg__(152)
             // probabilities are 0 (the padded columns are never read)
             float* mr = s_m + pb * 64;
             float* thr = s_thr + pb * 64;
-            if (q == 0) {
+            if (warp == 0) {
                 const float kPosInf = __int_as_float(0x7f800000);
                 if (lane >= rows) mr[lane] = thr[lane] = kPosInf;
                 if (lane + 32 >= rows) mr[lane + 32] = thr[lane + 32] = kPosInf;
             }
-            // this token's share of the row sums: registers with 32 rows, TMEM columns
-            // of the token's lane with 64 (registers are short there)
-            constexpr bool kLT = NR == 64;
-            const uint32_t l_addr = tmem + lane_base + kLCol;
-            float l[kLT ? 1 : NR];
+            float l[kH];                                      // this token's share of its rows' sums
 #pragma unroll
-            for (int r = 0; r < (kLT ? 1 : NR); ++r) l[r] = 0.f;
-            if constexpr (kLT) {
-                uint32_t z[32];
-#pragma unroll
-                for (int r = 0; r < 32; ++r) z[r] = 0u;
-                tmem_st_32x32b_x32(l_addr, z);
-                tmem_st_32x32b_x32(l_addr + 32, z);
-                tmem_st_wait();
-            }
+            for (int r = 0; r < kH; ++r) l[r] = 0.f;
             for (int i = 0; i < n; ++i, ++pos) {
                 const int st = pos & 1;
                 const int* e = info + 8 + 4 * i;
@@ -466,19 +481,19 @@ __global__ void __maxnreg__(152)
                 const bool valid = mytok < nvj;
                 cta_wait(&bar[kBarSFull + st], (pos >> 1) & 1, s_abort);
                 tc_fence_after_sync();
-                float x[NR];                                  // raw scores q.k of this token
-                {
+                float x[kH];                                  // raw scores q.k of this token, rows r0..
+                if constexpr (kH == 16) {
+                    uint32_t v[16];
+                    tmem_ld_x16(tmem + lane_base + st * 64 + r0, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) x[r] = __uint_as_float(v[r]);
+                } else {
                     uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem + lane_base + st * 64, v);
+                    tmem_ld_32x32b_x32(tmem + lane_base + st * 64 + r0, v);
                     tmem_ld_wait();
 #pragma unroll
                     for (int r = 0; r < 32; ++r) x[r] = __uint_as_float(v[r]);
-                    if constexpr (NR == 64) {
-                        tmem_ld_32x32b_x32(tmem + lane_base + st * 64 + 32, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int r = 0; r < 32; ++r) x[32 + r] = __uint_as_float(v[r]);
-                    }
                 }
                 tc_fence_before_sync();
                 __syncwarp();
@@ -489,97 +504,80 @@ __global__ void __maxnreg__(152)
                     const int j0 = (__ffsll(static_cast<long long>(nvs)) - 1) >> 3;
                     if (tok == kBlockTokens * j0) {
 #pragma unroll
-                        for (int r = 0; r < NR; ++r)
-                            if (r < rows) {
+                        for (int r = 0; r < kH; ++r)
+                            if (r0 + r < rows) {
                                 const float m0 = x[r] * scale_log2;
-                                mr[r] = m0;
-                                thr[r] = (m0 + kAttnLazy) * inv_scale;
+                                mr[r0 + r] = m0;
+                                thr[r0 + r] = (m0 + kAttnLazy) * inv_scale;
                             }
                     }
-                    named_bar_sync(kNbSoftmax, 128);
+                    named_bar_sync(kNbSoftmax, kSm);
                 }
                 // does any row's running max move (by more than 2^32)?
                 bool up = false;
                 if (valid) {
 #pragma unroll
-                    for (int r = 0; r < NR; r += 4) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(thr + r);
+                    for (int r = 0; r < kH; r += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(thr + r0 + r);
                         up |= (x[r] > t4.x) | (x[r + 1] > t4.y) | (x[r + 2] > t4.z) | (x[r + 3] > t4.w);
                     }
                 }
-                if (named_bar_or(kNbSoftmaxVote, 128, up)) {
-                    // tile maxima (log2 units): lane t of each warp gets rows t and t + 32
+                if (named_bar_or(kNbSoftmaxVote, kSm, up)) {
+                    // tile maxima (log2 units): lane r of each warp keeps row r0 + r of its tokens
+                    float mine = kNegInf;
 #pragma unroll
-                    for (int hh = 0; hh < NR / 32; ++hh) {
-                        float t[32];
-#pragma unroll
-                        for (int r = 0; r < 32; ++r)
-                            t[r] = (valid && 32 * hh + r < rows) ? x[32 * hh + r] * scale_log2 : kNegInf;
-                        s_wmax[q * 64 + 32 * hh + lane] = warp_reduce_scatter32<true>(t, lane);
+                    for (int r = 0; r < kH; ++r) {
+                        const float wm = warp_max_f32((valid && r0 + r < rows) ? x[r] * scale_log2 : kNegInf);
+                        if (lane == r) mine = wm;
                     }
-                    named_bar_sync(kNbSoftmax, 128);
-                    if (q == 0) {
-#pragma unroll
-                        for (int hh = 0; hh < NR / 32; ++hh) {
-                            const int r = 32 * hh + lane;
-                            const float tmx = fmaxf(fmaxf(s_wmax[r], s_wmax[64 + r]), fmaxf(s_wmax[128 + r], s_wmax[192 + r]));
-                            const float mo = mr[r];
-                            float a = 1.f;
-                            if (r < rows && tmx > mo + kAttnLazy) {
-                                a = attn_exp2(mo - tmx);
-                                mr[r] = tmx;
-                                thr[r] = (tmx + kAttnLazy) * inv_scale;
-                            }
-                            s_alpha[r] = a;
+                    if (lane < kH) s_wmax[q * 64 + r0 + lane] = mine;
+                    named_bar_sync(kNbSoftmax, kSm);
+                    if (q == 0 && lane < kH) {                // warps 0 and 4: their rows
+                        const int r = r0 + lane;
+                        const float tmx = fmaxf(fmaxf(s_wmax[r], s_wmax[64 + r]), fmaxf(s_wmax[128 + r], s_wmax[192 + r]));
+                        const float mo = mr[r];
+                        float a = 1.f;
+                        if (r < rows && tmx > mo + kAttnLazy) {
+                            a = attn_exp2(mo - tmx);
+                            mr[r] = tmx;
+                            thr[r] = (tmx + kAttnLazy) * inv_scale;
                         }
+                        s_alpha[r] = a;
                     }
-                    named_bar_sync(kNbSoftmax, 128);
-                    if constexpr (kLT) {
+                    named_bar_sync(kNbSoftmax, kSm);
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            uint32_t lv[32];
-                            tmem_ld_32x32b_x32(l_addr + 32 * hh, lv);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int r = 0; r < 32; ++r)
-                                lv[r] = __float_as_uint(__uint_as_float(lv[r]) * s_alpha[32 * hh + r]);
-                            tmem_st_32x32b_x32(l_addr + 32 * hh, lv);
-                        }
-                        tmem_st_wait();
-                    } else {
-#pragma unroll
-                        for (int r = 0; r < NR; ++r) l[r] *= s_alpha[r];
-                    }
+                    for (int r = 0; r < kH; ++r) l[r] *= s_alpha[r0 + r];
                     if (i > 0) {
                         // the previous tile's product must have landed in O^T before it is rescaled
                         cta_wait(&bar[kBarPFree + (pos - 1) % kPBufs], ((pos - 1) / kPBufs) & 1, s_abort);
                         tc_fence_after_sync();
 #pragma unroll
-                        for (int hh = 0; hh < 2 * NR / 32; ++hh) {            // head and remainder columns
-                            const uint32_t oaddr = tmem + lane_base + kOCol + pb * kOStride + 32 * hh;
-                            const int r0 = (32 * hh) % NR;
-                            uint32_t o[32];
-                            tmem_ld_32x32b_x32(oaddr, o);
+                        for (int part = 0; part < 2 * kH / 16; ++part) {   // head and remainder columns
+                            const int c0 = (part & (kH / 16 - 1)) * 16;           // column within the half
+                            const uint32_t oaddr = tmem + lane_base + kOCol + pb * kOStride +
+                                                   (part >= kH / 16 ? NR : 0) + r0 + c0;
+                            uint32_t o[16];
+                            tmem_ld_x16(oaddr, o);
                             tmem_ld_wait();
 #pragma unroll
-                            for (int r = 0; r < 32; ++r)
-                                o[r] = __float_as_uint(__uint_as_float(o[r]) * s_alpha[r0 + r]);
-                            tmem_st_32x32b_x32(oaddr, o);
+                            for (int r = 0; r < 16; ++r)
+                                o[r] = __float_as_uint(__uint_as_float(o[r]) * s_alpha[r0 + c0 + r]);
+                            tmem_st_x16(oaddr, o);
                         }
                         tmem_st_wait();
                     }
                 }
-                // this token's probabilities for every row, head and remainder (bf16 each),
-                // once the product that last read this P^T buffer is done
+                // this token's probabilities for this warp's rows, head and remainder (bf16
+                // each), once the product that last read this P^T buffer is done
                 const int pbuf = pos % kPBufs;
                 if (pos >= kPBufs) cta_wait(&bar[kBarPFree + pbuf], ((pos / kPBufs) - 1) & 1, s_abort);
                 uint8_t* prow = sP + pbuf * kAttnHalf + tok * 128;
                 if (valid) {
 #pragma unroll
-                    for (int c8 = 0; c8 < NR / 8; ++c8) {
-                        const float4 ma = *reinterpret_cast<const float4*>(mr + 8 * c8);
-                        const float4 mb = *reinterpret_cast<const float4*>(mr + 8 * c8 + 4);
+                    for (int c8 = 0; c8 < kH / 8; ++c8) {
                         const int r = 8 * c8;
+                        const float4 ma = *reinterpret_cast<const float4*>(mr + r0 + r);
+                        const float4 mb = *reinterpret_cast<const float4*>(mr + r0 + r + 4);
                         const float p0 = attn_exp2(fmaf(x[r + 0], scale_log2, -ma.x));
                         const float p1 = attn_exp2(fmaf(x[r + 1], scale_log2, -ma.y));
                         const float p2 = attn_exp2(fmaf(x[r + 2], scale_log2, -ma.z));
@@ -588,29 +586,19 @@ __global__ void __maxnreg__(152)
                         const float p5 = attn_exp2(fmaf(x[r + 5], scale_log2, -mb.y));
                         const float p6 = attn_exp2(fmaf(x[r + 6], scale_log2, -mb.z));
                         const float p7 = attn_exp2(fmaf(x[r + 7], scale_log2, -mb.w));
-                        if constexpr (kLT) {
-                            x[r + 0] = p0;
-                            x[r + 1] = p1;
-                            x[r + 2] = p2;
-                            x[r + 3] = p3;
-                            x[r + 4] = p4;
-                            x[r + 5] = p5;
-                            x[r + 6] = p6;
-                            x[r + 7] = p7;
-                        } else {
-                            l[r + 0] += p0;
-                            l[r + 1] += p1;
-                            l[r + 2] += p2;
-                            l[r + 3] += p3;
-                            l[r + 4] += p4;
-                            l[r + 5] += p5;
-                            l[r + 6] += p6;
-                            l[r + 7] += p7;
-                        }
+                        l[r + 0] += p0;
+                        l[r + 1] += p1;
+                        l[r + 2] += p2;
+                        l[r + 3] += p3;
+                        l[r + 4] += p4;
+                        l[r + 5] += p5;
+                        l[r + 6] += p6;
+                        l[r + 7] += p7;
                         const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
                         const uint32_t h45 = pack_bf16x2(p4, p5), h67 = pack_bf16x2(p6, p7);
-                        const int off = (c8 ^ (tok & 7)) << 4;
-                        const int roff = NR == 32 ? (((c8 + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
+                        const int cg = r0 / 8 + c8;                           // 16-B chunk of the row
+                        const int off = (cg ^ (tok & 7)) << 4;
+                        const int roff = NR == 32 ? (((cg + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
                         *reinterpret_cast<uint4*>(prow + off) = make_uint4(h01, h23, h45, h67);
                         *reinterpret_cast<uint4*>(prow + roff) =
                             make_uint4(pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01)),
@@ -623,13 +611,14 @@ __global__ void __maxnreg__(152)
                     // slot its value row reads as zero too (zero times a stale non-finite
                     // value is not zero)
 #pragma unroll
-                    for (int c8 = 0; c8 < NR / 8; ++c8) {
-                        const int off = (c8 ^ (tok & 7)) << 4;
-                        const int roff = NR == 32 ? (((c8 + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
+                    for (int c8 = 0; c8 < kH / 8; ++c8) {
+                        const int cg = r0 / 8 + c8;
+                        const int off = (cg ^ (tok & 7)) << 4;
+                        const int roff = NR == 32 ? (((cg + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
                         *reinterpret_cast<uint4*>(prow + off) = make_uint4(0u, 0u, 0u, 0u);
                         *reinterpret_cast<uint4*>(prow + roff) = make_uint4(0u, 0u, 0u, 0u);
                     }
-                    if (nvj > 0) {
+                    if (nvj > 0 && r0 == 0) {
                         cta_wait(&bar[kBarVFull + st], (pos >> 1) & 1, s_abort);   // orders the copy first
                         uint8_t* vrow = sV + st * kAttnStageBytes + tok * 128;
 #pragma unroll
@@ -643,37 +632,16 @@ __global__ void __maxnreg__(152)
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[kBarPFull + pbuf]);
-                if constexpr (kLT) {                          // x holds the probabilities now
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t lv[32];
-                        tmem_ld_32x32b_x32(l_addr + 32 * hh, lv);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int r = 0; r < 32; ++r)
-                            lv[r] = __float_as_uint(__uint_as_float(lv[r]) + (valid ? x[32 * hh + r] : 0.f));
-                        tmem_st_32x32b_x32(l_addr + 32 * hh, lv);
-                    }
-                    tmem_st_wait();
-                }
             }
-            // the chunk's row sums over this warp's tokens: lane t gets rows t and t + 32
-            float* lw = s_lw + (pb * 4 + q) * 64;
-            if constexpr (kLT) {
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t lv[32];
-                    tmem_ld_32x32b_x32(l_addr + 32 * hh, lv);
-                    tmem_ld_wait();
-                    float t[32];
-#pragma unroll
-                    for (int r = 0; r < 32; ++r) t[r] = __uint_as_float(lv[r]);
-                    lw[32 * hh + lane] = warp_reduce_scatter32<false>(t, lane);
-                }
-            } else {
-                lw[lane] = warp_reduce_scatter32<false>(*reinterpret_cast<float(*)[32]>(l), lane);
-                lw[32 + lane] = 0.f;
-            }
+            // the chunk's row sums over this warp's tokens: lane r gets row r0 + r
+            float* lw = s_lw + (pb * 4 + q) * 64 + r0;
+            float sum;
+            if constexpr (kH == 16)
+                sum = warp_reduce_scatter16<false>(l, lane);
+            else
+                sum = warp_reduce_scatter32<false>(l, lane);
+            if (lane < kH) lw[lane] = sum;
+            if (NR == 32 && r0 == 0) lw[32 + lane] = 0.f;                  // unused rows
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&bar[kBarSMDone + pb]);
@@ -685,7 +653,7 @@ __global__ void __maxnreg__(152)
         const int q = warp & 3;                               // TMEM lane quadrant
         const int chn = 32 * q + lane;                        // head-dimension channel
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-        const bool leader = warp == 4 && lane == 0;
+        const bool leader = warp == kAttnEpiWarp && lane == 0;
         for (int p = 0;; ++p) {
             const int pb = p & 1;
             cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort);
@@ -707,45 +675,50 @@ __global__ void __maxnreg__(152)
                 f_inv[r] = L > 0.f ? 1.f / L : 0.f;
                 f_lse[r] = L > 0.f ? s_m[pb * 64 + r] + log2f(L) : kNegInf;
             }
-            float o[NR];
-            if (n > 0) {
+            named_bar_sync(kNbEpi, 128);                      // 1/sum and lse ready; m and sums read
+            const int b = u / d.Hkv, h = u - b * d.Hkv;
+            const bool direct = ncu == 1;
+            float* dst = ws_o + static_cast<long long>(c) * rows * kHeadDim;
+            // O^T, 32 rows at a time: head + remainder products of this thread's channel
 #pragma unroll
-                for (int hh = 0; hh < NR / 32; ++hh) {                 // head + remainder products
-                    uint32_t v[32], w[32];
+            for (int hh = 0; hh < NR / 32; ++hh) {
+                uint32_t v[32];
+                float o[32];
+                if (n > 0) {
                     tmem_ld_32x32b_x32(tmem + lane_base + kOCol + pb * kOStride + 32 * hh, v);
-                    tmem_ld_32x32b_x32(tmem + lane_base + kOCol + pb * kOStride + NR + 32 * hh, w);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int r = 0; r < 32; ++r) o[32 * hh + r] = __uint_as_float(v[r]) + __uint_as_float(w[r]);
-                }
-            } else {
+                    for (int r = 0; r < 32; ++r) o[r] = __uint_as_float(v[r]);
+                    tmem_ld_32x32b_x32(tmem + lane_base + kOCol + pb * kOStride + NR + 32 * hh, v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int r = 0; r < NR; ++r) o[r] = 0.f;
+                    for (int r = 0; r < 32; ++r) o[r] += __uint_as_float(v[r]);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) o[r] = 0.f;
+                }
+#pragma unroll
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = 32 * hh + rr;
+                    if (r >= rows) break;
+                    if (direct) {
+                        const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
+                        out[orow * kHeadDim + chn] = o[rr] * f_inv[r];
+                    } else {
+                        dst[r * kHeadDim + chn] = o[rr] * f_inv[r];
+                    }
+                }
             }
             tc_fence_before_sync();
-            named_bar_sync(kNbEpi, 128);       // O^T, running max and sums read; 1/sum and lse ready
+            named_bar_sync(kNbEpi, 128);                      // every thread has read its O^T
             if (leader) mbar_arrive(&bar[kBarOFree + pb]);
-            const int b = u / d.Hkv, h = u - b * d.Hkv;
-            if (ncu == 1) {
-                // the chunk is the whole unit: final output
-#pragma unroll
-                for (int r = 0; r < NR; ++r) {
-                    if (r >= rows) break;
-                    const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
-                    out[orow * kHeadDim + chn] = o[r] * f_inv[r];
-                }
+            if (direct) {
                 if (q < 2 && 32 * q + lane < rows) {
                     const int r = 32 * q + lane;
                     const long long orow = (static_cast<long long>(b) * d.Qn + r / G) * d.Hq + h * G + r % G;
                     lse_out[orow] = f_lse[r] * kLn2;
                 }
             } else {
-                float* dst = ws_o + static_cast<long long>(c) * rows * kHeadDim;
-#pragma unroll
-                for (int r = 0; r < NR; ++r) {
-                    if (r >= rows) break;
-                    dst[r * kHeadDim + chn] = o[r] * f_inv[r];
-                }
                 if (q < 2 && 32 * q + lane < rows) ws_lse[static_cast<long long>(c) * rows + 32 * q + lane] = f_lse[32 * q + lane];
                 __threadfence();
                 named_bar_sync(kNbEpi, 128);
@@ -779,14 +752,14 @@ __global__ void __maxnreg__(152)
                         lse_out[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : kNegInf;
                     }
                     named_bar_sync(kNbEpi, 128);
-                    // 32 threads per row (4 channels each), 4 rows per row-set, two row-sets per
-                    // pass: up to 16 float4 loads in flight per thread
+                    // 32 threads per row (4 channels each), 4 rows per pass: up to 8 float4
+                    // loads in flight per thread
                     const int et = 32 * q + lane;
                     const int rsub = et >> 5, c4 = (et & 31) * 4;
-                    for (int r0 = 0; r0 < rows; r0 += 8) {
-                        float4 xv[2][kAttnMaxChunks];
+                    for (int r0 = 0; r0 < rows; r0 += 4) {
+                        float4 xv[1][kAttnMaxChunks];
 #pragma unroll
-                        for (int s2 = 0; s2 < 2; ++s2) {
+                        for (int s2 = 0; s2 < 1; ++s2) {
                             const int r = r0 + 4 * s2 + rsub;
 #pragma unroll
                             for (int jj = 0; jj < kAttnMaxChunks; ++jj)
@@ -796,7 +769,7 @@ __global__ void __maxnreg__(152)
                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
                         }
 #pragma unroll
-                        for (int s2 = 0; s2 < 2; ++s2) {
+                        for (int s2 = 0; s2 < 1; ++s2) {
                             const int r = r0 + 4 * s2 + rsub;
                             if (r >= rows) continue;
                             const float* w = s_mw + r * kAttnMaxChunks;

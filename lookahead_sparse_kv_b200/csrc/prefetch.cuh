@@ -13,9 +13,9 @@
 // bandwidth-delay product (~55 GB/s x a few microseconds).  Measured on B200:
 // 16, 32 and 64 CTAs all gather at 51 GB/s, 8 at 45 GB/s; and an attention or
 // scoring CTA that shares an SM with a gather CTA runs 1.4-2.5x slower, so
-// the fewer SMs the gather occupies the better.  Its 48 registers a thread
-// (launch bound of 10 CTAs per SM) leave room beside an attention CTA
-// (384 threads x 152 registers) in the 64K-register file.  Only real fetches are visited: a CTA takes the prefix sum of
+// the fewer SMs the gather occupies the better.  It keeps to 48 registers a
+// thread (launch bound of 10 CTAs per SM) and 4 KB of shared memory, so it
+// fits beside a scoring CTA.  Only real fetches are visited: a CTA takes the prefix sum of
 // the units' fetch counts (1,024 units per pass, in shared memory), numbers
 // the fetches of all units consecutively, and takes every gridDim-th pair;
 // a binary search over the prefix maps a fetch number back to (unit, entry).
