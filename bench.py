@@ -457,6 +457,9 @@ def load_traffic(workload: str):
 
 
 # ------------------------------------------------------------------- run
+HOST_COVER_CYCLES = 400_000       # ~0.2 ms of device spin ahead of each isolated launch
+
+
 def isolated_kernel_ms(st, reps: int = 20) -> dict:
     """Each library call of one layer-step timed alone on one stream (no
     concurrent kernels), for per-kernel rooflines."""
@@ -488,6 +491,9 @@ def isolated_kernel_ms(st, reps: int = 20) -> dict:
         n = 3 if name == "build_summaries" else reps          # ~20 ms each: 1 GiB over PCIe
         for _ in range(n):
             flush.zero_()                                  # evict L2 between launches
+            # keep the device busy while the host enqueues the call, so the
+            # events time the kernel and not the host's launch work
+            torch.cuda._sleep(HOST_COVER_CYCLES)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(s)
             fn()

@@ -170,7 +170,7 @@ int oasis_score_select_rows(const oasis_dims* d, const void* q, int32_t row_begi
  * memory; ws: a workspace of oasis_workspace_bytes(d) bytes.  The plan reads
  * and rewrites slot_table / last_used, so it must run after any attention
  * that reads this layer's slot table.  EINVAL also when the fused kernel's
- * shared memory cannot hold one unit's N keys and plan (4*N + 8*K + 36*K
+ * shared memory cannot hold one unit's N keys and plan (up to 4*N + 64*K
  * bytes above 226 KiB, i.e. only near N = 32768 with a large K). */
 int oasis_score_select_plan(const oasis_dims* d, const void* q, const void* kmin,
                             const void* kmax, const int32_t* ctx_len, int32_t* sel,

@@ -480,6 +480,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int nvj = (static_cast<uint32_t>(myslot < 4 ? e[1] : e[2]) >> (8 * (myslot & 3))) & 0xFF;
                 const bool valid = mytok < nvj;
                 cta_wait(&bar[kBarSFull + st], (pos >> 1) & 1, s_abort);
+                __syncwarp();                                 // tcgen05.ld is warp-wide: lanes together
                 tc_fence_after_sync();
                 float x[kH];                                  // raw scores q.k of this token, rows r0..
                 if constexpr (kH == 16) {
@@ -550,6 +551,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (i > 0) {
                         // the previous tile's product must have landed in O^T before it is rescaled
                         cta_wait(&bar[kBarPFree + (pos - 1) % kPBufs], ((pos - 1) / kPBufs) & 1, s_abort);
+                        __syncwarp();
                         tc_fence_after_sync();
 #pragma unroll
                         for (int part = 0; part < 2 * kH / 16; ++part) {   // head and remainder columns

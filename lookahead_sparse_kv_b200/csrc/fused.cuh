@@ -24,16 +24,23 @@
 //             two TMEM accumulators;
 //   warps 2-5 read the accumulators back (one TMEM lane quadrant each: 32
 //             blocks per warp), take the max over the real columns and store
-//             the fp32 scores; after a chunk they add one to the unit's
-//             ticket;
-//   warps 6-9 claim units in order from a second counter (so every CTA
-//             selects and plans about B*Hkv / CTAs units, whichever CTAs
-//             scored them), wait until the unit's ticket shows all its chunks
-//             scored, read its scores back from L2 into shared memory and run
-//             the top-K selection (select_unit) and the plan (plan_unit),
-//             while the other warps score on.
+//             the fp32 scores;
+//   warps 6-9 run the top-K selection and the plan of a unit once all of it
+//             is scored, while the other warps score on.
+// Two ways a unit reaches the selection:
+//   - whole units (a chunk covers a unit, used when units >= CTAs): the
+//     epilogue also keeps the unit's keys in shared memory and hands them to
+//     the CTA's own selection warps (an mbarrier each way), which read them
+//     into registers;
+//   - split units: after a chunk the epilogue adds one to the unit's ticket;
+//     the selection warps claim units in order from a second counter (so
+//     every CTA selects about B*Hkv / CTAs units, whichever CTAs scored them),
+//     wait until the unit's ticket shows all its chunks scored and read its
+//     scores from L2 into registers.
+// The selection runs on keys in registers (select_unit_regs) up to 64 keys a
+// thread (N <= 8192), else on keys in shared memory (select_unit).
 // Results are those of the separate lookahead_score / select_topk / plan
-// kernels bit for bit (the same MMA, the same select_unit and plan_unit).
+// kernels bit for bit (the same MMA, the same selection rule and plan_unit).
 // The last CTA to exit resets the counters for the next call.
 #pragma once
 
@@ -62,15 +69,19 @@ constexpr int kSspQFull = 12;     // [2] unit's query rows landed in the operand
 constexpr int kSspCFull = 14;     // [2] chunk description written (producer)
 constexpr int kSspCFree = 16;     // [2] description read (MMA issuer, epilogue leader)
 constexpr int kSspFinal = 18;
-constexpr int kSspNumBars = 19;
+constexpr int kSspKFull = 19;     // whole units: the unit's keys are in shared memory (epilogue leader)
+constexpr int kSspKFree = 20;     // whole units: the selection warps have read them
+constexpr int kSspNumBars = 21;
 constexpr uint32_t kSspNbEpiVote = 3;                      // named barrier of the epilogue's stop vote
 
 // Chunking of the scoring work (host and device agree through these).
 struct SspChunks {
-    int cts;   // tiles per chunk
-    int cpu;   // chunks per unit (ceil(ceil(N / 128) / cts))
-    int nc;    // chunks in all
+    int cts;     // tiles per chunk
+    int cpu;     // chunks per unit (ceil(ceil(N / 128) / cts))
+    int nc;      // chunks in all
+    int whole;   // cts covers every unit (cpu == 1): keys handed over in shared memory
 };
+constexpr int kSspRegKeys = 64;                            // keys a tail thread holds in registers at most
 
 template <int NPAD>
 struct SspSmem {
@@ -82,13 +93,40 @@ struct SspSmem {
     static constexpr int kAccStride = NPAD <= 16 ? 16 : (NPAD <= 32 ? 32 : 64);   // TMEM columns per accumulator
     static constexpr int kTmemCols = 2 * kAccStride < 32 ? 32 : 2 * kAccStride;
     // total dynamic bytes for nbuf operand buffers, budget K and N blocks
-    // (candidates, plan scratch, the unit's keys; +1024 alignment slack)
+    // (candidates, plan scratch, the unit's keys rounded up to 4; +1024
+    // alignment slack)
     static constexpr int bytes(int nbuf, int K, int N) {
         int kp = 2;                                  // >= 2 keeps the plan scratch 16-B aligned
         while (kp < K) kp <<= 1;
-        return kOffCand(nbuf) + kp * 8 + plan_smem_ints(K) * 4 + N * 4 + 1024;
+        return kOffCand(nbuf) + kp * 8 + plan_smem_ints(K) * 4 + ((N + 3) & ~3) * 4 + 1024;
     }
 };
+
+// The i-th tile a chunk of nt tiles starting at t0 of unit u takes: the
+// chunk's tiles rotated by a unit-dependent amount.
+__device__ __forceinline__ int ssp_tile(int u, int t0, int nt, int i) {
+    const int r = i + (u * 7) % nt;
+    return t0 + (r >= nt ? r - nt : r);
+}
+
+// Selection of one unit by the tail warps with PER keys a thread in
+// registers, read from the handed-over keys in shared memory (whole units;
+// kfree is then arrived once they are read) or from the scores in L2.
+template <int PER>
+__device__ __forceinline__ void ssp_select_regs(bool from_smem, const uint32_t* keys, const float* su, bool vec4, int nv,
+                                                int K, unsigned long long* cand, SelScratch* sc, int32_t* sel_u,
+                                                float* ss_u, int32_t* s_sel, uint64_t* kfree) {
+    uint32_t kk[PER];
+    if (from_smem)
+        rk_load_keys<SspTailGroup, PER>(kk, keys, nv);
+    else
+        rk_load_scores<SspTailGroup, PER>(kk, su, nv, vec4);
+    if (kfree) {
+        SspTailGroup::sync();                                  // every thread has its keys
+        if (SspTailGroup::tid() == 0) mbar_arrive(kfree);
+    }
+    select_unit_regs<SspTailGroup, PER>(kk, nv, K, cand, sc, su, sel_u, ss_u, s_sel);
+}
 
 template <int NPAD, bool kScored>
 __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
@@ -111,6 +149,7 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
     volatile int* s_abort = misc + 1;
     int* s_info = misc + 8;                               // [2][kSspInfoInts] chunk descriptions
     volatile int* s_claim = misc + 24;                    // the tail group's claimed unit
+    volatile int* s_kunit = misc + 25;                    // whole units: the unit whose keys are handed over
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + S::kOffCand(nbuf));
     int kp = 2;
     while (kp < d.K) kp <<= 1;
@@ -124,7 +163,7 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
         for (int i = 0; i < kSspNumBars; ++i)
             mbar_init(&bar[i], (i == kSspAccFree || i == kSspAccFree + 1) ? 4
                                : (i == kSspCFree || i == kSspCFree + 1) ? 2
-                                                                         : 1);
+                                                                         : 1);   // KFull, KFree: 1
         fence_mbar_init();
         *s_abort = 0;
     }
@@ -194,9 +233,12 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
                 break;
             }
             const int ts = min(t0 + ch.cts, (nv + kScoreTile - 1) / kScoreTile);   // scored tiles [t0, ts)
+            // the chunk's tiles are taken in a rotated order (ssp_tile), so CTAs that
+            // start together read different offsets of their units
+            const int nt = ts - t0;
             // as many tiles as the ring holds go out first: they wait only on earlier
             // chunks' products; the rest wait on this chunk's, so the operand comes first
-            const int t_pre = min(ts, t0 + kSspStages);
+            const int n_pre = min(nt, kSspStages);
             if (lane == 0) {
                 info[0] = 0;
                 info[1] = u;
@@ -205,7 +247,7 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
                 info[4] = ts;
                 info[5] = vt;
                 mbar_arrive(&bar[kSspCFull + pb]);
-                for (int t = t0; t < t_pre; ++t) load_tile(u, t);
+                for (int i = 0; i < n_pre; ++i) load_tile(u, ssp_tile(u, t0, nt, i));
             }
             __syncwarp();
             if (ts > t0) {
@@ -244,7 +286,7 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&bar[kSspBFull + bb]);
-                    for (int t = t_pre; t < ts; ++t) load_tile(u, t);
+                    for (int i = n_pre; i < nt; ++i) load_tile(u, ssp_tile(u, t0, nt, i));
                 }
                 ++nb;
             }
@@ -308,10 +350,21 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             cta_wait(&bar[kSspCFull + pb], (p >> 1) & 1, s_abort);
             const int* info = s_info + pb * kSspInfoInts;
             const int end = info[0], u = info[1], nv = info[2], t0 = info[3], ts = info[4];
-            if (named_bar_or(kSspNbEpiVote, 128, end != 0 || *s_abort)) break;
-            for (int t = t0; t < ts; ++t, ++pos) {
+            // whole units: the previous unit's keys must have been read before
+            // this unit's (or the end mark) go into shared memory
+            if (ch.whole && p > 0) cta_wait(&bar[kSspKFree], (p - 1) & 1, s_abort);
+            if (named_bar_or(kSspNbEpiVote, 128, end != 0 || *s_abort)) {
+                if (ch.whole && leader) {
+                    *s_kunit = -1;
+                    mbar_arrive(&bar[kSspKFull]);
+                }
+                break;
+            }
+            for (int i = 0; i < ts - t0; ++i, ++pos) {
+                const int t = ssp_tile(u, t0, ts - t0, i);
                 const int ab = pos & 1;
                 const bool ok = cta_wait(&bar[kSspAccFull + ab], (pos >> 1) & 1, s_abort);
+                __syncwarp();                                      // tcgen05.ld is warp-wide: lanes together
                 tc_fence_after_sync();
                 float best = -__int_as_float(0x7f800000);
                 if (ok) {
@@ -329,60 +382,124 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[kSspAccFree + ab]);
                 const int n = t * kScoreTile + qd * 32 + lane;
-                if (ok && n < nv) scores[u * N + n] = best;
+                if (ok && n < nv) {
+                    scores[u * N + n] = best;
+                    if (ch.whole) keys[n] = ordered_key(best);
+                }
             }
-            // the chunk's scores are out: one more chunk of the unit done
-            __threadfence();
-            SspEpiGroup::sync();
-            if (leader) {
-                atomicAdd(ticket + u, 1);
-                mbar_arrive(&bar[kSspCFree + pb]);
+            if (ch.whole) {
+                // the unit's keys (and scores) are out: hand them to the selection warps
+                SspEpiGroup::sync();
+                if (leader) {
+                    *s_kunit = u;
+                    mbar_arrive(&bar[kSspKFull]);
+                    mbar_arrive(&bar[kSspCFree + pb]);
+                }
+            } else {
+                // the chunk's scores are out: one more chunk of the unit done
+                __threadfence();
+                SspEpiGroup::sync();
+                if (leader) {
+                    atomicAdd(ticket + u, 1);
+                    mbar_arrive(&bar[kSspCFree + pb]);
+                }
             }
         }
     } else {
         // ====================================== top-K + plan tail (6..9)
         const int ttid = SspTailGroup::tid();
         const int units = d.B * d.Hkv;
-        while (true) {
-            // claim the next unit; wait until every chunk of it holding valid blocks is scored
-            if (ttid == 0) {
-                int u = *s_abort ? units : atomicAdd(sched + 2, 1);
-                if (u < units) {
-                    const int nvu = n_valid_blocks(ctx_len[u / d.Hkv], d.N);
-                    const int vt = max(1, (nvu + kScoreTile - 1) / kScoreTile);
-                    const int chunks = (vt + ch.cts - 1) / ch.cts;
-                    const uint64_t t0 = global_timer_ns();
-                    while (ld_acquire_gpu(ticket + u) < chunks) {
-                        if (global_timer_ns() - t0 > kWaitLimitNs) {   // bounded: give up, flag it
-                            *s_abort = 1;
-                            raise_dev_error(OASIS_DEVERR_TIMEOUT);
-                            u = units;
-                            break;
-                        }
-                        __nanosleep(64);
+        const bool vec4 = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
+        int32_t* s_sel = slot_table != nullptr ? plan_sel_smem(sp, d.K) : nullptr;
+        for (int k = 0;; ++k) {
+            int u;
+            if (ch.whole) {
+                // the next unit this CTA scored (one thread waits, the others at the barrier)
+                if (ttid == 0) {
+                    bool ok = !*s_abort;
+                    if (ok && !mbar_wait_idle(&bar[kSspKFull], k & 1)) {
+                        *s_abort = 1;
+                        raise_dev_error(OASIS_DEVERR_TIMEOUT);
+                        ok = false;
                     }
+                    *s_claim = ok ? *s_kunit : -1;
                 }
-                *s_claim = u;
+                SspTailGroup::sync();
+                u = *s_claim;
+                SspTailGroup::sync();
+                if (u < 0) break;
+            } else {
+                // claim the next unit; wait until every chunk of it holding valid blocks is scored
+                if (ttid == 0) {
+                    int c = *s_abort ? units : atomicAdd(sched + 2, 1);
+                    if (c < units) {
+                        const int nvu = n_valid_blocks(ctx_len[c / d.Hkv], d.N);
+                        const int vt = max(1, (nvu + kScoreTile - 1) / kScoreTile);
+                        const int chunks = (vt + ch.cts - 1) / ch.cts;
+                        const uint64_t t0 = global_timer_ns();
+                        while (ld_acquire_gpu(ticket + c) < chunks) {
+                            if (global_timer_ns() - t0 > kWaitLimitNs) {   // bounded: give up, flag it
+                                *s_abort = 1;
+                                raise_dev_error(OASIS_DEVERR_TIMEOUT);
+                                c = units;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                    }
+                    *s_claim = c;
+                }
+                SspTailGroup::sync();
+                u = *s_claim;
+                SspTailGroup::sync();
+                if (u >= units) break;
+                if (ttid == 0) ticket[u] = 0;                  // ready for the next call
             }
-            SspTailGroup::sync();
-            const int u = *s_claim;
-            SspTailGroup::sync();
-            if (u >= units) break;
-            if (ttid == 0) ticket[u] = 0;                      // ready for the next call
             const int nv = n_valid_blocks(ctx_len[u / d.Hkv], d.N);
             const float* su = scores + u * N;
-            for (int i = ttid; i < nv; i += SspTailGroup::kThreads) keys[i] = ordered_key(__ldcg(su + i));
-            SspTailGroup::sync();
-            int32_t* sel_u = sel + static_cast<long long>(u) * d.K;
-            select_unit<SspTailGroup>(SmemKeys{keys}, nv, d.K, cand, &sc, su, sel_u,
-                                      sel_score ? sel_score + static_cast<long long>(u) * d.K : nullptr);
-            if (slot_table == nullptr) continue;
-            SspTailGroup::sync();                              // the selection is in memory
-            const int stp = step_dev != nullptr ? *step_dev : step;
             const long long uk = static_cast<long long>(u) * d.K, uc = static_cast<long long>(u) * d.C;
-            plan_unit<SspTailGroup, kScored>(d.K, d.C, d.N, sel_u, kScored ? su : nullptr, slot_table + uk,
+            // the unit's slot table and recency, loaded now and used by the plan
+            // after the selection (the loads are in flight meanwhile)
+            const bool pre = slot_table != nullptr && d.K <= 2 * SspTailGroup::kThreads;
+            int32_t pst[2] = {-1, -1}, plu[2] = {0, 0};
+            if (pre) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int i = ttid + h * SspTailGroup::kThreads;
+                    if (i < d.K) {
+                        pst[h] = __ldcg(slot_table + uk + i);
+                        plu[h] = __ldcg(last_used + uk + i);
+                    }
+                }
+            }
+            int32_t* sel_u = sel + static_cast<long long>(u) * d.K;
+            float* ss_u = sel_score ? sel_score + static_cast<long long>(u) * d.K : nullptr;
+            uint64_t* kfree = ch.whole ? &bar[kSspKFree] : nullptr;
+            if (nv <= 16 * SspTailGroup::kThreads) {
+                ssp_select_regs<16>(ch.whole != 0, keys, su, vec4, nv, d.K, cand, &sc, sel_u, ss_u, s_sel, kfree);
+            } else if (nv <= kSspRegKeys * SspTailGroup::kThreads) {
+                ssp_select_regs<kSspRegKeys>(ch.whole != 0, keys, su, vec4, nv, d.K, cand, &sc, sel_u, ss_u, s_sel,
+                                             kfree);
+            } else {
+                // more keys than registers: the unit's keys in shared memory
+                if (!ch.whole) {
+                    for (int i = ttid; i < nv; i += SspTailGroup::kThreads) keys[i] = ordered_key(__ldcg(su + i));
+                    SspTailGroup::sync();
+                }
+                select_unit<SspTailGroup>(SmemKeys{keys}, nv, d.K, cand, &sc, su, sel_u, ss_u, s_sel);
+                if (kfree) {
+                    SspTailGroup::sync();                      // keys no longer read
+                    if (ttid == 0) mbar_arrive(kfree);
+                }
+            }
+            if (slot_table == nullptr) {
+                SspTailGroup::sync();                          // cand / scratch free for the next unit
+                continue;
+            }
+            const int stp = step_dev != nullptr ? *step_dev : step;
+            plan_unit<SspTailGroup, kScored>(d.K, d.C, d.N, s_sel, kScored ? su : nullptr, slot_table + uk,
                                              last_used + uk, stp, fetch_slot + uc, fetch_block + uc, n_fetch + u, sp,
-                                             tmp);
+                                             tmp, pre ? pst : nullptr, pre ? plu : nullptr);
             SspTailGroup::sync();                              // scratch free for the next unit
         }
     }

@@ -311,6 +311,7 @@ int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const CUtenso
     ch.cts = (tpu + want - 1) / want;
     ch.cpu = (tpu + ch.cts - 1) / ch.cts;
     ch.nc = static_cast<int>(units * ch.cpu);
+    ch.whole = ch.cpu == 1 ? 1 : 0;
     const int ctas = std::min(sm_count(), ch.nc);
     k<<<ctas, oasis::kSspThreads, smem, s>>>(tmax, tmin, tq, d, q, ctx, scores, row0, rows, ticket, sched, sel, sel_score,
                                              st, lu, step, step_dev, fs, fb, nf, ch, nbuf);
@@ -411,11 +412,11 @@ int plan(const oasis_dims* dp, const int32_t* sel, const float* scores, int32_t*
     const int smem = oasis::plan_smem_ints(d.K) * static_cast<int>(sizeof(int32_t));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (scores != nullptr) {
-        if (int rc = carveout(oasis::plan_fetch_kernel<true>, "plan carve-out")) return rc;
+        if (int rc = set_smem(oasis::plan_fetch_kernel<true>, smem, "plan smem")) return rc;
         oasis::plan_fetch_kernel<true><<<d.B * d.Hkv, oasis::kPlanThreads, smem, s>>>(
             d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
     } else {
-        if (int rc = carveout(oasis::plan_fetch_kernel<false>, "plan carve-out")) return rc;
+        if (int rc = set_smem(oasis::plan_fetch_kernel<false>, smem, "plan smem")) return rc;
         oasis::plan_fetch_kernel<false><<<d.B * d.Hkv, oasis::kPlanThreads, smem, s>>>(
             d, sel, scores, slot_table, last_used, step, step_dev, fetch_slot, fetch_block, n_fetch);
     }
@@ -505,9 +506,7 @@ int oasis_select_topk(const oasis_dims* dp, const float* scores, const int32_t* 
     if (int rc = check_ptr(ctx_len, "ctx_len")) return rc;
     if (int rc = check_ptr(sel, "sel")) return rc;
     if (int rc = check_ptr(sel_score, "sel_score", true)) return rc;
-    const int smem = d.N * static_cast<int>(sizeof(uint32_t));
-    if (int rc = set_smem(oasis::select_topk_kernel, smem, "select smem")) return rc;
-    oasis::select_topk_kernel<<<d.B * d.Hkv, oasis::kSelThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+    oasis::select_topk_kernel<<<d.B * d.Hkv, oasis::kSelThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         d, scores, ctx_len, sel, sel_score);
     return check_launch("select_topk launch");
 }

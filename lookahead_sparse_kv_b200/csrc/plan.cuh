@@ -6,14 +6,17 @@
 // Table 2 (LRU eviction), Figure 9 (a per-KV-head table maps each GPU
 // block slot to a CPU block), "Terms in this paper" (capped eviction).
 //
-// One CTA per (b, h) with one thread per slot / rank (K <= 1024):
-//   1. thread i looks up sel[i] in the slot table (K compares in smem);
-//      hits protect their slot and stamp it with the step;
-//   2. misses are numbered in rank order by a block-wide scan; the first
+// One group of threads per (b, h), each thread looping over slots / ranks
+// (K <= 1024):
+//   1. the resident blocks go into a hash table in shared memory (block id ->
+//      lowest slot holding it; a second slot with the same block is an
+//      error); each selected block looks itself up there, and hits protect
+//      their slot and stamp it with the step;
+//   2. misses are numbered in rank order by a group-wide scan; the first
 //      min(C, |M|) are fetched;
-//   3. every unprotected slot j gets a 64-bit victim key - free slots
-//      (0, j), stale slots (1, order, block id) - and its rank among the
-//      candidates by counting smaller keys; rank r < nF receives fetch r.
+//   3. every unprotected slot j has a 64-bit victim key - free slots (0, j),
+//      stale slots (1, order, block id) - and its rank among the candidates
+//      by counting smaller keys; rank r < nF receives fetch r.
 //      order = last_used (LRU, Table 2) or, for the score-based variant of
 //      the eviction ablation, the block's current lookahead score mapped to
 //      a monotone integer key (lowest score evicted first).
@@ -34,18 +37,33 @@ __device__ __forceinline__ unsigned long long victim_key(int slot, int blk, uint
 
 constexpr int kPlanThreads = 256;
 
-// Shared-memory ints plan_unit needs for budget K (nine arrays of K rounded
-// up to a multiple of 4, so the scans over slots read 16 B at a time).
+// Shared-memory layout of plan_unit for budget K, in ints: eight arrays of K
+// rounded up to a multiple of 4 (so the scans over slots read 16 B at a
+// time), the victim keys (64-bit, same count) and the hash table (2 entries
+// per slot, a power of two).
 __host__ __device__ constexpr int plan_k4(int K) { return (K + 3) & ~3; }
-__host__ __device__ constexpr int plan_smem_ints(int K) { return 9 * plan_k4(K); }
+__host__ __device__ constexpr int plan_pow2(int K) { return K <= 1 ? 1 : 2 * plan_pow2((K + 1) / 2); }
+__host__ __device__ constexpr int plan_hash_size(int K) { return K <= 2 ? 4 : 2 * plan_pow2(K); }   // >= 4: 16-B multiple
+__host__ __device__ constexpr int plan_smem_ints(int K) { return 10 * plan_k4(K) + plan_hash_size(K); }
+// The selection's place in that layout: a caller may write the selection
+// there itself and pass this pointer as `sel`.
+__device__ __forceinline__ int32_t* plan_sel_smem(int32_t* sp, int K) { return sp + 6 * plan_k4(K); }
+
+constexpr uint32_t kPlanHashEmpty = 0xFFFFFFFFu;
+__device__ __forceinline__ uint32_t plan_hash(uint32_t blk, int log2_size) {
+    return (blk * 0x9E3779B1u) >> (32 - log2_size);
+}
 
 // Plan of one (b, h) by a group of threads (each loops over slots /
 // ranks): sel, st, lu point at the unit's K entries, fs/fb at its C fetch
 // entries, nf at its fetch count; scores_u (kScored) at its N block scores.
-// sp: plan_smem_ints(K) ints of shared memory; tmp: 32 ints.
+// sp: plan_smem_ints(K) ints of shared memory, 16-B aligned; tmp: 32 ints.
+// pre_st / pre_lu (K <= 2 * NT, may be NULL): st[tid + h * NT] and
+// lu[tid + h * NT] for h = 0, 1, already loaded by the caller.
 template <class Grp, bool kScored>
 __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* scores_u, int32_t* st, int32_t* lu,
-                          int step, int32_t* fs, int32_t* fb, int32_t* nf, int32_t* sp, int* tmp) {
+                          int step, int32_t* fs, int32_t* fb, int32_t* nf, int32_t* sp, int* tmp,
+                          const int32_t* pre_st = nullptr, const int32_t* pre_lu = nullptr) {
     constexpr int NT = Grp::kThreads;
     const int K4 = plan_k4(K);
     int32_t* s_st = sp;
@@ -54,58 +72,90 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
     int32_t* s_vict = sp + 3 * K4;
     int32_t* s_nst = sp + 4 * K4;
     int32_t* s_nlu = sp + 5 * K4;
-    uint32_t* s_ord = reinterpret_cast<uint32_t*>(sp + 6 * K4);
-    int32_t* s_sel = sp + 7 * K4;
-    int32_t* s_mpos = sp + 8 * K4;         // miss flag, then the miss's position in rank order (-1: no miss)
+    int32_t* s_sel = sp + 6 * K4;          // == plan_sel_smem(sp, K)
+    int32_t* s_mpos = sp + 7 * K4;         // miss flag, then the miss's position in rank order (-1: no miss)
+    unsigned long long* s_vk = reinterpret_cast<unsigned long long*>(sp + 8 * K4);   // victim keys, ~0: not a victim
+    uint32_t* s_hash = reinterpret_cast<uint32_t*>(sp + 10 * K4);
+    const int hs = plan_hash_size(K), hlog = __ffs(hs) - 1;
     const int tid = Grp::tid();
     for (int i = K + tid; i < K4; i += NT) {   // padding: never matches, never a victim
         s_st[i] = -2;
         s_prot[i] = 1;
-        s_ord[i] = 0u;
+        s_vk[i] = ~0ull;
     }
-    for (int i = tid; i < K; i += NT) {
-        int x = st[i];
+    for (int i = tid; i < hs; i += NT) s_hash[i] = kPlanHashEmpty;
+    const bool sel_here = sel == s_sel;
+    auto stage = [&](int i, int x, int l) {
         if (x < -1 || x >= N) {
             raise_dev_error(OASIS_DEVERR_ID_RANGE);
             x = -1;
         }
         s_st[i] = x;
-        s_lu[i] = lu[i];
+        s_lu[i] = l;
         s_prot[i] = 0;
+        uint32_t ord;
         if constexpr (kScored)
-            s_ord[i] = x >= 0 ? ordered_key(__ldcg(scores_u + x)) : 0u;
+            ord = x >= 0 ? ordered_key(__ldcg(scores_u + x)) : 0u;
         else
-            s_ord[i] = static_cast<uint32_t>(s_lu[i]) ^ 0x80000000u;   // signed order
-        int sv = sel[i];
-        if (sv < -1 || sv >= N) {
-            raise_dev_error(OASIS_DEVERR_ID_RANGE);
-            sv = -1;
+            ord = static_cast<uint32_t>(l) ^ 0x80000000u;   // signed order
+        s_vk[i] = victim_key(i, x, ord);
+        if (!sel_here) {
+            int sv = sel[i];
+            if (sv < -1 || sv >= N) {
+                raise_dev_error(OASIS_DEVERR_ID_RANGE);
+                sv = -1;
+            }
+            s_sel[i] = sv;
         }
-        s_sel[i] = sv;
+    };
+    if (pre_st != nullptr) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            if (tid + h * NT < K) stage(tid + h * NT, pre_st[h], pre_lu[h]);
+    } else {
+        for (int i = tid; i < K; i += NT) stage(i, st[i], lu[i]);
     }
     Grp::sync();
-    // 1. residency lookup of every selected block (hits are protected), and a
-    //    check that no block is resident twice; 4 slots per shared-memory read
-    const int4* st4 = reinterpret_cast<const int4*>(s_st);
+    // 1a. resident blocks into the table: entry (block << 10 | slot); a block
+    //     found there already is resident twice (the lower slot is kept)
     for (int i = tid; i < K; i += NT) {
-        const int sv = s_sel[i], own = s_st[i];
-        int hit = 0x7FFFFFFF;
-        bool dup = false;
-#pragma unroll 4
-        for (int j4 = 0; j4 < K4 / 4; ++j4) {
-            const int4 x = st4[j4];
-            const int j = 4 * j4;
-            if (x.w == sv) hit = min(hit, j + 3);
-            if (x.z == sv) hit = min(hit, j + 2);
-            if (x.y == sv) hit = min(hit, j + 1);
-            if (x.x == sv) hit = min(hit, j);
-            dup |= (x.x == own && j < i) | (x.y == own && j + 1 < i) | (x.z == own && j + 2 < i) |
-                   (x.w == own && j + 3 < i);
+        const int x = s_st[i];
+        if (x < 0) continue;
+        const uint32_t e = (static_cast<uint32_t>(x) << 10) | static_cast<uint32_t>(i);
+        uint32_t pos = plan_hash(static_cast<uint32_t>(x), hlog);
+        for (int probe = 0; probe < hs; ++probe) {
+            const uint32_t old = atomicCAS(s_hash + pos, kPlanHashEmpty, e);
+            if (old == kPlanHashEmpty) break;
+            if ((old >> 10) == static_cast<uint32_t>(x)) {
+                raise_dev_error(OASIS_DEVERR_DUPLICATE);
+                atomicMin(s_hash + pos, e);
+                break;
+            }
+            pos = (pos + 1) & (hs - 1);
         }
-        if (sv < 0) hit = 0x7FFFFFFF;
-        if (own >= 0 && dup) raise_dev_error(OASIS_DEVERR_DUPLICATE);
-        if (hit != 0x7FFFFFFF) s_prot[hit] = 1;
-        s_mpos[i] = (sv >= 0 && hit == 0x7FFFFFFF) ? 1 : 0;
+    }
+    Grp::sync();
+    // 1b. residency lookup of every selected block (hits are protected)
+    for (int i = tid; i < K; i += NT) {
+        const int sv = s_sel[i];
+        int hit = -1;
+        if (sv >= 0) {
+            uint32_t pos = plan_hash(static_cast<uint32_t>(sv), hlog);
+            for (int probe = 0; probe < hs; ++probe) {
+                const uint32_t e = s_hash[pos];
+                if (e == kPlanHashEmpty) break;
+                if ((e >> 10) == static_cast<uint32_t>(sv)) {
+                    hit = static_cast<int>(e & 1023u);
+                    break;
+                }
+                pos = (pos + 1) & (hs - 1);
+            }
+        }
+        if (hit >= 0) {
+            s_prot[hit] = 1;
+            s_vk[hit] = ~0ull;
+        }
+        s_mpos[i] = (sv >= 0 && hit < 0) ? 1 : 0;
     }
     Grp::sync();
     // 2. misses numbered in rank order
@@ -125,18 +175,16 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
         s_nst[i] = s_st[i];
         s_nlu[i] = prot ? step : s_lu[i];
         if (!prot && nF > 0) {
-            const unsigned long long mine = victim_key(i, s_st[i], s_ord[i]);
-            const int4* pr4 = reinterpret_cast<const int4*>(s_prot);
-            const uint4* or4 = reinterpret_cast<const uint4*>(s_ord);
-            int rank = 0;
-#pragma unroll 2
-            for (int j4 = 0; j4 < K4 / 4; ++j4) {
-                const int4 pr = pr4[j4], x = st4[j4];
-                const uint4 od = or4[j4];
-                const int j = 4 * j4;
-                rank += (!pr.x && victim_key(j, x.x, od.x) < mine) + (!pr.y && victim_key(j + 1, x.y, od.y) < mine) +
-                        (!pr.z && victim_key(j + 2, x.z, od.z) < mine) + (!pr.w && victim_key(j + 3, x.w, od.w) < mine);
+            const unsigned long long mine = s_vk[i];
+            const ulonglong2* vk2 = reinterpret_cast<const ulonglong2*>(s_vk);
+            int r0 = 0, r1 = 0;
+#pragma unroll 4
+            for (int j2 = 0; j2 < K4 / 2; j2 += 2) {
+                const ulonglong2 x = vk2[j2], y = vk2[j2 + 1];
+                r0 += (x.x < mine) + (x.y < mine);
+                r1 += (y.x < mine) + (y.y < mine);
             }
+            const int rank = r0 + r1;
             if (rank < nF) s_vict[rank] = i;
         }
     }

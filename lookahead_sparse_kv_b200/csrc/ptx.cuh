@@ -83,6 +83,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// As mbar_wait for a long wait by a thread with nothing else to do: it
+// sleeps between polls, leaving the issue slots to the working warps.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) return false;
+        __nanosleep(128);
+    }
+    return true;
+}
+
 // Load with acquire semantics at GPU scope (pairs with a release by a
 // __threadfence() + atomic in another CTA).
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
