@@ -307,7 +307,18 @@ int launch_fused(const CUtensorMap& tmax, const CUtensorMap& tmin, const CUtenso
     const int tpu = (d.N + oasis::kScoreTile - 1) / oasis::kScoreTile;
     oasis::SspChunks ch;
     const long long units = static_cast<long long>(d.B) * d.Hkv;
-    const int want = static_cast<int>(std::max<long long>(1, sm_count() / std::max(1ll, units)));
+    // Whole units when there are at least half as many units as SMs (the
+    // epilogue hands the keys over in shared memory; cutting units would not
+    // shorten the longest CTA's share by more than the hand-off saves).
+    // Fewer units: about two chunks per SM (a power of two per unit, at least
+    // two tiles a chunk), so every SM scores and the units finish one after
+    // another, their selections overlapping the scoring of later units.
+    int want = 1;
+    if (2 * units < sm_count()) {
+        const long long per = (2ll * sm_count() + units - 1) / units;
+        while (want < per) want <<= 1;
+        want = std::max(1, std::min(want, tpu / 2));
+    }
     ch.cts = (tpu + want - 1) / want;
     ch.cpu = (tpu + ch.cts - 1) / ch.cts;
     ch.nc = static_cast<int>(units * ch.cpu);
