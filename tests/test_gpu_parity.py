@@ -331,6 +331,85 @@ def test_score_select_plan_matches_separate_kernels_and_oracle(Hq, Hkv, Qn, N, K
         st, lu = plan["slot_table"], plan["last_used"]
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,Qn,N,K,C,victims", [
+    (12, 32, 8, 5, 600, 128, 16, "lru"),      # 96 units: whole units, keys handed over in shared memory
+    (10, 64, 8, 8, 300, 64, 8, "score"),      # 80 units, whole, score-ordered victims
+    (3, 16, 2, 2, 8192, 128, 8, "lru"),       # 6 units of 8192 blocks: many chunks a unit, 64 keys a thread
+    (3, 8, 2, 2, 9000, 64, 8, "lru"),         # more keys than the registers hold: shared-memory selection
+])
+def test_score_select_plan_modes(B, Hq, Hkv, Qn, N, K, C, victims):
+    """The fused launch in each of its ways of reaching the selection (whole
+    units handed over in shared memory, split units read back from L2 into
+    registers, and the shared-memory fallback past 64 keys a thread) against
+    the separate kernels bit for bit and against the oracle.  Summaries are
+    drawn directly (no KV), with a context that fills every block, one inside
+    the budget, one empty, and random lengths for the rest."""
+    d = _dims(B, Hq, Hkv, N, K, Qn, C)
+    g = _gen(900 + N + K + B)
+    kmin_h = (torch.randn(B, Hkv, N, 128, generator=g) - 0.5).to(torch.bfloat16)
+    kmax_h = (kmin_h.float() + torch.rand(B, Hkv, N, 128, generator=g) * 2).to(torch.bfloat16)
+    lens = [N * 16 - 7, min(N, K) * 16 - 20, 0] + [int(x) for x in torch.randint(1, N * 16, (B - 3,), generator=g)]
+    ctx = torch.tensor(lens[:B], dtype=torch.int32)
+    ctx_d = ctx.to(DEV)
+    kmin, kmax = kmin_h.to(DEV), kmax_h.to(DEV)
+    ws = torch.zeros(lsk.workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    ws2 = torch.zeros_like(ws)
+    okmin, okmax = f64(kmin_h), f64(kmax_h)
+    rng = np.random.default_rng(N + K + B)
+    st0 = np.full((B, Hkv, K), -1, dtype=np.int32)
+    nv = O.n_valid_blocks(ctx.numpy(), 16)
+    for b in range(B):
+        for h in range(Hkv):
+            if nv[b]:
+                ids = rng.permutation(int(nv[b]))[: rng.integers(0, min(K, int(nv[b])) + 1)]
+                st0[b, h, :len(ids)] = ids
+                st0[b, h] = rng.permutation(st0[b, h])
+    lu0 = np.where(st0 >= 0, rng.integers(-1, 5, size=st0.shape), -1).astype(np.int32)
+    F = {k: torch.from_numpy(v.copy()).to(DEV) for k, v in (("st", st0), ("lu", lu0))}
+    S = {k: torch.from_numpy(v.copy()).to(DEV) for k, v in (("st", st0), ("lu", lu0))}
+    for X in (F, S):
+        X.update(sel=torch.empty((B, Hkv, K), dtype=torch.int32, device=DEV),
+                 sel_score=torch.empty((B, Hkv, K), device=DEV),
+                 fs=torch.full((B, Hkv, max(C, 1)), -9, dtype=torch.int32, device=DEV),
+                 fb=torch.full((B, Hkv, max(C, 1)), -9, dtype=torch.int32, device=DEV),
+                 nf=torch.full((B, Hkv), -9, dtype=torch.int32, device=DEV),
+                 scores=torch.zeros((B, Hkv, N), device=DEV))
+    scored = victims == "score"
+    st, lu = st0, lu0
+    for step in range(5, 8):
+        q = (torch.randn(B, Qn, Hq, 128, generator=g) * 1.3).to(torch.bfloat16)
+        qd = q.to(DEV)
+        lsk.score_select_plan(d, qd, kmin, kmax, ctx_d, F["sel"], F["sel_score"], F["scores"] if scored else None,
+                              F["st"], F["lu"], step, None, F["fs"], F["fb"], F["nf"], ws)
+        if scored:
+            lsk.lookahead_scores(d, qd, kmin, kmax, ctx_d, S["scores"])
+            lsk.select_topk(d, S["scores"], ctx_d, S["sel"], S["sel_score"])
+            lsk.plan_fetch_scored(d, S["sel"], S["scores"], S["st"], S["lu"], step, S["fs"], S["fb"], S["nf"])
+        else:
+            lsk.score_select(d, qd, kmin, kmax, ctx_d, S["sel"], S["sel_score"], ws2)
+            lsk.plan_fetch(d, S["sel"], S["st"], S["lu"], step, S["fs"], S["fb"], S["nf"])
+        torch.cuda.synchronize()
+        assert lsk.read_device_error(clear=True) == 0
+        for key in ("sel", "sel_score", "st", "lu", "nf"):
+            assert torch.equal(F[key], S[key]), f"{key} differs from the separate kernels at step {step}"
+        for b in range(B):
+            for h in range(Hkv):
+                n = int(np_i32(F["nf"])[b, h])
+                assert n <= C
+                assert torch.equal(F["fs"][b, h, :n], S["fs"][b, h, :n])
+                assert torch.equal(F["fb"][b, h, :n], S["fb"][b, h, :n])
+        sc = O.lookahead_scores(f64(q), okmin, okmax, ctx.numpy(), 16)
+        ref_sel, _ = O.select_topk(sc, ctx.numpy(), K, 16)
+        sel = np_i32(F["sel"])
+        assert_selection_matches(sel, ref_sel, sc, ctx.numpy(), K)
+        assert (sel[2] == -1).all()
+        plan = O.plan_fetch(sel, st, lu, step, C, scores=F["scores"].cpu().numpy() if scored else None)
+        np.testing.assert_array_equal(np_i32(F["st"]), plan["slot_table"])
+        np.testing.assert_array_equal(np_i32(F["lu"]), plan["last_used"])
+        np.testing.assert_array_equal(np_i32(F["nf"]), plan["n_fetch"])
+        st, lu = plan["slot_table"], plan["last_used"]
+
+
 # --------------------------------------------------------------- prefetch
 def test_prefetch_bytes_exact():
     B, H, N, K, C = 2, 3, 50, 16, 6
