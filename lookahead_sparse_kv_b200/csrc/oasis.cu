@@ -743,7 +743,12 @@ int oasis_sparse_attn(const oasis_dims* dp, const void* q, const void* pool, con
     const float scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const oasis::AttnChunks chunks = attn_chunks(d, sm_count());
-    const unsigned ctas = static_cast<unsigned>(std::min(sm_count(), chunks.nc));
+    // An attention CTA fills an SM's register file, so no gather CTA fits
+    // beside it: leave the gather's SMs free, so a gather on the copy stream
+    // keeps running while the attention of another layer does (the chunks
+    // are taken from a counter, so fewer CTAs only take more chunks each).
+    const int grid_max = std::max(1, sm_count() - oasis::kPrefetchCtas);
+    const unsigned ctas = static_cast<unsigned>(std::min(grid_max, chunks.nc));
     auto kern = d.Qn * d.G() <= 32 ? oasis::sparse_attn_kernel<32> : oasis::sparse_attn_kernel<64>;
     if (int rc = set_smem(kern, oasis::kAttnSmem, "sparse_attn smem")) return rc;
     kern<<<ctas, oasis::kAttnThreads, oasis::kAttnSmem, s>>>(tk, tv, tq, d, slot_table, ctx_len, scale_log2, chunks,
