@@ -460,6 +460,20 @@ def load_traffic(workload: str):
 HOST_COVER_CYCLES = 400_000       # ~0.2 ms of device spin ahead of each isolated launch
 
 
+def fetch_history(steps: int, layers, device=None):
+    """Per-step, per-layer fetch counts of a timed run, in pinned host memory
+    filled by asynchronous device-to-host copies on the main stream: a copy
+    engine moves them, so no SM kernel runs between the pipeline's own
+    launches (a reduction kernel there changed the SMs' shared-memory split
+    under the pipeline and cost up to a third of the layer-step rate)."""
+    return torch.zeros((steps, len(layers)) + tuple(layers[0].n_fetch.shape), dtype=torch.int32, pin_memory=True)
+
+
+def record_fetches(hist, i: int, layers):
+    for l, L in enumerate(layers):
+        hist[i, l].copy_(L.n_fetch, non_blocking=True)
+
+
 def isolated_kernel_ms(st, reps: int = 20) -> dict:
     """Each library call of one layer-step timed alone on one stream (no
     concurrent kernels), for per-kernel rooflines.  Before every timed launch
@@ -666,21 +680,20 @@ def run_ablation(args, device):
                 pipe.step(t, [p[t] for p in qpaths])
             pipe.wait_all()
             torch.cuda.synchronize()
-            fetched = torch.zeros((), dtype=torch.int64, device=device)
+            hist = fetch_history(args.steps, layers, device)
             resident_sel = torch.zeros((), dtype=torch.int64, device=device)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(pipe.main)
             for t in range(1 + warm, total):
                 pipe.step(t, [p[t] for p in qpaths])
                 if exact is None:
-                    for L in layers:
-                        fetched += L.n_fetch.sum()
+                    record_fetches(hist, t - 1 - warm, layers)
             pipe.wait_all()
             e1.record(pipe.main)
             torch.cuda.synchronize()
             if exact is None:
                 ms = e0.elapsed_time(e1)
-                nfetch = fetched.item() / (nl * args.steps)           # blocks per layer-step
+                nfetch = hist.sum().item() / (nl * args.steps)        # blocks per layer-step
                 for L in layers:                                       # final plan's fetches landed
                     lsk.block_overlap(d, L.slot_table, L.sel, cover)
                     resident_sel += cover.sum()
@@ -754,18 +767,18 @@ def run_longctx(args, device):
                 pipe.step(t, [p[t] for p in qpaths])
             pipe.wait_all()
             torch.cuda.synchronize()
-            fetched = torch.zeros((), dtype=torch.int64, device=device)
+            hist = fetch_history(steps, layers, device)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(pipe.main)
             for t in range(1 + warm, total):
                 pipe.step(t, [p[t] for p in qpaths])
-                for L in layers:
-                    fetched += L.n_fetch.sum()
+                record_fetches(hist, t - 1 - warm, layers)
             pipe.wait_all()
             e1.record(pipe.main)
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1)
             per_ls = ms / (nl * steps)
+            fetched = hist.sum()
             gbs = fetched.item() * w.block_bytes / (ms * 1e-3) / 1e9
             iso = isolated_kernel_ms({"pipe": pipe, "layers": layers, "dims": d, "qrings": [[qpaths[0][total - 1]]]},
                                      reps=5)
@@ -852,18 +865,18 @@ def run_reasoning(args, device):
             pipe.step(t, qs_at(t), appended=app_at(t))
         pipe.wait_all()
         torch.cuda.synchronize()
-        fetched = torch.zeros((), dtype=torch.int64, device=device)
+        hist = fetch_history(steps, layers, device)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(pipe.main)
         h0 = time.perf_counter()
         for t in range(1 + warm, total):
             pipe.step(t, qs_at(t), appended=app_at(t))
-            for L in layers:
-                fetched += L.n_fetch.sum()
+            record_fetches(hist, t - 1 - warm, layers)
         pipe.wait_all()
         e1.record(pipe.main)
         host_ms = (time.perf_counter() - h0) * 1e3
         torch.cuda.synchronize()
+        fetched = hist.sum()
         ms = e0.elapsed_time(e1)
         ctx_end = int(pipe.ctx_len[0].item())
         per_ls = ms / (nl * steps)
@@ -1007,7 +1020,7 @@ def run_gpu(args, rank, world, device):
     timer = KernelTimer(args.steps * nl)
     pipe.timer = timer
     main = pipe.main
-    fetch_hist = torch.zeros((args.steps, nl, w.batch, w.n_kv_heads), dtype=torch.int32, device=device)
+    fetch_hist = fetch_history(args.steps, layers)
 
     def qs_at(t):
         i = ring_index(t, nq)
@@ -1037,8 +1050,7 @@ def run_gpu(args, rank, world, device):
         h0 = time.perf_counter()
         for i in range(args.steps):
             pipe.step(t, qs_at(t), evict=ms_at(t))
-            for l, L in enumerate(layers):
-                fetch_hist[i, l].copy_(L.n_fetch, non_blocking=True)
+            record_fetches(fetch_hist, i, layers)
             t += 1
         pipe.wait_all()
         ev1.record(main)
