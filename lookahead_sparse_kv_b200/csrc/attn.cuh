@@ -110,13 +110,13 @@ constexpr int kBarPFree = 14;    // P^T read by O^T (commit)
 constexpr int kBarQFull = 16;    // chunk's query rows landed
 constexpr int kBarQFree = 18;    // query rows no longer read (commit after the chunk's last S^T)
 constexpr int kBarLFull = 20;    // chunk description written (producer)
-constexpr int kBarLFree = 22;    // description read by all 11 consumer warps
+constexpr int kBarLFree = 22;    // description read by every consumer (kAttnLFreeCount arrivals)
 constexpr int kBarODone = 24;    // chunk's last O^T product completed (commit)
 constexpr int kBarOFree = 26;    // O^T accumulator, running max and row sums read by the epilogue
 constexpr int kBarSMDone = 28;   // chunk's row sums written by the 4 softmax warps
 constexpr int kBarFinalS = 30;   // teardown: every S^T issued has completed
 constexpr int kBarFinalO = 31;   // teardown: every O^T issued has completed
-constexpr int kAttnLFreeCount = 15;
+constexpr int kAttnLFreeCount = 16;   // 14 consumer warps + the loader's K and V lanes
 
 // named barriers (0 is __syncthreads)
 constexpr uint32_t kNbSoftmax = 1, kNbSoftmaxVote = 2, kNbEpi = 3, kNbEpiVote = 4;
@@ -318,12 +318,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp == kAttnLoaderWarp) {
         // ======================================================= loader
-        if (lane == 0) {
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
+        // lane 0 streams K, lane 1 streams V, each through its own 2-stage
+        // ring: a K tile is requested as soon as its stage's S^T product is
+        // done, without waiting behind the V stage, which stays held until
+        // the O^T product of its tile (after that tile's softmax)
+        if (lane < 2) {
+            const bool is_k = lane == 0;
+            const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+            uint8_t* ring = is_k ? sK : sV;
+            const int bar_full = is_k ? kBarKFull : kBarVFull, bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
+            prefetch_tensormap(tm);
             const uint64_t pol_kv = l2_policy_evict_first();
             int pos = 0;
-            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+            int last[2] = {-1, -1};
             for (int p = 0;; ++p) {
                 const int pb = p & 1;
                 if (!cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort)) break;
@@ -334,30 +341,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int i = 0; i < n; ++i, ++pos) {
                     const int st = pos & 1;
                     const int z = zu + info[8 + 4 * i];              // first pool slot of the tile
-                    if (pos >= 2) cta_wait(&bar[kBarKEmpty + st], ((pos >> 1) - 1) & 1, s_abort);
-                    mbar_arrive_expect_tx(&bar[kBarKFull + st], kAttnStageBytes);
+                    if (pos >= 2) cta_wait(&bar[bar_empty + st], ((pos >> 1) - 1) & 1, s_abort);
+                    mbar_arrive_expect_tx(&bar[bar_full + st], kAttnStageBytes);
                     if (!*s_abort) {
-                        last_k[st] = pos;
-                        uint8_t* dk = sK + st * kAttnStageBytes;
-                        tma_load_3d(dk, &tm_k, &bar[kBarKFull + st], 0, 0, z, pol_kv);
-                        tma_load_3d(dk + kAttnHalf, &tm_k, &bar[kBarKFull + st], 64, 0, z, pol_kv);
-                    }
-                    if (pos >= 2) cta_wait(&bar[kBarVEmpty + st], ((pos >> 1) - 1) & 1, s_abort);
-                    mbar_arrive_expect_tx(&bar[kBarVFull + st], kAttnStageBytes);
-                    if (!*s_abort) {
-                        last_v[st] = pos;
-                        uint8_t* dv = sV + st * kAttnStageBytes;
-                        tma_load_3d(dv, &tm_v, &bar[kBarVFull + st], 0, 0, z, pol_kv);
-                        tma_load_3d(dv + kAttnHalf, &tm_v, &bar[kBarVFull + st], 64, 0, z, pol_kv);
+                        last[st] = pos;
+                        uint8_t* dst = ring + st * kAttnStageBytes;
+                        tma_load_3d(dst, tm, &bar[bar_full + st], 0, 0, z, pol_kv);
+                        tma_load_3d(dst + kAttnHalf, tm, &bar[bar_full + st], 64, 0, z, pol_kv);
                     }
                 }
                 mbar_arrive(&bar[kBarLFree + pb]);
             }
             // no copy may still be writing this CTA's shared memory when it exits
-            for (int st = 0; st < 2; ++st) {
-                if (last_k[st] >= 0) mbar_wait(&bar[kBarKFull + st], static_cast<uint32_t>((last_k[st] >> 1) & 1));
-                if (last_v[st] >= 0) mbar_wait(&bar[kBarVFull + st], static_cast<uint32_t>((last_v[st] >> 1) & 1));
-            }
+            for (int st = 0; st < 2; ++st)
+                if (last[st] >= 0) mbar_wait(&bar[bar_full + st], static_cast<uint32_t>((last[st] >> 1) & 1));
         }
         __syncwarp();
     } else if (warp == kAttnSWarp) {
