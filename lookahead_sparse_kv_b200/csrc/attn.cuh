@@ -41,8 +41,8 @@
 //              current one is listed), lists a chunk's tiles that hold a
 //              valid token (valid-token count of each slot) and loads the
 //              unit's query rows;
-//   warp 12    loader: streams the listed tiles' K and V through two 2-stage
-//              TMA rings (per tile and tensor two 16-KiB boxes of 8 slots x
+//   warp 12    loader: lane 0 streams the listed tiles' K, lane 1 their V,
+//              through two 2-stage TMA rings (per tile and tensor two 16-KiB boxes of 8 slots x
 //              16 rows x 64 columns, 128-byte swizzle).
 //   warp 13    issues S^T (and holds the TMEM allocation).
 //   warp 14    issues O^T; a free slot's product is not issued.
