@@ -149,7 +149,8 @@ def test_lookahead_scores(Hq, Hkv, Qn, N):
 
 # ----------------------------------------------------------------- select
 @pytest.mark.parametrize("N,K,nv_blocks", [(300, 32, 300), (300, 32, 20), (2048, 128, 2048),
-                                           (8192, 256, 8000), (64, 64, 64), (1000, 1000, 999)])
+                                           (8192, 256, 8000), (64, 64, 64), (1000, 1000, 999),
+                                           (301, 32, 297), (4097, 128, 4097)])
 def test_select_topk_bit_exact(N, K, nv_blocks):
     B, H = 2, 3
     d = _dims(B, 6, H, N, K, 2, 1)
@@ -535,6 +536,38 @@ def test_sparse_attention_full_budget_is_dense():
 
 
 # ------------------------------------------------------------ error word
+def test_duplicate_resident_block_sets_error_word_without_fault():
+    """A slot table that holds one block in two slots is an invalid state: the
+    planner (standalone and inside the fused launch) flags it in the device
+    error word and finishes; the other unit's plan is unaffected."""
+    B, H, N, K, C = 1, 2, 64, 8, 3
+    d = _dims(B, 4, H, N, K, 1, C)
+    assert lsk.read_device_error(clear=True) == 0
+    st0 = torch.tensor([[[5, 9, 5, -1, 12, -1, 7, -1], [1, 2, 3, -1, -1, -1, -1, -1]]], dtype=torch.int32)
+    sel = torch.tensor([[[5, 40, 41, 9, -1, -1, -1, -1], [1, 2, 50, 51, 52, -1, -1, -1]]], dtype=torch.int32, device=DEV)
+    st, lu = st0.to(DEV), torch.zeros_like(st0).to(DEV)
+    fs = torch.empty((B, H, C), dtype=torch.int32, device=DEV)
+    fb = torch.empty_like(fs)
+    nf = torch.empty((B, H), dtype=torch.int32, device=DEV)
+    lsk.plan_fetch(d, sel, st, lu, 1, fs, fb, nf)
+    assert lsk.read_device_error(clear=True) & lsk.DEVERR_DUPLICATE
+    # the valid unit: misses 50, 51, 52 into its free slots 3, 4, 5 in slot order
+    ref = O.plan_fetch(np_i32(sel)[:, 1:], st0.numpy()[:, 1:], np.zeros((1, 1, K), np.int32), 1, C)
+    np.testing.assert_array_equal(np_i32(st)[:, 1:], ref["slot_table"])
+    np.testing.assert_array_equal(np_i32(nf)[:, 1:], ref["n_fetch"])
+    # the fused launch on the same state
+    g = _gen(77)
+    q = torch.randn((B, 1, 4, 128), generator=g).to(torch.bfloat16).to(DEV)
+    kmin = (torch.randn((B, H, N, 128), generator=g) - 1).to(torch.bfloat16).to(DEV)
+    kmax = (kmin.float() + 2).to(torch.bfloat16)
+    ctx = torch.tensor([N * 16], dtype=torch.int32, device=DEV)
+    ws = torch.zeros(lsk.workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    st2, lu2 = st0.to(DEV), torch.zeros_like(st0).to(DEV)
+    sel2 = torch.empty_like(sel)
+    lsk.score_select_plan(d, q, kmin, kmax, ctx, sel2, None, None, st2, lu2, 1, None, fs, fb, nf, ws)
+    assert lsk.read_device_error(clear=True) & lsk.DEVERR_DUPLICATE
+
+
 def test_out_of_range_ids_set_error_word_without_fault():
     B, H, N, K = 1, 1, 10, 4
     d = _dims(B, 2, H, N, K, 1, 2)
