@@ -28,7 +28,8 @@
 //   warps 6-9 run the top-K selection and the plan of a unit once all of it
 //             is scored, while the other warps score on.
 // Two ways a unit reaches the selection:
-//   - whole units (a chunk covers a unit, used when units >= CTAs): the
+//   - whole units (a chunk covers a unit; the host picks this with at least
+//     half as many units as SMs, else about two chunks per SM): the
 //     epilogue also keeps the unit's keys in shared memory and hands them to
 //     the CTA's own selection warps (an mbarrier each way), which read them
 //     into registers;
