@@ -244,8 +244,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // ======================================================= lister
         if (lane == 0) prefetch_tensormap(&tm_q);
         const uint64_t pol_q = l2_policy_evict_last();
-        int c_next = 0;
-        if (lane == 0) c_next = atomicAdd(ws_sched, 1);
+        // the first chunk of each CTA is its block index (grid <= chunks), the
+        // rest come from the counter, numbered from the grid size on
+        int c_next = static_cast<int>(blockIdx.x);
         for (int p = 0;; ++p) {
             const int pb = p & 1;
             int* info = s_info + pb * kAttnInfoInts;
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 break;
             }
-            if (lane == 0) c_next = atomicAdd(ws_sched, 1);    // lands while this chunk is listed
+            if (lane == 0) c_next = static_cast<int>(gridDim.x) + atomicAdd(ws_sched, 1);   // lands while this chunk is listed
             const int u = c / ch.cpu, j = c - u * ch.cpu;
             const int lo = j * ch.ct * kAttnTileSlots, hi = min(lo + ch.ct * kAttnTileSlots, K);
             const int b = u / d.Hkv, h = u - b * d.Hkv;

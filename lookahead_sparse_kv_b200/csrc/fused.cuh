@@ -205,8 +205,9 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             }
             ++pos;
         };
-        int c_next = 0;                                    // requested one chunk ahead
-        if (lane == 0) c_next = atomicAdd(sched, 1);
+        // requested one chunk ahead: the first is the CTA's block index (grid <=
+        // chunks), the rest come from the counter, numbered from the grid size on
+        int c_next = static_cast<int>(blockIdx.x);
         for (int p = 0;; ++p) {
             const int pb = p & 1;
             int* info = s_info + pb * kSspInfoInts;
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             while (true) {
                 if (lane == 0) {
                     c = *s_abort ? ch.nc : c_next;
-                    if (c < ch.nc) c_next = atomicAdd(sched, 1);
+                    if (c < ch.nc) c_next = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);
                 }
                 c = __shfl_sync(0xFFFFFFFFu, c, 0);
                 if (c >= ch.nc) break;
