@@ -90,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, u
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (global_timer_ns() - t0 > limit_ns) return false;
-        __nanosleep(128);
+        __nanosleep(32);
     }
     return true;
 }
