@@ -460,20 +460,10 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             const int nv = n_valid_blocks(ctx_len[u / d.Hkv], d.N);
             const float* su = scores + u * N;
             const long long uk = static_cast<long long>(u) * d.K, uc = static_cast<long long>(u) * d.C;
-            // the unit's slot table and recency, loaded now and used by the plan
-            // after the selection (the loads are in flight meanwhile)
-            const bool pre = slot_table != nullptr && d.K <= 2 * SspTailGroup::kThreads;
-            int32_t pst[2] = {-1, -1}, plu[2] = {0, 0};
-            if (pre) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int i = ttid + h * SspTailGroup::kThreads;
-                    if (i < d.K) {
-                        pst[h] = __ldcg(slot_table + uk + i);
-                        plu[h] = __ldcg(last_used + uk + i);
-                    }
-                }
-            }
+            // the unit's slot table and recency, copied into the plan's shared
+            // memory now (asynchronously) and used by the plan after the selection
+            const bool pre = slot_table != nullptr;
+            if (pre) plan_stage_async<SspTailGroup>(d.K, slot_table + uk, last_used + uk, sp);
             int32_t* sel_u = sel + static_cast<long long>(u) * d.K;
             float* ss_u = sel_score ? sel_score + static_cast<long long>(u) * d.K : nullptr;
             uint64_t* kfree = ch.whole ? &bar[kSspKFree] : nullptr;
@@ -501,7 +491,7 @@ __global__ void __launch_bounds__(kSspThreads, 1) score_select_plan_kernel(
             const int stp = step_dev != nullptr ? *step_dev : step;
             plan_unit<SspTailGroup, kScored>(d.K, d.C, d.N, s_sel, kScored ? su : nullptr, slot_table + uk,
                                              last_used + uk, stp, fetch_slot + uc, fetch_block + uc, n_fetch + u, sp,
-                                             tmp, pre ? pst : nullptr, pre ? plu : nullptr);
+                                             tmp, pre);
             SspTailGroup::sync();                              // scratch free for the next unit
         }
     }

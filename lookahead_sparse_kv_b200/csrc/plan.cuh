@@ -49,6 +49,19 @@ __host__ __device__ constexpr int plan_smem_ints(int K) { return 10 * plan_k4(K)
 // there itself and pass this pointer as `sel`.
 __device__ __forceinline__ int32_t* plan_sel_smem(int32_t* sp, int K) { return sp + 6 * plan_k4(K); }
 
+// Starts copying a unit's slot table and recency into the plan's shared
+// memory (each thread its slots tid, tid + NT, ...), for plan_unit(...,
+// staged = true) to use once they have landed.
+template <class Grp>
+__device__ __forceinline__ void plan_stage_async(int K, const int32_t* st, const int32_t* lu, int32_t* sp) {
+    const int K4 = plan_k4(K);
+    for (int i = Grp::tid(); i < K; i += Grp::kThreads) {
+        cp_async_4(sp + i, st + i);
+        cp_async_4(sp + K4 + i, lu + i);
+    }
+    cp_async_commit();
+}
+
 constexpr uint32_t kPlanHashEmpty = 0xFFFFFFFFu;
 __device__ __forceinline__ uint32_t plan_hash(uint32_t blk, int log2_size) {
     return (blk * 0x9E3779B1u) >> (32 - log2_size);
@@ -58,12 +71,12 @@ __device__ __forceinline__ uint32_t plan_hash(uint32_t blk, int log2_size) {
 // ranks): sel, st, lu point at the unit's K entries, fs/fb at its C fetch
 // entries, nf at its fetch count; scores_u (kScored) at its N block scores.
 // sp: plan_smem_ints(K) ints of shared memory, 16-B aligned; tmp: 32 ints.
-// pre_st / pre_lu (K <= 2 * NT, may be NULL): st[tid + h * NT] and
-// lu[tid + h * NT] for h = 0, 1, already loaded by the caller.
+// staged: the caller has already copied st and lu into the first two arrays
+// of sp (plan_stage_async, each thread its own slots tid, tid + NT, ...).
 template <class Grp, bool kScored>
 __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* scores_u, int32_t* st, int32_t* lu,
                           int step, int32_t* fs, int32_t* fb, int32_t* nf, int32_t* sp, int* tmp,
-                          const int32_t* pre_st = nullptr, const int32_t* pre_lu = nullptr) {
+                          bool staged = false) {
     constexpr int NT = Grp::kThreads;
     const int K4 = plan_k4(K);
     int32_t* s_st = sp;
@@ -108,10 +121,9 @@ __device__ void plan_unit(int K, int C, int N, const int32_t* sel, const float* 
             s_sel[i] = sv;
         }
     };
-    if (pre_st != nullptr) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-            if (tid + h * NT < K) stage(tid + h * NT, pre_st[h], pre_lu[h]);
+    if (staged) {
+        cp_async_wait_all();                 // this thread's own copies have landed
+        for (int i = tid; i < K; i += NT) stage(i, s_st[i], s_lu[i]);
     } else {
         for (int i = tid; i < K; i += NT) stage(i, st[i], lu[i]);
     }

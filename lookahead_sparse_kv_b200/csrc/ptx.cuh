@@ -95,6 +95,14 @@ __device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, u
     return true;
 }
 
+// 4-byte asynchronous copy from global to shared memory (no register on the
+// way; completes in the background until cp_async_wait_all).
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Load with acquire semantics at GPU scope (pairs with a release by a
 // __threadfence() + atomic in another CTA).
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
