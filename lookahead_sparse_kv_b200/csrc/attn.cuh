@@ -17,8 +17,9 @@
 //                             bf16 remainder (~16 significant bits), side by
 //                             side along N, so head and remainder products land
 //                             in two column ranges that the epilogue adds; with
-//                             32 rows the two share a 128-B row and P^T is
-//                             double-buffered, with 64 they take a region each
+//                             32 rows the two share a 128-B row, with 64 they
+//                             take a region each; P^T is double-buffered, so a
+//                             tile's softmax overlaps the previous tile's product
 // NR = 32 or 64 is the row count padded to the MMA's N.  A tile is 8 pool
 // slots (128 tokens).  In TMEM, lane i of S^T is token i of the tile (a
 // softmax thread owns a token and reads its NR scores), lane i of O^T is
@@ -79,12 +80,11 @@ constexpr int kAttnTmemCols = 512;                                 // S^T x 2 (6
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kAttnLazy = 32.f;                                  // rescale when a score passes m + 32 (log2)
 
-// shared memory, from the 1024-B aligned base
+// shared memory, from the 1024-B aligned base: the K and V rings, the small
+// arrays, then the query rows and P^T, whose size depends on the row count
 constexpr int kAttnOffK = 0;                                       // K ring, 2 stages
 constexpr int kAttnOffV = kAttnOffK + 2 * kAttnStageBytes;         // V ring, 2 stages
-constexpr int kAttnOffQ = kAttnOffV + 2 * kAttnStageBytes;         // 2 buffers x 2 halves
-constexpr int kAttnOffP = kAttnOffQ + 4 * kAttnQHalf;              // P^T: two [128 tokens][128 B] regions
-constexpr int kAttnOffInfo = kAttnOffP + 2 * kAttnHalf;            // 2 chunk descriptions
+constexpr int kAttnOffInfo = kAttnOffV + 2 * kAttnStageBytes;      // 2 chunk descriptions
 constexpr int kAttnOffBar = kAttnOffInfo + 2 * kAttnInfoInts * 4;
 constexpr int kAttnNumBars = 32;
 constexpr int kAttnOffMisc = kAttnOffBar + kAttnNumBars * 8;       // 8 ints
@@ -96,7 +96,17 @@ constexpr int kAttnOffFin = kAttnOffLw + 2 * 4 * 64 * 4;           // [2][64] 1/
 constexpr int kAttnMaxChunks = 8;                                  // chunks per unit (merge weights)
 constexpr int kAttnOffMw = kAttnOffFin + 4 * 64 * 4;               // [64][8] merge weights
 constexpr int kAttnOffThr = kAttnOffMw + 64 * kAttnMaxChunks * 4;  // [2][64] raw-score thresholds
-constexpr int kAttnSmem = kAttnOffThr + 2 * 64 * 4 + 1024;         // + alignment slack
+constexpr int kAttnOffQ = (kAttnOffThr + 2 * 64 * 4 + 1023) / 1024 * 1024;
+// Query buffers (2 halves each) and P^T buffers.  With 32 rows a 128-B row
+// per token holds P^T's head (bytes 0-63 of the row before swizzling) and
+// remainder (64-127), and the query rows are double-buffered across chunks;
+// with 64 rows head and remainder fill a [128 tokens][128 B] region each, and
+// a single query buffer leaves room for the second P^T buffer.
+constexpr int attn_q_bufs(int nr) { return nr == 64 ? 1 : 2; }
+constexpr int attn_p_buf_bytes(int nr) { return (nr == 64 ? 2 : 1) * kAttnHalf; }
+constexpr int attn_off_p(int nr) { return kAttnOffQ + attn_q_bufs(nr) * 2 * kAttnQHalf; }
+constexpr int attn_smem(int nr) { return attn_off_p(nr) + 2 * attn_p_buf_bytes(nr) + 1024; }   // + alignment slack
+static_assert(attn_smem(32) <= 227 * 1024 && attn_smem(64) <= 227 * 1024, "attention shared memory");
 
 // mbarriers ([2] = one per ring stage / buffer)
 constexpr int kBarKFull = 0;     // K tile landed (producer expect_tx)
@@ -118,8 +128,10 @@ constexpr int kBarFinalS = 30;   // teardown: every S^T issued has completed
 constexpr int kBarFinalO = 31;   // teardown: every O^T issued has completed
 constexpr int kAttnLFreeCount = 16;   // 14 consumer warps + the loader's K and V lanes
 
-// named barriers (0 is __syncthreads)
+// named barriers (0 is __syncthreads); the softmax warps of the low rows (warps
+// 0-3) and of the high rows (warps 4-7) each have their own pair
 constexpr uint32_t kNbSoftmax = 1, kNbSoftmaxVote = 2, kNbEpi = 3, kNbEpiVote = 4;
+constexpr uint32_t kNbSoftmaxHi = 5, kNbSoftmaxVoteHi = 6;
 
 // Chunking of the attention work (host and device agree through these).
 struct AttnChunks {
@@ -184,10 +196,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        float* __restrict__ out, float* __restrict__ lse_out, float* ws_o, float* ws_lse,
                        int* ws_ticket, int* ws_sched) {
     static_assert(NR == 32 || NR == 64, "rows are padded to 32 or 64");
-    // P^T buffers: with 32 rows one 128-B row per token holds the head (bytes
-    // 0-63 of the row before swizzling) and the remainder (64-127), two
-    // buffers; with 64 rows head and remainder fill one region each, one buffer.
-    constexpr int kPBufs = NR == 32 ? 2 : 1;
+    constexpr int kPBufs = 2;                                     // P^T buffers
+    constexpr int kPBufBytes = attn_p_buf_bytes(NR);
+    constexpr int kQBufs = attn_q_bufs(NR);                      // query-row buffers
     // TMEM columns: S^T buffers at 0 and 64, O^T buffers (head and remainder
     // products side by side) at 128 and 128 + 2 NR, 64-row sums after them
     constexpr uint32_t kOCol = 128, kOStride = 2 * NR;
@@ -197,7 +208,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t* sK = smem + kAttnOffK;
     uint8_t* sV = smem + kAttnOffV;
     uint8_t* sQ = smem + kAttnOffQ;
-    uint8_t* sP = smem + kAttnOffP;
+    uint8_t* sP = smem + attn_off_p(NR);
     int* s_info = reinterpret_cast<int*>(smem + kAttnOffInfo);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kAttnOffBar);
     int* misc = reinterpret_cast<int*>(smem + kAttnOffMisc);
@@ -307,10 +318,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 info[3] = ch.cpu;
                 mbar_arrive(&bar[kBarLFull + pb]);
                 // the unit's query rows: box {64 columns, G heads, Qn rows} per 64-column half
-                if (p >= 2) cta_wait(&bar[kBarQFree + pb], ((p >> 1) - 1) & 1, s_abort);
+                // (after the S^T products of the chunk that last used the buffer)
+                if (p >= kQBufs) cta_wait(&bar[kBarQFree + ((p - kQBufs) & 1)], ((p - kQBufs) >> 1) & 1, s_abort);
                 mbar_arrive_expect_tx(&bar[kBarQFull + pb], static_cast<uint32_t>(rows) * kRowBytes);
                 if (!*s_abort) {
-                    uint8_t* q_dst = sQ + pb * 2 * kAttnQHalf;
+                    uint8_t* q_dst = sQ + (p % kQBufs) * 2 * kAttnQHalf;
                     tma_load_3d(q_dst, &tm_q, &bar[kBarQFull + pb], 0, h * G, b * d.Qn, pol_q);
                     tma_load_3d(q_dst + kAttnQHalf, &tm_q, &bar[kBarQFull + pb], 64, h * G, b * d.Qn, pol_q);
                 }
@@ -369,7 +381,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int n = s_info[pb * kAttnInfoInts];
                 if (n < 0) break;
                 cta_wait(&bar[kBarQFull + pb], (p >> 1) & 1, s_abort);
-                const uint32_t qa = smem_addr(sQ + pb * 2 * kAttnQHalf);
+                const uint32_t qa = smem_addr(sQ + (p % kQBufs) * 2 * kAttnQHalf);
                 for (int i = 0; i < n; ++i, ++sp) {
                     const int st = sp & 1;
                     bool ok = cta_wait(&bar[kBarKFull + st], (sp >> 1) & 1, s_abort);
@@ -418,7 +430,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const uint32_t nvlo = static_cast<uint32_t>(info[8 + 4 * i + 1]);
                         const uint32_t nvhi = static_cast<uint32_t>(info[8 + 4 * i + 2]);
                         const uint32_t va = smem_addr(sV + st * kAttnStageBytes);
-                        const uint32_t pa = smem_addr(sP + pbuf * kAttnHalf);
+                        const uint32_t pa = smem_addr(sP + pbuf * kPBufBytes);
 #pragma unroll
                         for (int kk = 0; kk < kAttnTileSlots; ++kk) {
                             const uint32_t nv = ((kk < 4 ? nvlo : nvhi) >> (8 * (kk & 3))) & 0xFFu;
@@ -441,10 +453,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
     } else if (warp < kAttnSoftmaxWarps) {
         // ================================== softmax (token / thread, half the rows / warp)
+        // The two row halves share no running max, sum or O^T column, so each
+        // half (one warp per TMEM lane quadrant) votes and syncs on its own.
         constexpr int kH = NR / 2;                            // rows per thread
-        constexpr int kSm = 32 * kAttnSoftmaxWarps;           // softmax threads
+        constexpr int kSm = 32 * kAttnSoftmaxWarps / 2;       // softmax threads of a row half
         const int q = warp & 3;                               // TMEM lane quadrant
         const int r0 = (warp >> 2) * kH;                      // first row of this warp
+        const uint32_t nb_sync = r0 == 0 ? kNbSoftmax : kNbSoftmaxHi;
+        const uint32_t nb_vote = r0 == 0 ? kNbSoftmaxVote : kNbSoftmaxVoteHi;
         const int tok = 32 * q + lane;                        // token of the tile this thread owns
         const int myslot = tok >> 4, mytok = tok & 15;
         const float inv_scale = 1.f / scale_log2;             // thresholds in raw-score units
@@ -455,7 +471,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             cta_wait(&bar[kBarLFull + pb], (p >> 1) & 1, s_abort);
             const int* info = s_info + pb * kAttnInfoInts;
             const int n = info[0];
-            if (named_bar_or(kNbSoftmaxVote, kSm, n < 0 || *s_abort)) break;
+            if (named_bar_or(nb_vote, kSm, n < 0 || *s_abort)) break;
             // the epilogue of chunk p-2 has read this buffer's running max and sums
             if (p >= 2) cta_wait(&bar[kBarOFree + pb], ((p >> 1) - 1) & 1, s_abort);
             // running max m (log2 units) and the raw-score threshold (m + 32) / scale of
@@ -464,10 +480,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // probabilities are 0 (the padded columns are never read)
             float* mr = s_m + pb * 64;
             float* thr = s_thr + pb * 64;
-            if (warp == 0) {
+            if (q == 0 && lane < kH && r0 + lane >= rows) {
                 const float kPosInf = __int_as_float(0x7f800000);
-                if (lane >= rows) mr[lane] = thr[lane] = kPosInf;
-                if (lane + 32 >= rows) mr[lane + 32] = thr[lane + 32] = kPosInf;
+                mr[r0 + lane] = thr[r0 + lane] = kPosInf;
             }
             float l[kH];                                      // this token's share of its rows' sums
 #pragma unroll
@@ -510,7 +525,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                 thr[r0 + r] = (m0 + kAttnLazy) * inv_scale;
                             }
                     }
-                    named_bar_sync(kNbSoftmax, kSm);
+                    named_bar_sync(nb_sync, kSm);
                 }
                 // does any row's running max move (by more than 2^32)?
                 bool up = false;
@@ -521,7 +536,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         up |= (x[r] > t4.x) | (x[r + 1] > t4.y) | (x[r + 2] > t4.z) | (x[r + 3] > t4.w);
                     }
                 }
-                if (named_bar_or(kNbSoftmaxVote, kSm, up)) {
+                if (named_bar_or(nb_vote, kSm, up)) {
                     // tile maxima (log2 units): lane r of each warp keeps row r0 + r of its tokens
                     float mine = kNegInf;
 #pragma unroll
@@ -530,7 +545,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         if (lane == r) mine = wm;
                     }
                     if (lane < kH) s_wmax[q * 64 + r0 + lane] = mine;
-                    named_bar_sync(kNbSoftmax, kSm);
+                    named_bar_sync(nb_sync, kSm);
                     if (q == 0 && lane < kH) {                // warps 0 and 4: their rows
                         const int r = r0 + lane;
                         const float tmx = fmaxf(fmaxf(s_wmax[r], s_wmax[64 + r]), fmaxf(s_wmax[128 + r], s_wmax[192 + r]));
@@ -543,7 +558,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         }
                         s_alpha[r] = a;
                     }
-                    named_bar_sync(kNbSoftmax, kSm);
+                    named_bar_sync(nb_sync, kSm);
 #pragma unroll
                     for (int r = 0; r < kH; ++r) l[r] *= s_alpha[r0 + r];
                     if (i > 0) {
@@ -567,11 +582,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         tmem_st_wait();
                     }
                 }
-                // this token's probabilities for this warp's rows, head and remainder (bf16
-                // each), once the product that last read this P^T buffer is done
-                const int pbuf = pos % kPBufs;
-                if (pos >= kPBufs) cta_wait(&bar[kBarPFree + pbuf], ((pos / kPBufs) - 1) & 1, s_abort);
-                uint8_t* prow = sP + pbuf * kAttnHalf + tok * 128;
+                // this token's probabilities for this warp's rows as bf16 head and
+                // remainder words, computed before the wait for the product that last
+                // read this P^T buffer (with one buffer, the previous tile's), so the
+                // exponentials overlap that product; the words of rows r..r+7 replace
+                // their scores in x (head words first, then remainder words)
                 if (valid) {
 #pragma unroll
                     for (int c8 = 0; c8 < kH / 8; ++c8) {
@@ -596,15 +611,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         l[r + 7] += p7;
                         const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
                         const uint32_t h45 = pack_bf16x2(p4, p5), h67 = pack_bf16x2(p6, p7);
+                        x[r + 0] = __uint_as_float(h01);
+                        x[r + 1] = __uint_as_float(h23);
+                        x[r + 2] = __uint_as_float(h45);
+                        x[r + 3] = __uint_as_float(h67);
+                        x[r + 4] = __uint_as_float(pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01)));
+                        x[r + 5] = __uint_as_float(pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23)));
+                        x[r + 6] = __uint_as_float(pack_bf16x2(p4 - bf16_lo(h45), p5 - bf16_hi(h45)));
+                        x[r + 7] = __uint_as_float(pack_bf16x2(p6 - bf16_lo(h67), p7 - bf16_hi(h67)));
+                    }
+                }
+                const int pbuf = pos % kPBufs;
+                if (pos >= kPBufs) cta_wait(&bar[kBarPFree + pbuf], ((pos / kPBufs) - 1) & 1, s_abort);
+                uint8_t* prow = sP + pbuf * kPBufBytes + tok * 128;
+                if (valid) {
+#pragma unroll
+                    for (int c8 = 0; c8 < kH / 8; ++c8) {
                         const int cg = r0 / 8 + c8;                           // 16-B chunk of the row
                         const int off = (cg ^ (tok & 7)) << 4;
                         const int roff = NR == 32 ? (((cg + 4) ^ (tok & 7)) << 4) : kAttnHalf + off;
-                        *reinterpret_cast<uint4*>(prow + off) = make_uint4(h01, h23, h45, h67);
+                        const int r = 8 * c8;
+                        *reinterpret_cast<uint4*>(prow + off) =
+                            make_uint4(__float_as_uint(x[r]), __float_as_uint(x[r + 1]),
+                                       __float_as_uint(x[r + 2]), __float_as_uint(x[r + 3]));
                         *reinterpret_cast<uint4*>(prow + roff) =
-                            make_uint4(pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01)),
-                                       pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23)),
-                                       pack_bf16x2(p4 - bf16_lo(h45), p5 - bf16_hi(h45)),
-                                       pack_bf16x2(p6 - bf16_lo(h67), p7 - bf16_hi(h67)));
+                            make_uint4(__float_as_uint(x[r + 4]), __float_as_uint(x[r + 5]),
+                                       __float_as_uint(x[r + 6]), __float_as_uint(x[r + 7]));
                     }
                 } else {
                     // a token past the context or in a free slot: zero weights; in an occupied

@@ -749,9 +749,11 @@ int oasis_sparse_attn(const oasis_dims* dp, const void* q, const void* pool, con
     // are taken from a counter, so fewer CTAs only take more chunks each).
     const int grid_max = std::max(1, sm_count() - oasis::kPrefetchCtas);
     const unsigned ctas = static_cast<unsigned>(std::min(grid_max, chunks.nc));
-    auto kern = d.Qn * d.G() <= 32 ? oasis::sparse_attn_kernel<32> : oasis::sparse_attn_kernel<64>;
-    if (int rc = set_smem(kern, oasis::kAttnSmem, "sparse_attn smem")) return rc;
-    kern<<<ctas, oasis::kAttnThreads, oasis::kAttnSmem, s>>>(tk, tv, tq, d, slot_table, ctx_len, scale_log2, chunks,
+    const bool r32 = d.Qn * d.G() <= 32;
+    auto kern = r32 ? oasis::sparse_attn_kernel<32> : oasis::sparse_attn_kernel<64>;
+    const int smem = oasis::attn_smem(r32 ? 32 : 64);
+    if (int rc = set_smem(kern, smem, "sparse_attn smem")) return rc;
+    kern<<<ctas, oasis::kAttnThreads, smem, s>>>(tk, tv, tq, d, slot_table, ctx_len, scale_log2, chunks,
                                                              out, lse, ws_o, ws_lse, ws_ticket, ws_sched);
     return check_launch("sparse_attn launch");
 }
