@@ -485,6 +485,48 @@ def test_sparse_attention(Hq, Hkv, Qn, K):
         assert_attention_close(out, lse, o_ref, lse_ref)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,Qn,K", [(40, 32, 4, 8, 16),     # 64 rows, 160 whole units
+                                           (35, 16, 2, 8, 128),    # 64 rows, 70 units of 2 chunks
+                                           (40, 16, 4, 5, 16)])    # 20 rows, 160 whole units
+def test_sparse_attention_more_chunks_than_ctas(B, Hq, Hkv, Qn, K):
+    """More chunks than the launch has CTAs (at most one per SM, less the
+    gather's 16), so CTAs take further chunks from the counter: a chunk's
+    query rows land in the buffer the CTA's previous chunk read (the only one
+    with 64 rows) once that chunk's S^T products are done, and split units
+    are merged by whichever of their chunks finishes last."""
+    N = K + 7
+    d = _dims(B, Hq, Hkv, N, K, Qn, 4)
+    g = _gen(900 + B + K)
+    kv = random_kv(B, Hkv, N, g)
+    q = torch.randn(B, Qn, Hq, 128, generator=g).to(torch.bfloat16)
+    rng = np.random.default_rng(B * K)
+    ctx = torch.from_numpy(rng.integers(K * 16 - 40, N * 16 + 1, size=B).astype(np.int32))
+    nvb = O.n_valid_blocks(ctx.numpy(), 16)
+    st = np.full((B, Hkv, K), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(Hkv):
+            blocks = rng.permutation(N)[:K]          # includes blocks beyond the context
+            st[b, h] = np.where(rng.random(K) < 0.85, blocks, -1)
+            st[b, h][st[b, h] == nvb[b] - 1] = -1
+            st[b, h, rng.integers(K)] = nvb[b] - 1   # the partial last block
+    st[B - 1, Hkv - 1] = -1                          # a head with nothing resident
+    idx = torch.from_numpy(np.maximum(st, 0)).long()
+    pool = kv[torch.arange(B)[:, None, None], torch.arange(Hkv)[None, :, None], idx]
+    pool[torch.from_numpy(st < 0)] = 0
+    scale = 1 / math.sqrt(128)
+    out = torch.empty((B, Qn, Hq, 128), device=DEV)
+    lse = torch.empty((B, Qn, Hq), device=DEV)
+    ws = torch.zeros(lsk.workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    pk, pv = kv_split(pool)
+    o_ref, lse_ref = O.sparse_attention(f64(q), pk, pv, st, ctx.numpy(), scale)
+    for _ in range(2):                                # second call reuses the zeroed counters
+        out.fill_(float("nan"))
+        lsk.sparse_attn(d, q.to(DEV), pool.to(DEV), torch.from_numpy(st).to(DEV), ctx.to(DEV),
+                        scale, out, lse, ws)
+        torch.cuda.synchronize()
+        assert_attention_close(out, lse, o_ref, lse_ref)
+
+
 def test_sparse_attention_masks_garbage_beyond_context():
     """Values of tokens beyond ctx_len (NaN here) never reach the output."""
     B, Hq, Hkv, K, N = 1, 4, 1, 8, 20
